@@ -1,0 +1,249 @@
+"""fp64 CPU oracle for the BaKron solver.
+
+TEST INFRASTRUCTURE ONLY. Nothing in the product path may import this module: only ``tests/``,
+``__graft_entry__.smoke()`` and the CPU-baseline leg of ``bench.py`` use it. It shares no code
+with the CUDA path.
+
+Sources (web pages on the method):
+* [BaKron] "BaKron: Efficient Quantization with Kronecker-Factored Hessians", summary and
+  abstract (insight.aitobox.com, 2026-08-07 post): two-sided adaptive rounding in the
+  BoA/YAQA formulation, anti-diagonal parallelism, O(m+n) sequential steps,
+  O(mn(m+n)) total work.
+* [YAQA] YAQA article (news.43b.com.cn/a/479517.html):
+  - section 2: the layer objective 1/2 (W-W*)^T (grad^2 L) (W-W*) with the Kronecker
+    approximation grad^2 L ~ H_O (m x m) (x) H_I (n x n);
+  - section 4: the rounding rule
+        W_ij = Q(W*_ij + a_i^T (W*-W)[:i,:j] b_j + a_i^T (W*-W)[:i,j] + (W*-W)[i,:j] b_j),
+    a_i column i of the strictly upper triangular m x m L_O, b_j column j of the strictly upper
+    triangular n x n L_I, Q nearest (or stochastic) rounding;
+  - section 4: the factorisation H_O = (L_O + I) D_O (L_O + I)^T (likewise H_I) and the bound
+    dW (H_O (x) H_I) dW^T <= tr(D_I) tr(D_O) sigma^2.
+
+Readings taken where the pages are garbled or silent (each one is listed in the design notes):
+* index ranges ``:i`` / ``:j`` are exclusive (rows k < i, columns l < j);
+* L is strictly *upper* triangular, so H = (I+L) D (I+L)^T is a U D U^T factorisation
+  (the section-4 text also calls it "unit lower"; only the upper reading makes the rule causal
+  and the bound hold);
+* Q is round-half-to-even of pre/s_i followed by a clamp to [-2^(b-1), 2^(b-1)-1], per-row
+  scale s_i; s_i = 0 gives code 0;
+* E = W* - W always includes the clamp error;
+* the proxy loss is tr(H_O dW H_I dW^T) with no factor 1/2.
+
+Parity status: every function below is pinned by ``tests/test_oracle.py`` against closed
+forms, textbook routines (numpy Cholesky, the GPTQ/OBS update on the vectorised problem),
+special cases and brute force. No worked numerical example is printed on the pages, so there
+is no golden value from the pages themselves.
+"""
+from __future__ import annotations
+
+import itertools
+
+import numpy as np
+
+__all__ = [
+    "udu", "quantize", "round_naive", "round_row_sweep", "fixed_point_pre",
+    "proxy_loss", "proxy_loss_kron", "brute_force_fixed_points", "gptq_obs",
+    "code_range",
+]
+
+
+def code_range(bits: int) -> tuple[int, int]:
+    return -(1 << (bits - 1)), (1 << (bits - 1)) - 1
+
+
+# ---------------------------------------------------------------------------------------------
+# Factorisation: H = (I + L) D (I + L)^T, L strictly upper triangular ([YAQA] section 4).
+# ---------------------------------------------------------------------------------------------
+def udu(H: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
+    """Textbook U D U^T factorisation, last index first, in fp64.
+
+    For j = d-1 down to 0:
+        D_j      = H_jj - sum_{k>j} U_jk^2 D_k
+        U_ij     = (H_ij - sum_{k>j} U_ik U_jk D_k) / D_j      for i < j
+    with U = I + L. Returns (L, D): L strictly upper (zeros on and below the diagonal).
+    Raises ValueError on a non-positive or non-finite pivot.
+    """
+    H = np.asarray(H, dtype=np.float64)
+    d = H.shape[0]
+    U = np.eye(d)
+    D = np.zeros(d)
+    for j in range(d - 1, -1, -1):
+        tail = slice(j + 1, d)
+        D[j] = H[j, j] - np.dot(U[j, tail] ** 2, D[tail])
+        if not np.isfinite(D[j]) or D[j] <= 0.0:
+            raise ValueError(f"non-positive pivot at index {j}: {D[j]}")
+        if j > 0:
+            U[:j, j] = (H[:j, j] - U[:j, tail] @ (U[j, tail] * D[tail])) / D[j]
+    L = U - np.eye(d)
+    return L, D
+
+
+# ---------------------------------------------------------------------------------------------
+# Base quantizer Q ([YAQA] section 4: nearest rounding; reading: half-even, then clamp).
+# ---------------------------------------------------------------------------------------------
+def quantize(pre: float, s: float, bits: int) -> int:
+    """Code for one entry: clamp(round_half_even(pre / s)); s == 0 gives 0."""
+    lo, hi = code_range(bits)
+    if s == 0.0:
+        return 0
+    c = float(np.rint(pre / s))
+    return int(min(max(c, lo), hi))
+
+
+# ---------------------------------------------------------------------------------------------
+# The rule, entry by entry, in raster order ([YAQA] section 4). Raster order is a valid order
+# because entry (i, j) reads only entries (k, l) with k <= i and l <= j, (k, l) != (i, j).
+# ---------------------------------------------------------------------------------------------
+def round_naive(Wstar, L_O, L_I, scales, bits, return_pre=False):
+    """Plain definition, O(m^2 n^2 / 4) multiply-adds.
+
+    pre_ij = W*_ij + a_i^T E[:i,:j] b_j + a_i^T E[:i,j] + E[i,:j] b_j,   E = W* - W
+    with a_i = L_O[:i, i] and b_j = L_I[:j, j].
+    Returns (codes int64 m x n, W fp64 m x n[, pre fp64 m x n]).
+    """
+    Ws = np.asarray(Wstar, dtype=np.float64)
+    LO = np.asarray(L_O, dtype=np.float64)
+    LI = np.asarray(L_I, dtype=np.float64)
+    s = np.asarray(scales, dtype=np.float64)
+    m, n = Ws.shape
+    E = np.zeros((m, n))
+    W = np.zeros((m, n))
+    C = np.zeros((m, n), dtype=np.int64)
+    P = np.zeros((m, n))
+    for i in range(m):
+        a = LO[:i, i]
+        for j in range(n):
+            b = LI[:j, j]
+            pre = Ws[i, j]
+            if i > 0 and j > 0:
+                pre += (a @ E[:i, :j]) @ b
+            if i > 0:
+                pre += a @ E[:i, j]
+            if j > 0:
+                pre += E[i, :j] @ b
+            c = quantize(pre, s[i], bits)
+            C[i, j] = c
+            W[i, j] = s[i] * c
+            E[i, j] = Ws[i, j] - W[i, j]
+            P[i, j] = pre
+    return (C, W, P) if return_pre else (C, W)
+
+
+def round_row_sweep(Wstar, L_O, L_I, scales, bits, return_pre=False):
+    """Same result as ``round_naive`` in O(mn(m+n)) work (the row-by-row reading).
+
+    Row i sees every earlier row only through T_i = sum_{k<i} L_O[k,i] E_k (a row vector).
+    Substituting into the rule gives pre_ij = r_j + sum_{l<j} E_il L_I[l,j] with
+    r = W*_i + T_i + T_i L_I, i.e. one-sided LDLQ of the biased row (a left-to-right pass).
+    """
+    Ws = np.asarray(Wstar, dtype=np.float64)
+    LO = np.asarray(L_O, dtype=np.float64)
+    LI = np.asarray(L_I, dtype=np.float64)
+    s = np.asarray(scales, dtype=np.float64)
+    m, n = Ws.shape
+    E = np.zeros((m, n))
+    W = np.zeros((m, n))
+    C = np.zeros((m, n), dtype=np.int64)
+    P = np.zeros((m, n))
+    for i in range(m):
+        T = LO[:i, i] @ E[:i, :] if i > 0 else np.zeros(n)
+        r = Ws[i] + T + T @ LI
+        for j in range(n):
+            pre = r[j] + E[i, :j] @ LI[:j, j]
+            c = quantize(pre, s[i], bits)
+            C[i, j] = c
+            W[i, j] = s[i] * c
+            E[i, j] = Ws[i, j] - W[i, j]
+            P[i, j] = pre
+    return (C, W, P) if return_pre else (C, W)
+
+
+def fixed_point_pre(Wstar, W, L_O, L_I):
+    """Closed form of the pre-rounding values given the final W:
+
+        pre = W* + (I + L_O)^T E (I + L_I) - E,    E = W* - W,
+
+    evaluated with fp64 matrix products. Because (I + L_O)^T is lower and (I + L_I) upper
+    triangular, entry (i, j) only sees E_kl with k <= i, l <= j; the -E removes the (i, j)
+    self-term. A correct solve satisfies W_ij = Q(pre_ij) at every entry.
+    """
+    Ws = np.asarray(Wstar, dtype=np.float64)
+    E = Ws - np.asarray(W, dtype=np.float64)
+    m, n = E.shape
+    Ao = np.eye(m) + np.asarray(L_O, dtype=np.float64)
+    Ai = np.eye(n) + np.asarray(L_I, dtype=np.float64)
+    return Ws + (Ao.T @ E) @ Ai - E
+
+
+def proxy_loss(dW, H_O, H_I) -> float:
+    """tr(H_O dW H_I dW^T) in fp64 ([YAQA] section 4 proxy; no factor 1/2)."""
+    d = np.asarray(dW, dtype=np.float64)
+    return float(np.trace(np.asarray(H_O, np.float64) @ d @ np.asarray(H_I, np.float64) @ d.T))
+
+
+def proxy_loss_kron(dW, H_O, H_I) -> float:
+    """vec(dW)^T (H_O (x) H_I) vec(dW) with row-major vec, by the explicit Kronecker product
+    (tiny shapes only)."""
+    v = np.asarray(dW, dtype=np.float64).reshape(-1)
+    K = np.kron(np.asarray(H_O, np.float64), np.asarray(H_I, np.float64))
+    return float(v @ K @ v)
+
+
+# ---------------------------------------------------------------------------------------------
+# Independent algorithms used only to pin the rule.
+# ---------------------------------------------------------------------------------------------
+def gptq_obs(w_star: np.ndarray, H: np.ndarray, scales: np.ndarray, bits: int):
+    """GPTQ in its optimal-brain-surgeon form on a vector w (length N) with Hessian H.
+
+    Coordinates are fixed in index order. After fixing coordinate q to its quantised value,
+    every still-free coordinate f moves by  -(w_q - Q(w_q)) [H_F^{-1}]_{f q} / [H_F^{-1}]_{q q},
+    where H_F is H restricted to the free set (q included). ``scales[q]`` is the grid step of
+    coordinate q. Returns integer codes. Uses an explicit inverse per step: tiny N only.
+    """
+    w = np.asarray(w_star, dtype=np.float64).copy()
+    H = np.asarray(H, dtype=np.float64)
+    N = w.shape[0]
+    codes = np.zeros(N, dtype=np.int64)
+    for q in range(N):
+        c = quantize(w[q], float(scales[q]), bits)
+        codes[q] = c
+        wq = float(scales[q]) * c
+        F = np.arange(q, N)
+        Hinv = np.linalg.inv(H[np.ix_(F, F)])
+        delta = (w[q] - wq) / Hinv[0, 0]
+        w[F] -= delta * Hinv[:, 0]
+        w[q] = wq
+    return codes
+
+
+def brute_force_fixed_points(Wstar, L_O, L_I, scales, bits, chunk=4096):
+    """All code matrices C with C = Q(pre(C)) under the closed form, by enumeration.
+
+    Every candidate C in [lo, hi]^(m x n) is tried: W = s * C, pre is the closed form of
+    ``fixed_point_pre`` (evaluated for a batch of candidates at once with the same fp64
+    products), and C is kept when clamp(rint(pre / s)) == C at every entry. Tiny shapes only
+    ((2^bits)^(mn) candidates). Rows with s_i = 0 are not supported here.
+    """
+    Ws = np.asarray(Wstar, dtype=np.float64)
+    s = np.asarray(scales, dtype=np.float64)
+    m, n = Ws.shape
+    lo, hi = code_range(bits)
+    Ao = np.eye(m) + np.asarray(L_O, dtype=np.float64)
+    Ai = np.eye(n) + np.asarray(L_I, dtype=np.float64)
+    values = np.arange(lo, hi + 1)
+    total = len(values) ** (m * n)
+    found = []
+    for start in range(0, total, chunk):
+        idx = np.arange(start, min(start + chunk, total))
+        digits = np.empty((idx.size, m * n), dtype=np.int64)
+        rest = idx.copy()
+        for p in range(m * n - 1, -1, -1):
+            digits[:, p] = values[rest % len(values)]
+            rest //= len(values)
+        C = digits.reshape(-1, m, n)
+        E = Ws[None] - s[None, :, None] * C
+        pre = Ws[None] + np.einsum("ki,bkl,lj->bij", Ao, E, Ai) - E
+        Q = np.clip(np.rint(pre / s[None, :, None]), lo, hi)
+        ok = np.all(Q == C, axis=(1, 2))
+        found.extend(C[ok])
+    return found
