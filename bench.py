@@ -1,0 +1,352 @@
+"""Benchmark of the BaKron solve path on synthetic LLM-layer workloads.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+One step = the whole path on one layer with inputs resident in HBM:
+    bakron_ldl(H_O), bakron_ldl(H_I), bakron_round(W*, L_O, L_I, scales, bits),
+    bakron_proxy_loss(W* - W, H_O, H_I).
+Metric: quantized weights per second, m*n / step time (whole job: summed over replicas, one
+independent layer per GPU, no collective on the data path; timed as the max over ranks).
+
+--impl reference times the fp64 CPU oracle (the deliberately slow reference) on a bounded
+sample of the same workload: the oracle's whole path (U D U^T, the raster-order rule, the proxy
+loss) on the leading r x c sub-layer of the workload (W*[:r, :c], H_O[:r, :r], H_I[:c, :c]).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "BaKron solver quantized weights/s (m·n/s) and % of B200 tensor roofline"
+UNIT = "weights/s"
+DEFAULT_WORKLOAD = "down_4096x14336"
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "sm_max_mhz": 1965.0}, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples taken while the timed region runs."""
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines: list[str] = []
+
+    def __enter__(self):
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def _dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def oracle_sample(wl, arrays=None, seconds_target: float = 12.0):
+    """Times the oracle's whole path on leading r x 2r sub-layers of the workload, growing r by
+    1.25x until one run takes a quarter of ``seconds_target``; returns the last (r, c, s)."""
+    from threadpoolctl import threadpool_limits
+
+    import oracle
+    from two_sided_adaptive_bakron_b200.workloads import make_workload
+    if arrays is None:
+        arrays = make_workload(wl, device="cuda" if wl.m * wl.n > (1 << 22) else None)
+    Ws, HO, HI, s, bits = arrays
+    r = 16.0
+    with threadpool_limits(limits=1):
+        while True:
+            rr = min(wl.m, int(r))
+            c = min(wl.n, 2 * int(r))
+            t0 = time.perf_counter()
+            oracle_path(oracle, Ws, HO, HI, s, bits, rr, c)
+            dt = time.perf_counter() - t0
+            if dt > seconds_target / 4 or (rr == wl.m and c == wl.n):
+                return rr, c, dt
+            r *= 1.25
+
+
+def oracle_path(oracle, Ws, HO, HI, s, bits, rr, c):
+    LO, _ = oracle.udu(HO[:rr, :rr])
+    LI, _ = oracle.udu(HI[:c, :c])
+    C, W = oracle.round_naive(Ws[:rr, :c], LO, LI, s[:rr], bits)
+    return oracle.proxy_loss(Ws[:rr, :c] - W, HO[:rr, :rr], HI[:c, :c])
+
+
+def run_reference(args):
+    ws, rank, _ = _dist()
+    if rank != 0:
+        return 0
+    from threadpoolctl import threadpool_limits
+
+    import oracle
+    from two_sided_adaptive_bakron_b200.workloads import WORKLOADS, make_workload
+    wl = WORKLOADS[args.workload]
+    arrays = make_workload(wl, device="cuda" if wl.m * wl.n > (1 << 22) else None)
+    Ws, HO, HI, s, bits = arrays
+    # sizing run (also the first warm-up), then the remaining warm-ups, then K timed steps
+    rr, c, _ = oracle_sample(wl, arrays, seconds_target=args.ref_seconds)
+    times = []
+    with threadpool_limits(limits=1):
+        for _ in range(max(0, args.warmup - 1)):
+            oracle_path(oracle, Ws, HO, HI, s, bits, rr, c)
+        for _ in range(args.steps):
+            t0 = time.perf_counter()
+            oracle_path(oracle, Ws, HO, HI, s, bits, rr, c)
+            times.append(time.perf_counter() - t0)
+    t = sum(times) / len(times)
+    v = rr * c / t
+    sample = (f"oracle whole path (udu, raster rule, proxy loss) on the leading {rr}x{c} "
+              f"sub-layer of {wl.name}, fp64 numpy, 1 thread")
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": ws,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": wl.name, "m": wl.m, "n": wl.n, "bits": wl.bits,
+                       "sample_rows": rr, "sample_cols": c},
+            "cpu_baseline": {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run(args):
+    import torch
+    import numpy as np
+
+    ws, rank, local = _dist()
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", torch.cuda.current_device())
+
+    from two_sided_adaptive_bakron_b200 import bakron as bk
+    from two_sided_adaptive_bakron_b200.workloads import WORKLOADS, make_workload
+    wl = WORKLOADS[args.workload]
+    m, n = wl.m, wl.n
+    Ws_np, HO_np, HI_np, s_np, bits = make_workload(wl, device=str(dev))
+    Ws = torch.from_numpy(Ws_np).to(dev)
+    HO = torch.from_numpy(HO_np).to(dev)
+    HI = torch.from_numpy(HI_np).to(dev)
+    sc = torch.from_numpy(s_np).to(dev)
+    solver = bk.Solver(m, n, dev)
+    stream = torch.cuda.current_stream(dev)
+
+    # ---- per-call timing events on the launching stream (device-timed breakdown)
+    names = ["ldl_O", "ldl_I", "round", "loss"]
+
+    def step(evs=None):
+        calls = [
+            lambda: bk.bakron_ldl(HO, solver.L_O, solver.D_O, solver.ws, solver.status, stream),
+            lambda: bk.bakron_ldl(HI, solver.L_I, solver.D_I, solver.ws, solver.status, stream),
+            lambda: bk.bakron_round(Ws, solver.L_O, solver.L_I, sc, bits, solver.codes, solver.W,
+                                    solver.ws_round, solver.status, stream),
+            lambda: bk.bakron_proxy_loss(solver.E, HO, HI, solver.loss, solver.ws, stream),
+        ]
+        for k, f in enumerate(calls):
+            if evs is not None:
+                evs[k][0].record(stream)
+            rc = f()
+            if rc != 0:
+                raise bk.BakronError(rc, names[k])
+            if evs is not None:
+                evs[k][1].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    st = bk.bakron_read_status(solver.status, stream)
+    if st != 0:
+        raise bk.BakronError(st, "warm-up")
+
+    evs = [[[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)]
+            for _ in names] for _ in range(args.steps)]
+    l0 = bk.bakron_kernel_launches()
+    if ws > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev.index if dev.index is not None else 0) as clk:
+        t_start.record(stream)
+        for k in range(args.steps):
+            step(evs[k])
+        t_end.record(stream)
+        torch.cuda.synchronize()
+    launches = bk.bakron_kernel_launches() - l0
+    ms_total = t_start.elapsed_time(t_end)
+    if ws > 1:
+        t = torch.tensor([ms_total], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms_total = float(t.item())
+    st = bk.bakron_read_status(solver.status, stream)
+    if st != 0:
+        raise bk.BakronError(st, "timed region")
+    ms_step = ms_total / args.steps
+    value = ws * m * n / (ms_step * 1e-3)
+    per = {nm: statistics.mean(evs[k][i][0].elapsed_time(evs[k][i][1]) for k in range(args.steps))
+           for i, nm in enumerate(names)}
+
+    # ---- end to end through the public API with host buffers (pinned), copies timed
+    hW = torch.from_numpy(Ws_np).pin_memory()
+    hO = torch.from_numpy(HO_np).pin_memory()
+    hI = torch.from_numpy(HI_np).pin_memory()
+    hs = torch.from_numpy(s_np).pin_memory()
+    hcodes = torch.empty((m, n), dtype=torch.int8).pin_memory()
+    hloss = torch.empty((1,), dtype=torch.float64).pin_memory()
+    dW2, dO2, dI2, ds2 = (torch.empty_like(Ws), torch.empty_like(HO), torch.empty_like(HI),
+                          torch.empty_like(sc))
+    h2d = sum(x.numel() * x.element_size() for x in (hW, hO, hI, hs))
+    d2h = m * n + 8
+
+    def e2e_step():
+        dW2.copy_(hW, non_blocking=True)
+        dO2.copy_(hO, non_blocking=True)
+        dI2.copy_(hI, non_blocking=True)
+        ds2.copy_(hs, non_blocking=True)
+        solver.run(dW2, dO2, dI2, ds2, bits, stream)
+        hcodes.copy_(solver.codes, non_blocking=True)
+        hloss.copy_(solver.loss, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    if ws > 1:
+        torch.distributed.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / args.steps
+    if ws > 1:
+        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = ws * m * n / (e2e_ms * 1e-3)
+
+    # ---- roofline of the dominant call
+    peaks, peak_kind = _peaks()
+    sm_max = float(peaks.get("sm_max_mhz", 1965.0))
+    fp32_simt_tflops = 148 * 128 * 2 * sm_max * 1e6 / 1e12
+    work = {
+        "ldl_O": m ** 3 / 3.0, "ldl_I": n ** 3 / 3.0,
+        "round": float(m) * n * (m + n),          # minimal (triangular) multiply-add work, x2 flops
+        "loss": 2.0 * m * n * (m + n),
+    }
+    dom = max(per, key=lambda k: per[k])
+    achieved = work[dom] / (per[dom] * 1e-3) / 1e12
+    roofline = {"bound": "alu", "kernel": dom, "achieved": achieved, "peak": fp32_simt_tflops,
+                "unit": "TFLOP/s", "frac": achieved / fp32_simt_tflops, "traffic": None,
+                "peak_source": (f"FP32 SIMT: 148 SMs x 128 lanes x 2 flop x {sm_max:.0f} MHz "
+                                f"(max SM clock of {peak_kind} peaks file)")}
+
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        rr, c, dt = oracle_sample(wl, (Ws_np, HO_np, HI_np, s_np, bits))
+        cpu = {"value": rr * c / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
+               "sample": f"oracle whole path on the leading {rr}x{c} sub-layer of {wl.name}, "
+                         f"fp64 numpy, 1 thread, {dt:.1f} s"}
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+                "config": {"workload": wl.name, "m": m, "n": n, "bits": bits,
+                           "parallelism": f"replicas x{ws}" if ws > 1 else "single",
+                           "l2": "inputs larger than L2 (H_I alone is "
+                                 f"{4 * n * n / 2**20:.0f} MiB), no flush"},
+                "breakdown_ms": per,
+                "round_weights_per_s": m * n / (per["round"] * 1e-3),
+                "roofline": roofline, "cpu_baseline": cpu,
+                "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                        "d2h_bytes_per_step": d2h},
+                "gpu_launches": int(launches), "clocks": clk.summary()}
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-seconds", type=float, default=12.0)
+    args = ap.parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,133 @@
+/*
+ * bakron.h -- C ABI of the BaKron two-sided adaptive rounding library (CUDA, sm_100a).
+ *
+ * The library rounds an m x n weight matrix W* (rows = output features, columns = input
+ * features) under a Kronecker-factored Hessian H ~ H_O (x) H_I, H_O m x m, H_I n x n
+ * (YAQA article, news.43b.com.cn/a/479517.html, section 2: Kronecker approximation of the
+ * Fisher; BaKron page "BaKron: Efficient Quantization with Kronecker-Factored Hessians",
+ * abstract: the two-sided adaptive-rounding formulation of BoA/YAQA).
+ *
+ * Conventions for every entry point:
+ *   - All array pointers are DEVICE pointers unless stated otherwise. Matrices are dense,
+ *     row-major, leading dimension = number of columns. fp32 unless stated otherwise.
+ *   - The caller owns every buffer, including the workspace; the library never allocates
+ *     device memory. Outputs must not alias inputs or the workspace.
+ *   - Work is enqueued asynchronously on `stream` (a cudaStream_t passed as void*; NULL is the
+ *     legacy default stream). The return value reports host-side argument checks and launch
+ *     errors only. Errors found on the device (non-positive pivot, non-finite input, a
+ *     dependency wait that timed out) are written to `*dev_status`, a device int that the
+ *     caller owns and initialises to 0 (BAKRON_OK). Calls never reset it: the first error of
+ *     a chain of calls sticks, and bakron_read_status() reads it.
+ *   - Nothing traps: device-side waits are bounded and give up with BAKRON_ERR_TIMEOUT.
+ *   - Identical inputs give bitwise identical outputs.
+ */
+#ifndef BAKRON_H_
+#define BAKRON_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    BAKRON_OK = 0,
+    BAKRON_ERR_INVALID_ARG = -1,  /* bad size, NULL pointer, unsupported bits          */
+    BAKRON_ERR_NOT_PD = -2,       /* a pivot D_j <= 0 or non-finite in bakron_ldl        */
+    BAKRON_ERR_CUDA = -3,         /* a CUDA launch or runtime call failed                */
+    BAKRON_ERR_TIMEOUT = -4,      /* a device-side dependency wait gave up               */
+    BAKRON_ERR_WORKSPACE = -5,    /* workspace NULL, too small or misaligned (256 B)     */
+    BAKRON_ERR_NONFINITE = -6     /* a non-finite value met on the device                */
+} bakron_status;
+
+/* ------------------------------------------------------------------------------------------
+ * bakron_ldl -- U D U^T factorisation of one damped Kronecker factor.
+ *
+ * Computes H = (I + L) D (I + L)^T with L strictly UPPER triangular and D diagonal > 0
+ * (YAQA article, section 4: the factor L_O of the rounding rule is taken from the LDL
+ * decomposition H_O = (L_O + I) D_O (L_O + I)^T; the rule of the same section makes L_O
+ * strictly upper triangular, since a_i, the i-th column of L_O, only has entries above row i).
+ * Equivalently it is the LDL^T factorisation of H with its index order reversed.
+ *
+ *   H        [in]  n x n, symmetric positive definite, already damped by the caller. Only the
+ *                  upper triangle (j >= i) is read.
+ *   n        [in]  1 <= n <= 65536.
+ *   L        [out] n x n; written in full: the strictly upper part holds L, every entry on
+ *                  and below the diagonal is 0.
+ *   D        [out] n pivots.
+ *   ws       [in]  workspace of at least bakron_ldl_workspace_bytes(n) bytes, 256-B aligned.
+ *   dev_status [out] device int; BAKRON_ERR_NOT_PD if a pivot is <= 0 or non-finite (L and D
+ *                  are then unspecified).
+ * ---------------------------------------------------------------------------------------- */
+size_t bakron_ldl_workspace_bytes(int n);
+int bakron_ldl(const float* H, int n, float* L, float* D,
+               void* ws, size_t ws_bytes, int* dev_status, void* stream);
+
+/* ------------------------------------------------------------------------------------------
+ * bakron_round -- the BaKron solve of the two-sided adaptive rounding rule.
+ *
+ * For every entry, in any order compatible with "(k,l) before (i,j) when k <= i and l <= j"
+ * (the anti-diagonal order of the BaKron page, abstract: O(m+n) sequential steps):
+ *
+ *   pre_ij = W*_ij + a_i^T E[:i,:j] b_j + a_i^T E[:i,j] + E[i,:j] b_j      (YAQA, section 4)
+ *   code_ij = clamp(round_half_even(pre_ij / s_i), -2^(bits-1), 2^(bits-1) - 1)
+ *   W_ij    = s_i * code_ij,      E_ij = W*_ij - W_ij
+ *
+ * where a_i is column i of L_O (entries k < i), b_j is column j of L_I (entries l < j), and
+ * ":i" means indices 0..i-1. Equivalently W = Q(W* + (I+L_O)^T E (I+L_I) - E) holds at every
+ * entry (the closed form used to check results).
+ *
+ *   Wstar    [in]  m x n.
+ *   m, n     [in]  1 <= m, n; m*n < 2^31.
+ *   L_O      [in]  m x m, strictly upper part used (the output format of bakron_ldl).
+ *   L_I      [in]  n x n, strictly upper part used.
+ *   scales   [in]  m per-row grid steps s_i >= 0 (s_i == 0: the row gets code 0, W 0).
+ *   bits     [in]  2..8.
+ *   codes    [out] m x n int8.
+ *   W        [out] m x n dequantised weights s_i * code_ij.
+ *   ws       [in/out] at least bakron_round_workspace_bytes(m, n) bytes, 256-B aligned. When
+ *                  the call has run, its first m*n floats hold the residual E = W* - W
+ *                  (row-major), ready to be passed to bakron_proxy_loss as dW.
+ *   dev_status [out] BAKRON_ERR_TIMEOUT if a dependency wait gave up, BAKRON_ERR_NONFINITE if a
+ *                  pre-rounding value was not finite.
+ * ---------------------------------------------------------------------------------------- */
+size_t bakron_round_workspace_bytes(int m, int n);
+int bakron_round(const float* Wstar, int m, int n, const float* L_O, const float* L_I,
+                 const float* scales, int bits, int8_t* codes, float* W,
+                 void* ws, size_t ws_bytes, int* dev_status, void* stream);
+
+/* ------------------------------------------------------------------------------------------
+ * bakron_proxy_loss -- tr(H_O dW H_I dW^T) = vec(dW)^T (H_O (x) H_I) vec(dW).
+ *
+ * The layer proxy of the YAQA article (section 4 error bound, section 2 second-order
+ * objective without its factor 1/2), row-major vec.
+ *
+ *   dW       [in]  m x n (e.g. W* - W).
+ *   H_O, H_I [in]  m x m and n x n, symmetric (both triangles are read).
+ *   loss     [out] one DEVICE double.
+ *   ws       [in]  at least bakron_proxy_loss_workspace_bytes(m, n) bytes, 256-B aligned.
+ * ---------------------------------------------------------------------------------------- */
+size_t bakron_proxy_loss_workspace_bytes(int m, int n);
+int bakron_proxy_loss(const float* dW, int m, int n, const float* H_O, const float* H_I,
+                      double* loss, void* ws, size_t ws_bytes, void* stream);
+
+/* Synchronises `stream`, then returns the device status word (a bakron_status value), or
+ * BAKRON_ERR_CUDA if the synchronisation itself failed. */
+int bakron_read_status(const int* dev_status, void* stream);
+
+/* Static, NUL-terminated description of a bakron_status value. */
+const char* bakron_status_string(int code);
+
+/* Number of CUDA kernels this library has launched in the calling process so far
+ * (diagnostics: lets a benchmark count its launches). */
+unsigned long long bakron_kernel_launches(void);
+
+/* Library version as 10000*major + 100*minor + patch. */
+int bakron_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BAKRON_H_ */

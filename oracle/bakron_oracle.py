@@ -43,7 +43,7 @@ import numpy as np
 __all__ = [
     "udu", "quantize", "round_naive", "round_row_sweep", "fixed_point_pre",
     "proxy_loss", "proxy_loss_kron", "brute_force_fixed_points", "gptq_obs",
-    "code_range",
+    "code_range", "fixed_point_pre_rows", "band_check",
 ]
 
 
@@ -173,6 +173,39 @@ def fixed_point_pre(Wstar, W, L_O, L_I):
     Ao = np.eye(m) + np.asarray(L_O, dtype=np.float64)
     Ai = np.eye(n) + np.asarray(L_I, dtype=np.float64)
     return Ws + (Ao.T @ E) @ Ai - E
+
+
+def fixed_point_pre_rows(Wstar, W, L_O, L_I, rows):
+    """``fixed_point_pre`` restricted to the given rows (same closed form, fp64):
+    pre[R] = W*[R] + ((I + L_O)^T)[R, :] E (I + L_I) - E[R]."""
+    rows = np.asarray(rows)
+    Ws = np.asarray(Wstar, dtype=np.float64)
+    E = Ws - np.asarray(W, dtype=np.float64)
+    m, n = E.shape
+    LO = np.asarray(L_O, dtype=np.float64)
+    LI = np.asarray(L_I, dtype=np.float64)
+    AoT_R = LO[:, rows].T.copy()
+    AoT_R[np.arange(rows.size), rows] += 1.0
+    T = AoT_R @ E
+    return Ws[rows] + T + T @ LI - E[rows]
+
+
+def band_check(pre, codes, scales, bits, band=1e-3):
+    """Compare codes with Q(pre) under the exemption band of the tolerance rule.
+
+    An entry may disagree only if pre/s lies within ``band`` grid steps of a rounding boundary
+    (a half-integer). Returns (n_mismatch, n_mismatch_outside_band, n_in_band).
+    """
+    s = np.asarray(scales, dtype=np.float64)[:, None]
+    lo, hi = code_range(bits)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        x = np.where(s > 0, pre / np.where(s > 0, s, 1.0), 0.0)
+    q = np.clip(np.rint(x), lo, hi)
+    q = np.where(s > 0, q, 0.0)
+    frac = np.abs(x - np.floor(x) - 0.5)
+    in_band = frac < band
+    mism = q != np.asarray(codes, dtype=np.float64)
+    return int(mism.sum()), int((mism & ~in_band).sum()), int(in_band.sum())
 
 
 def proxy_loss(dW, H_O, H_I) -> float:

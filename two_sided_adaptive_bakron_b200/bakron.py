@@ -1,0 +1,254 @@
+"""Python binding of libbakron.so (ctypes): argument marshalling only.
+
+The functions named like the C ABI (``bakron_ldl``, ``bakron_round``, ``bakron_proxy_loss``,
+``bakron_read_status``, ``bakron_status_string`` and the ``*_workspace_bytes`` queries) take
+torch CUDA tensors, pass their device pointers and the current CUDA stream to the library and
+return its status code. ``ldl``, ``round_weights``, ``proxy_loss`` and ``solve`` additionally
+allocate outputs and workspaces with torch and raise on any error.
+
+Every step of the computation runs in the library's CUDA kernels; there is no CPU path. If
+the shared library is missing the first call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libbakron.so")
+HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "bakron.h")
+
+BAKRON_OK = 0
+BAKRON_ERR_INVALID_ARG = -1
+BAKRON_ERR_NOT_PD = -2
+BAKRON_ERR_CUDA = -3
+BAKRON_ERR_TIMEOUT = -4
+BAKRON_ERR_WORKSPACE = -5
+BAKRON_ERR_NONFINITE = -6
+
+_c_size_t, _c_int, _vp = ctypes.c_size_t, ctypes.c_int, ctypes.c_void_p
+_SIGNATURES = {
+    "bakron_ldl_workspace_bytes": (_c_size_t, [_c_int]),
+    "bakron_ldl": (_c_int, [_vp, _c_int, _vp, _vp, _vp, _c_size_t, _vp, _vp]),
+    "bakron_round_workspace_bytes": (_c_size_t, [_c_int, _c_int]),
+    "bakron_round": (_c_int, [_vp, _c_int, _c_int, _vp, _vp, _vp, _c_int, _vp, _vp, _vp,
+                              _c_size_t, _vp, _vp]),
+    "bakron_proxy_loss_workspace_bytes": (_c_size_t, [_c_int, _c_int]),
+    "bakron_proxy_loss": (_c_int, [_vp, _c_int, _c_int, _vp, _vp, _vp, _vp, _c_size_t, _vp]),
+    "bakron_read_status": (_c_int, [_vp, _vp]),
+    "bakron_status_string": (ctypes.c_char_p, [_c_int]),
+    "bakron_version": (_c_int, []),
+    "bakron_kernel_launches": (ctypes.c_ulonglong, []),
+}
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+class BakronError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        super().__init__(f"{where}: {status_string(code)} ({code})")
+        self.code = code
+
+
+def header_functions() -> list[str]:
+    """Names of the functions that include/bakron.h declares."""
+    text = open(HEADER_PATH).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(bakron_\w+)\s*\(", text)))
+
+
+def lib() -> ctypes.CDLL:
+    """Loads libbakron.so (once). Raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m two_sided_adaptive_bakron_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGNATURES.items():
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+def status_string(code: int) -> str:
+    return lib().bakron_status_string(int(code)).decode()
+
+
+bakron_status_string = status_string
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _check_cuda(t: torch.Tensor, dtype: torch.dtype, shape: tuple, name: str):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype or tuple(t.shape) != tuple(shape) or not t.is_contiguous():
+        raise ValueError(f"{name}: expected contiguous {dtype} of shape {tuple(shape)}, got "
+                         f"{t.dtype} {tuple(t.shape)} contiguous={t.is_contiguous()}")
+
+
+# ----------------------------------------------------------------------------- C-ABI mirrors
+def bakron_ldl_workspace_bytes(n: int) -> int:
+    return int(lib().bakron_ldl_workspace_bytes(int(n)))
+
+
+def bakron_round_workspace_bytes(m: int, n: int) -> int:
+    return int(lib().bakron_round_workspace_bytes(int(m), int(n)))
+
+
+def bakron_proxy_loss_workspace_bytes(m: int, n: int) -> int:
+    return int(lib().bakron_proxy_loss_workspace_bytes(int(m), int(n)))
+
+
+def bakron_ldl(H, L, D, ws, dev_status, stream=None) -> int:
+    n = H.shape[0]
+    _check_cuda(H, torch.float32, (n, n), "H")
+    _check_cuda(L, torch.float32, (n, n), "L")
+    _check_cuda(D, torch.float32, (n,), "D")
+    return lib().bakron_ldl(_ptr(H), n, _ptr(L), _ptr(D), _ptr(ws), ws.numel() * ws.element_size(),
+                            _ptr(dev_status), _stream(stream))
+
+
+def bakron_round(Wstar, L_O, L_I, scales, bits, codes, W, ws, dev_status, stream=None) -> int:
+    m, n = Wstar.shape
+    _check_cuda(Wstar, torch.float32, (m, n), "Wstar")
+    _check_cuda(L_O, torch.float32, (m, m), "L_O")
+    _check_cuda(L_I, torch.float32, (n, n), "L_I")
+    _check_cuda(scales, torch.float32, (m,), "scales")
+    _check_cuda(codes, torch.int8, (m, n), "codes")
+    _check_cuda(W, torch.float32, (m, n), "W")
+    return lib().bakron_round(_ptr(Wstar), m, n, _ptr(L_O), _ptr(L_I), _ptr(scales), int(bits),
+                              _ptr(codes), _ptr(W), _ptr(ws), ws.numel() * ws.element_size(),
+                              _ptr(dev_status), _stream(stream))
+
+
+def bakron_proxy_loss(dW, H_O, H_I, loss, ws, stream=None) -> int:
+    m, n = dW.shape
+    _check_cuda(dW, torch.float32, (m, n), "dW")
+    _check_cuda(H_O, torch.float32, (m, m), "H_O")
+    _check_cuda(H_I, torch.float32, (n, n), "H_I")
+    _check_cuda(loss, torch.float64, (1,), "loss")
+    return lib().bakron_proxy_loss(_ptr(dW), m, n, _ptr(H_O), _ptr(H_I), _ptr(loss), _ptr(ws),
+                                   ws.numel() * ws.element_size(), _stream(stream))
+
+
+def bakron_read_status(dev_status, stream=None) -> int:
+    return int(lib().bakron_read_status(_ptr(dev_status), _stream(stream)))
+
+
+def bakron_kernel_launches() -> int:
+    return int(lib().bakron_kernel_launches())
+
+
+def bakron_version() -> int:
+    return int(lib().bakron_version())
+
+
+# ----------------------------------------------------------------------------- conveniences
+def workspace(nbytes: int, device) -> torch.Tensor:
+    """A 256-byte aligned byte buffer (torch's caching allocator aligns to 512 bytes)."""
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+def new_status(device) -> torch.Tensor:
+    return torch.zeros(1, dtype=torch.int32, device=device)
+
+
+def _raise(code: int, where: str):
+    if code != BAKRON_OK:
+        raise BakronError(code, where)
+
+
+def ldl(H: torch.Tensor, stream=None, check: bool = True):
+    """(L, D) with H = (I + L) diag(D) (I + L)^T, L strictly upper."""
+    n = H.shape[0]
+    L = torch.empty((n, n), dtype=torch.float32, device=H.device)
+    D = torch.empty((n,), dtype=torch.float32, device=H.device)
+    ws = workspace(bakron_ldl_workspace_bytes(n), H.device)
+    st = new_status(H.device)
+    _raise(bakron_ldl(H, L, D, ws, st, stream), "bakron_ldl")
+    if check:
+        _raise(bakron_read_status(st, stream), "bakron_ldl (device)")
+    return L, D
+
+
+def round_weights(Wstar, L_O, L_I, scales, bits, stream=None, check: bool = True):
+    """(codes int8, W fp32) of the BaKron solve."""
+    m, n = Wstar.shape
+    codes = torch.empty((m, n), dtype=torch.int8, device=Wstar.device)
+    W = torch.empty((m, n), dtype=torch.float32, device=Wstar.device)
+    ws = workspace(bakron_round_workspace_bytes(m, n), Wstar.device)
+    st = new_status(Wstar.device)
+    _raise(bakron_round(Wstar, L_O, L_I, scales, bits, codes, W, ws, st, stream), "bakron_round")
+    if check:
+        _raise(bakron_read_status(st, stream), "bakron_round (device)")
+    return codes, W
+
+
+def proxy_loss(dW, H_O, H_I, stream=None) -> torch.Tensor:
+    """tr(H_O dW H_I dW^T) as a one-element float64 CUDA tensor."""
+    m, n = dW.shape
+    loss = torch.empty((1,), dtype=torch.float64, device=dW.device)
+    ws = workspace(bakron_proxy_loss_workspace_bytes(m, n), dW.device)
+    _raise(bakron_proxy_loss(dW, H_O, H_I, loss, ws, stream), "bakron_proxy_loss")
+    return loss
+
+
+class Solver:
+    """Reusable buffers for the whole path: ldl(H_O), ldl(H_I), round, proxy loss.
+
+    The round workspace keeps E = W* - W at its start (see bakron.h), which is the dW handed
+    to the proxy loss.
+    """
+
+    def __init__(self, m: int, n: int, device="cuda"):
+        self.m, self.n, self.device = m, n, torch.device(device)
+        f32 = dict(dtype=torch.float32, device=self.device)
+        self.L_O = torch.empty((m, m), **f32)
+        self.D_O = torch.empty((m,), **f32)
+        self.L_I = torch.empty((n, n), **f32)
+        self.D_I = torch.empty((n,), **f32)
+        self.codes = torch.empty((m, n), dtype=torch.int8, device=self.device)
+        self.W = torch.empty((m, n), **f32)
+        self.loss = torch.empty((1,), dtype=torch.float64, device=self.device)
+        self.ws_round = workspace(bakron_round_workspace_bytes(m, n), self.device)
+        self.ws = workspace(max(bakron_ldl_workspace_bytes(m), bakron_ldl_workspace_bytes(n),
+                                bakron_proxy_loss_workspace_bytes(m, n)), self.device)
+        self.E = self.ws_round[: 4 * m * n].view(torch.float32).view(m, n)
+        self.status = new_status(self.device)
+
+    def run(self, Wstar, H_O, H_I, scales, bits, stream=None, with_loss=True):
+        """Enqueues the whole path (reads: self.codes, self.W, self.E, self.loss)."""
+        _raise(bakron_ldl(H_O, self.L_O, self.D_O, self.ws, self.status, stream), "bakron_ldl")
+        _raise(bakron_ldl(H_I, self.L_I, self.D_I, self.ws, self.status, stream), "bakron_ldl")
+        _raise(bakron_round(Wstar, self.L_O, self.L_I, scales, bits, self.codes, self.W,
+                            self.ws_round, self.status, stream), "bakron_round")
+        if with_loss:
+            _raise(bakron_proxy_loss(self.E, H_O, H_I, self.loss, self.ws, stream),
+                   "bakron_proxy_loss")
+
+    def check(self, stream=None):
+        _raise(bakron_read_status(self.status, stream), "bakron (device)")
+
+
+def solve(Wstar, H_O, H_I, scales, bits, stream=None):
+    """Whole path on device tensors: returns (codes, W, loss, (L_O, D_O), (L_I, D_I))."""
+    s = Solver(Wstar.shape[0], Wstar.shape[1], Wstar.device)
+    s.run(Wstar, H_O, H_I, scales, bits, stream)
+    s.check(stream)
+    return s.codes, s.W, s.loss, (s.L_O, s.D_O), (s.L_I, s.D_I)
