@@ -25,7 +25,9 @@ Readings taken where the pages are garbled or silent (each one is listed in the 
   (the section-4 text also calls it "unit lower"; only the upper reading makes the rule causal
   and the bound hold);
 * Q is round-half-to-even of pre/s_i followed by a clamp to [-2^(b-1), 2^(b-1)-1], per-row
-  scale s_i; s_i = 0 gives code 0;
+  scale s_i; s_i = 0 gives code 0. The pages fix no precision for this integer decision, so
+  it is taken in the precision of the CUDA kernels: pre is rounded to fp32 and divided by s_i
+  with one correctly rounded fp32 division before round-half-even (pre itself stays fp64);
 * E = W* - W always includes the clamp error;
 * the proxy loss is tr(H_O dW H_I dW^T) with no factor 1/2.
 
@@ -43,7 +45,7 @@ import numpy as np
 __all__ = [
     "udu", "quantize", "round_naive", "round_row_sweep", "fixed_point_pre",
     "proxy_loss", "proxy_loss_kron", "brute_force_fixed_points", "gptq_obs",
-    "code_range", "fixed_point_pre_rows", "band_check",
+    "code_range", "fixed_point_pre_rows", "band_check", "grid_quotient",
 ]
 
 
@@ -81,12 +83,21 @@ def udu(H: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
 # ---------------------------------------------------------------------------------------------
 # Base quantizer Q ([YAQA] section 4: nearest rounding; reading: half-even, then clamp).
 # ---------------------------------------------------------------------------------------------
+def grid_quotient(pre, s):
+    """pre / s as the rounding decision sees it: fp32(pre) / fp32(s), one correctly rounded
+    fp32 division (elementwise on arrays), returned as fp64."""
+    with np.errstate(divide="ignore", invalid="ignore"):
+        q = np.float32(pre) / np.float32(s) if np.isscalar(pre) and np.isscalar(s) else \
+            np.asarray(pre, dtype=np.float32) / np.asarray(s, dtype=np.float32)
+    return np.asarray(q, dtype=np.float64)
+
+
 def quantize(pre: float, s: float, bits: int) -> int:
     """Code for one entry: clamp(round_half_even(pre / s)); s == 0 gives 0."""
     lo, hi = code_range(bits)
     if s == 0.0:
         return 0
-    c = float(np.rint(pre / s))
+    c = float(np.rint(grid_quotient(pre, s)))
     return int(min(max(c, lo), hi))
 
 
@@ -198,9 +209,11 @@ def band_check(pre, codes, scales, bits, band=1e-3):
     """
     s = np.asarray(scales, dtype=np.float64)[:, None]
     lo, hi = code_range(bits)
+    s_safe = np.where(s > 0, s, 1.0)
     with np.errstate(divide="ignore", invalid="ignore"):
-        x = np.where(s > 0, pre / np.where(s > 0, s, 1.0), 0.0)
-    q = np.clip(np.rint(x), lo, hi)
+        x = np.where(s > 0, pre / s_safe, 0.0)
+    xq = np.where(s > 0, grid_quotient(pre, np.broadcast_to(s_safe, pre.shape)), 0.0)
+    q = np.clip(np.rint(xq), lo, hi)
     q = np.where(s > 0, q, 0.0)
     frac = np.abs(x - np.floor(x) - 0.5)
     in_band = frac < band
@@ -276,7 +289,8 @@ def brute_force_fixed_points(Wstar, L_O, L_I, scales, bits, chunk=4096):
         C = digits.reshape(-1, m, n)
         E = Ws[None] - s[None, :, None] * C
         pre = Ws[None] + np.einsum("ki,bkl,lj->bij", Ao, E, Ai) - E
-        Q = np.clip(np.rint(pre / s[None, :, None]), lo, hi)
+        Q = np.clip(np.rint(grid_quotient(pre, np.broadcast_to(s[None, :, None], pre.shape))),
+                    lo, hi)
         ok = np.all(Q == C, axis=(1, 2))
         found.extend(C[ok])
     return found

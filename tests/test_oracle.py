@@ -17,7 +17,7 @@ transposed factor, a wrong triangle, a wrong sign, the wrong rounding mode) fail
 import numpy as np
 import pytest
 
-from oracle import (brute_force_fixed_points, code_range, fixed_point_pre, gptq_obs,
+from oracle import (brute_force_fixed_points, code_range, fixed_point_pre, gptq_obs, grid_quotient,
                     proxy_loss, proxy_loss_kron, quantize, round_naive, round_row_sweep, udu)
 from two_sided_adaptive_bakron_b200.workloads import make_workload, random_problem
 
@@ -63,6 +63,9 @@ def test_quantize_half_even_and_clamp():
     assert quantize(-9.7, 1.0, 4) == -8
     assert quantize(3.0, 0.0, 4) == 0     # zero scale row
     assert code_range(3) == (-4, 3)
+    # the decision is taken on the fp32 quotient: 0.7499999999 rounds to fp32 0.75 -> 1
+    assert quantize(0.7499999999, 1.0, 4) == 1
+    assert quantize(-7.5, 1.0, 4) == -8
 
 
 # ----------------------------------------------------------------------------- special cases
@@ -72,7 +75,8 @@ def test_identity_factors_give_round_to_nearest(m, n, bits, seed):
     LO, _, LI, _ = _factors(HO, HI)
     C, _ = round_naive(Ws, LO, LI, s, bits)
     lo, hi = code_range(bits)
-    rtn = np.clip(np.rint(Ws.astype(np.float64) / s[:, None].astype(np.float64)), lo, hi)
+    # round to nearest, the quotient taken as one fp32 division (the decision precision)
+    rtn = np.clip(np.rint(Ws.astype(np.float32) / s[:, None].astype(np.float32)), lo, hi)
     np.testing.assert_array_equal(C, rtn)
 
 
@@ -145,7 +149,8 @@ def test_closed_form_fixed_point_holds():
     pre = fixed_point_pre(Ws, W, LO, LI)
     np.testing.assert_allclose(pre, P, rtol=0, atol=1e-12)
     lo, hi = code_range(bits)
-    np.testing.assert_array_equal(np.clip(np.rint(pre / s[:, None]), lo, hi), C)
+    q = np.rint(grid_quotient(pre, np.broadcast_to(s[:, None], pre.shape)))
+    np.testing.assert_array_equal(np.clip(q, lo, hi), C)
 
 
 def test_zero_scale_row_gives_zero_codes():
