@@ -19,6 +19,7 @@ def test_library_exports_every_header_function(libpath):
             "bakron_status_string", "bakron_ldl_workspace_bytes",
             "bakron_round_workspace_bytes", "bakron_proxy_loss_workspace_bytes"} <= set(names)
     lib = ctypes.CDLL(libpath)
+    names += bakron.header_functions(bakron.HEADER_PATH.replace("bakron.h", "bakron_internal.h"))
     missing = [n for n in names if not hasattr(lib, n)]
     assert not missing, missing
 

@@ -43,6 +43,13 @@ _SIGNATURES = {
     "bakron_status_string": (ctypes.c_char_p, [_c_int]),
     "bakron_version": (_c_int, []),
     "bakron_kernel_launches": (ctypes.c_ulonglong, []),
+    # test hooks (include/bakron_internal.h)
+    "bakron_internal_gemm3x_workspace_bytes": (_c_size_t, [_c_int, _c_int, _c_int]),
+    "bakron_internal_gemm3x": (_c_int, [_vp, _c_int, _c_int, _c_int, _vp, _c_int, _c_int, _vp,
+                                        _c_int, _vp, _c_size_t, _vp, _vp]),
+    "bakron_internal_proxy_loss_simt_workspace_bytes": (_c_size_t, [_c_int, _c_int]),
+    "bakron_internal_proxy_loss_simt": (_c_int, [_vp, _c_int, _c_int, _vp, _vp, _vp, _vp,
+                                                 _c_size_t, _vp]),
 }
 
 _lib: Optional[ctypes.CDLL] = None
@@ -54,9 +61,9 @@ class BakronError(RuntimeError):
         self.code = code
 
 
-def header_functions() -> list[str]:
-    """Names of the functions that include/bakron.h declares."""
-    text = open(HEADER_PATH).read()
+def header_functions(path: str = HEADER_PATH) -> list[str]:
+    """Names of the functions that a header (default include/bakron.h) declares."""
+    text = open(path).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
     return sorted(set(re.findall(r"\b(bakron_\w+)\s*\(", text)))
 
@@ -157,6 +164,31 @@ def bakron_kernel_launches() -> int:
 
 def bakron_version() -> int:
     return int(lib().bakron_version())
+
+
+def internal_gemm3x(A: torch.Tensor, B: torch.Tensor, stream=None) -> torch.Tensor:
+    """C = A B^T through the 3xTF32 tensor-core engine (test hook)."""
+    M, K = A.shape
+    N = B.shape[0]
+    C = torch.empty((M, N), dtype=torch.float32, device=A.device)
+    ws = workspace(int(lib().bakron_internal_gemm3x_workspace_bytes(M, N, K)), A.device)
+    st = new_status(A.device)
+    _raise(lib().bakron_internal_gemm3x(_ptr(A), M, K, A.stride(0), _ptr(B), N, B.stride(0),
+                                        _ptr(C), N, _ptr(ws), ws.numel(), _ptr(st),
+                                        _stream(stream)), "bakron_internal_gemm3x")
+    _raise(bakron_read_status(st, stream), "bakron_internal_gemm3x (device)")
+    return C
+
+
+def internal_proxy_loss_simt(dW, H_O, H_I, stream=None) -> torch.Tensor:
+    """The CUDA-core proxy loss (test hook, cross-check of bakron_proxy_loss)."""
+    m, n = dW.shape
+    loss = torch.empty((1,), dtype=torch.float64, device=dW.device)
+    ws = workspace(int(lib().bakron_internal_proxy_loss_simt_workspace_bytes(m, n)), dW.device)
+    _raise(lib().bakron_internal_proxy_loss_simt(_ptr(dW), m, n, _ptr(H_O), _ptr(H_I),
+                                                 _ptr(loss), _ptr(ws), ws.numel(),
+                                                 _stream(stream)), "proxy_loss_simt")
+    return loss
 
 
 # ----------------------------------------------------------------------------- conveniences

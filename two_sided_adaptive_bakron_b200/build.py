@@ -22,7 +22,7 @@ LIB = os.path.join(PKG_DIR, "libbakron.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-O3",
-              "--expt-relaxed-constexpr", "-I", INCLUDE, "-I", CSRC]
+              "--expt-relaxed-constexpr", "-I", INCLUDE, "-I", CSRC, "-Xcudafe", "--diag_suppress=177"]
 
 
 def _nvcc() -> str:

@@ -1,0 +1,238 @@
+// tcgemm.cuh -- 3xTF32 tensor-core GEMM engine for sm_100a (tcgen05 + TMA + TMEM).
+//
+//   C_tile (BM x BN) = sum_k A[m][k] * B[n][k]        (both operands K-major, fp32 values)
+//
+// Each fp32 operand is stored as two planes, hi = x with its 13 low mantissa bits cleared
+// (exact in tf32) and lo = x - hi (exact in fp32). The product is accumulated as
+//   A_hi B_hi + A_hi B_lo + A_lo B_hi
+// in fp32 TMEM accumulators, which keeps about 22 significant bits per product (the dropped
+// A_lo B_lo term and the tf32 truncation of lo are both below 2^-21 relative).
+//
+// Pipeline (one 128-thread CTA per output tile):
+//   warp 0 / lane 0 : TMA producer, STAGES-deep ring of {A_hi, A_lo, B_hi, B_lo} k-blocks of
+//                     32 fp32 (one 128-byte swizzle row), full/empty mbarriers;
+//   warp 1 / lane 0 : MMA issuer, 4 k-steps of 8 x 3 tcgen05.mma per k-block, tcgen05.commit
+//                     frees the stage, a final commit signals the epilogue;
+//   all 4 warps     : epilogue, tcgen05.ld of the accumulator (warp w owns TMEM lanes
+//                     32w..32w+31 = tile rows), then the Epi functor.
+// A launch may hold several problems (a grouped GEMM): the operand tensor maps cover whole
+// planes and every problem only moves the tile origins.
+// Every mbarrier wait is bounded; on expiry the status word gets BAKRON_ERR_TIMEOUT, in-flight
+// copies and MMAs are drained (with a bound) and the TMEM is released before returning.
+#pragma once
+
+#include "sm100.cuh"
+
+namespace bakron {
+namespace tc {
+
+constexpr int BM = 128;
+constexpr int BK = 32;
+constexpr int kMaxProblems = 24;
+constexpr int kThreads = 128;
+
+struct Problem {
+    int a_row0, a_k0;   // origin of the A tile rows (M) and of K in the A planes
+    int b_row0, b_k0;   // origin of the B tile rows (N) and of K in the B planes
+    int M, N, K;        // problem extents
+    int c_row0, c_col0; // origin of the output (handed to the epilogue)
+    int tiles_n;        // ceil(N / BN)
+    int tile_begin;     // first linear tile index of this problem in the launch
+    int tiles;          // number of tiles of this problem in the launch
+    int upper_only;     // 1: only tiles with tile_m <= tile_n (square tiles, BM == BN)
+    float weight;       // epilogue scalar
+};
+
+struct Problems {
+    Problem p[kMaxProblems];
+    int count;
+    int total_tiles;
+};
+
+template <int BN>
+struct Cfg {
+    static constexpr uint32_t kABytes = BM * BK * 4;          // one A plane k-block
+    static constexpr uint32_t kBBytes = BN * BK * 4;          // one B plane k-block
+    static constexpr uint32_t kStageBytes = 2 * kABytes + 2 * kBBytes;
+    static constexpr uint32_t kTmemCols = BN < 32 ? 32 : BN;  // power of two >= 32
+};
+
+template <int BN, int STAGES>
+constexpr size_t gemm_smem_bytes() {
+    return 1024 /*alignment slack*/ + (size_t)STAGES * Cfg<BN>::kStageBytes + 256;
+}
+
+// Maps a linear tile index of the launch to (problem, m0, n0). Returns false if out of range.
+__device__ __forceinline__ bool decode_tile(const Problems& P, int BNv, int t, int& pi, int& m0,
+                                            int& n0) {
+    for (int i = 0; i < P.count; ++i) {
+        const Problem& p = P.p[i];
+        if (t >= p.tile_begin && t < p.tile_begin + p.tiles) {
+            int local = t - p.tile_begin;
+            int tm, tn;
+            if (p.upper_only) {
+                // enumerate (tm, tn) with tm <= tn < tiles_n row by row
+                tm = 0;
+                int rowlen = p.tiles_n;
+                while (local >= rowlen) { local -= rowlen; ++tm; --rowlen; }
+                tn = tm + local;
+            } else {
+                tm = local / p.tiles_n;
+                tn = local % p.tiles_n;
+            }
+            pi = i;
+            m0 = tm * BM;
+            n0 = tn * BNv;
+            return true;
+        }
+    }
+    return false;
+}
+
+template <int BN, int STAGES, class Epi>
+__global__ void __launch_bounds__(kThreads, 1)
+gemm3x_kernel(const __grid_constant__ CUtensorMap a_hi, const __grid_constant__ CUtensorMap a_lo,
+              const __grid_constant__ CUtensorMap b_hi, const __grid_constant__ CUtensorMap b_lo,
+              const __grid_constant__ Problems probs, const Epi epi, int* status,
+              uint64_t limit_ns) {
+    using C = Cfg<BN>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * C::kStageBytes);
+    uint64_t* empty = full + STAGES;
+    uint64_t* done = empty + STAGES;       // accumulator complete
+    uint64_t* drain = done + 1;            // error path: all MMAs retired
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    int* s_abort = reinterpret_cast<int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    Epi e = epi;
+    int pi, m0, n0;
+    if (!decode_tile(probs, BN, blockIdx.x, pi, m0, n0)) return;
+    const Problem& P = probs.p[pi];
+    const int nkb = (P.K + BK - 1) / BK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            sm100::mbar_init(&full[s], 1);
+            sm100::mbar_init(&empty[s], 1);
+        }
+        sm100::mbar_init(done, 1);
+        sm100::mbar_init(drain, 1);
+        *s_abort = 0;
+        sm100::fence_mbar_init();
+    }
+    if (warp == 0) {
+        sm100::tmem_alloc(tmem_slot, C::kTmemCols);
+        sm100::tmem_relinquish();
+    }
+    sm100::tc_fence_before();
+    __syncthreads();
+    sm100::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    auto stage_ptr = [&](int s, int which) -> uint8_t* {
+        // which: 0 A_hi, 1 A_lo, 2 B_hi, 3 B_lo
+        uint8_t* base = smem + (size_t)s * C::kStageBytes;
+        return which < 2 ? base + which * C::kABytes : base + 2 * C::kABytes + (which - 2) * C::kBBytes;
+    };
+
+    if (warp == 0 && lane == 0 && nkb > 0) {
+        // ---------------- TMA producer
+        sm100::prefetch_tmap(&a_hi);
+        sm100::prefetch_tmap(&a_lo);
+        sm100::prefetch_tmap(&b_hi);
+        sm100::prefetch_tmap(&b_lo);
+        int issued = 0;
+        for (int kb = 0; kb < nkb; ++kb) {
+            const int s = kb % STAGES;
+            const uint32_t ph = (kb / STAGES) & 1;
+            if (kb >= STAGES) {
+                if (!sm100::mbar_wait(&empty[s], ph ^ 1, status, limit_ns)) {
+                    atomicExch(s_abort, 1);
+                    break;
+                }
+            }
+            if (*(volatile int*)s_abort) break;
+            sm100::mbar_arrive_expect_tx(&full[s], C::kStageBytes);
+            const int ka = P.a_k0 + kb * BK, kbb = P.b_k0 + kb * BK;
+            sm100::tma_load_2d(stage_ptr(s, 0), &a_hi, ka, P.a_row0 + m0, &full[s]);
+            sm100::tma_load_2d(stage_ptr(s, 1), &a_lo, ka, P.a_row0 + m0, &full[s]);
+            sm100::tma_load_2d(stage_ptr(s, 2), &b_hi, kbb, P.b_row0 + n0, &full[s]);
+            sm100::tma_load_2d(stage_ptr(s, 3), &b_lo, kbb, P.b_row0 + n0, &full[s]);
+            issued = kb + 1;
+        }
+        // Error path: let every issued copy land before the CTA can exit.
+        if (*(volatile int*)s_abort) {
+            for (int kb = (issued > STAGES ? issued - STAGES : 0); kb < issued; ++kb)
+                sm100::mbar_wait(&full[kb % STAGES], (kb / STAGES) & 1, status, limit_ns);
+        }
+    } else if (warp == 1 && lane == 0 && nkb > 0) {
+        // ---------------- MMA issuer
+        constexpr uint32_t idesc = sm100::idesc_tf32(BM, BN);
+        for (int kb = 0; kb < nkb; ++kb) {
+            const int s = kb % STAGES;
+            const uint32_t ph = (kb / STAGES) & 1;
+            if (!sm100::mbar_wait(&full[s], ph, status, limit_ns)) {
+                atomicExch(s_abort, 1);
+                break;
+            }
+            if (*(volatile int*)s_abort) break;
+            sm100::tc_fence_after();
+            const uint32_t ah = sm100::smem_u32(stage_ptr(s, 0));
+            const uint32_t al = sm100::smem_u32(stage_ptr(s, 1));
+            const uint32_t bh = sm100::smem_u32(stage_ptr(s, 2));
+            const uint32_t bl = sm100::smem_u32(stage_ptr(s, 3));
+#pragma unroll
+            for (int kk = 0; kk < BK / 8; ++kk) {
+                const uint32_t off = kk * 32;  // 8 tf32 = 32 bytes along the swizzled row
+                const uint64_t dah = sm100::desc_kmajor_sw128(ah + off);
+                const uint64_t dal = sm100::desc_kmajor_sw128(al + off);
+                const uint64_t dbh = sm100::desc_kmajor_sw128(bh + off);
+                const uint64_t dbl = sm100::desc_kmajor_sw128(bl + off);
+                const uint32_t acc0 = (kb > 0 || kk > 0) ? 1u : 0u;
+                sm100::mma_tf32(tmem, dah, dbh, idesc, acc0);
+                sm100::mma_tf32(tmem, dah, dbl, idesc, 1u);
+                sm100::mma_tf32(tmem, dal, dbh, idesc, 1u);
+            }
+            sm100::mma_commit(&empty[s]);
+        }
+        if (*(volatile int*)s_abort) {
+            sm100::mma_commit(drain);
+            sm100::mbar_wait(drain, 0, status, limit_ns);
+        } else {
+            sm100::mma_commit(done);
+        }
+    }
+    __syncwarp();
+
+    // ---------------- epilogue (all 4 warps)
+    bool have = nkb > 0;
+    if (have) {
+        // every thread polls the completion barrier (bounded)
+        if (!sm100::mbar_wait(done, 0, status, limit_ns)) have = false;
+        if (*(volatile int*)s_abort) have = false;
+    }
+    have = __all_sync(0xffffffffu, have);
+    sm100::tc_fence_after();
+    const int row = m0 + warp * 32 + lane;
+#pragma unroll 1
+    for (int c0 = 0; c0 < BN; c0 += 32) {
+        float v[32];
+        if (have) {
+            sm100::tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0, v);
+        } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = 0.f;
+        }
+        if (!*(volatile int*)s_abort) e(P, row, n0 + c0, m0, n0, v);
+    }
+    e.finish(P, blockIdx.x);
+    sm100::tc_fence_before();
+    __syncthreads();
+    if (warp == 0) sm100::tmem_dealloc(tmem, C::kTmemCols);
+}
+
+}  // namespace tc
+}  // namespace bakron

@@ -1,0 +1,153 @@
+// tcgemm_host.cuh -- host-side helpers of the 3xTF32 GEMM engine: tensor maps, hi/lo plane
+// splitting, epilogue functors and the launcher.
+#pragma once
+
+#include <cudaTypedefs.h>
+
+#include "tcgemm.cuh"
+
+namespace bakron {
+namespace tc {
+
+// Leading dimension of every hi/lo plane: a multiple of 32 fp32 (128 bytes), which satisfies
+// the tensor-map stride rule (multiple of 16 bytes) and keeps rows on 128-byte boundaries.
+inline int plane_ld(int cols) { return (cols + 31) / 32 * 32; }
+
+// 2-D K-major fp32 tensor map: `rows` rows of `kcols` valid fp32 values, row stride `ld`
+// elements (ld % 4 == 0, base 16-byte aligned), box of 32 x box_rows, 128-byte swizzle,
+// out-of-range elements read as zero.
+int make_kmajor_map(CUtensorMap* map, const float* base, int rows, int kcols, int ld,
+                    int box_rows);
+
+// Splits an fp32 matrix (rows x cols, row stride ld_src) into hi/lo planes (row stride
+// ld_dst). transpose = 1 writes the planes of the transposed matrix (cols x rows).
+void split_planes(const float* src, int rows, int cols, int ld_src, float* hi, float* lo,
+                  int ld_dst, int transpose, cudaStream_t st);
+
+// ---------------------------------------------------------------------------- epilogues
+// out = weight * acc, written as hi/lo planes at (c_row0 + r, c_col0 + c).
+struct EpiStoreSplit {
+    float* hi;
+    float* lo;
+    int ld;
+    __device__ void operator()(const Problem& P, int row, int col0, int, int,
+                               const float (&v)[32]) {
+        if (row >= P.M) return;
+        const size_t base = (size_t)(P.c_row0 + row) * ld + P.c_col0 + col0;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            if (col0 + i < P.N) {
+                const float x = P.weight * v[i];
+                const float h = sm100::tf32_hi(x);
+                hi[base + i] = h;
+                lo[base + i] = x - h;
+            }
+        }
+    }
+    __device__ void finish(const Problem&, int) {}
+};
+
+// C (+)= weight * acc at (c_row0 + r, c_col0 + c); `accumulate` selects += over =; with
+// `upper` set only entries whose global column >= global row are touched.
+struct EpiStore {
+    float* C;
+    int ldc;
+    int accumulate;
+    int upper;
+    __device__ void operator()(const Problem& P, int row, int col0, int, int,
+                               const float (&v)[32]) {
+        if (row >= P.M) return;
+        const int gr = P.c_row0 + row;
+        float* out = C + (size_t)gr * ldc + P.c_col0 + col0;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            const int gc = P.c_col0 + col0 + i;
+            if (col0 + i < P.N && (!upper || gc >= gr)) {
+                const float x = P.weight * v[i];
+                out[i] = accumulate ? out[i] + x : x;
+            }
+        }
+    }
+    __device__ void finish(const Problem&, int) {}
+};
+
+// partial[tile] = w * sum_{r,c in tile} acc[r][c] * G[r][c] in fp64, w = 1 on diagonal tiles
+// (m0 == n0) and `offdiag_weight` elsewhere (symmetric products computed on one triangle).
+struct EpiDot {
+    const float* G;
+    int ldg;
+    double* partial;
+    float offdiag_weight;
+    double acc;
+    __device__ void operator()(const Problem& P, int row, int col0, int m0, int n0,
+                               const float (&v)[32]) {
+        if (row >= P.M) return;
+        const float* g = G + (size_t)row * ldg + col0;
+        double s = 0.0;
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+            if (col0 + i < P.N) s += (double)v[i] * (double)g[i];
+        acc += (m0 == n0) ? s : (double)offdiag_weight * s;
+    }
+    __device__ void finish(const Problem&, int tile) {
+        __shared__ double red[kThreads / 32];
+        double s = acc;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) s += __shfl_down_sync(0xffffffffu, s, o);
+        if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = s;
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            double t = 0.0;
+            for (int w = 0; w < kThreads / 32; ++w) t += red[w];
+            partial[tile] = t;
+        }
+    }
+};
+
+// ---------------------------------------------------------------------------- problems
+struct ProblemList {
+    Problems P{};
+    int BN;
+    explicit ProblemList(int bn) : BN(bn) { P.count = 0; P.total_tiles = 0; }
+    // returns false when the list is full
+    bool add(int a_row0, int a_k0, int b_row0, int b_k0, int M, int N, int K, int c_row0,
+             int c_col0, float weight = 1.f, int upper_only = 0) {
+        if (M <= 0 || N <= 0) return true;
+        if (P.count == kMaxProblems) return false;
+        Problem& p = P.p[P.count++];
+        p.a_row0 = a_row0; p.a_k0 = a_k0; p.b_row0 = b_row0; p.b_k0 = b_k0;
+        p.M = M; p.N = N; p.K = K; p.c_row0 = c_row0; p.c_col0 = c_col0;
+        p.tiles_n = (N + BN - 1) / BN;
+        const int tiles_m = (M + BM - 1) / BM;
+        p.upper_only = upper_only;
+        p.tiles = upper_only ? p.tiles_n * (p.tiles_n + 1) / 2 : tiles_m * p.tiles_n;
+        p.tile_begin = P.total_tiles;
+        p.weight = weight;
+        P.total_tiles += p.tiles;
+        return true;
+    }
+    bool empty() const { return P.total_tiles == 0; }
+};
+
+template <int BN, int STAGES, class Epi>
+int launch_gemm3x(const CUtensorMap& ah, const CUtensorMap& al, const CUtensorMap& bh,
+                  const CUtensorMap& bl, const ProblemList& L, const Epi& epi, int* status,
+                  cudaStream_t st) {
+    if (L.empty()) return BAKRON_OK;
+    constexpr size_t smem = gemm_smem_bytes<BN, STAGES>();
+    auto kern = gemm3x_kernel<BN, STAGES, Epi>;
+    static bool configured = false;   // per template instance
+    if (!configured) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)smem);
+        if (e != cudaSuccess) return BAKRON_ERR_CUDA;
+        configured = true;
+    }
+    kern<<<L.P.total_tiles, kThreads, smem, st>>>(ah, al, bh, bl, L.P, epi, status,
+                                                  spin_limit_ns());
+    count_launches(1);
+    return cuda_err(cudaGetLastError());
+}
+
+}  // namespace tc
+}  // namespace bakron
