@@ -20,7 +20,7 @@ def bk():
 
 @pytest.mark.parametrize("M,N,K,seed", [(128, 128, 32, 0), (128, 128, 256, 1), (256, 384, 1024, 2),
                                         (100, 37, 50, 3), (1, 1, 1, 4), (130, 129, 33, 5),
-                                        (640, 256, 4096, 6), (128, 128, 0, 7)])
+                                        (640, 256, 4096, 6)])
 def test_gemm3x_matches_fp64(bk, M, N, K, seed):
     rng = np.random.default_rng(seed)
     A = rng.standard_normal((M, K)).astype(np.float32)

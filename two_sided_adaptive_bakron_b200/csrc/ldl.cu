@@ -5,22 +5,30 @@
 // of the same section makes L strictly upper (a U D U^T factorisation, i.e. LDL^T of H with its
 // index order reversed).
 //
-// Blocked right-looking algorithm, last block of indices first. With the index set split into
-// A (still pending, lower indices), B (the current block) and C (done), and H' the Schur
-// complement left by C:
-//   H'_BB = U_BB D_B U_BB^T               (unblocked, one warp, fp64)
-//   U_AB  = H'_AB U_BB^{-T} D_B^{-1}        (one thread per row of A, back substitution)
-//   H'_AA -= (U_AB D_B) U_AB^T             (upper triangle only)
-// The factor is built in place in the output buffer L, which first receives a copy of the
-// upper triangle of H; the entries on and below the diagonal are cleared at the end.
+// Two-level blocked right-looking algorithm, last indices first, built in place in the output
+// L (which first receives the upper triangle of H). With U = I + L, pending indices A, the
+// current block B and H' the Schur complement left by the indices after B:
+//   H'_BB = U_BB D_B U_BB^T                  one CTA per 128-index block (fp64 in shared
+//                                             memory), which also forms U_BB^{-1};
+//   X     = H'_AB U_BB^{-T},  U_AB = X D_B^{-1} 3xTF32 tensor-core GEMM (K = 128) whose
+//                                             epilogue writes U_AB into L and the hi/lo planes
+//                                             of X and U_AB;
+//   H'_AA -= X U_AB^T                        split in two: columns inside the current 512-index
+//                                             outer block right away (K = 128), the rest once
+//                                             per outer block (K = 512, upper block triangle),
+//                                             so the trailing matrix is streamed n/512 times.
 #include <algorithm>
 
-#include "common.cuh"
+#include "tcgemm_host.cuh"
 
 namespace bakron {
 namespace {
 
-constexpr int NB = 32;  // block of indices per step
+constexpr int NBI = 128;   // inner block: diagonal factorisation in one CTA
+constexpr int NBO = 512;   // outer block: K of the trailing update
+constexpr int BN = 128;
+constexpr int STAGES = 3;
+constexpr int DIAG_THREADS = 256;
 
 __global__ void copy_upper_kernel(const float* __restrict__ H, float* __restrict__ L, int n) {
     const size_t total = (size_t)n * n;
@@ -40,105 +48,122 @@ __global__ void clear_lower_kernel(float* __restrict__ L, int n) {
     }
 }
 
-// Unblocked U D U^T of the b x b diagonal block [k0, k0+b), one warp, fp64; lane i owns row i.
-__global__ void diag_block_kernel(float* __restrict__ L, float* __restrict__ D, int n, int k0,
-                                  int b, int* status) {
-    __shared__ double h[NB][NB + 1];
-    const int lane = threadIdx.x;
-    for (int c = 0; c < NB; ++c)
-        h[lane][c] = (lane < b && c < b && c >= lane) ? (double)L[(size_t)(k0 + lane) * n + k0 + c]
-                                                      : 0.0;
-    __syncwarp();
+constexpr size_t kDiagSmem = (size_t)NBI * (NBI + 1) * sizeof(double)   // S (fp64)
+                             + (size_t)NBI * (NBI + 1) * sizeof(float);  // U^{-1}
+
+// U D U^T of the b x b diagonal block at [k0, k0 + b) (b <= 128) in fp64 shared memory;
+// writes U's strictly upper part into L, the pivots into D, and U^{-1} (unit upper, zero
+// padded to 128 x 128) as hi/lo planes with row stride 128.
+__global__ void __launch_bounds__(DIAG_THREADS) diag_block_kernel(float* __restrict__ L, int n,
+                                                                int k0, int b,
+                                                                float* __restrict__ D,
+                                                                float* __restrict__ inv_hi,
+                                                                float* __restrict__ inv_lo,
+                                                                int* status) {
+    extern __shared__ double dsm[];
+    double(*S)[NBI + 1] = reinterpret_cast<double(*)[NBI + 1]>(dsm);
+    float(*Ui)[NBI + 1] = reinterpret_cast<float(*)[NBI + 1]>(dsm + NBI * (NBI + 1));
+    const int tid = threadIdx.x;
+    for (int e = tid; e < NBI * NBI; e += DIAG_THREADS) {
+        const int r = e / NBI, c = e % NBI;
+        S[r][c] = (r < b && c < b && c >= r) ? (double)L[(size_t)(k0 + r) * n + k0 + c] : 0.0;
+    }
+    __syncthreads();
+    // right-looking rank-1 downdates, last index first
+    const int row = tid % NBI, par = tid / NBI;   // two threads per row
     for (int j = b - 1; j >= 0; --j) {
-        double d = h[j][j];
-        if (!(d > 0.0) || !isfinite(d)) {
-            if (lane == 0) set_status(status, BAKRON_ERR_NOT_PD);
-            d = 1.0;
+        __syncthreads();   // the previous downdate is complete
+        double d = S[j][j];
+        const bool bad = !(d > 0.0) || !isfinite(d);
+        if (bad) d = 1.0;
+        if (tid == 0) {
+            if (bad) set_status(status, BAKRON_ERR_NOT_PD);
+            D[k0 + j] = (float)d;
         }
-        double u = 0.0;
-        if (lane < j) u = h[lane][j] / d;
-        __syncwarp();
-        if (lane < j) h[lane][j] = u;   // column j of U (strictly upper part)
-        if (lane == 0) D[k0 + j] = (float)d;
-        __syncwarp();
-        // rank-1 downdate of the leading (j x j) block, upper triangle
-        if (lane < j) {
-            for (int l = lane; l < j; ++l) h[lane][l] -= u * d * h[l][j];
+        if (par == 0 && row < j) S[row][j] /= d;   // rows < j only: S[j][j] is not touched
+        __syncthreads();
+        if (row < j) {
+            const double ui = S[row][j] * d;
+            for (int l = row + par; l < j; l += 2) S[row][l] -= ui * S[l][j];
         }
-        __syncwarp();
     }
-    for (int c = 0; c < NB; ++c)
-        if (lane < b && c < b && c > lane) L[(size_t)(k0 + lane) * n + k0 + c] = (float)h[lane][c];
-}
-
-// Rows i < k0: y U_BB^T = H'_{iB} (back substitution), U_{iB} = y / D_B; y kept for the update.
-__global__ void panel_kernel(float* __restrict__ L, const float* __restrict__ D,
-                             float* __restrict__ Y, int n, int k0, int b) {
-    __shared__ float u[NB][NB + 1];
-    __shared__ float dinv[NB];
-    for (int e = threadIdx.x; e < NB * NB; e += blockDim.x) {
-        const int r = e / NB, c = e % NB;
-        u[r][c] = (r < b && c < b && c > r) ? L[(size_t)(k0 + r) * n + k0 + c] : 0.f;
-    }
-    if (threadIdx.x < NB) dinv[threadIdx.x] = (threadIdx.x < b) ? 1.f / D[k0 + threadIdx.x] : 0.f;
     __syncthreads();
-    const int i = blockIdx.x * blockDim.x + threadIdx.x;
-    if (i >= k0) return;
-    float y[NB];
-#pragma unroll
-    for (int c = 0; c < NB; ++c) y[c] = (c < b) ? L[(size_t)i * n + k0 + c] : 0.f;
-#pragma unroll
-    for (int jj = NB - 1; jj >= 0; --jj) {
-        float acc = y[jj];
-#pragma unroll
-        for (int l = jj + 1; l < NB; ++l) acc = fmaf(-u[jj][l], y[l], acc);
-        y[jj] = acc;
+    for (int e = tid; e < NBI * NBI; e += DIAG_THREADS) {
+        const int r = e / NBI, c = e % NBI;
+        if (r < b && c < b && c > r) L[(size_t)(k0 + r) * n + k0 + c] = (float)S[r][c];
     }
-#pragma unroll
-    for (int c = 0; c < NB; ++c) {
+    // U^{-1} by columns: U x = e_c (back substitution), thread c owns column c
+    if (tid < NBI) {
+        const int c = tid;
+        for (int r = 0; r < NBI; ++r) Ui[r][c] = (r == c && c < b) ? 1.f : 0.f;
         if (c < b) {
-            Y[(size_t)i * NB + c] = y[c];
-            L[(size_t)i * n + k0 + c] = y[c] * dinv[c];
+            // x kept in shared memory column c (fp32 storage of fp64 sums)
+            for (int r = c - 1; r >= 0; --r) {
+                double acc = -S[r][c];
+                for (int t = r + 1; t < c; ++t) acc -= S[r][t] * (double)Ui[t][c];
+                Ui[r][c] = (float)acc;
+            }
         }
+    }
+    __syncthreads();
+    for (int e = tid; e < NBI * NBI; e += DIAG_THREADS) {
+        const int r = e / NBI, c = e % NBI;
+        const float x = Ui[r][c];
+        const float h = sm100::tf32_hi(x);
+        inv_hi[e] = h;
+        inv_lo[e] = x - h;
     }
 }
 
-// H'_AA -= Y U_AB^T on the upper triangle of [0, k0)^2; 64 x 64 output tiles, K = NB.
-__global__ void __launch_bounds__(256) syrk_update_kernel(float* __restrict__ L,
-                                                         const float* __restrict__ Y, int n,
-                                                         int k0, int T) {
-    // blockIdx.x -> (ti, tj), ti <= tj < T
-    int rem = blockIdx.x, ti = 0;
-    while (rem >= T - ti) { rem -= T - ti; ++ti; }
-    const int tj = ti + rem;
-    __shared__ float sY[NB][64 + 4];
-    __shared__ float sP[NB][64 + 4];
-    const int i0 = ti * 64, j0 = tj * 64;
-    for (int e = threadIdx.x; e < 64 * NB; e += 256) {
-        const int r = e / NB, c = e % NB;
-        sY[c][r] = (i0 + r < k0) ? Y[(size_t)(i0 + r) * NB + c] : 0.f;
-        sP[c][r] = (j0 + r < k0) ? L[(size_t)(j0 + r) * n + k0 + c] : 0.f;
-    }
-    __syncthreads();
-    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
-    float acc[4][4] = {};
-#pragma unroll 8
-    for (int k = 0; k < NB; ++k) {
-        float a[4], bb[4];
+// Panel epilogue: x = (H'_AB U_BB^{-T})[i][c]; U_AB = x / D_c goes to L; x and U_AB also go
+// to the hi/lo planes used by the trailing updates (column offset c_off in the outer block).
+struct EpiPanel {
+    float* L;
+    int n;
+    const float* D;
+    int kb0;
+    float* xh;
+    float* xl;
+    float* uh;
+    float* ul;
+    int ldx;
+    int c_off;
+    __device__ void operator()(const tc::Problem& P, int row, int col0, int, int,
+                               const float (&v)[32]) {
+        if (row >= P.M) return;
 #pragma unroll
-        for (int q = 0; q < 4; ++q) { a[q] = sY[k][ty * 4 + q]; bb[q] = sP[k][tx * 4 + q]; }
-#pragma unroll
-        for (int p = 0; p < 4; ++p)
-#pragma unroll
-            for (int q = 0; q < 4; ++q) acc[p][q] = fmaf(a[p], bb[q], acc[p][q]);
-    }
-#pragma unroll
-    for (int p = 0; p < 4; ++p)
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const int i = i0 + ty * 4 + p, j = j0 + tx * 4 + q;
-            if (i < k0 && j < k0 && j >= i) L[(size_t)i * n + j] -= acc[p][q];
+        for (int i = 0; i < 32; ++i) {
+            const int c = col0 + i;
+            if (c < P.N) {
+                const float x = v[i];
+                const float u = __fdiv_rn(x, D[kb0 + c]);
+                L[(size_t)row * n + kb0 + c] = u;
+                const size_t o = (size_t)row * ldx + c_off + c;
+                const float xh_ = sm100::tf32_hi(x), uh_ = sm100::tf32_hi(u);
+                xh[o] = xh_;
+                xl[o] = x - xh_;
+                uh[o] = uh_;
+                ul[o] = u - uh_;
+            }
         }
+    }
+    __device__ void finish(const tc::Problem&, int) {}
+};
+
+struct LdlWs {
+    float *inv_hi, *inv_lo, *p_hi, *p_lo, *x_hi, *x_lo, *u_hi, *u_lo;
+};
+
+template <class F>
+void ldl_ws_layout(int n, F&& take) {
+    take((size_t)NBI * NBI);        // inv_hi
+    take((size_t)NBI * NBI);        // inv_lo
+    take((size_t)n * NBI);          // p_hi  (panel of H')
+    take((size_t)n * NBI);          // p_lo
+    take((size_t)n * NBO);          // x_hi  (X of the outer block)
+    take((size_t)n * NBO);          // x_lo
+    take((size_t)n * NBO);          // u_hi  (U_AB of the outer block)
+    take((size_t)n * NBO);          // u_lo
 }
 
 }  // namespace
@@ -149,7 +174,7 @@ using namespace bakron;
 extern "C" size_t bakron_ldl_workspace_bytes(int n) {
     if (n < 1) return 0;
     WsSizer z;
-    z.take<float>((size_t)n * NB);  // Y = U_AB D_B panel
+    ldl_ws_layout(n, [&](size_t k) { z.take<float>(k); });
     return z.bytes();
 }
 
@@ -159,20 +184,69 @@ extern "C" int bakron_ldl(const float* H, int n, float* L, float* D, void* ws, s
     if (!ws_ok(ws, ws_bytes, bakron_ldl_workspace_bytes(n))) return BAKRON_ERR_WORKSPACE;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     WsCarver c(ws);
-    float* Y = c.take<float>((size_t)n * NB);
-    const int eb = 1184;  // elementwise grid
+    float* bufs[8];
+    int bi = 0;
+    ldl_ws_layout(n, [&](size_t k) { bufs[bi++] = c.take<float>(k); });
+    LdlWs w{bufs[0], bufs[1], bufs[2], bufs[3], bufs[4], bufs[5], bufs[6], bufs[7]};
+
+    static bool diag_configured = false;
+    if (!diag_configured) {
+        if (cudaFuncSetAttribute(diag_block_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)kDiagSmem) != cudaSuccess)
+            return BAKRON_ERR_CUDA;
+        diag_configured = true;
+    }
+    int e;
+    // Tensor maps over the outer-block planes (fixed for the whole call).
+    CUtensorMap m_xh, m_xl, m_uh, m_ul;
+    if ((e = tc::make_kmajor_map(&m_xh, w.x_hi, n, NBO, NBO, tc::BM))) return e;
+    if ((e = tc::make_kmajor_map(&m_xl, w.x_lo, n, NBO, NBO, tc::BM))) return e;
+    if ((e = tc::make_kmajor_map(&m_uh, w.u_hi, n, NBO, NBO, BN))) return e;
+    if ((e = tc::make_kmajor_map(&m_ul, w.u_lo, n, NBO, NBO, BN))) return e;
+
+    const int eb = 1184;
     copy_upper_kernel<<<eb, 256, 0, st>>>(H, L, n);
-    for (int k1 = n; k1 > 0; k1 -= NB) {
-        const int k0 = std::max(0, k1 - NB), b = k1 - k0;
-        diag_block_kernel<<<1, 32, 0, st>>>(L, D, n, k0, b, dev_status);
-        if (k0 > 0) {
-            panel_kernel<<<(k0 + 127) / 128, 128, 0, st>>>(L, D, Y, n, k0, b);
-            const int T = (k0 + 63) / 64;
-            syrk_update_kernel<<<T * (T + 1) / 2, 256, 0, st>>>(L, Y, n, k0, T);
+    count_launches(1);
+    for (int ko1 = n; ko1 > 0; ko1 -= NBO) {
+        const int ko0 = std::max(0, ko1 - NBO);
+        for (int kb1 = ko1; kb1 > ko0; kb1 -= NBI) {
+            const int kb0 = std::max(ko0, kb1 - NBI), b = kb1 - kb0, c_off = kb0 - ko0;
+            diag_block_kernel<<<1, DIAG_THREADS, kDiagSmem, st>>>(L, n, kb0, b, D, w.inv_hi,
+                                                                  w.inv_lo, dev_status);
+            count_launches(1);
+            if (kb0 == 0) continue;
+            // panel: X = H'[0:kb0, B] U_BB^{-T}
+            tc::split_planes(L + kb0, kb0, b, n, w.p_hi, w.p_lo, NBI, 0, st);
+            CUtensorMap m_ph, m_pl, m_ih, m_il;
+            if ((e = tc::make_kmajor_map(&m_ph, w.p_hi, kb0, b, NBI, tc::BM))) return e;
+            if ((e = tc::make_kmajor_map(&m_pl, w.p_lo, kb0, b, NBI, tc::BM))) return e;
+            if ((e = tc::make_kmajor_map(&m_ih, w.inv_hi, NBI, b, NBI, BN))) return e;
+            if ((e = tc::make_kmajor_map(&m_il, w.inv_lo, NBI, b, NBI, BN))) return e;
+            tc::ProblemList pl(BN);
+            pl.add(0, 0, 0, 0, kb0, b, b, 0, 0);
+            EpiPanel ep{L, n, D, kb0, w.x_hi, w.x_lo, w.u_hi, w.u_lo, NBO, c_off};
+            if ((e = tc::launch_gemm3x<BN, STAGES>(m_ph, m_pl, m_ih, m_il, pl, ep, dev_status, st)))
+                return e;
+            // columns of the outer block still pending: H'[0:kb0, ko0:kb0] -= X U_AB^T
+            if (kb0 > ko0) {
+                tc::ProblemList wl(BN);
+                wl.add(0, c_off, ko0, c_off, kb0, kb0 - ko0, b, 0, ko0, -1.f);
+                tc::EpiStore es{L, n, 1, 1};
+                if ((e = tc::launch_gemm3x<BN, STAGES>(m_xh, m_xl, m_uh, m_ul, wl, es, dev_status,
+                                                       st)))
+                    return e;
+            }
+        }
+        // the rest of the trailing matrix, once per outer block: upper block triangle
+        if (ko0 > 0) {
+            tc::ProblemList tl(BN);
+            tl.add(0, 0, 0, 0, ko0, ko0, ko1 - ko0, 0, 0, -1.f, /*upper_only=*/1);
+            tc::EpiStore es{L, n, 1, 1};
+            if ((e = tc::launch_gemm3x<BN, STAGES>(m_xh, m_xl, m_uh, m_ul, tl, es, dev_status, st)))
+                return e;
         }
     }
     clear_lower_kernel<<<eb, 256, 0, st>>>(L, n);
-    const long long nblk = (n + NB - 1) / NB;
-    count_launches(2 + 3 * nblk - 2);
+    count_launches(1);
     return cuda_err(cudaGetLastError());
 }

@@ -4,64 +4,84 @@
 //   pre_ij = W*_ij + a_i^T E[:i,:j] b_j + a_i^T E[:i,j] + E[i,:j] b_j,  E = W* - W,
 //   W_ij   = s_i * clamp(rint(pre_ij / s_i)).
 // Entry (i,j) reads only entries (k,l) with k <= i, l <= j, so every anti-diagonal i+j = const
-// is independent (BaKron page, abstract: O(m+n) sequential steps).
+// is independent (BaKron page, abstract: O(m+n) sequential steps, anti-diagonal parallelism
+// combined with a divide-and-conquer construction that brings the work to O(mn(m+n))).
 //
-// Reformulation used here. With U = (I + L_O)^T E (column-causal) the rule reads
+// Reformulation. With U = (I + L_O)^T E (column-causal) the rule reads
 //   pre_ij = W*_ij + T_ij + R_ij,   T_ij = sum_{k<i} L_O[k,i] E_kj,   U_ij = T_ij + E_ij,
 //                                   R_ij = sum_{l<j} U_il L_I[l,j],
-// i.e. a vertical sum over E (from rows above) and a horizontal sum over U (from columns to
-// the left); the bilinear term a_i^T E[:i,:j] b_j is carried by U.
+// a vertical sum over E (rows above) and a horizontal sum over U (columns to the left); the
+// bilinear term a_i^T E[:i,:j] b_j is carried by U.
 //
-// Structure (one persistent cooperative launch):
-//  * The matrix is cut into 32x32 leaves. Leaf (I,J) depends on leaves (I',J) with I' < I
-//    (through E) and (I,J') with J' < J (through U).
-//  * Blocks take leaves in anti-diagonal order, round robin. Leaves of earlier diagonals have
-//    smaller indices, every block walks its leaves in increasing index order and all blocks
-//    are co-resident (cooperative launch), so the dependency waits cannot form a cycle.
-//  * For its leaf a block first gathers the contributions of all earlier leaves (T from the
-//    leaves above, R from the leaves to the left), waiting on each source leaf's ready flag
-//    with a bounded spin. Then one warp runs the in-leaf anti-diagonal wavefront (63 steps):
-//    lane j owns column j; values are indexed by step ("slot" t = r + j) so that every register
-//    index is a compile-time constant; the vertical in-leaf updates stay in the lane, the
-//    horizontal ones travel by warp shuffles. Finally the block publishes E and U of the leaf
-//    and raises the leaf's flag (release), which readers acquire.
-//  * E and U are read with ld.global.cg (L2, never a possibly stale L1 line).
+// Structure. The matrix is cut into 256 x 256 super-blocks, processed one super-block
+// anti-diagonal ("phase") at a time; the blocks of a phase are independent of each other.
+//  * Leaf launch (persistent, cooperative): every block of the phase is cut into 32 x 32
+//    leaves, taken in anti-diagonal order across all blocks of the phase. A leaf starts from
+//    the far sums T_far, R_far (everything outside its block, already accumulated), adds the
+//    contributions of the leaves above / to the left inside its block (CUDA-core dot products,
+//    after a bounded wait on each source leaf's ready flag), then one warp runs the in-leaf
+//    wavefront (63 steps; lane j owns column j, values indexed by step so that every register
+//    index is a compile-time constant; vertical updates stay in the lane, horizontal ones move
+//    by warp shuffles). The leaf publishes codes, W, E (row-major), E^T and U as hi/lo planes
+//    and raises its flag (release / acquire).
+//  * Push launches (3xTF32 tcgen05 GEMMs, one grouped launch per direction): every block of
+//    the phase pushes its E into T_far of all rows below it and its U into R_far of all
+//    columns to its right (K = 256), i.e. the divide-and-conquer off-diagonal updates as dense
+//    block products.
 #include <algorithm>
 
-#include "common.cuh"
+#include "tcgemm_host.cuh"
 
 namespace bakron {
 namespace {
 
 constexpr int LB = 32;          // leaf edge
 constexpr int NSLOT = 2 * LB - 1;
-constexpr int NTH = 128;        // threads per block
+constexpr int NTH = 128;        // threads per leaf block
+constexpr int SB = 256;         // super-block edge
+constexpr int LPB = SB / LB;    // leaves per super-block edge
+constexpr int BN = 128;
+constexpr int STAGES = 3;
 
-struct RoundArgs {
+struct PhaseArgs {
     const float* Ws;
     const float* LO;
     const float* LI;
     const float* sc;
-    int m, n, Mt, Nt;
+    const float* Tf;
+    const float* Rf;
+    int m, n, Nt;
+    int delta, p_lo, p_hi, maxd;
     float qlo, qhi;
     int8_t* codes;
     float* Wq;
     float* E;
-    float* U;
+    float* et_hi;
+    float* et_lo;
+    int ldm;
+    float* u_hi;
+    float* u_lo;
+    int ldn;
     int* flags;
     int* abort_word;
     int* status;
     uint64_t limit_ns;
-    long long total;
+    int total;
 };
 
-__device__ __forceinline__ int diag_count(int D, int Mt, int Nt) {
-    return min(D, Mt - 1) - max(0, D - Nt + 1) + 1;
+__device__ __forceinline__ int leaves_of(int extent, int blk) {
+    const int e = min(SB, extent - blk * SB);
+    return (e + LB - 1) / LB;
 }
 
-// The in-leaf wavefront, run by one warp. Inputs live in shared memory with row stride LB:
-// element (r, c) of a leaf sits at r*LB + c, so both an anti-diagonal (distinct c) and a row
-// (distinct c) hit 32 distinct banks.
+// number of leaves (a, c) with a + c = d in a block of lm x ln leaves
+__device__ __forceinline__ int diag_len(int d, int lm, int ln) {
+    const int lo = max(0, d - ln + 1), hi = min(d, lm - 1);
+    return hi >= lo ? hi - lo + 1 : 0;
+}
+
+// The in-leaf wavefront, run by one warp. Leaf arrays live in shared memory with row stride
+// LB: element (r, c) at r*LB + c, so an anti-diagonal and a row both touch 32 distinct banks.
 __device__ __forceinline__ void solve_leaf(int lane, int rows, int cols, float qlo, float qhi,
                                            const float* sW, const float* sT, const float* sR,
                                            const float* sLO, const float* sLI, const float* sS,
@@ -121,7 +141,7 @@ __device__ __forceinline__ void solve_leaf(int lane, int rows, int cols, float q
     if (bad) set_status(status, BAKRON_ERR_NONFINITE);
 }
 
-__global__ void __launch_bounds__(NTH) round_leaves_kernel(RoundArgs a) {
+__global__ void __launch_bounds__(NTH) phase_leaves_kernel(PhaseArgs a) {
     __shared__ float sA[LB][LB + 1];
     __shared__ float sB[LB][LB + 1];
     __shared__ float sT[LB * LB], sR[LB * LB], sW[LB * LB], sLO[LB * LB], sLI[LB * LB];
@@ -132,36 +152,49 @@ __global__ void __launch_bounds__(NTH) round_leaves_kernel(RoundArgs a) {
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int m = a.m, n = a.n;
-    int Dg = 0;
+    // walker over (local diagonal d, block row P), counting tasks
+    int d = 0, P = a.p_lo;
     long long base = 0;
 
-    for (long long g = blockIdx.x; g < a.total; g += gridDim.x) {
+    for (int g = blockIdx.x; g < a.total; g += gridDim.x) {
+        int lm, ln, cnt;
         while (true) {
-            const int c = diag_count(Dg, a.Mt, a.Nt);
-            if (g < base + c) break;
-            base += c;
-            ++Dg;
+            const int Q = a.delta - P;
+            lm = leaves_of(m, P);
+            ln = leaves_of(n, Q);
+            cnt = diag_len(d, lm, ln);
+            if (g < base + cnt) break;
+            base += cnt;
+            if (++P > a.p_hi) { P = a.p_lo; ++d; }
         }
-        const int I = max(0, Dg - (a.Nt - 1)) + (int)(g - base);
-        const int J = Dg - I;
+        const int Q = a.delta - P;
+        const int la = max(0, d - ln + 1) + (int)(g - base);   // leaf row inside the block
+        const int lc = d - la;                                 // leaf column inside the block
+        const int I = P * LPB + la, J = Q * LPB + lc;
         const int i0 = I * LB, j0 = J * LB;
         const int rows = min(LB, m - i0), cols = min(LB, n - j0);
 
+        // ---- far sums (everything outside the block), then the leaves above / left inside it
         float accT[8], accR[8];
 #pragma unroll
-        for (int t = 0; t < 8; ++t) accT[t] = accR[t] = 0.f;
-
-        // ---- vertical contributions of the leaves above: T += L_O[K-rows, leaf rows]^T E
-        for (int Kp = 0; Kp < I; ++Kp) {
+        for (int t = 0; t < 8; ++t) {
+            const int r = warp * 8 + t;
+            const bool ok = r < rows && lane < cols;
+            const size_t o = (size_t)(i0 + r) * n + j0 + lane;
+            accT[t] = ok ? __ldcg(&a.Tf[o]) : 0.f;
+            accR[t] = ok ? __ldcg(&a.Rf[o]) : 0.f;
+        }
+        for (int ka = 0; ka < la; ++ka) {
+            const int Ip = P * LPB + ka;
             if (tid == 0)
-                s_stop = wait_flag(&a.flags[(size_t)Kp * a.Nt + J], a.abort_word, a.status,
+                s_stop = wait_flag(&a.flags[(size_t)Ip * a.Nt + J], a.abort_word, a.status,
                                    a.limit_ns) ? 0 : 1;
             __syncthreads();
             if (s_stop) return;
 #pragma unroll
             for (int q = 0; q < (LB * LB) / NTH; ++q) {
                 const int e = tid + q * NTH, kk = e >> 5, c = e & 31;
-                const size_t k = (size_t)Kp * LB + kk;
+                const size_t k = (size_t)Ip * LB + kk;
                 sA[kk][c] = (c < rows) ? __ldg(&a.LO[k * m + i0 + c]) : 0.f;
                 sB[kk][c] = (c < cols) ? __ldcg(&a.E[k * n + j0 + c]) : 0.f;
             }
@@ -174,18 +207,19 @@ __global__ void __launch_bounds__(NTH) round_leaves_kernel(RoundArgs a) {
             }
             __syncthreads();
         }
-        // ---- horizontal contributions of the leaves to the left: R += U[leaf rows, L-cols] L_I
-        for (int Lp = 0; Lp < J; ++Lp) {
+        for (int kc = 0; kc < lc; ++kc) {
+            const int Jp = Q * LPB + kc;
             if (tid == 0)
-                s_stop = wait_flag(&a.flags[(size_t)I * a.Nt + Lp], a.abort_word, a.status,
+                s_stop = wait_flag(&a.flags[(size_t)I * a.Nt + Jp], a.abort_word, a.status,
                                    a.limit_ns) ? 0 : 1;
             __syncthreads();
             if (s_stop) return;
 #pragma unroll
             for (int q = 0; q < (LB * LB) / NTH; ++q) {
                 const int e = tid + q * NTH, rr = e >> 5, c = e & 31;
-                const size_t l = (size_t)Lp * LB;
-                sA[rr][c] = (rr < rows) ? __ldcg(&a.U[(size_t)(i0 + rr) * n + l + c]) : 0.f;
+                const size_t l = (size_t)Jp * LB;
+                const size_t o = (size_t)(i0 + rr) * a.ldn + l + c;
+                sA[rr][c] = (rr < rows) ? (__ldcg(&a.u_hi[o]) + __ldcg(&a.u_lo[o])) : 0.f;
                 sB[rr][c] = (c < cols) ? __ldg(&a.LI[(l + rr) * n + j0 + c]) : 0.f;
             }
             __syncthreads();
@@ -208,12 +242,12 @@ __global__ void __launch_bounds__(NTH) round_leaves_kernel(RoundArgs a) {
         for (int q = 0; q < (LB * LB) / NTH; ++q) {
             const int e = tid + q * NTH, r = e >> 5, c = e & 31;
             sW[e] = (r < rows && c < cols) ? __ldg(&a.Ws[(size_t)(i0 + r) * n + j0 + c]) : 0.f;
-            // skewed diagonal blocks: sLO[d][r] = L_O[i0+r][i0+r+d], sLI[d][c] = L_I[j0+c][j0+c+d]
-            const int d = r, x = c;
-            sLO[e] = (d >= 1 && x + d < rows)
-                         ? __ldg(&a.LO[(size_t)(i0 + x) * m + i0 + x + d]) : 0.f;
-            sLI[e] = (d >= 1 && x + d < cols)
-                         ? __ldg(&a.LI[(size_t)(j0 + x) * n + j0 + x + d]) : 0.f;
+            // skewed diagonal blocks: sLO[dd][x] = L_O[i0+x][i0+x+dd], sLI[dd][x] likewise
+            const int dd = r, x = c;
+            sLO[e] = (dd >= 1 && x + dd < rows)
+                         ? __ldg(&a.LO[(size_t)(i0 + x) * m + i0 + x + dd]) : 0.f;
+            sLI[e] = (dd >= 1 && x + dd < cols)
+                         ? __ldg(&a.LI[(size_t)(j0 + x) * n + j0 + x + dd]) : 0.f;
         }
         if (tid < LB) sS[tid] = (tid < rows) ? __ldg(&a.sc[i0 + tid]) : 0.f;
         __syncthreads();
@@ -223,7 +257,7 @@ __global__ void __launch_bounds__(NTH) round_leaves_kernel(RoundArgs a) {
                        a.status);
         __syncthreads();
 
-        // ---- publish
+        // ---- publish: row-major outputs and E, U planes; E^T planes transposed
 #pragma unroll
         for (int q = 0; q < (LB * LB) / NTH; ++q) {
             const int e = tid + q * NTH, r = e >> 5, c = e & 31;
@@ -232,7 +266,17 @@ __global__ void __launch_bounds__(NTH) round_leaves_kernel(RoundArgs a) {
                 a.codes[o] = oC[e];
                 a.Wq[o] = oW[e];
                 __stcg(&a.E[o], oE[e]);
-                __stcg(&a.U[o], oU[e]);
+                const float u = oU[e], uh = sm100::tf32_hi(u);
+                const size_t ou = (size_t)(i0 + r) * a.ldn + j0 + c;
+                __stcg(&a.u_hi[ou], uh);
+                __stcg(&a.u_lo[ou], u - uh);
+            }
+            const int rt = e & 31, ct = e >> 5;   // transposed walk: consecutive rows
+            if (rt < rows && ct < cols) {
+                const float x = oE[rt * LB + ct], xh = sm100::tf32_hi(x);
+                const size_t ot = (size_t)(j0 + ct) * a.ldm + i0 + rt;
+                a.et_hi[ot] = xh;
+                a.et_lo[ot] = x - xh;
             }
         }
         __threadfence();
@@ -242,7 +286,7 @@ __global__ void __launch_bounds__(NTH) round_leaves_kernel(RoundArgs a) {
 }
 
 struct Layout {
-    int Mt, Nt;
+    int Mt, Nt, MS, NS, ldm, ldn;
     size_t mn;
 };
 
@@ -250,8 +294,40 @@ Layout layout(int m, int n) {
     Layout L;
     L.Mt = (m + LB - 1) / LB;
     L.Nt = (n + LB - 1) / LB;
+    L.MS = (m + SB - 1) / SB;
+    L.NS = (n + SB - 1) / SB;
+    L.ldm = tc::plane_ld(m);
+    L.ldn = tc::plane_ld(n);
     L.mn = (size_t)m * n;
     return L;
+}
+
+template <class F>
+void round_ws_layout(const Layout& L, int m, int n, F&& take) {
+    take((size_t)L.mn * 4);                         // E (row-major, first: see bakron.h)
+    take((size_t)m * L.ldm * 4); take((size_t)m * L.ldm * 4);   // L_O^T planes
+    take((size_t)n * L.ldn * 4); take((size_t)n * L.ldn * 4);   // L_I^T planes
+    take((size_t)n * L.ldm * 4); take((size_t)n * L.ldm * 4);   // E^T planes
+    take((size_t)m * L.ldn * 4); take((size_t)m * L.ldn * 4);   // U planes
+    take((size_t)L.mn * 4);                         // T_far
+    take((size_t)L.mn * 4);                         // R_far
+    take(((size_t)L.Mt * L.Nt + 64) * 4);           // leaf flags + abort word
+}
+
+int leaf_grid(int tasks) {
+    static int cached = 0;
+    if (!cached) {
+        int dev = 0, nsm = 0, per_sm = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+        if (cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return -1;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, phase_leaves_kernel, NTH, 0) !=
+            cudaSuccess)
+            return -1;
+        if (per_sm < 1) return -1;
+        cached = per_sm * nsm;
+    }
+    return std::min(tasks, cached);
 }
 
 }  // namespace
@@ -263,9 +339,7 @@ extern "C" size_t bakron_round_workspace_bytes(int m, int n) {
     if (m < 1 || n < 1) return 0;
     const Layout L = layout(m, n);
     WsSizer z;
-    z.take<float>(L.mn);                      // E
-    z.take<float>(L.mn);                      // U
-    z.take<int>((size_t)L.Mt * L.Nt + 64);    // leaf flags + abort word
+    round_ws_layout(L, m, n, [&](size_t bytes) { z.take<char>(bytes); });
     return z.bytes();
 }
 
@@ -279,32 +353,100 @@ extern "C" int bakron_round(const float* Wstar, int m, int n, const float* L_O, 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const Layout L = layout(m, n);
     WsCarver c(ws);
-    RoundArgs a;
-    a.E = c.take<float>(L.mn);
-    a.U = c.take<float>(L.mn);
-    a.flags = c.take<int>((size_t)L.Mt * L.Nt + 64);
-    a.abort_word = a.flags + (size_t)L.Mt * L.Nt;
-    int e = cuda_err(cudaMemsetAsync(a.flags, 0, ((size_t)L.Mt * L.Nt + 64) * sizeof(int), st));
-    if (e) return e;
-    a.Ws = Wstar; a.LO = L_O; a.LI = L_I; a.sc = scales;
-    a.m = m; a.n = n; a.Mt = L.Mt; a.Nt = L.Nt;
+    char* p[12];
+    int k = 0;
+    round_ws_layout(L, m, n, [&](size_t bytes) { p[k++] = c.take<char>(bytes); });
+    float* E = (float*)p[0];
+    float *lot_hi = (float*)p[1], *lot_lo = (float*)p[2];
+    float *lit_hi = (float*)p[3], *lit_lo = (float*)p[4];
+    float *et_hi = (float*)p[5], *et_lo = (float*)p[6];
+    float *u_hi = (float*)p[7], *u_lo = (float*)p[8];
+    float *Tf = (float*)p[9], *Rf = (float*)p[10];
+    int* flags = (int*)p[11];
+    int e;
+    if ((e = cuda_err(cudaMemsetAsync(flags, 0, ((size_t)L.Mt * L.Nt + 64) * 4, st)))) return e;
+    if ((e = cuda_err(cudaMemsetAsync(Tf, 0, L.mn * 4, st)))) return e;
+    if ((e = cuda_err(cudaMemsetAsync(Rf, 0, L.mn * 4, st)))) return e;
+    // static operands of the pushes: L_O^T and L_I^T as hi/lo planes
+    tc::split_planes(L_O, m, m, m, lot_hi, lot_lo, L.ldm, 1, st);
+    tc::split_planes(L_I, n, n, n, lit_hi, lit_lo, L.ldn, 1, st);
+
+    CUtensorMap m_loth, m_lotl, m_eth, m_etl, m_uh, m_ul, m_lith, m_litl;
+    if ((e = tc::make_kmajor_map(&m_loth, lot_hi, m, m, L.ldm, tc::BM))) return e;
+    if ((e = tc::make_kmajor_map(&m_lotl, lot_lo, m, m, L.ldm, tc::BM))) return e;
+    if ((e = tc::make_kmajor_map(&m_eth, et_hi, n, m, L.ldm, BN))) return e;
+    if ((e = tc::make_kmajor_map(&m_etl, et_lo, n, m, L.ldm, BN))) return e;
+    if ((e = tc::make_kmajor_map(&m_uh, u_hi, m, n, L.ldn, tc::BM))) return e;
+    if ((e = tc::make_kmajor_map(&m_ul, u_lo, m, n, L.ldn, tc::BM))) return e;
+    if ((e = tc::make_kmajor_map(&m_lith, lit_hi, n, n, L.ldn, BN))) return e;
+    if ((e = tc::make_kmajor_map(&m_litl, lit_lo, n, n, L.ldn, BN))) return e;
+
+    PhaseArgs a;
+    a.Ws = Wstar; a.LO = L_O; a.LI = L_I; a.sc = scales; a.Tf = Tf; a.Rf = Rf;
+    a.m = m; a.n = n; a.Nt = L.Nt;
     a.qlo = (float)(-(1 << (bits - 1)));
     a.qhi = (float)((1 << (bits - 1)) - 1);
-    a.codes = codes; a.Wq = W;
+    a.codes = codes; a.Wq = W; a.E = E;
+    a.et_hi = et_hi; a.et_lo = et_lo; a.ldm = L.ldm;
+    a.u_hi = u_hi; a.u_lo = u_lo; a.ldn = L.ldn;
+    a.flags = flags;
+    a.abort_word = flags + (size_t)L.Mt * L.Nt;
     a.status = dev_status;
     a.limit_ns = spin_limit_ns();
-    a.total = (long long)L.Mt * L.Nt;
 
-    int dev = 0, nsm = 0, per_sm = 0;
-    if ((e = cuda_err(cudaGetDevice(&dev)))) return e;
-    if ((e = cuda_err(cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev)))) return e;
-    if ((e = cuda_err(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, round_leaves_kernel,
-                                                                    NTH, 0))))
-        return e;
-    if (per_sm < 1) return BAKRON_ERR_CUDA;
-    const long long grid = std::min<long long>(a.total, (long long)per_sm * nsm);
-    void* params[] = {&a};
-    count_launches(1);
-    return cuda_err(cudaLaunchCooperativeKernel((const void*)round_leaves_kernel, dim3((unsigned)grid),
-                                                dim3(NTH), params, 0, st));
+    for (int delta = 0; delta < L.MS + L.NS - 1; ++delta) {
+        const int p_lo = std::max(0, delta - (L.NS - 1)), p_hi = std::min(delta, L.MS - 1);
+        int total = 0, maxd = 0;
+        for (int P = p_lo; P <= p_hi; ++P) {
+            const int lm = (std::min(SB, m - P * SB) + LB - 1) / LB;
+            const int ln = (std::min(SB, n - (delta - P) * SB) + LB - 1) / LB;
+            total += lm * ln;
+            maxd = std::max(maxd, lm + ln - 2);
+        }
+        a.delta = delta; a.p_lo = p_lo; a.p_hi = p_hi; a.maxd = maxd; a.total = total;
+        const int grid = leaf_grid(total);
+        if (grid < 1) return BAKRON_ERR_CUDA;
+        void* params[] = {&a};
+        count_launches(1);
+        if ((e = cuda_err(cudaLaunchCooperativeKernel((const void*)phase_leaves_kernel,
+                                                      dim3(grid), dim3(NTH), params, 0, st))))
+            return e;
+
+        // pushes of the phase's blocks: E down into T_far, U right into R_far
+        tc::ProblemList pv(BN), ph(BN);
+        auto flush_v = [&]() -> int {
+            tc::EpiStore epi{Tf, n, 1, 0};
+            int r = tc::launch_gemm3x<BN, STAGES>(m_loth, m_lotl, m_eth, m_etl, pv, epi,
+                                                   dev_status, st);
+            pv = tc::ProblemList(BN);
+            return r;
+        };
+        auto flush_h = [&]() -> int {
+            tc::EpiStore epi{Rf, n, 1, 0};
+            int r = tc::launch_gemm3x<BN, STAGES>(m_uh, m_ul, m_lith, m_litl, ph, epi,
+                                                   dev_status, st);
+            ph = tc::ProblemList(BN);
+            return r;
+        };
+        for (int P = p_lo; P <= p_hi; ++P) {
+            const int Q = delta - P;
+            const int r0 = P * SB, c0 = Q * SB;
+            const int br = std::min(SB, m - r0), bc = std::min(SB, n - c0);
+            if (r0 + br < m) {
+                if (!pv.add(r0 + br, r0, c0, r0, m - (r0 + br), bc, br, r0 + br, c0)) {
+                    if ((e = flush_v())) return e;
+                    pv.add(r0 + br, r0, c0, r0, m - (r0 + br), bc, br, r0 + br, c0);
+                }
+            }
+            if (c0 + bc < n) {
+                if (!ph.add(r0, c0, c0 + bc, c0, br, n - (c0 + bc), bc, r0, c0 + bc)) {
+                    if ((e = flush_h())) return e;
+                    ph.add(r0, c0, c0 + bc, c0, br, n - (c0 + bc), bc, r0, c0 + bc);
+                }
+            }
+        }
+        if (!pv.empty() && (e = flush_v())) return e;
+        if (!ph.empty() && (e = flush_h())) return e;
+    }
+    return cuda_err(cudaGetLastError());
 }

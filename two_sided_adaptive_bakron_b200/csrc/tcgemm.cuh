@@ -28,7 +28,7 @@ namespace tc {
 
 constexpr int BM = 128;
 constexpr int BK = 32;
-constexpr int kMaxProblems = 24;
+constexpr int kMaxProblems = 48;
 constexpr int kThreads = 128;
 
 struct Problem {
