@@ -28,7 +28,7 @@ constexpr int NBI = 128;   // inner block: diagonal factorisation in one CTA
 constexpr int NBO = 512;   // outer block: K of the trailing update
 constexpr int BN = 128;
 constexpr int STAGES = 3;
-constexpr int DIAG_THREADS = 256;
+constexpr int DIAG_THREADS = 512;
 
 __global__ void copy_upper_kernel(const float* __restrict__ H, float* __restrict__ L, int n) {
     const size_t total = (size_t)n * n;
@@ -48,8 +48,7 @@ __global__ void clear_lower_kernel(float* __restrict__ L, int n) {
     }
 }
 
-constexpr size_t kDiagSmem = (size_t)NBI * (NBI + 1) * sizeof(double)   // S (fp64)
-                             + (size_t)NBI * (NBI + 1) * sizeof(float);  // U^{-1}
+constexpr size_t kDiagSmem = (size_t)NBI * (NBI + 1) * sizeof(double);  // S and W^T, fp64
 
 // U D U^T of the b x b diagonal block at [k0, k0 + b) (b <= 128) in fp64 shared memory;
 // writes U's strictly upper part into L, the pivots into D, and U^{-1} (unit upper, zero
@@ -62,17 +61,20 @@ __global__ void __launch_bounds__(DIAG_THREADS) diag_block_kernel(float* __restr
                                                                 int* status) {
     extern __shared__ double dsm[];
     double(*S)[NBI + 1] = reinterpret_cast<double(*)[NBI + 1]>(dsm);
-    float(*Ui)[NBI + 1] = reinterpret_cast<float(*)[NBI + 1]>(dsm + NBI * (NBI + 1));
     const int tid = threadIdx.x;
     for (int e = tid; e < NBI * NBI; e += DIAG_THREADS) {
         const int r = e / NBI, c = e % NBI;
         S[r][c] = (r < b && c < b && c >= r) ? (double)L[(size_t)(k0 + r) * n + k0 + c] : 0.0;
     }
-    __syncthreads();
-    // right-looking rank-1 downdates, last index first
-    const int row = tid % NBI, par = tid / NBI;   // two threads per row
+    // Right-looking rank-1 downdates, last index first. Column j of U is u_j + e_j, and
+    // U = G_{b-1} ... G_1 with G_j = I + u_j e_j^T, so U^{-1} = G_1^{-1} ... G_{b-1}^{-1}
+    // with G_j^{-1} = I - u_j e_j^T: the inverse W is accumulated alongside, W <- G_j^{-1} W
+    // (rows i < j: W[i][:] -= u_j[i] W[j][:]), stored transposed in the strictly lower
+    // triangle of S (S[c][i] = W[i][c], c > i; its unit diagonal is implicit).
+    const int row = tid % NBI, par = tid / NBI;   // DIAG_THREADS / NBI threads per row
+    constexpr int PAR = DIAG_THREADS / NBI;
     for (int j = b - 1; j >= 0; --j) {
-        __syncthreads();   // the previous downdate is complete
+        __syncthreads();   // the previous step is complete
         double d = S[j][j];
         const bool bad = !(d > 0.0) || !isfinite(d);
         if (bad) d = 1.0;
@@ -83,32 +85,20 @@ __global__ void __launch_bounds__(DIAG_THREADS) diag_block_kernel(float* __restr
         if (par == 0 && row < j) S[row][j] /= d;   // rows < j only: S[j][j] is not touched
         __syncthreads();
         if (row < j) {
-            const double ui = S[row][j] * d;
-            for (int l = row + par; l < j; l += 2) S[row][l] -= ui * S[l][j];
+            const double u = S[row][j];
+            const double ud = u * d;
+            for (int l = row + par; l < j; l += PAR) S[row][l] -= ud * S[l][j];
+            // W[row][c] -= u * W[j][c] for c >= j (W[j][j] = 1)
+            if (par == 0) S[j][row] = -u;
+            for (int c = j + 1 + par; c < b; c += PAR) S[c][row] -= u * S[c][j];
         }
     }
     __syncthreads();
     for (int e = tid; e < NBI * NBI; e += DIAG_THREADS) {
         const int r = e / NBI, c = e % NBI;
         if (r < b && c < b && c > r) L[(size_t)(k0 + r) * n + k0 + c] = (float)S[r][c];
-    }
-    // U^{-1} by columns: U x = e_c (back substitution), thread c owns column c
-    if (tid < NBI) {
-        const int c = tid;
-        for (int r = 0; r < NBI; ++r) Ui[r][c] = (r == c && c < b) ? 1.f : 0.f;
-        if (c < b) {
-            // x kept in shared memory column c (fp32 storage of fp64 sums)
-            for (int r = c - 1; r >= 0; --r) {
-                double acc = -S[r][c];
-                for (int t = r + 1; t < c; ++t) acc -= S[r][t] * (double)Ui[t][c];
-                Ui[r][c] = (float)acc;
-            }
-        }
-    }
-    __syncthreads();
-    for (int e = tid; e < NBI * NBI; e += DIAG_THREADS) {
-        const int r = e / NBI, c = e % NBI;
-        const float x = Ui[r][c];
+        // U^{-1}[r][c] (zero padded to 128 x 128), hi/lo planes
+        const float x = (r < b && c < b) ? (c > r ? (float)S[c][r] : (c == r ? 1.f : 0.f)) : 0.f;
         const float h = sm100::tf32_hi(x);
         inv_hi[e] = h;
         inv_lo[e] = x - h;
@@ -209,8 +199,10 @@ extern "C" int bakron_ldl(const float* H, int n, float* L, float* D, void* ws, s
     count_launches(1);
     for (int ko1 = n; ko1 > 0; ko1 -= NBO) {
         const int ko0 = std::max(0, ko1 - NBO);
-        for (int kb1 = ko1; kb1 > ko0; kb1 -= NBI) {
-            const int kb0 = std::max(ko0, kb1 - NBI), b = kb1 - kb0, c_off = kb0 - ko0;
+        for (int t = 0, kb1 = ko1; kb1 > ko0; ++t, kb1 -= NBI) {
+            // plane columns of this inner block, counted from the end of the outer block so
+            // that they stay 128-aligned even when the outer block is a partial one
+            const int kb0 = std::max(ko0, kb1 - NBI), b = kb1 - kb0, c_off = NBO - NBI * (t + 1);
             diag_block_kernel<<<1, DIAG_THREADS, kDiagSmem, st>>>(L, n, kb0, b, D, w.inv_hi,
                                                                   w.inv_lo, dev_status);
             count_launches(1);

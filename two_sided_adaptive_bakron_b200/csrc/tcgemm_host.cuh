@@ -134,6 +134,9 @@ int launch_gemm3x(const CUtensorMap& ah, const CUtensorMap& al, const CUtensorMa
                   const CUtensorMap& bl, const ProblemList& L, const Epi& epi, int* status,
                   cudaStream_t st) {
     if (L.empty()) return BAKRON_OK;
+    // A TMA tile load must start on a 16-byte boundary: every K origin a multiple of 4 fp32.
+    for (int i = 0; i < L.P.count; ++i)
+        if ((L.P.p[i].a_k0 & 3) || (L.P.p[i].b_k0 & 3)) return BAKRON_ERR_INVALID_ARG;
     constexpr size_t smem = gemm_smem_bytes<BN, STAGES>();
     auto kern = gemm3x_kernel<BN, STAGES, Epi>;
     static bool configured = false;   // per template instance
