@@ -48,11 +48,28 @@ __global__ void clear_lower_kernel(float* __restrict__ L, int n) {
     }
 }
 
-constexpr size_t kDiagSmem = (size_t)NBI * (NBI + 1) * sizeof(double);  // S and W^T, fp64
+constexpr int SUB = 32;                                   // sub-block of the diagonal block
+constexpr int NSUB = NBI / SUB;
+constexpr size_t kSOff = 0;                               // S: [NBI][NBI+1] fp64
+constexpr size_t kXOff = kSOff + (size_t)NBI * (NBI + 1); // X: [NBI-SUB][SUB+1] fp64
+constexpr size_t kTOff = kXOff + (size_t)(NBI - SUB) * (SUB + 1);  // T: [NSUB-1][SUB][SUB+1]
+constexpr size_t kDiagSmem =
+    (kTOff + (size_t)(NSUB - 1) * SUB * (SUB + 1) + NBI) * sizeof(double);
 
 // U D U^T of the b x b diagonal block at [k0, k0 + b) (b <= 128) in fp64 shared memory;
 // writes U's strictly upper part into L, the pivots into D, and U^{-1} (unit upper, zero
 // padded to 128 x 128) as hi/lo planes with row stride 128.
+//
+// Indices >= b are padded with the identity (pivot 1, no coupling), so the block is always
+// 128 wide. It is processed in 32-index sub-blocks, last first:
+//  (1) one warp factors the 32 x 32 diagonal sub-block by rank-1 steps and accumulates its
+//      inverse alongside: column j of U is u_j + e_j and U = G_31 ... G_1 with
+//      G_j = I + u_j e_j^T, so U^{-1} = G_1^{-1} ... G_31^{-1}, G_j^{-1} = I - u_j e_j^T;
+//  (2) all threads: X = H'[rows above, sub-block] W_JJ^T and U = X D^{-1} for the rows above;
+//  (3) all threads: H'[rows above]^2 -= X U^T on the upper triangle.
+// The inverse's off-diagonal blocks follow by block back substitution,
+// W_IJ = -W_II sum_{I<K<=J} U_IK W_KJ. S keeps U in its strict upper triangle and W^T in its
+// strict lower triangle (both unit diagonals implicit).
 __global__ void __launch_bounds__(DIAG_THREADS) diag_block_kernel(float* __restrict__ L, int n,
                                                                 int k0, int b,
                                                                 float* __restrict__ D,
@@ -60,44 +77,111 @@ __global__ void __launch_bounds__(DIAG_THREADS) diag_block_kernel(float* __restr
                                                                 float* __restrict__ inv_lo,
                                                                 int* status) {
     extern __shared__ double dsm[];
-    double(*S)[NBI + 1] = reinterpret_cast<double(*)[NBI + 1]>(dsm);
-    const int tid = threadIdx.x;
+    double(*S)[NBI + 1] = reinterpret_cast<double(*)[NBI + 1]>(dsm + kSOff);
+    double(*X)[SUB + 1] = reinterpret_cast<double(*)[SUB + 1]>(dsm + kXOff);
+    double(*T)[SUB][SUB + 1] = reinterpret_cast<double(*)[SUB][SUB + 1]>(dsm + kTOff);
+    double* sD = dsm + kTOff + (size_t)(NSUB - 1) * SUB * (SUB + 1);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     for (int e = tid; e < NBI * NBI; e += DIAG_THREADS) {
         const int r = e / NBI, c = e % NBI;
-        S[r][c] = (r < b && c < b && c >= r) ? (double)L[(size_t)(k0 + r) * n + k0 + c] : 0.0;
-    }
-    // Right-looking rank-1 downdates, last index first. Column j of U is u_j + e_j, and
-    // U = G_{b-1} ... G_1 with G_j = I + u_j e_j^T, so U^{-1} = G_1^{-1} ... G_{b-1}^{-1}
-    // with G_j^{-1} = I - u_j e_j^T: the inverse W is accumulated alongside, W <- G_j^{-1} W
-    // (rows i < j: W[i][:] -= u_j[i] W[j][:]), stored transposed in the strictly lower
-    // triangle of S (S[c][i] = W[i][c], c > i; its unit diagonal is implicit).
-    const int row = tid % NBI, par = tid / NBI;   // DIAG_THREADS / NBI threads per row
-    constexpr int PAR = DIAG_THREADS / NBI;
-    for (int j = b - 1; j >= 0; --j) {
-        __syncthreads();   // the previous step is complete
-        double d = S[j][j];
-        const bool bad = !(d > 0.0) || !isfinite(d);
-        if (bad) d = 1.0;
-        if (tid == 0) {
-            if (bad) set_status(status, BAKRON_ERR_NOT_PD);
-            D[k0 + j] = (float)d;
-        }
-        if (par == 0 && row < j) S[row][j] /= d;   // rows < j only: S[j][j] is not touched
-        __syncthreads();
-        if (row < j) {
-            const double u = S[row][j];
-            const double ud = u * d;
-            for (int l = row + par; l < j; l += PAR) S[row][l] -= ud * S[l][j];
-            // W[row][c] -= u * W[j][c] for c >= j (W[j][j] = 1)
-            if (par == 0) S[j][row] = -u;
-            for (int c = j + 1 + par; c < b; c += PAR) S[c][row] -= u * S[c][j];
-        }
+        double v = 0.0;
+        if (r < b && c < b) v = (c >= r) ? (double)L[(size_t)(k0 + r) * n + k0 + c] : 0.0;
+        else if (r == c) v = 1.0;
+        S[r][c] = v;
     }
     __syncthreads();
+    for (int J = NSUB - 1; J >= 0; --J) {
+        const int j0 = J * SUB;
+        // (1) the diagonal sub-block, one warp
+        if (warp == 0) {
+            for (int jj = SUB - 1; jj >= 0; --jj) {
+                const int j = j0 + jj;
+                double d = S[j][j];
+                const bool bad = !(d > 0.0) || !isfinite(d);
+                if (bad) d = 1.0;
+                if (lane == 0) {
+                    sD[j] = d;
+                    if (j < b) {
+                        if (bad) set_status(status, BAKRON_ERR_NOT_PD);
+                        D[k0 + j] = (float)d;
+                    }
+                }
+                double u = 0.0;
+                if (lane < jj) {
+                    u = S[j0 + lane][j] / d;
+                    S[j0 + lane][j] = u;
+                }
+                __syncwarp();
+                if (lane < jj) {
+                    const int r = j0 + lane;
+                    const double ud = u * d;
+                    for (int l = r; l < j; ++l) S[r][l] -= ud * S[l][j];
+                    S[j][r] = -u;
+                    for (int c = j + 1; c < j0 + SUB; ++c) S[c][r] -= u * S[c][j];
+                }
+                __syncwarp();
+            }
+        }
+        __syncthreads();
+        if (J == 0) break;
+        // (2) X[r][c] = sum_{t >= c} H'[r][j0+t] W_JJ[c][t], rows r < j0
+        for (int e = tid; e < j0 * SUB; e += DIAG_THREADS) {
+            const int r = e / SUB, c = e % SUB;
+            double acc = S[r][j0 + c];
+            for (int t = c + 1; t < SUB; ++t) acc += S[r][j0 + t] * S[j0 + t][j0 + c];
+            X[r][c] = acc;
+        }
+        __syncthreads();
+        for (int e = tid; e < j0 * SUB; e += DIAG_THREADS) {
+            const int r = e / SUB, c = e % SUB;
+            S[r][j0 + c] = X[r][c] / sD[j0 + c];
+        }
+        __syncthreads();
+        // (3) H'[r][l] -= sum_c X[r][c] U[l][c], r <= l < j0
+        for (int e = tid; e < j0 * j0; e += DIAG_THREADS) {
+            const int r = e / j0, l = e % j0;
+            if (l < r) continue;
+            double acc = 0.0;
+#pragma unroll 8
+            for (int c = 0; c < SUB; ++c) acc += X[r][c] * S[l][j0 + c];
+            S[r][l] -= acc;
+        }
+        __syncthreads();
+    }
+    // off-diagonal blocks of W = U^{-1}, by distance J - I = 1 .. NSUB-1
+    for (int dist = 1; dist < NSUB; ++dist) {
+        const int npairs = NSUB - dist;
+        // T_p = sum_{K=I+1..J} U_IK W_KJ, pair p = I
+        for (int e = tid; e < npairs * SUB * SUB; e += DIAG_THREADS) {
+            const int I = e / (SUB * SUB), t = (e / SUB) % SUB, c = e % SUB;
+            const int Jb = I + dist, i0 = I * SUB, jb0 = Jb * SUB;
+            double acc = 0.0;
+            for (int K = I + 1; K <= Jb; ++K) {
+                const int kk0 = K * SUB;
+                for (int s = 0; s < SUB; ++s) {
+                    double w;   // W_KJ[s][c]
+                    if (K < Jb) w = S[jb0 + c][kk0 + s];
+                    else w = (c > s) ? S[jb0 + c][jb0 + s] : (c == s ? 1.0 : 0.0);
+                    acc += S[i0 + t][kk0 + s] * w;
+                }
+            }
+            T[I][t][c] = acc;
+        }
+        __syncthreads();
+        // W_IJ[a][c] = -sum_t W_II[a][t] T[t][c], stored as S[J0+c][I0+a]
+        for (int e = tid; e < npairs * SUB * SUB; e += DIAG_THREADS) {
+            const int I = e / (SUB * SUB), a = (e / SUB) % SUB, c = e % SUB;
+            const int Jb = I + dist, i0 = I * SUB, jb0 = Jb * SUB;
+            double acc = T[I][a][c];
+            for (int t = a + 1; t < SUB; ++t) acc += S[i0 + t][i0 + a] * T[I][t][c];
+            S[jb0 + c][i0 + a] = -acc;
+        }
+        __syncthreads();
+    }
     for (int e = tid; e < NBI * NBI; e += DIAG_THREADS) {
         const int r = e / NBI, c = e % NBI;
         if (r < b && c < b && c > r) L[(size_t)(k0 + r) * n + k0 + c] = (float)S[r][c];
-        // U^{-1}[r][c] (zero padded to 128 x 128), hi/lo planes
+        // U^{-1}[r][c] (zero padded beyond b), hi/lo planes
         const float x = (r < b && c < b) ? (c > r ? (float)S[c][r] : (c == r ? 1.f : 0.f)) : 0.f;
         const float h = sm100::tf32_hi(x);
         inv_hi[e] = h;
@@ -118,24 +202,16 @@ struct EpiPanel {
     float* ul;
     int ldx;
     int c_off;
-    __device__ void operator()(const tc::Problem& P, int row, int col0, int, int,
-                               const float (&v)[32]) {
-        if (row >= P.M) return;
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            const int c = col0 + i;
-            if (c < P.N) {
-                const float x = v[i];
-                const float u = __fdiv_rn(x, D[kb0 + c]);
-                L[(size_t)row * n + kb0 + c] = u;
-                const size_t o = (size_t)row * ldx + c_off + c;
-                const float xh_ = sm100::tf32_hi(x), uh_ = sm100::tf32_hi(u);
-                xh[o] = xh_;
-                xl[o] = x - xh_;
-                uh[o] = uh_;
-                ul[o] = u - uh_;
-            }
-        }
+    __device__ void operator()(const tc::Problem& P, int row, int c, int, int, float x) {
+        if (row >= P.M || c >= P.N) return;
+        const float u = __fdiv_rn(x, D[kb0 + c]);
+        L[(size_t)row * n + kb0 + c] = u;
+        const size_t o = (size_t)row * ldx + c_off + c;
+        const float xh_ = sm100::tf32_hi(x), uh_ = sm100::tf32_hi(u);
+        xh[o] = xh_;
+        xl[o] = x - xh_;
+        uh[o] = uh_;
+        ul[o] = u - uh_;
     }
     __device__ void finish(const tc::Problem&, int) {}
 };

@@ -80,62 +80,99 @@ __device__ __forceinline__ int diag_len(int d, int lm, int ln) {
     return hi >= lo ? hi - lo + 1 : 0;
 }
 
-// The in-leaf wavefront, run by one warp. Leaf arrays live in shared memory with row stride
-// LB: element (r, c) at r*LB + c, so an anti-diagonal and a row both touch 32 distinct banks.
+constexpr int UW = 4;            // wavefront steps per unrolled group
+constexpr int WIN = LB + UW;     // register window of slots
+constexpr int LS = LB + 4;       // row stride of the skewed diagonal blocks (16-byte rows)
+
+// The in-leaf wavefront, run by one warp; lane j owns column j and the element of row r is
+// handled at step s = r + j. Leaf arrays live in shared memory with row stride LB, element
+// (r, c) at r*LB + c, so an anti-diagonal and a row both touch 32 distinct banks.
+// Per lane, slot s of wT / wR holds the vertical / horizontal sum of its element of step s.
+// A step reads slot s, then pushes E down its column into slots s+1..s+31 (in-lane) and U
+// along its row into slot s+d of lane j+d (warp shuffles). The step loop stays rolled
+// (4 steps per iteration) over a sliding window of 36 slot registers, which keeps every
+// register index static while the code stays small enough for the instruction cache.
+//   sLOr[r*LS + d] = L_O[i0+r][i0+r+d]    (row r of the diagonal block, shifted)
+//   sLIc[c*LS + d] = L_I[j0+c-d][j0+c]    (column c of the diagonal block, shifted)
 __device__ __forceinline__ void solve_leaf(int lane, int rows, int cols, float qlo, float qhi,
                                            const float* sW, const float* sT, const float* sR,
-                                           const float* sLO, const float* sLI, const float* sS,
-                                           int8_t* oC, float* oW, float* oE, float* oU,
-                                           int* status) {
+                                           const float* sLOr, const float* sLIc,
+                                           const float* sS, int8_t* oC, float* oW, float* oE,
+                                           float* oU, int* status) {
     const int j = lane;
     const bool colok = j < cols;
-    float aT[NSLOT], aR[NSLOT];
+    float li[LB];
 #pragma unroll
-    for (int t = 0; t < NSLOT; ++t) {
+    for (int q = 0; q < LB / 4; ++q) {
+        const float4 v = *reinterpret_cast<const float4*>(&sLIc[j * LS + 4 * q]);
+        li[4 * q] = v.x; li[4 * q + 1] = v.y; li[4 * q + 2] = v.z; li[4 * q + 3] = v.w;
+    }
+    float wT[WIN], wR[WIN];
+#pragma unroll
+    for (int t = 0; t < WIN; ++t) {
         const int r = t - j;
         const bool ok = (r >= 0) && (r < LB);
         const int rr = ok ? r : 0;
-        aT[t] = ok ? sT[rr * LB + j] : 0.f;
-        aR[t] = ok ? sR[rr * LB + j] : 0.f;
+        wT[t] = ok ? sT[rr * LB + j] : 0.f;
+        wR[t] = ok ? sR[rr * LB + j] : 0.f;
     }
     bool bad = false;
+#pragma unroll 1
+    for (int s0 = 0; s0 < NSLOT; s0 += UW) {
 #pragma unroll
-    for (int s = 0; s < NSLOT; ++s) {
-        const int r = s - j;
-        const bool inleaf = (r >= 0) && (r < LB);
-        const int rr = inleaf ? r : 0;
-        const bool act = inleaf && (r < rows) && colok;
-        float e = 0.f, u = 0.f;
-        if (act) {
-            const float w_star = sW[rr * LB + j];
-            const float pre = w_star + aT[s] + aR[s];
-            const float sr = sS[rr];
-            float q = 0.f;
-            if (sr > 0.f) {
-                q = rintf(__fdiv_rn(pre, sr));
-                q = fminf(fmaxf(q, qlo), qhi);
+        for (int k = 0; k < UW; ++k) {
+            const int r = s0 + k - j;
+            const bool inleaf = (r >= 0) && (r < LB);
+            const int rr = inleaf ? r : 0;
+            const bool act = inleaf && (r < rows) && colok;
+            float e = 0.f, u = 0.f;
+            if (act) {
+                const float w_star = sW[rr * LB + j];
+                const float pre = w_star + wT[k] + wR[k];
+                const float sr = sS[rr];
+                float q = 0.f;
+                if (sr > 0.f) {
+                    q = rintf(__fdiv_rn(pre, sr));
+                    q = fminf(fmaxf(q, qlo), qhi);
+                }
+                bad |= !isfinite(pre);
+                const float w = sr * q;
+                e = w_star - w;
+                u = wT[k] + e;
+                oC[rr * LB + j] = (int8_t)q;
+                oW[rr * LB + j] = w;
+                oE[rr * LB + j] = e;
+                oU[rr * LB + j] = u;
             }
-            bad |= !isfinite(pre);
-            const float w = sr * q;
-            e = w_star - w;
-            u = aT[s] + e;
-            oC[rr * LB + j] = (int8_t)q;
-            oW[rr * LB + j] = w;
-            oE[rr * LB + j] = e;
-            oU[rr * LB + j] = u;
-        }
-        // vertical: E_rj feeds rows r+d of the same column (slot s+d of this lane)
+            // vertical: E_rj feeds rows r+d of the same column
+            float lo[LB];
 #pragma unroll
-        for (int d = 1; d < LB; ++d) {
-            if (s + d < NSLOT) aT[s + d] = fmaf(sLO[d * LB + rr], e, aT[s + d]);
-        }
-        // horizontal: U_rj feeds columns j+d of the same row (slot s+d of lane j+d)
+            for (int q = 0; q < LB / 4; ++q) {
+                const float4 v = *reinterpret_cast<const float4*>(&sLOr[rr * LS + 4 * q]);
+                lo[4 * q] = v.x; lo[4 * q + 1] = v.y; lo[4 * q + 2] = v.z; lo[4 * q + 3] = v.w;
+            }
 #pragma unroll
-        for (int d = 1; d < LB; ++d) {
-            if (s + d < NSLOT) {
+            for (int d = 1; d < LB; ++d) wT[k + d] = fmaf(lo[d], e, wT[k + d]);
+            // horizontal: U_rj feeds columns j+d of the same row (lane j+d)
+#pragma unroll
+            for (int d = 1; d < LB; ++d) {
                 const float v = __shfl_up_sync(0xffffffffu, u, d);
-                if (j >= d) aR[s + d] = fmaf(v, sLI[d * LB + (j - d)], aR[s + d]);
+                if (j >= d) wR[k + d] = fmaf(v, li[d], wR[k + d]);
             }
+        }
+        // slide the window by UW slots
+#pragma unroll
+        for (int t = 0; t < WIN - UW; ++t) {
+            wT[t] = wT[t + UW];
+            wR[t] = wR[t + UW];
+        }
+#pragma unroll
+        for (int t = WIN - UW; t < WIN; ++t) {
+            const int r = s0 + UW + t - j;
+            const bool ok = (r >= 0) && (r < LB);
+            const int rr = ok ? r : 0;
+            wT[t] = ok ? sT[rr * LB + j] : 0.f;
+            wR[t] = ok ? sR[rr * LB + j] : 0.f;
         }
     }
     if (bad) set_status(status, BAKRON_ERR_NONFINITE);
@@ -144,7 +181,9 @@ __device__ __forceinline__ void solve_leaf(int lane, int rows, int cols, float q
 __global__ void __launch_bounds__(NTH) phase_leaves_kernel(PhaseArgs a) {
     __shared__ float sA[LB][LB + 1];
     __shared__ float sB[LB][LB + 1];
-    __shared__ float sT[LB * LB], sR[LB * LB], sW[LB * LB], sLO[LB * LB], sLI[LB * LB];
+    __shared__ float sT[LB * LB], sR[LB * LB], sW[LB * LB];
+    __shared__ __align__(16) float sLO[LB * LS];
+    __shared__ __align__(16) float sLI[LB * LS];
     __shared__ float oW[LB * LB], oE[LB * LB], oU[LB * LB];
     __shared__ int8_t oC[LB * LB];
     __shared__ float sS[LB];
@@ -238,18 +277,22 @@ __global__ void __launch_bounds__(NTH) phase_leaves_kernel(PhaseArgs a) {
             sT[(warp * 8 + t) * LB + lane] = accT[t];
             sR[(warp * 8 + t) * LB + lane] = accR[t];
         }
+        // diagonal blocks of L_O and L_I: coalesced row loads into sA / sB first
 #pragma unroll
         for (int q = 0; q < (LB * LB) / NTH; ++q) {
             const int e = tid + q * NTH, r = e >> 5, c = e & 31;
             sW[e] = (r < rows && c < cols) ? __ldg(&a.Ws[(size_t)(i0 + r) * n + j0 + c]) : 0.f;
-            // skewed diagonal blocks: sLO[dd][x] = L_O[i0+x][i0+x+dd], sLI[dd][x] likewise
-            const int dd = r, x = c;
-            sLO[e] = (dd >= 1 && x + dd < rows)
-                         ? __ldg(&a.LO[(size_t)(i0 + x) * m + i0 + x + dd]) : 0.f;
-            sLI[e] = (dd >= 1 && x + dd < cols)
-                         ? __ldg(&a.LI[(size_t)(j0 + x) * n + j0 + x + dd]) : 0.f;
+            sA[r][c] = (r < rows && c < rows) ? __ldg(&a.LO[(size_t)(i0 + r) * m + i0 + c]) : 0.f;
+            sB[r][c] = (r < cols && c < cols) ? __ldg(&a.LI[(size_t)(j0 + r) * n + j0 + c]) : 0.f;
         }
         if (tid < LB) sS[tid] = (tid < rows) ? __ldg(&a.sc[i0 + tid]) : 0.f;
+        __syncthreads();
+        // skewed copies: sLO[x*LS + d] = L_O[i0+x][i0+x+d], sLI[x*LS + d] = L_I[j0+x-d][j0+x]
+        for (int e = tid; e < LB * LS; e += NTH) {
+            const int x = e / LS, dd = e % LS;
+            sLO[e] = (dd >= 1 && dd < LB && x + dd < LB) ? sA[x][x + dd] : 0.f;
+            sLI[e] = (dd >= 1 && dd < LB && x - dd >= 0) ? sB[x - dd][x] : 0.f;
+        }
         __syncthreads();
 
         if (warp == 0)

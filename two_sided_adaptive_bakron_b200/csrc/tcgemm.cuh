@@ -215,18 +215,31 @@ gemm3x_kernel(const __grid_constant__ CUtensorMap a_hi, const __grid_constant__ 
         if (*(volatile int*)s_abort) have = false;
     }
     have = __all_sync(0xffffffffu, have);
+    const bool aborted = __any_sync(0xffffffffu, *(volatile int*)s_abort != 0);
     sm100::tc_fence_after();
-    const int row = m0 + warp * 32 + lane;
+    // Each warp moves its 32 x 32 accumulator chunks through a private, padded shared-memory
+    // tile (the operand ring is idle once the last MMA has completed) so that the epilogue
+    // sees one row per warp-wide step with lanes on consecutive columns: coalesced global
+    // accesses.
+    float* stage = reinterpret_cast<float*>(smem) + warp * (32 * 33);
+    if (!aborted) {
 #pragma unroll 1
-    for (int c0 = 0; c0 < BN; c0 += 32) {
-        float v[32];
-        if (have) {
-            sm100::tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0, v);
-        } else {
+        for (int c0 = 0; c0 < BN; c0 += 32) {
+            float v[32];
+            if (have) {
+                sm100::tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0, v);
+            } else {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = 0.f;
+                for (int i = 0; i < 32; ++i) v[i] = 0.f;
+            }
+#pragma unroll
+            for (int i = 0; i < 32; ++i) stage[lane * 33 + i] = v[i];
+            __syncwarp();
+#pragma unroll 4
+            for (int rr = 0; rr < 32; ++rr)
+                e(P, m0 + warp * 32 + rr, n0 + c0 + lane, m0, n0, stage[rr * 33 + lane]);
+            __syncwarp();
         }
-        if (!*(volatile int*)s_abort) e(P, row, n0 + c0, m0, n0, v);
     }
     e.finish(P, blockIdx.x);
     sm100::tc_fence_before();

@@ -25,24 +25,22 @@ void split_planes(const float* src, int rows, int cols, int ld_src, float* hi, f
                   int ld_dst, int transpose, cudaStream_t st);
 
 // ---------------------------------------------------------------------------- epilogues
+// An epilogue functor is called once per accumulator element, (row, col) relative to the
+// problem origin, warp-wide with one row per call and lanes on consecutive columns; m0, n0
+// give the tile origin. finish() runs once per CTA, by all threads.
+
 // out = weight * acc, written as hi/lo planes at (c_row0 + r, c_col0 + c).
 struct EpiStoreSplit {
     float* hi;
     float* lo;
     int ld;
-    __device__ void operator()(const Problem& P, int row, int col0, int, int,
-                               const float (&v)[32]) {
-        if (row >= P.M) return;
-        const size_t base = (size_t)(P.c_row0 + row) * ld + P.c_col0 + col0;
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            if (col0 + i < P.N) {
-                const float x = P.weight * v[i];
-                const float h = sm100::tf32_hi(x);
-                hi[base + i] = h;
-                lo[base + i] = x - h;
-            }
-        }
+    __device__ void operator()(const Problem& P, int row, int col, int, int, float v) {
+        if (row >= P.M || col >= P.N) return;
+        const size_t o = (size_t)(P.c_row0 + row) * ld + P.c_col0 + col;
+        const float x = P.weight * v;
+        const float h = sm100::tf32_hi(x);
+        hi[o] = h;
+        lo[o] = x - h;
     }
     __device__ void finish(const Problem&, int) {}
 };
@@ -54,19 +52,13 @@ struct EpiStore {
     int ldc;
     int accumulate;
     int upper;
-    __device__ void operator()(const Problem& P, int row, int col0, int, int,
-                               const float (&v)[32]) {
-        if (row >= P.M) return;
-        const int gr = P.c_row0 + row;
-        float* out = C + (size_t)gr * ldc + P.c_col0 + col0;
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            const int gc = P.c_col0 + col0 + i;
-            if (col0 + i < P.N && (!upper || gc >= gr)) {
-                const float x = P.weight * v[i];
-                out[i] = accumulate ? out[i] + x : x;
-            }
-        }
+    __device__ void operator()(const Problem& P, int row, int col, int, int, float v) {
+        if (row >= P.M || col >= P.N) return;
+        const int gr = P.c_row0 + row, gc = P.c_col0 + col;
+        if (upper && gc < gr) return;
+        float* out = C + (size_t)gr * ldc + gc;
+        const float x = P.weight * v;
+        *out = accumulate ? *out + x : x;
     }
     __device__ void finish(const Problem&, int) {}
 };
@@ -79,14 +71,9 @@ struct EpiDot {
     double* partial;
     float offdiag_weight;
     double acc;
-    __device__ void operator()(const Problem& P, int row, int col0, int m0, int n0,
-                               const float (&v)[32]) {
-        if (row >= P.M) return;
-        const float* g = G + (size_t)row * ldg + col0;
-        double s = 0.0;
-#pragma unroll
-        for (int i = 0; i < 32; ++i)
-            if (col0 + i < P.N) s += (double)v[i] * (double)g[i];
+    __device__ void operator()(const Problem& P, int row, int col, int m0, int n0, float v) {
+        if (row >= P.M || col >= P.N) return;
+        const double s = (double)v * (double)G[(size_t)row * ldg + col];
         acc += (m0 == n0) ? s : (double)offdiag_weight * s;
     }
     __device__ void finish(const Problem&, int tile) {
