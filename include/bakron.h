@@ -65,6 +65,25 @@ int bakron_ldl(const float* H, int n, float* L, float* D,
                void* ws, size_t ws_bytes, int* dev_status, void* stream);
 
 /* ------------------------------------------------------------------------------------------
+ * bakron_ldl_noalloc -- bakron_ldl without a caller workspace. (The pages have no counterpart:
+ * this serves callers that cannot allocate device memory, e.g. a process whose framework
+ * allocator already holds the device's memory, or a latency-critical loop that must not call
+ * cudaMalloc / cudaFree, which can synchronise the device.)
+ *
+ * Same contract and results as bakron_ldl, with the scratch in a fixed array that is part of
+ * the library (20 MiB, held on every GPU that loads the library until the process exits).
+ *   n        [in]  1 <= n <= bakron_ldl_noalloc_max_n() (2048); larger n returns
+ *                  BAKRON_ERR_INVALID_ARG without touching the device.
+ * The first call on a device looks up the array's device address (cudaGetSymbolAddress) with
+ * that device current; make that first call before any stream capture. Calls share the
+ * array: two calls that overlap on the GPU (different streams or host threads) race. Nothing
+ * in the array needs to start at zero. Allocates nothing.
+ * ---------------------------------------------------------------------------------------- */
+int bakron_ldl_noalloc(const float* H, int n, float* L, float* D, int* dev_status,
+                       void* stream);
+int bakron_ldl_noalloc_max_n(void);
+
+/* ------------------------------------------------------------------------------------------
  * bakron_round -- the BaKron solve of the two-sided adaptive rounding rule.
  *
  * For every entry, in any order compatible with "(k,l) before (i,j) when k <= i and l <= j"

@@ -43,6 +43,8 @@ _SIGNATURES = {
     "bakron_status_string": (ctypes.c_char_p, [_c_int]),
     "bakron_version": (_c_int, []),
     "bakron_kernel_launches": (ctypes.c_ulonglong, []),
+    "bakron_ldl_noalloc": (_c_int, [_vp, _c_int, _vp, _vp, _vp, _vp]),
+    "bakron_ldl_noalloc_max_n": (_c_int, []),
     # test hooks (include/bakron_internal.h)
     "bakron_internal_gemm3x_workspace_bytes": (_c_size_t, [_c_int, _c_int, _c_int]),
     "bakron_internal_gemm3x": (_c_int, [_vp, _c_int, _c_int, _c_int, _vp, _c_int, _c_int, _vp,
@@ -152,6 +154,20 @@ def bakron_proxy_loss(dW, H_O, H_I, loss, ws, stream=None) -> int:
     _check_cuda(loss, torch.float64, (1,), "loss")
     return lib().bakron_proxy_loss(_ptr(dW), m, n, _ptr(H_O), _ptr(H_I), _ptr(loss), _ptr(ws),
                                    ws.numel() * ws.element_size(), _stream(stream))
+
+
+def bakron_ldl_noalloc(H, L, D, dev_status, stream=None) -> int:
+    """bakron_ldl with the library's own fixed scratch (no workspace argument)."""
+    n = H.shape[0]
+    _check_cuda(H, torch.float32, (n, n), "H")
+    _check_cuda(L, torch.float32, (n, n), "L")
+    _check_cuda(D, torch.float32, (n,), "D")
+    return lib().bakron_ldl_noalloc(_ptr(H), n, _ptr(L), _ptr(D), _ptr(dev_status),
+                                    _stream(stream))
+
+
+def bakron_ldl_noalloc_max_n() -> int:
+    return int(lib().bakron_ldl_noalloc_max_n())
 
 
 def bakron_read_status(dev_status, stream=None) -> int:
