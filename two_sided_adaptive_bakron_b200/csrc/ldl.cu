@@ -94,6 +94,9 @@ __global__ void __launch_bounds__(DIAG_THREADS) diag_block_kernel(float* __restr
         const int j0 = J * SUB;
         // (1) the diagonal sub-block, one warp
         if (warp == 0) {
+            // lane = row r of the sub-block; the pivot column and the W row are read into
+            // registers first (broadcast loads), then every update has a static offset
+            double* Srow = &S[j0 + lane][j0];          // S[r][j0 + l]
             for (int jj = SUB - 1; jj >= 0; --jj) {
                 const int j = j0 + jj;
                 double d = S[j][j];
@@ -106,18 +109,28 @@ __global__ void __launch_bounds__(DIAG_THREADS) diag_block_kernel(float* __restr
                         D[k0 + j] = (float)d;
                     }
                 }
-                double u = 0.0;
-                if (lane < jj) {
-                    u = S[j0 + lane][j] / d;
-                    S[j0 + lane][j] = u;
-                }
+                const double u = (lane < jj) ? S[j0 + lane][j] / d : 0.0;
                 __syncwarp();
-                if (lane < jj) {
-                    const int r = j0 + lane;
-                    const double ud = u * d;
-                    for (int l = r; l < j; ++l) S[r][l] -= ud * S[l][j];
-                    S[j][r] = -u;
-                    for (int c = j + 1; c < j0 + SUB; ++c) S[c][r] -= u * S[c][j];
+                if (lane < jj) S[j0 + lane][j] = u;
+                const double ud = u * d;
+                const bool act = lane < jj;
+                // S[r][l] -= u_r d u_l for r <= l < j (u_l by shuffle: no shared-memory alias)
+#pragma unroll
+                for (int l = 0; l < SUB; ++l) {
+                    const double ul = __shfl_sync(0xffffffffu, u, l);
+                    if (act && l >= lane && l < jj) Srow[l] -= ud * ul;
+                }
+                // W[r][c] -= u_r W[j][c] for c > j, stored at S[j0+c][j0+r]; W[r][j] = -u_r.
+                // W[j][c] = S[j0+c][j] is read 8 columns at a time before the 8 updates.
+                if (act) S[j][j0 + lane] = -u;
+#pragma unroll
+                for (int c0 = 0; c0 < SUB; c0 += 8) {
+                    double wrow[8];
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) wrow[q] = (c0 + q > jj) ? S[j0 + c0 + q][j] : 0.0;
+#pragma unroll
+                    for (int q = 0; q < 8; ++q)
+                        if (act && c0 + q > jj) S[j0 + c0 + q][j0 + lane] -= u * wrow[q];
                 }
                 __syncwarp();
             }
@@ -202,16 +215,23 @@ struct EpiPanel {
     float* ul;
     int ldx;
     int c_off;
-    __device__ void operator()(const tc::Problem& P, int row, int c, int, int, float x) {
-        if (row >= P.M || c >= P.N) return;
-        const float u = __fdiv_rn(x, D[kb0 + c]);
-        L[(size_t)row * n + kb0 + c] = u;
-        const size_t o = (size_t)row * ldx + c_off + c;
-        const float xh_ = sm100::tf32_hi(x), uh_ = sm100::tf32_hi(u);
-        xh[o] = xh_;
-        xl[o] = x - xh_;
-        uh[o] = uh_;
-        ul[o] = u - uh_;
+    __device__ void chunk(const tc::Problem& P, int row0, int c, int, int, const float* v) {
+        if (c >= P.N) return;
+        const float dc = D[kb0 + c];
+#pragma unroll 8
+        for (int rr = 0; rr < 32; ++rr) {
+            const int row = row0 + rr;
+            if (row >= P.M) break;
+            const float x = v[rr * 33];
+            const float u = __fdiv_rn(x, dc);
+            L[(size_t)row * n + kb0 + c] = u;
+            const size_t o = (size_t)row * ldx + c_off + c;
+            const float xh_ = sm100::tf32_hi(x), uh_ = sm100::tf32_hi(u);
+            xh[o] = xh_;
+            xl[o] = x - xh_;
+            uh[o] = uh_;
+            ul[o] = u - uh_;
+        }
     }
     __device__ void finish(const tc::Problem&, int) {}
 };

@@ -235,9 +235,8 @@ gemm3x_kernel(const __grid_constant__ CUtensorMap a_hi, const __grid_constant__ 
 #pragma unroll
             for (int i = 0; i < 32; ++i) stage[lane * 33 + i] = v[i];
             __syncwarp();
-#pragma unroll 4
-            for (int rr = 0; rr < 32; ++rr)
-                e(P, m0 + warp * 32 + rr, n0 + c0 + lane, m0, n0, stage[rr * 33 + lane]);
+            // lane = column n0 + c0 + lane, element rr of the chunk at stage[rr * 33 + lane]
+            e.chunk(P, m0 + warp * 32, n0 + c0 + lane, m0, n0, stage + lane);
             __syncwarp();
         }
     }

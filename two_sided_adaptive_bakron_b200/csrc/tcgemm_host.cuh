@@ -25,22 +25,29 @@ void split_planes(const float* src, int rows, int cols, int ld_src, float* hi, f
                   int ld_dst, int transpose, cudaStream_t st);
 
 // ---------------------------------------------------------------------------- epilogues
-// An epilogue functor is called once per accumulator element, (row, col) relative to the
-// problem origin, warp-wide with one row per call and lanes on consecutive columns; m0, n0
-// give the tile origin. finish() runs once per CTA, by all threads.
+// An epilogue functor's chunk() is called once per 32 x 32 accumulator chunk of a warp:
+// row0 is the chunk's first row, col = this lane's column (both relative to the problem
+// origin), element rr of the lane's column is v[rr * 33]; m0, n0 give the tile origin.
+// Global loads of a chunk are all issued before its stores (32 in flight per thread).
+// finish() runs once per CTA, by all threads.
 
 // out = weight * acc, written as hi/lo planes at (c_row0 + r, c_col0 + c).
 struct EpiStoreSplit {
     float* hi;
     float* lo;
     int ld;
-    __device__ void operator()(const Problem& P, int row, int col, int, int, float v) {
-        if (row >= P.M || col >= P.N) return;
-        const size_t o = (size_t)(P.c_row0 + row) * ld + P.c_col0 + col;
-        const float x = P.weight * v;
-        const float h = sm100::tf32_hi(x);
-        hi[o] = h;
-        lo[o] = x - h;
+    __device__ void chunk(const Problem& P, int row0, int col, int, int, const float* v) {
+        if (col >= P.N) return;
+#pragma unroll
+        for (int rr = 0; rr < 32; ++rr) {
+            if (row0 + rr < P.M) {
+                const size_t o = (size_t)(P.c_row0 + row0 + rr) * ld + P.c_col0 + col;
+                const float x = P.weight * v[rr * 33];
+                const float h = sm100::tf32_hi(x);
+                hi[o] = h;
+                lo[o] = x - h;
+            }
+        }
     }
     __device__ void finish(const Problem&, int) {}
 };
@@ -52,13 +59,22 @@ struct EpiStore {
     int ldc;
     int accumulate;
     int upper;
-    __device__ void operator()(const Problem& P, int row, int col, int, int, float v) {
-        if (row >= P.M || col >= P.N) return;
-        const int gr = P.c_row0 + row, gc = P.c_col0 + col;
-        if (upper && gc < gr) return;
-        float* out = C + (size_t)gr * ldc + gc;
-        const float x = P.weight * v;
-        *out = accumulate ? *out + x : x;
+    __device__ void chunk(const Problem& P, int row0, int col, int, int, const float* v) {
+        if (col >= P.N) return;
+        const int gc = P.c_col0 + col;
+        float old[32];
+#pragma unroll
+        for (int rr = 0; rr < 32; ++rr) {
+            const int gr = P.c_row0 + row0 + rr;
+            const bool ok = (row0 + rr < P.M) && (!upper || gc >= gr);
+            old[rr] = (ok && accumulate) ? C[(size_t)gr * ldc + gc] : 0.f;
+        }
+#pragma unroll
+        for (int rr = 0; rr < 32; ++rr) {
+            const int gr = P.c_row0 + row0 + rr;
+            const bool ok = (row0 + rr < P.M) && (!upper || gc >= gr);
+            if (ok) C[(size_t)gr * ldc + gc] = old[rr] + P.weight * v[rr * 33];
+        }
     }
     __device__ void finish(const Problem&, int) {}
 };
@@ -71,9 +87,15 @@ struct EpiDot {
     double* partial;
     float offdiag_weight;
     double acc;
-    __device__ void operator()(const Problem& P, int row, int col, int m0, int n0, float v) {
-        if (row >= P.M || col >= P.N) return;
-        const double s = (double)v * (double)G[(size_t)row * ldg + col];
+    __device__ void chunk(const Problem& P, int row0, int col, int m0, int n0, const float* v) {
+        if (col >= P.N) return;
+        float g[32];
+#pragma unroll
+        for (int rr = 0; rr < 32; ++rr)
+            g[rr] = (row0 + rr < P.M) ? G[(size_t)(row0 + rr) * ldg + col] : 0.f;
+        double s = 0.0;
+#pragma unroll
+        for (int rr = 0; rr < 32; ++rr) s += (double)v[rr * 33] * (double)g[rr];
         acc += (m0 == n0) ? s : (double)offdiag_weight * s;
     }
     __device__ void finish(const Problem&, int tile) {
