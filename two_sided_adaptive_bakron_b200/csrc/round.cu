@@ -15,15 +15,14 @@
 //
 // Structure. The matrix is cut into 256 x 256 super-blocks, processed one super-block
 // anti-diagonal ("phase") at a time; the blocks of a phase are independent of each other.
-//  * Leaf launch (persistent, cooperative): every block of the phase is cut into 32 x 32
-//    leaves, taken in anti-diagonal order across all blocks of the phase. A leaf starts from
-//    the far sums T_far, R_far (everything outside its block, already accumulated), adds the
-//    contributions of the leaves above / to the left inside its block (CUDA-core dot products,
-//    after a bounded wait on each source leaf's ready flag), then one warp runs the in-leaf
-//    wavefront (63 steps; lane j owns column j, values indexed by step so that every register
-//    index is a compile-time constant; vertical updates stay in the lane, horizontal ones move
-//    by warp shuffles). The leaf publishes codes, W, E (row-major), E^T and U as hi/lo planes
-//    and raises its flag (release / acquire).
+//  * Leaf launch (persistent, cooperative, one CTA per SM): every block of the phase is cut
+//    into 32 x 32 leaves, taken in anti-diagonal order across all blocks of the phase, round
+//    robin over the CTAs. In each CTA four loader warps stage a leaf: the far sums T_far,
+//    R_far (everything outside its block, already accumulated) plus the contributions of the
+//    leaves above / to the left inside its block (CUDA-core dot products, after a bounded wait
+//    on each source leaf's ready flag). A fifth, solver warp runs the in-leaf wavefront of the
+//    previous leaf meanwhile (two staging buffers, mbarrier handoff) and publishes it: codes,
+//    W, E (row-major), E^T and U as hi/lo planes, then the leaf's release flag.
 //  * Push launches (3xTF32 tcgen05 GEMMs, one grouped launch per direction): every block of
 //    the phase pushes its E into T_far of all rows below it and its U into R_far of all
 //    columns to its right (K = 256), i.e. the divide-and-conquer off-diagonal updates as dense
@@ -37,7 +36,6 @@ namespace {
 
 constexpr int LB = 32;          // leaf edge
 constexpr int NSLOT = 2 * LB - 1;
-constexpr int NTH = 128;        // threads per leaf block
 constexpr int SB = 256;         // super-block edge
 constexpr int LPB = SB / LB;    // leaves per super-block edge
 constexpr int BN = 128;
@@ -83,28 +81,51 @@ __device__ __forceinline__ int diag_len(int d, int lm, int ln) {
 constexpr int UW = 4;            // wavefront steps per unrolled group
 constexpr int WIN = LB + UW;     // register window of slots
 constexpr int LS = LB + 4;       // row stride of the skewed diagonal blocks (16-byte rows)
+constexpr int NLOAD = 128;       // loader threads (warps 0-3)
+constexpr int NTHW = NLOAD + 32; // + the solver warp (warp 4)
 
-// The in-leaf wavefront, run by one warp; lane j owns column j and the element of row r is
-// handled at step s = r + j. Leaf arrays live in shared memory with row stride LB, element
-// (r, c) at r*LB + c, so an anti-diagonal and a row both touch 32 distinct banks.
-// Per lane, slot s of wT / wR holds the vertical / horizontal sum of its element of step s.
-// A step reads slot s, then pushes E down its column into slots s+1..s+31 (in-lane) and U
-// along its row into slot s+d of lane j+d (warp shuffles). The step loop stays rolled
-// (4 steps per iteration) over a sliding window of 36 slot registers, which keeps every
-// register index static while the code stays small enough for the instruction cache.
-//   sLOr[r*LS + d] = L_O[i0+r][i0+r+d]    (row r of the diagonal block, shifted)
-//   sLIc[c*LS + d] = L_I[j0+c-d][j0+c]    (column c of the diagonal block, shifted)
+// One staging buffer: a leaf's inputs and outputs (shared memory, floats).
+struct LeafBuf {
+    float W[LB * LB];            // W* of the leaf, row stride LB
+    float T[LB * LB];            // vertical sums (everything above the leaf)
+    float R[LB * LB];            // horizontal sums (everything left of the leaf)
+    float LOr[LB * LS];          // LOr[r*LS + d] = L_O[i0+r][i0+r+d]
+    float LIc[LB * LS];          // LIc[c*LS + d] = L_I[j0+c-d][j0+c]
+    float S[2 * LB];             // s_r and its reciprocal
+    float oW[LB * LB], oE[LB * LB], oU[LB * LB];
+    float oEt[LB * LB];          // E transposed (for the transposed planes)
+    int8_t oC[LB * LB];
+    int meta[4];                 // I, J, rows, cols
+};
+
+struct LeafSmem {
+    LeafBuf buf[2];
+    float sA[LB][LB + 1];        // pull staging
+    float sB[LB][LB + 1];
+    uint64_t full[2], empty[2];
+    int stop;
+};
+
+// The in-leaf wavefront, run by the solver warp; lane j owns column j and the element of row
+// r is handled at step s = r + j. Leaf arrays use row stride LB, element (r, c) at r*LB + c,
+// so an anti-diagonal and a row both touch 32 distinct banks. Per lane, slot s of wT / wR
+// holds the vertical / horizontal sum of its element of step s. A step reads slot s, then
+// pushes E down its column into slots s+1..s+31 (in-lane) and U along its row into slot s+d
+// of lane j+d (warp shuffles); the d = 1 pushes, the only ones the next step needs, go
+// first. The step loop stays rolled (4 steps per iteration) over a sliding window of 36
+// slot registers: every register index is static and the code stays small.
+// Q divides by s_r as one correctly rounded fp32 division; the quotient is formed as
+// pre * (1/s_r), whose distance to the division's result is below 2e-7 |x|, and the exact
+// division is taken instead whenever that quotient lies within 1e-6 max(1,|x|) of a rounding
+// boundary, so the decision always equals the division's.
 __device__ __forceinline__ void solve_leaf(int lane, int rows, int cols, float qlo, float qhi,
-                                           const float* sW, const float* sT, const float* sR,
-                                           const float* sLOr, const float* sLIc,
-                                           const float* sS, int8_t* oC, float* oW, float* oE,
-                                           float* oU, int* status) {
+                                           LeafBuf& B, int* status) {
     const int j = lane;
     const bool colok = j < cols;
     float li[LB];
 #pragma unroll
     for (int q = 0; q < LB / 4; ++q) {
-        const float4 v = *reinterpret_cast<const float4*>(&sLIc[j * LS + 4 * q]);
+        const float4 v = *reinterpret_cast<const float4*>(&B.LIc[j * LS + 4 * q]);
         li[4 * q] = v.x; li[4 * q + 1] = v.y; li[4 * q + 2] = v.z; li[4 * q + 3] = v.w;
     }
     float wT[WIN], wR[WIN];
@@ -113,8 +134,8 @@ __device__ __forceinline__ void solve_leaf(int lane, int rows, int cols, float q
         const int r = t - j;
         const bool ok = (r >= 0) && (r < LB);
         const int rr = ok ? r : 0;
-        wT[t] = ok ? sT[rr * LB + j] : 0.f;
-        wR[t] = ok ? sR[rr * LB + j] : 0.f;
+        wT[t] = ok ? B.T[rr * LB + j] : 0.f;
+        wR[t] = ok ? B.R[rr * LB + j] : 0.f;
     }
     bool bad = false;
 #pragma unroll 1
@@ -125,37 +146,43 @@ __device__ __forceinline__ void solve_leaf(int lane, int rows, int cols, float q
             const bool inleaf = (r >= 0) && (r < LB);
             const int rr = inleaf ? r : 0;
             const bool act = inleaf && (r < rows) && colok;
+            float lo[LB];
+#pragma unroll
+            for (int q = 0; q < LB / 4; ++q) {
+                const float4 v = *reinterpret_cast<const float4*>(&B.LOr[rr * LS + 4 * q]);
+                lo[4 * q] = v.x; lo[4 * q + 1] = v.y; lo[4 * q + 2] = v.z; lo[4 * q + 3] = v.w;
+            }
+            const float w_star = B.W[rr * LB + j];
+            const float sr = B.S[rr], inv = B.S[LB + rr];
             float e = 0.f, u = 0.f;
             if (act) {
-                const float w_star = sW[rr * LB + j];
                 const float pre = w_star + wT[k] + wR[k];
-                const float sr = sS[rr];
                 float q = 0.f;
                 if (sr > 0.f) {
-                    q = rintf(__fdiv_rn(pre, sr));
-                    q = fminf(fmaxf(q, qlo), qhi);
+                    float x = pre * inv;
+                    const float t = fabsf(x - rintf(x));
+                    if (0.5f - t < 1e-6f * fmaxf(1.f, fabsf(x))) x = __fdiv_rn(pre, sr);
+                    q = fminf(fmaxf(rintf(x), qlo), qhi);
                 }
                 bad |= !isfinite(pre);
                 const float w = sr * q;
                 e = w_star - w;
                 u = wT[k] + e;
-                oC[rr * LB + j] = (int8_t)q;
-                oW[rr * LB + j] = w;
-                oE[rr * LB + j] = e;
-                oU[rr * LB + j] = u;
+                B.oC[rr * LB + j] = (int8_t)q;
+                B.oW[rr * LB + j] = w;
+                B.oE[rr * LB + j] = e;
+                B.oEt[j * LB + rr] = e;
+                B.oU[rr * LB + j] = u;
             }
-            // vertical: E_rj feeds rows r+d of the same column
-            float lo[LB];
-#pragma unroll
-            for (int q = 0; q < LB / 4; ++q) {
-                const float4 v = *reinterpret_cast<const float4*>(&sLOr[rr * LS + 4 * q]);
-                lo[4 * q] = v.x; lo[4 * q + 1] = v.y; lo[4 * q + 2] = v.z; lo[4 * q + 3] = v.w;
+            wT[k + 1] = fmaf(lo[1], e, wT[k + 1]);
+            {
+                const float v = __shfl_up_sync(0xffffffffu, u, 1);
+                if (j >= 1) wR[k + 1] = fmaf(v, li[1], wR[k + 1]);
             }
 #pragma unroll
-            for (int d = 1; d < LB; ++d) wT[k + d] = fmaf(lo[d], e, wT[k + d]);
-            // horizontal: U_rj feeds columns j+d of the same row (lane j+d)
+            for (int d = 2; d < LB; ++d) wT[k + d] = fmaf(lo[d], e, wT[k + d]);
 #pragma unroll
-            for (int d = 1; d < LB; ++d) {
+            for (int d = 2; d < LB; ++d) {
                 const float v = __shfl_up_sync(0xffffffffu, u, d);
                 if (j >= d) wR[k + d] = fmaf(v, li[d], wR[k + d]);
             }
@@ -171,160 +198,220 @@ __device__ __forceinline__ void solve_leaf(int lane, int rows, int cols, float q
             const int r = s0 + UW + t - j;
             const bool ok = (r >= 0) && (r < LB);
             const int rr = ok ? r : 0;
-            wT[t] = ok ? sT[rr * LB + j] : 0.f;
-            wR[t] = ok ? sR[rr * LB + j] : 0.f;
+            wT[t] = ok ? B.T[rr * LB + j] : 0.f;
+            wR[t] = ok ? B.R[rr * LB + j] : 0.f;
         }
     }
     if (bad) set_status(status, BAKRON_ERR_NONFINITE);
 }
 
-__global__ void __launch_bounds__(NTH) phase_leaves_kernel(PhaseArgs a) {
-    __shared__ float sA[LB][LB + 1];
-    __shared__ float sB[LB][LB + 1];
-    __shared__ float sT[LB * LB], sR[LB * LB], sW[LB * LB];
-    __shared__ __align__(16) float sLO[LB * LS];
-    __shared__ __align__(16) float sLI[LB * LS];
-    __shared__ float oW[LB * LB], oE[LB * LB], oU[LB * LB];
-    __shared__ int8_t oC[LB * LB];
-    __shared__ float sS[LB];
-    __shared__ int s_stop;
+__device__ __forceinline__ void loader_sync() {
+    asm volatile("bar.sync 1, %0;" ::"n"(NLOAD) : "memory");
+}
 
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int m = a.m, n = a.n;
-    // walker over (local diagonal d, block row P), counting tasks
-    int d = 0, P = a.p_lo;
-    long long base = 0;
-
-    for (int g = blockIdx.x; g < a.total; g += gridDim.x) {
-        int lm, ln, cnt;
+// Walks the phase's tasks: (local anti-diagonal d, block row P) in order, counting leaves.
+struct TaskWalker {
+    int d, P;
+    long long base;
+    __device__ void init(int p_lo) { d = 0; P = p_lo; base = 0; }
+    __device__ void find(const PhaseArgs& a, int g, int& I, int& J) {
+        int ln;
         while (true) {
             const int Q = a.delta - P;
-            lm = leaves_of(m, P);
-            ln = leaves_of(n, Q);
-            cnt = diag_len(d, lm, ln);
+            const int lm = leaves_of(a.m, P);
+            ln = leaves_of(a.n, Q);
+            const int cnt = diag_len(d, lm, ln);
             if (g < base + cnt) break;
             base += cnt;
             if (++P > a.p_hi) { P = a.p_lo; ++d; }
         }
-        const int Q = a.delta - P;
-        const int la = max(0, d - ln + 1) + (int)(g - base);   // leaf row inside the block
-        const int lc = d - la;                                 // leaf column inside the block
-        const int I = P * LPB + la, J = Q * LPB + lc;
-        const int i0 = I * LB, j0 = J * LB;
-        const int rows = min(LB, m - i0), cols = min(LB, n - j0);
+        const int la = max(0, d - ln + 1) + (int)(g - base);
+        I = P * LPB + la;
+        J = (a.delta - P) * LPB + (d - la);
+    }
+};
 
-        // ---- far sums (everything outside the block), then the leaves above / left inside it
-        float accT[8], accR[8];
-#pragma unroll
-        for (int t = 0; t < 8; ++t) {
-            const int r = warp * 8 + t;
-            const bool ok = r < rows && lane < cols;
-            const size_t o = (size_t)(i0 + r) * n + j0 + lane;
-            accT[t] = ok ? __ldcg(&a.Tf[o]) : 0.f;
-            accR[t] = ok ? __ldcg(&a.Rf[o]) : 0.f;
+// Warps 0-3 stage leaf k into buffer k&1 (far sums, the in-block contributions of the leaves
+// above / left after a bounded wait on each one's ready flag, the diagonal blocks of L_O and
+// L_I) while warp 4 solves leaf k-1 from the other buffer and publishes it (outputs, planes,
+// release flag). The solver warp never runs the staging code and the loaders never run the
+// solver, so each keeps its own instruction stream.
+__global__ void __launch_bounds__(NTHW, 1) phase_leaves_kernel(PhaseArgs a) {
+    extern __shared__ __align__(16) uint8_t leaf_smem_raw[];
+    LeafSmem& sm = *reinterpret_cast<LeafSmem*>(leaf_smem_raw);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int m = a.m, n = a.n;
+    if (tid == 0) {
+        for (int b = 0; b < 2; ++b) {
+            sm100::mbar_init(&sm.full[b], 1);
+            sm100::mbar_init(&sm.empty[b], 1);
         }
-        for (int ka = 0; ka < la; ++ka) {
-            const int Ip = P * LPB + ka;
-            if (tid == 0)
-                s_stop = wait_flag(&a.flags[(size_t)Ip * a.Nt + J], a.abort_word, a.status,
-                                   a.limit_ns) ? 0 : 1;
-            __syncthreads();
-            if (s_stop) return;
-#pragma unroll
-            for (int q = 0; q < (LB * LB) / NTH; ++q) {
-                const int e = tid + q * NTH, kk = e >> 5, c = e & 31;
-                const size_t k = (size_t)Ip * LB + kk;
-                sA[kk][c] = (c < rows) ? __ldg(&a.LO[k * m + i0 + c]) : 0.f;
-                sB[kk][c] = (c < cols) ? __ldcg(&a.E[k * n + j0 + c]) : 0.f;
+        sm.stop = 0;
+        sm100::fence_mbar_init();
+    }
+    __syncthreads();
+    TaskWalker wk;
+    wk.init(a.p_lo);
+
+    if (warp < 4) {
+        // ------------------------------------------------------------ loaders
+        int k = 0;
+        for (int g = blockIdx.x; g < a.total; g += gridDim.x, ++k) {
+            const int b = k & 1;
+            LeafBuf& B = sm.buf[b];
+            if (k >= 2) {
+                if (tid == 0 && !sm100::mbar_wait(&sm.empty[b], ((k >> 1) - 1) & 1, a.status,
+                                                  a.limit_ns)) {
+                    atomicExch(a.abort_word, 1);
+                    sm.stop = 1;
+                }
+                loader_sync();
+                if (*(volatile int*)&sm.stop) break;
             }
-            __syncthreads();
+            int I, J;
+            wk.find(a, g, I, J);
+            const int P = wk.P, Q = a.delta - P;
+            const int la = I - P * LPB, lc = J - Q * LPB;
+            const int i0 = I * LB, j0 = J * LB;
+            const int rows = min(LB, m - i0), cols = min(LB, n - j0);
+            float accT[8], accR[8];
+#pragma unroll
+            for (int t = 0; t < 8; ++t) {
+                const int r = warp * 8 + t;
+                const bool ok = r < rows && lane < cols;
+                const size_t o = (size_t)(i0 + r) * n + j0 + lane;
+                accT[t] = ok ? __ldcg(&a.Tf[o]) : 0.f;
+                accR[t] = ok ? __ldcg(&a.Rf[o]) : 0.f;
+            }
+            bool stop = false;
+            for (int ka = 0; ka < la && !stop; ++ka) {
+                const int Ip = P * LPB + ka;
+                if (tid == 0)
+                    sm.stop = wait_flag(&a.flags[(size_t)Ip * a.Nt + J], a.abort_word, a.status,
+                                        a.limit_ns) ? 0 : 1;
+                loader_sync();
+                if (*(volatile int*)&sm.stop) { stop = true; break; }
+#pragma unroll
+                for (int q = 0; q < (LB * LB) / NLOAD; ++q) {
+                    const int e = tid + q * NLOAD, kk = e >> 5, c = e & 31;
+                    const size_t kr = (size_t)Ip * LB + kk;
+                    sm.sA[kk][c] = (c < rows) ? __ldg(&a.LO[kr * m + i0 + c]) : 0.f;
+                    sm.sB[kk][c] = (c < cols) ? __ldcg(&a.E[kr * n + j0 + c]) : 0.f;
+                }
+                loader_sync();
 #pragma unroll 8
-            for (int kk = 0; kk < LB; ++kk) {
-                const float b = sB[kk][lane];
+                for (int kk = 0; kk < LB; ++kk) {
+                    const float bv = sm.sB[kk][lane];
 #pragma unroll
-                for (int t = 0; t < 8; ++t) accT[t] = fmaf(sA[kk][warp * 8 + t], b, accT[t]);
+                    for (int t = 0; t < 8; ++t) accT[t] = fmaf(sm.sA[kk][warp * 8 + t], bv, accT[t]);
+                }
+                loader_sync();
             }
-            __syncthreads();
-        }
-        for (int kc = 0; kc < lc; ++kc) {
-            const int Jp = Q * LPB + kc;
-            if (tid == 0)
-                s_stop = wait_flag(&a.flags[(size_t)I * a.Nt + Jp], a.abort_word, a.status,
-                                   a.limit_ns) ? 0 : 1;
-            __syncthreads();
-            if (s_stop) return;
+            for (int kc = 0; kc < lc && !stop; ++kc) {
+                const int Jp = Q * LPB + kc;
+                if (tid == 0)
+                    sm.stop = wait_flag(&a.flags[(size_t)I * a.Nt + Jp], a.abort_word, a.status,
+                                        a.limit_ns) ? 0 : 1;
+                loader_sync();
+                if (*(volatile int*)&sm.stop) { stop = true; break; }
 #pragma unroll
-            for (int q = 0; q < (LB * LB) / NTH; ++q) {
-                const int e = tid + q * NTH, rr = e >> 5, c = e & 31;
-                const size_t l = (size_t)Jp * LB;
-                const size_t o = (size_t)(i0 + rr) * a.ldn + l + c;
-                sA[rr][c] = (rr < rows) ? (__ldcg(&a.u_hi[o]) + __ldcg(&a.u_lo[o])) : 0.f;
-                sB[rr][c] = (c < cols) ? __ldg(&a.LI[(l + rr) * n + j0 + c]) : 0.f;
-            }
-            __syncthreads();
+                for (int q = 0; q < (LB * LB) / NLOAD; ++q) {
+                    const int e = tid + q * NLOAD, rr = e >> 5, c = e & 31;
+                    const size_t l = (size_t)Jp * LB;
+                    const size_t o = (size_t)(i0 + rr) * a.ldn + l + c;
+                    sm.sA[rr][c] = (rr < rows) ? (__ldcg(&a.u_hi[o]) + __ldcg(&a.u_lo[o])) : 0.f;
+                    sm.sB[rr][c] = (c < cols) ? __ldg(&a.LI[(l + rr) * n + j0 + c]) : 0.f;
+                }
+                loader_sync();
 #pragma unroll 8
-            for (int ll = 0; ll < LB; ++ll) {
-                const float b = sB[ll][lane];
+                for (int ll = 0; ll < LB; ++ll) {
+                    const float bv = sm.sB[ll][lane];
 #pragma unroll
-                for (int t = 0; t < 8; ++t) accR[t] = fmaf(sA[warp * 8 + t][ll], b, accR[t]);
+                    for (int t = 0; t < 8; ++t) accR[t] = fmaf(sm.sA[warp * 8 + t][ll], bv, accR[t]);
+                }
+                loader_sync();
             }
-            __syncthreads();
-        }
-
-        // ---- stage the leaf
+            if (stop) break;
+            // stage the leaf into buffer b
 #pragma unroll
-        for (int t = 0; t < 8; ++t) {
-            sT[(warp * 8 + t) * LB + lane] = accT[t];
-            sR[(warp * 8 + t) * LB + lane] = accR[t];
-        }
-        // diagonal blocks of L_O and L_I: coalesced row loads into sA / sB first
-#pragma unroll
-        for (int q = 0; q < (LB * LB) / NTH; ++q) {
-            const int e = tid + q * NTH, r = e >> 5, c = e & 31;
-            sW[e] = (r < rows && c < cols) ? __ldg(&a.Ws[(size_t)(i0 + r) * n + j0 + c]) : 0.f;
-            sA[r][c] = (r < rows && c < rows) ? __ldg(&a.LO[(size_t)(i0 + r) * m + i0 + c]) : 0.f;
-            sB[r][c] = (r < cols && c < cols) ? __ldg(&a.LI[(size_t)(j0 + r) * n + j0 + c]) : 0.f;
-        }
-        if (tid < LB) sS[tid] = (tid < rows) ? __ldg(&a.sc[i0 + tid]) : 0.f;
-        __syncthreads();
-        // skewed copies: sLO[x*LS + d] = L_O[i0+x][i0+x+d], sLI[x*LS + d] = L_I[j0+x-d][j0+x]
-        for (int e = tid; e < LB * LS; e += NTH) {
-            const int x = e / LS, dd = e % LS;
-            sLO[e] = (dd >= 1 && dd < LB && x + dd < LB) ? sA[x][x + dd] : 0.f;
-            sLI[e] = (dd >= 1 && dd < LB && x - dd >= 0) ? sB[x - dd][x] : 0.f;
-        }
-        __syncthreads();
-
-        if (warp == 0)
-            solve_leaf(lane, rows, cols, a.qlo, a.qhi, sW, sT, sR, sLO, sLI, sS, oC, oW, oE, oU,
-                       a.status);
-        __syncthreads();
-
-        // ---- publish: row-major outputs and E, U planes; E^T planes transposed
-#pragma unroll
-        for (int q = 0; q < (LB * LB) / NTH; ++q) {
-            const int e = tid + q * NTH, r = e >> 5, c = e & 31;
-            if (r < rows && c < cols) {
-                const size_t o = (size_t)(i0 + r) * n + j0 + c;
-                a.codes[o] = oC[e];
-                a.Wq[o] = oW[e];
-                __stcg(&a.E[o], oE[e]);
-                const float u = oU[e], uh = sm100::tf32_hi(u);
-                const size_t ou = (size_t)(i0 + r) * a.ldn + j0 + c;
-                __stcg(&a.u_hi[ou], uh);
-                __stcg(&a.u_lo[ou], u - uh);
+            for (int t = 0; t < 8; ++t) {
+                B.T[(warp * 8 + t) * LB + lane] = accT[t];
+                B.R[(warp * 8 + t) * LB + lane] = accR[t];
             }
-            const int rt = e & 31, ct = e >> 5;   // transposed walk: consecutive rows
-            if (rt < rows && ct < cols) {
-                const float x = oE[rt * LB + ct], xh = sm100::tf32_hi(x);
-                const size_t ot = (size_t)(j0 + ct) * a.ldm + i0 + rt;
-                a.et_hi[ot] = xh;
-                a.et_lo[ot] = x - xh;
+#pragma unroll
+            for (int q = 0; q < (LB * LB) / NLOAD; ++q) {
+                const int e = tid + q * NLOAD, r = e >> 5, c = e & 31;
+                B.W[e] = (r < rows && c < cols) ? __ldg(&a.Ws[(size_t)(i0 + r) * n + j0 + c]) : 0.f;
+                sm.sA[r][c] = (r < rows && c < rows) ? __ldg(&a.LO[(size_t)(i0 + r) * m + i0 + c]) : 0.f;
+                sm.sB[r][c] = (r < cols && c < cols) ? __ldg(&a.LI[(size_t)(j0 + r) * n + j0 + c]) : 0.f;
+            }
+            if (tid < LB) {
+                const float sv = (tid < rows) ? __ldg(&a.sc[i0 + tid]) : 0.f;
+                B.S[tid] = sv;
+                B.S[LB + tid] = sv > 0.f ? __frcp_rn(sv) : 0.f;
+            }
+            if (tid == 0) { B.meta[0] = I; B.meta[1] = J; B.meta[2] = rows; B.meta[3] = cols; }
+            loader_sync();
+            for (int e = tid; e < LB * LS; e += NLOAD) {
+                const int x = e / LS, dd = e % LS;
+                B.LOr[e] = (dd >= 1 && dd < LB && x + dd < LB) ? sm.sA[x][x + dd] : 0.f;
+                B.LIc[e] = (dd >= 1 && dd < LB && x - dd >= 0) ? sm.sB[x - dd][x] : 0.f;
+            }
+            loader_sync();
+            if (tid == 0) {
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(sm100::smem_u32(&sm.full[b])) : "memory");
             }
         }
-        __threadfence();
-        __syncthreads();
-        if (tid == 0) st_release_gpu(&a.flags[(size_t)I * a.Nt + J], 1);
+        if (tid == 0) {
+            // loaders ended early: let the solver warp see it
+            if (*(volatile int*)&sm.stop) atomicExch(a.abort_word, 1);
+        }
+    } else {
+        // ------------------------------------------------------------ solver warp
+        int k = 0;
+        for (int g = blockIdx.x; g < a.total; g += gridDim.x, ++k) {
+            const int b = k & 1;
+            LeafBuf& B = sm.buf[b];
+            bool ok = true;
+            if (lane == 0) ok = sm100::mbar_wait(&sm.full[b], (k >> 1) & 1, a.status, a.limit_ns);
+            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+            if (!ok || ld_acquire_gpu(a.abort_word) != 0) {
+                if (lane == 0) atomicExch(a.abort_word, 1);
+                break;
+            }
+            const int I = B.meta[0], J = B.meta[1], rows = B.meta[2], cols = B.meta[3];
+            const int i0 = I * LB, j0 = J * LB;
+            solve_leaf(lane, rows, cols, a.qlo, a.qhi, B, a.status);
+            __syncwarp();
+            // publish: lane = column for row-major outputs, lane = row for the E^T planes
+            if (lane < cols) {
+                for (int r = 0; r < rows; ++r) {
+                    const size_t o = (size_t)(i0 + r) * n + j0 + lane;
+                    a.codes[o] = B.oC[r * LB + lane];
+                    a.Wq[o] = B.oW[r * LB + lane];
+                    __stcg(&a.E[o], B.oE[r * LB + lane]);
+                    const float u = B.oU[r * LB + lane], uh = sm100::tf32_hi(u);
+                    const size_t ou = (size_t)(i0 + r) * a.ldn + j0 + lane;
+                    __stcg(&a.u_hi[ou], uh);
+                    __stcg(&a.u_lo[ou], u - uh);
+                }
+            }
+            if (lane < rows) {
+                for (int c = 0; c < cols; ++c) {
+                    const float x = B.oEt[c * LB + lane], xh = sm100::tf32_hi(x);
+                    const size_t ot = (size_t)(j0 + c) * a.ldm + i0 + lane;
+                    a.et_hi[ot] = xh;
+                    a.et_lo[ot] = x - xh;
+                }
+            }
+            __threadfence();
+            __syncwarp();
+            if (lane == 0) {
+                st_release_gpu(&a.flags[(size_t)I * a.Nt + J], 1);
+                asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(sm100::smem_u32(&sm.empty[b])) : "memory");
+            }
+        }
     }
 }
 
@@ -364,8 +451,11 @@ int leaf_grid(int tasks) {
         if (cudaGetDevice(&dev) != cudaSuccess) return -1;
         if (cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
             return -1;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, phase_leaves_kernel, NTH, 0) !=
-            cudaSuccess)
+        if (cudaFuncSetAttribute(phase_leaves_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)sizeof(LeafSmem)) != cudaSuccess)
+            return -1;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, phase_leaves_kernel, NTHW,
+                                                          sizeof(LeafSmem)) != cudaSuccess)
             return -1;
         if (per_sm < 1) return -1;
         cached = per_sm * nsm;
@@ -452,7 +542,8 @@ extern "C" int bakron_round(const float* Wstar, int m, int n, const float* L_O, 
         void* params[] = {&a};
         count_launches(1);
         if ((e = cuda_err(cudaLaunchCooperativeKernel((const void*)phase_leaves_kernel,
-                                                      dim3(grid), dim3(NTH), params, 0, st))))
+                                                      dim3(grid), dim3(NTHW), params,
+                                                      sizeof(LeafSmem), st))))
             return e;
 
         // pushes of the phase's blocks: E down into T_far, U right into R_far
