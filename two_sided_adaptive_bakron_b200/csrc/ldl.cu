@@ -137,12 +137,28 @@ __global__ void __launch_bounds__(DIAG_THREADS) diag_block_kernel(float* __restr
         }
         __syncthreads();
         if (J == 0) break;
-        // (2) X[r][c] = sum_{t >= c} H'[r][j0+t] W_JJ[c][t], rows r < j0
-        for (int e = tid; e < j0 * SUB; e += DIAG_THREADS) {
-            const int r = e / SUB, c = e % SUB;
-            double acc = S[r][j0 + c];
-            for (int t = c + 1; t < SUB; ++t) acc += S[r][j0 + t] * S[j0 + t][j0 + c];
-            X[r][c] = acc;
+        // (2) X[r][c] = sum_{t >= c} H'[r][j0+t] W_JJ[c][t], rows r < j0 (4x4 register tiles)
+        for (int e = tid; e < (j0 / 4) * (SUB / 4); e += DIAG_THREADS) {
+            const int r0 = (e / (SUB / 4)) * 4, c0 = (e % (SUB / 4)) * 4;
+            double acc[4][4] = {};
+            for (int t = 0; t < SUB; ++t) {
+                double h[4], w[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) h[i] = S[r0 + i][j0 + t];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int c = c0 + q;
+                    w[q] = (t > c) ? S[j0 + t][j0 + c] : (t == c ? 1.0 : 0.0);
+                }
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) acc[i][q] += h[i] * w[q];
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int q = 0; q < 4; ++q) X[r0 + i][c0 + q] = acc[i][q];
         }
         __syncthreads();
         for (int e = tid; e < j0 * SUB; e += DIAG_THREADS) {
@@ -150,44 +166,92 @@ __global__ void __launch_bounds__(DIAG_THREADS) diag_block_kernel(float* __restr
             S[r][j0 + c] = X[r][c] / sD[j0 + c];
         }
         __syncthreads();
-        // (3) H'[r][l] -= sum_c X[r][c] U[l][c], r <= l < j0
-        for (int e = tid; e < j0 * j0; e += DIAG_THREADS) {
-            const int r = e / j0, l = e % j0;
-            if (l < r) continue;
-            double acc = 0.0;
-#pragma unroll 8
-            for (int c = 0; c < SUB; ++c) acc += X[r][c] * S[l][j0 + c];
-            S[r][l] -= acc;
+        // (3) H'[r][l] -= sum_c X[r][c] U[l][c], r <= l < j0, 4x4 tiles on the upper triangle
+        {
+            const int n4 = j0 / 4;
+            for (int e = tid; e < n4 * (n4 + 1) / 2; e += DIAG_THREADS) {
+                int R = 0, rem = e, rowlen = n4;
+                while (rem >= rowlen) { rem -= rowlen; ++R; --rowlen; }
+                const int Lt = R + rem, r0 = R * 4, l0 = Lt * 4;
+                double acc[4][4] = {};
+                for (int c = 0; c < SUB; ++c) {
+                    double x[4], u[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) x[i] = X[r0 + i][c];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) u[q] = S[l0 + q][j0 + c];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) acc[i][q] += x[i] * u[q];
+                }
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        if (l0 + q >= r0 + i) S[r0 + i][l0 + q] -= acc[i][q];
+            }
         }
         __syncthreads();
     }
-    // off-diagonal blocks of W = U^{-1}, by distance J - I = 1 .. NSUB-1
+    // off-diagonal blocks of W = U^{-1}, by distance J - I = 1 .. NSUB-1 (4x4 register tiles)
     for (int dist = 1; dist < NSUB; ++dist) {
         const int npairs = NSUB - dist;
-        // T_p = sum_{K=I+1..J} U_IK W_KJ, pair p = I
-        for (int e = tid; e < npairs * SUB * SUB; e += DIAG_THREADS) {
-            const int I = e / (SUB * SUB), t = (e / SUB) % SUB, c = e % SUB;
+        // T_I = sum_{K=I+1..J} U_IK W_KJ
+        for (int e = tid; e < npairs * (SUB / 4) * (SUB / 4); e += DIAG_THREADS) {
+            const int I = e / ((SUB / 4) * (SUB / 4));
+            const int t0 = ((e / (SUB / 4)) % (SUB / 4)) * 4, c0 = (e % (SUB / 4)) * 4;
             const int Jb = I + dist, i0 = I * SUB, jb0 = Jb * SUB;
-            double acc = 0.0;
+            double acc[4][4] = {};
             for (int K = I + 1; K <= Jb; ++K) {
                 const int kk0 = K * SUB;
-                for (int s = 0; s < SUB; ++s) {
-                    double w;   // W_KJ[s][c]
-                    if (K < Jb) w = S[jb0 + c][kk0 + s];
-                    else w = (c > s) ? S[jb0 + c][jb0 + s] : (c == s ? 1.0 : 0.0);
-                    acc += S[i0 + t][kk0 + s] * w;
+                for (int sx = 0; sx < SUB; ++sx) {
+                    double uu[4], w[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) uu[i] = S[i0 + t0 + i][kk0 + sx];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const int c = c0 + q;   // W_KJ[sx][c]
+                        w[q] = (K < Jb) ? S[jb0 + c][kk0 + sx]
+                                        : ((c > sx) ? S[jb0 + c][jb0 + sx] : (c == sx ? 1.0 : 0.0));
+                    }
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) acc[i][q] += uu[i] * w[q];
                 }
             }
-            T[I][t][c] = acc;
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int q = 0; q < 4; ++q) T[I][t0 + i][c0 + q] = acc[i][q];
         }
         __syncthreads();
-        // W_IJ[a][c] = -sum_t W_II[a][t] T[t][c], stored as S[J0+c][I0+a]
-        for (int e = tid; e < npairs * SUB * SUB; e += DIAG_THREADS) {
-            const int I = e / (SUB * SUB), a = (e / SUB) % SUB, c = e % SUB;
+        // W_IJ[a][c] = -sum_{t >= a} W_II[a][t] T[t][c], stored as S[J0+c][I0+a]
+        for (int e = tid; e < npairs * (SUB / 4) * (SUB / 4); e += DIAG_THREADS) {
+            const int I = e / ((SUB / 4) * (SUB / 4));
+            const int a0 = ((e / (SUB / 4)) % (SUB / 4)) * 4, c0 = (e % (SUB / 4)) * 4;
             const int Jb = I + dist, i0 = I * SUB, jb0 = Jb * SUB;
-            double acc = T[I][a][c];
-            for (int t = a + 1; t < SUB; ++t) acc += S[i0 + t][i0 + a] * T[I][t][c];
-            S[jb0 + c][i0 + a] = -acc;
+            double acc[4][4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int q = 0; q < 4; ++q) acc[i][q] = T[I][a0 + i][c0 + q];
+            for (int t = a0 + 1; t < SUB; ++t) {
+                double wi[4], tt[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) wi[i] = (t > a0 + i) ? S[i0 + t][i0 + a0 + i] : 0.0;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) tt[q] = T[I][t][c0 + q];
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) acc[i][q] += wi[i] * tt[q];
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int q = 0; q < 4; ++q) S[jb0 + c0 + q][i0 + a0 + i] = -acc[i][q];
         }
         __syncthreads();
     }

@@ -284,50 +284,57 @@ __global__ void __launch_bounds__(NTHW, 1) phase_leaves_kernel(PhaseArgs a) {
                 accR[t] = ok ? __ldcg(&a.Rf[o]) : 0.f;
             }
             bool stop = false;
-            for (int ka = 0; ka < la && !stop; ++ka) {
-                const int Ip = P * LPB + ka;
+            // In-block sources: the leaves above (vertical, via E) and to the left (horizontal,
+            // via U). The two most recent ones, (la-1, lc) and (la, lc-1), finish last, so every
+            // older source is pulled first and those two close the list.
+            const int nv = max(la - 1, 0), nh = max(lc - 1, 0);
+            const int nsrc = la + lc;
+            for (int idx = 0; idx < nsrc && !stop; ++idx) {
+                bool vert;
+                int src;
+                if (idx < nv) { vert = true; src = idx; }
+                else if (idx < nv + nh) { vert = false; src = idx - nv; }
+                else if (idx == nv + nh && la > 0) { vert = true; src = la - 1; }
+                else { vert = false; src = lc - 1; }
+                const int Is = vert ? P * LPB + src : I, Js = vert ? J : Q * LPB + src;
                 if (tid == 0)
-                    sm.stop = wait_flag(&a.flags[(size_t)Ip * a.Nt + J], a.abort_word, a.status,
+                    sm.stop = wait_flag(&a.flags[(size_t)Is * a.Nt + Js], a.abort_word, a.status,
                                         a.limit_ns) ? 0 : 1;
                 loader_sync();
                 if (*(volatile int*)&sm.stop) { stop = true; break; }
+                if (vert) {
 #pragma unroll
-                for (int q = 0; q < (LB * LB) / NLOAD; ++q) {
-                    const int e = tid + q * NLOAD, kk = e >> 5, c = e & 31;
-                    const size_t kr = (size_t)Ip * LB + kk;
-                    sm.sA[kk][c] = (c < rows) ? __ldg(&a.LO[kr * m + i0 + c]) : 0.f;
-                    sm.sB[kk][c] = (c < cols) ? __ldcg(&a.E[kr * n + j0 + c]) : 0.f;
-                }
-                loader_sync();
+                    for (int q = 0; q < (LB * LB) / NLOAD; ++q) {
+                        const int e = tid + q * NLOAD, kk = e >> 5, c = e & 31;
+                        const size_t kr = (size_t)Is * LB + kk;
+                        sm.sA[kk][c] = (c < rows) ? __ldg(&a.LO[kr * m + i0 + c]) : 0.f;
+                        sm.sB[kk][c] = (c < cols) ? __ldcg(&a.E[kr * n + j0 + c]) : 0.f;
+                    }
+                    loader_sync();
 #pragma unroll 8
-                for (int kk = 0; kk < LB; ++kk) {
-                    const float bv = sm.sB[kk][lane];
+                    for (int kk = 0; kk < LB; ++kk) {
+                        const float bv = sm.sB[kk][lane];
 #pragma unroll
-                    for (int t = 0; t < 8; ++t) accT[t] = fmaf(sm.sA[kk][warp * 8 + t], bv, accT[t]);
-                }
-                loader_sync();
-            }
-            for (int kc = 0; kc < lc && !stop; ++kc) {
-                const int Jp = Q * LPB + kc;
-                if (tid == 0)
-                    sm.stop = wait_flag(&a.flags[(size_t)I * a.Nt + Jp], a.abort_word, a.status,
-                                        a.limit_ns) ? 0 : 1;
-                loader_sync();
-                if (*(volatile int*)&sm.stop) { stop = true; break; }
+                        for (int t = 0; t < 8; ++t)
+                            accT[t] = fmaf(sm.sA[kk][warp * 8 + t], bv, accT[t]);
+                    }
+                } else {
 #pragma unroll
-                for (int q = 0; q < (LB * LB) / NLOAD; ++q) {
-                    const int e = tid + q * NLOAD, rr = e >> 5, c = e & 31;
-                    const size_t l = (size_t)Jp * LB;
-                    const size_t o = (size_t)(i0 + rr) * a.ldn + l + c;
-                    sm.sA[rr][c] = (rr < rows) ? (__ldcg(&a.u_hi[o]) + __ldcg(&a.u_lo[o])) : 0.f;
-                    sm.sB[rr][c] = (c < cols) ? __ldg(&a.LI[(l + rr) * n + j0 + c]) : 0.f;
-                }
-                loader_sync();
+                    for (int q = 0; q < (LB * LB) / NLOAD; ++q) {
+                        const int e = tid + q * NLOAD, rr = e >> 5, c = e & 31;
+                        const size_t l = (size_t)Js * LB;
+                        const size_t o = (size_t)(i0 + rr) * a.ldn + l + c;
+                        sm.sA[rr][c] = (rr < rows) ? (__ldcg(&a.u_hi[o]) + __ldcg(&a.u_lo[o])) : 0.f;
+                        sm.sB[rr][c] = (c < cols) ? __ldg(&a.LI[(l + rr) * n + j0 + c]) : 0.f;
+                    }
+                    loader_sync();
 #pragma unroll 8
-                for (int ll = 0; ll < LB; ++ll) {
-                    const float bv = sm.sB[ll][lane];
+                    for (int ll = 0; ll < LB; ++ll) {
+                        const float bv = sm.sB[ll][lane];
 #pragma unroll
-                    for (int t = 0; t < 8; ++t) accR[t] = fmaf(sm.sA[warp * 8 + t][ll], bv, accR[t]);
+                        for (int t = 0; t < 8; ++t)
+                            accR[t] = fmaf(sm.sA[warp * 8 + t][ll], bv, accR[t]);
+                    }
                 }
                 loader_sync();
             }
