@@ -8,8 +8,8 @@
 // Two-level blocked right-looking algorithm, last indices first, built in place in the output
 // L (which first receives the upper triangle of H). With U = I + L, pending indices A, the
 // current block B and H' the Schur complement left by the indices after B:
-//   H'_BB = U_BB D_B U_BB^T                  one CTA per 128-index block (fp64 in shared
-//                                             memory), which also forms U_BB^{-1};
+//   H'_BB = U_BB D_B U_BB^T                  one CTA per 128-index block (fp64 register
+//                                             tiles, ldl_diag.cuh), which also forms U_BB^{-1};
 //   X     = H'_AB U_BB^{-T},  U_AB = X D_B^{-1} 3xTF32 tensor-core GEMM (K = 128) whose
 //                                             epilogue writes U_AB into L and the hi/lo planes
 //                                             of X and U_AB;
@@ -19,16 +19,17 @@
 //                                             so the trailing matrix is streamed n/512 times.
 #include <algorithm>
 
+#include "ldl_diag.cuh"
 #include "tcgemm_host.cuh"
 
 namespace bakron {
 namespace {
 
 constexpr int NBI = 128;   // inner block: diagonal factorisation in one CTA
+static_assert(NBI == ldl_diag::NB, "diagonal kernel block width");
 constexpr int NBO = 512;   // outer block: K of the trailing update
 constexpr int BN = 128;
 constexpr int STAGES = 3;
-constexpr int DIAG_THREADS = 512;
 
 __global__ void copy_upper_kernel(const float* __restrict__ H, float* __restrict__ L, int n) {
     const size_t total = (size_t)n * n;
@@ -45,224 +46,6 @@ __global__ void clear_lower_kernel(float* __restrict__ L, int n) {
          e += (size_t)gridDim.x * blockDim.x) {
         const int i = (int)(e / n), j = (int)(e % n);
         if (j <= i) L[e] = 0.f;
-    }
-}
-
-constexpr int SUB = 32;                                   // sub-block of the diagonal block
-constexpr int NSUB = NBI / SUB;
-constexpr size_t kSOff = 0;                               // S: [NBI][NBI+1] fp64
-constexpr size_t kXOff = kSOff + (size_t)NBI * (NBI + 1); // X: [NBI-SUB][SUB+1] fp64
-constexpr size_t kTOff = kXOff + (size_t)(NBI - SUB) * (SUB + 1);  // T: [NSUB-1][SUB][SUB+1]
-constexpr size_t kDiagSmem =
-    (kTOff + (size_t)(NSUB - 1) * SUB * (SUB + 1) + NBI) * sizeof(double);
-
-// U D U^T of the b x b diagonal block at [k0, k0 + b) (b <= 128) in fp64 shared memory;
-// writes U's strictly upper part into L, the pivots into D, and U^{-1} (unit upper, zero
-// padded to 128 x 128) as hi/lo planes with row stride 128.
-//
-// Indices >= b are padded with the identity (pivot 1, no coupling), so the block is always
-// 128 wide. It is processed in 32-index sub-blocks, last first:
-//  (1) one warp factors the 32 x 32 diagonal sub-block by rank-1 steps and accumulates its
-//      inverse alongside: column j of U is u_j + e_j and U = G_31 ... G_1 with
-//      G_j = I + u_j e_j^T, so U^{-1} = G_1^{-1} ... G_31^{-1}, G_j^{-1} = I - u_j e_j^T;
-//  (2) all threads: X = H'[rows above, sub-block] W_JJ^T and U = X D^{-1} for the rows above;
-//  (3) all threads: H'[rows above]^2 -= X U^T on the upper triangle.
-// The inverse's off-diagonal blocks follow by block back substitution,
-// W_IJ = -W_II sum_{I<K<=J} U_IK W_KJ. S keeps U in its strict upper triangle and W^T in its
-// strict lower triangle (both unit diagonals implicit).
-__global__ void __launch_bounds__(DIAG_THREADS) diag_block_kernel(float* __restrict__ L, int n,
-                                                                int k0, int b,
-                                                                float* __restrict__ D,
-                                                                float* __restrict__ inv_hi,
-                                                                float* __restrict__ inv_lo,
-                                                                int* status) {
-    extern __shared__ double dsm[];
-    double(*S)[NBI + 1] = reinterpret_cast<double(*)[NBI + 1]>(dsm + kSOff);
-    double(*X)[SUB + 1] = reinterpret_cast<double(*)[SUB + 1]>(dsm + kXOff);
-    double(*T)[SUB][SUB + 1] = reinterpret_cast<double(*)[SUB][SUB + 1]>(dsm + kTOff);
-    double* sD = dsm + kTOff + (size_t)(NSUB - 1) * SUB * (SUB + 1);
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    for (int e = tid; e < NBI * NBI; e += DIAG_THREADS) {
-        const int r = e / NBI, c = e % NBI;
-        double v = 0.0;
-        if (r < b && c < b) v = (c >= r) ? (double)L[(size_t)(k0 + r) * n + k0 + c] : 0.0;
-        else if (r == c) v = 1.0;
-        S[r][c] = v;
-    }
-    __syncthreads();
-    for (int J = NSUB - 1; J >= 0; --J) {
-        const int j0 = J * SUB;
-        // (1) the diagonal sub-block, one warp
-        if (warp == 0) {
-            // lane = row r of the sub-block; the pivot column and the W row are read into
-            // registers first (broadcast loads), then every update has a static offset
-            double* Srow = &S[j0 + lane][j0];          // S[r][j0 + l]
-            for (int jj = SUB - 1; jj >= 0; --jj) {
-                const int j = j0 + jj;
-                double d = S[j][j];
-                const bool bad = !(d > 0.0) || !isfinite(d);
-                if (bad) d = 1.0;
-                if (lane == 0) {
-                    sD[j] = d;
-                    if (j < b) {
-                        if (bad) set_status(status, BAKRON_ERR_NOT_PD);
-                        D[k0 + j] = (float)d;
-                    }
-                }
-                const double u = (lane < jj) ? S[j0 + lane][j] / d : 0.0;
-                __syncwarp();
-                if (lane < jj) S[j0 + lane][j] = u;
-                const double ud = u * d;
-                const bool act = lane < jj;
-                // S[r][l] -= u_r d u_l for r <= l < j (u_l by shuffle: no shared-memory alias)
-#pragma unroll
-                for (int l = 0; l < SUB; ++l) {
-                    const double ul = __shfl_sync(0xffffffffu, u, l);
-                    if (act && l >= lane && l < jj) Srow[l] -= ud * ul;
-                }
-                // W[r][c] -= u_r W[j][c] for c > j, stored at S[j0+c][j0+r]; W[r][j] = -u_r.
-                // W[j][c] = S[j0+c][j] is read 8 columns at a time before the 8 updates.
-                if (act) S[j][j0 + lane] = -u;
-#pragma unroll
-                for (int c0 = 0; c0 < SUB; c0 += 8) {
-                    double wrow[8];
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) wrow[q] = (c0 + q > jj) ? S[j0 + c0 + q][j] : 0.0;
-#pragma unroll
-                    for (int q = 0; q < 8; ++q)
-                        if (act && c0 + q > jj) S[j0 + c0 + q][j0 + lane] -= u * wrow[q];
-                }
-                __syncwarp();
-            }
-        }
-        __syncthreads();
-        if (J == 0) break;
-        // (2) X[r][c] = sum_{t >= c} H'[r][j0+t] W_JJ[c][t], rows r < j0 (4x4 register tiles)
-        for (int e = tid; e < (j0 / 4) * (SUB / 4); e += DIAG_THREADS) {
-            const int r0 = (e / (SUB / 4)) * 4, c0 = (e % (SUB / 4)) * 4;
-            double acc[4][4] = {};
-            for (int t = 0; t < SUB; ++t) {
-                double h[4], w[4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) h[i] = S[r0 + i][j0 + t];
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const int c = c0 + q;
-                    w[q] = (t > c) ? S[j0 + t][j0 + c] : (t == c ? 1.0 : 0.0);
-                }
-#pragma unroll
-                for (int i = 0; i < 4; ++i)
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) acc[i][q] += h[i] * w[q];
-            }
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-#pragma unroll
-                for (int q = 0; q < 4; ++q) X[r0 + i][c0 + q] = acc[i][q];
-        }
-        __syncthreads();
-        for (int e = tid; e < j0 * SUB; e += DIAG_THREADS) {
-            const int r = e / SUB, c = e % SUB;
-            S[r][j0 + c] = X[r][c] / sD[j0 + c];
-        }
-        __syncthreads();
-        // (3) H'[r][l] -= sum_c X[r][c] U[l][c], r <= l < j0, 4x4 tiles on the upper triangle
-        {
-            const int n4 = j0 / 4;
-            for (int e = tid; e < n4 * (n4 + 1) / 2; e += DIAG_THREADS) {
-                int R = 0, rem = e, rowlen = n4;
-                while (rem >= rowlen) { rem -= rowlen; ++R; --rowlen; }
-                const int Lt = R + rem, r0 = R * 4, l0 = Lt * 4;
-                double acc[4][4] = {};
-                for (int c = 0; c < SUB; ++c) {
-                    double x[4], u[4];
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) x[i] = X[r0 + i][c];
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) u[q] = S[l0 + q][j0 + c];
-#pragma unroll
-                    for (int i = 0; i < 4; ++i)
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) acc[i][q] += x[i] * u[q];
-                }
-#pragma unroll
-                for (int i = 0; i < 4; ++i)
-#pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        if (l0 + q >= r0 + i) S[r0 + i][l0 + q] -= acc[i][q];
-            }
-        }
-        __syncthreads();
-    }
-    // off-diagonal blocks of W = U^{-1}, by distance J - I = 1 .. NSUB-1 (4x4 register tiles)
-    for (int dist = 1; dist < NSUB; ++dist) {
-        const int npairs = NSUB - dist;
-        // T_I = sum_{K=I+1..J} U_IK W_KJ
-        for (int e = tid; e < npairs * (SUB / 4) * (SUB / 4); e += DIAG_THREADS) {
-            const int I = e / ((SUB / 4) * (SUB / 4));
-            const int t0 = ((e / (SUB / 4)) % (SUB / 4)) * 4, c0 = (e % (SUB / 4)) * 4;
-            const int Jb = I + dist, i0 = I * SUB, jb0 = Jb * SUB;
-            double acc[4][4] = {};
-            for (int K = I + 1; K <= Jb; ++K) {
-                const int kk0 = K * SUB;
-                for (int sx = 0; sx < SUB; ++sx) {
-                    double uu[4], w[4];
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) uu[i] = S[i0 + t0 + i][kk0 + sx];
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const int c = c0 + q;   // W_KJ[sx][c]
-                        w[q] = (K < Jb) ? S[jb0 + c][kk0 + sx]
-                                        : ((c > sx) ? S[jb0 + c][jb0 + sx] : (c == sx ? 1.0 : 0.0));
-                    }
-#pragma unroll
-                    for (int i = 0; i < 4; ++i)
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) acc[i][q] += uu[i] * w[q];
-                }
-            }
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-#pragma unroll
-                for (int q = 0; q < 4; ++q) T[I][t0 + i][c0 + q] = acc[i][q];
-        }
-        __syncthreads();
-        // W_IJ[a][c] = -sum_{t >= a} W_II[a][t] T[t][c], stored as S[J0+c][I0+a]
-        for (int e = tid; e < npairs * (SUB / 4) * (SUB / 4); e += DIAG_THREADS) {
-            const int I = e / ((SUB / 4) * (SUB / 4));
-            const int a0 = ((e / (SUB / 4)) % (SUB / 4)) * 4, c0 = (e % (SUB / 4)) * 4;
-            const int Jb = I + dist, i0 = I * SUB, jb0 = Jb * SUB;
-            double acc[4][4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-#pragma unroll
-                for (int q = 0; q < 4; ++q) acc[i][q] = T[I][a0 + i][c0 + q];
-            for (int t = a0 + 1; t < SUB; ++t) {
-                double wi[4], tt[4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) wi[i] = (t > a0 + i) ? S[i0 + t][i0 + a0 + i] : 0.0;
-#pragma unroll
-                for (int q = 0; q < 4; ++q) tt[q] = T[I][t][c0 + q];
-#pragma unroll
-                for (int i = 0; i < 4; ++i)
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) acc[i][q] += wi[i] * tt[q];
-            }
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-#pragma unroll
-                for (int q = 0; q < 4; ++q) S[jb0 + c0 + q][i0 + a0 + i] = -acc[i][q];
-        }
-        __syncthreads();
-    }
-    for (int e = tid; e < NBI * NBI; e += DIAG_THREADS) {
-        const int r = e / NBI, c = e % NBI;
-        if (r < b && c < b && c > r) L[(size_t)(k0 + r) * n + k0 + c] = (float)S[r][c];
-        // U^{-1}[r][c] (zero padded beyond b), hi/lo planes
-        const float x = (r < b && c < b) ? (c > r ? (float)S[c][r] : (c == r ? 1.f : 0.f)) : 0.f;
-        const float h = sm100::tf32_hi(x);
-        inv_hi[e] = h;
-        inv_lo[e] = x - h;
     }
 }
 
@@ -339,13 +122,10 @@ extern "C" int bakron_ldl(const float* H, int n, float* L, float* D, void* ws, s
     ldl_ws_layout(n, [&](size_t k) { bufs[bi++] = c.take<float>(k); });
     LdlWs w{bufs[0], bufs[1], bufs[2], bufs[3], bufs[4], bufs[5], bufs[6], bufs[7]};
 
-    static bool diag_configured = false;
-    if (!diag_configured) {
-        if (cudaFuncSetAttribute(diag_block_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)kDiagSmem) != cudaSuccess)
-            return BAKRON_ERR_CUDA;
-        diag_configured = true;
-    }
+    if (cudaFuncSetAttribute(ldl_diag::diag_block_kernel,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)ldl_diag::kSmemBytes) != cudaSuccess)
+        return BAKRON_ERR_CUDA;
     int e;
     // Tensor maps over the outer-block planes (fixed for the whole call).
     CUtensorMap m_xh, m_xl, m_uh, m_ul;
@@ -363,7 +143,7 @@ extern "C" int bakron_ldl(const float* H, int n, float* L, float* D, void* ws, s
             // plane columns of this inner block, counted from the end of the outer block so
             // that they stay 128-aligned even when the outer block is a partial one
             const int kb0 = std::max(ko0, kb1 - NBI), b = kb1 - kb0, c_off = NBO - NBI * (t + 1);
-            diag_block_kernel<<<1, DIAG_THREADS, kDiagSmem, st>>>(L, n, kb0, b, D, w.inv_hi,
+            ldl_diag::diag_block_kernel<<<1, ldl_diag::THREADS, ldl_diag::kSmemBytes, st>>>(L, n, kb0, b, D, w.inv_hi,
                                                                   w.inv_lo, dev_status);
             count_launches(1);
             if (kb0 == 0) continue;
