@@ -199,21 +199,8 @@ def run(args):
     names = ["ldl_O", "ldl_I", "round", "loss"]
 
     def step(evs=None):
-        calls = [
-            lambda: bk.bakron_ldl(HO, solver.L_O, solver.D_O, solver.ws, solver.status, stream),
-            lambda: bk.bakron_ldl(HI, solver.L_I, solver.D_I, solver.ws, solver.status, stream),
-            lambda: bk.bakron_round(Ws, solver.L_O, solver.L_I, sc, bits, solver.codes, solver.W,
-                                    solver.ws_round, solver.status, stream),
-            lambda: bk.bakron_proxy_loss(solver.E, HO, HI, solver.loss, solver.ws, stream),
-        ]
-        for k, f in enumerate(calls):
-            if evs is not None:
-                evs[k][0].record(stream)
-            rc = f()
-            if rc != 0:
-                raise bk.BakronError(rc, names[k])
-            if evs is not None:
-                evs[k][1].record(stream)
+        timing = None if evs is None else dict(zip(names, evs))
+        solver.run(Ws, HO, HI, sc, bits, stream, timing=timing)
 
     for _ in range(args.warmup):
         step()

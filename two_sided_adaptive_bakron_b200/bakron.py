@@ -275,20 +275,45 @@ class Solver:
         self.W = torch.empty((m, n), **f32)
         self.loss = torch.empty((1,), dtype=torch.float64, device=self.device)
         self.ws_round = workspace(bakron_round_workspace_bytes(m, n), self.device)
-        self.ws = workspace(max(bakron_ldl_workspace_bytes(m), bakron_ldl_workspace_bytes(n),
+        self.ws_O = workspace(bakron_ldl_workspace_bytes(m), self.device)
+        self.ws = workspace(max(bakron_ldl_workspace_bytes(n),
                                 bakron_proxy_loss_workspace_bytes(m, n)), self.device)
         self.E = self.ws_round[: 4 * m * n].view(torch.float32).view(m, n)
         self.status = new_status(self.device)
+        # the two factorisations are independent: ldl(H_O) runs on a side stream while
+        # ldl(H_I) runs on the caller's stream
+        self.side = torch.cuda.Stream(device=self.device)
+        self._fork = torch.cuda.Event()
+        self._join = torch.cuda.Event()
 
-    def run(self, Wstar, H_O, H_I, scales, bits, stream=None, with_loss=True):
-        """Enqueues the whole path (reads: self.codes, self.W, self.E, self.loss)."""
-        _raise(bakron_ldl(H_O, self.L_O, self.D_O, self.ws, self.status, stream), "bakron_ldl")
-        _raise(bakron_ldl(H_I, self.L_I, self.D_I, self.ws, self.status, stream), "bakron_ldl")
-        _raise(bakron_round(Wstar, self.L_O, self.L_I, scales, bits, self.codes, self.W,
-                            self.ws_round, self.status, stream), "bakron_round")
+    def run(self, Wstar, H_O, H_I, scales, bits, stream=None, with_loss=True, timing=None):
+        """Enqueues the whole path (reads: self.codes, self.W, self.E, self.loss).
+
+        timing: optional {name: (start_event, end_event)} for any of "ldl_O", "ldl_I", "round",
+        "loss"; each pair is recorded around its call on the stream that runs it.
+        """
+        if stream is None:
+            stream = torch.cuda.current_stream(self.device)
+        timing = timing or {}
+
+        def call(name, st, fn, *a):
+            ev = timing.get(name)
+            if ev is not None:
+                ev[0].record(st)
+            _raise(fn(*a, st), "bakron " + name)
+            if ev is not None:
+                ev[1].record(st)
+
+        self._fork.record(stream)
+        self.side.wait_event(self._fork)
+        call("ldl_O", self.side, bakron_ldl, H_O, self.L_O, self.D_O, self.ws_O, self.status)
+        call("ldl_I", stream, bakron_ldl, H_I, self.L_I, self.D_I, self.ws, self.status)
+        self._join.record(self.side)
+        stream.wait_event(self._join)
+        call("round", stream, bakron_round, Wstar, self.L_O, self.L_I, scales, bits, self.codes,
+             self.W, self.ws_round, self.status)
         if with_loss:
-            _raise(bakron_proxy_loss(self.E, H_O, H_I, self.loss, self.ws, stream),
-                   "bakron_proxy_loss")
+            call("loss", stream, bakron_proxy_loss, self.E, H_O, H_I, self.loss, self.ws)
 
     def check(self, stream=None):
         _raise(bakron_read_status(self.status, stream), "bakron (device)")

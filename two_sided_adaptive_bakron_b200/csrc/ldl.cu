@@ -80,7 +80,7 @@ struct EpiPanel {
             ul[o] = u - uh_;
         }
     }
-    __device__ void finish(const tc::Problem&, int) {}
+    __device__ void tile_done(const tc::Problem&, int, int) {}
 };
 
 struct LdlWs {

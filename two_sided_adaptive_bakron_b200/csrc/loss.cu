@@ -52,7 +52,7 @@ LossLayout loss_layout(int m, int n) {
     L.ha = (size_t)L.p * L.ldp;
     L.v = (size_t)L.q * L.ldp;
     const size_t t = (L.q + BN - 1) / BN;
-    L.tiles2 = t * (t + 1) / 2;
+    L.tiles2 = t * (t + 1) / 2;   // upper block triangle of Z
     return L;
 }
 
@@ -68,7 +68,7 @@ extern "C" size_t bakron_proxy_loss_workspace_bytes(int m, int n) {
     z.take<float>(L.xt); z.take<float>(L.xt);
     z.take<float>(L.ha); z.take<float>(L.ha);
     z.take<float>(L.v);  z.take<float>(L.v);
-    z.take<double>(L.tiles2);
+    z.take<double>(4 * L.tiles2);   // one partial per tile and epilogue warp
     z.take<int>(64);
     return z.bytes();
 }
@@ -87,7 +87,7 @@ extern "C" int bakron_proxy_loss(const float* dW, int m, int n, const float* H_O
     float* ha_lo = c.take<float>(L.ha);
     float* v_hi = c.take<float>(L.v);
     float* v_lo = c.take<float>(L.v);
-    double* partial = c.take<double>(L.tiles2);
+    double* partial = c.take<double>(4 * L.tiles2);
     int* status = c.take<int>(64);   // engine timeouts (never expected) land here
     int e;
     if ((e = cuda_err(cudaMemsetAsync(status, 0, sizeof(int), st)))) return e;
@@ -120,7 +120,7 @@ extern "C" int bakron_proxy_loss(const float* dW, int m, int n, const float* H_O
     tc::EpiDot epi2{Hb, q, partial, 2.f, 0.0};
     if ((e = tc::launch_gemm3x<BN, STAGES>(m_xth, m_xtl, m_vh, m_vl, g2, epi2, status, st)))
         return e;
-    final_sum_kernel<<<1, 1024, 0, st>>>(partial, L.tiles2, status, loss);
+    final_sum_kernel<<<1, 1024, 0, st>>>(partial, 4 * L.tiles2, status, loss);
     count_launches(1);
     return cuda_err(cudaGetLastError());
 }

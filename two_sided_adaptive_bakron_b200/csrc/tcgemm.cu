@@ -57,6 +57,24 @@ __global__ void split_kernel(const float* __restrict__ src, int rows, int cols, 
 
 }  // namespace
 
+int sm_count() {
+    static std::mutex mu;
+    static int cached[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return 0;
+    if (dev >= 64) {
+        int v = 0;
+        return cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess ? v : 0;
+    }
+    std::lock_guard<std::mutex> lock(mu);
+    if (cached[dev] == 0) {
+        int v = 0;
+        if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+        cached[dev] = v;
+    }
+    return cached[dev];
+}
+
 int make_kmajor_map(CUtensorMap* map, const float* base, int rows, int kcols, int ld,
                     int box_rows) {
     auto fn = encode_fn();

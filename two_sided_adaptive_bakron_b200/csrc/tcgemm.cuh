@@ -8,17 +8,21 @@
 // in fp32 TMEM accumulators, which keeps about 22 significant bits per product (the dropped
 // A_lo B_lo term and the tf32 truncation of lo are both below 2^-21 relative).
 //
-// Pipeline (one 128-thread CTA per output tile):
+// Persistent pipeline (at most one 192-thread CTA per SM, tiles t = blockIdx.x + i * gridDim.x):
 //   warp 0 / lane 0 : TMA producer, STAGES-deep ring of {A_hi, A_lo, B_hi, B_lo} k-blocks of
-//                     32 fp32 (one 128-byte swizzle row), full/empty mbarriers;
-//   warp 1 / lane 0 : MMA issuer, 4 k-steps of 8 x 3 tcgen05.mma per k-block, tcgen05.commit
-//                     frees the stage, a final commit signals the epilogue;
-//   all 4 warps     : epilogue, tcgen05.ld of the accumulator (warp w owns TMEM lanes
-//                     32w..32w+31 = tile rows), then the Epi functor.
+//                     32 fp32 (one 128-byte swizzle row) that runs on across tiles;
+//   warp 1 / lane 0 : MMA issuer, 4 k-steps of 8 x 3 tcgen05.mma per k-block into one of two
+//                     TMEM accumulators (2 x BN columns); tcgen05.commit frees the stage and,
+//                     after a tile's last k-block, hands the accumulator to the epilogue;
+//   warps 2 .. 5    : epilogue, tcgen05.ld of the accumulator (warp w reads TMEM lanes
+//                     32 (w % 4) .. + 31 = tile rows), then the Epi functor, then the
+//                     accumulator goes back to the MMA issuer, so a tile's epilogue overlaps
+//                     the next tile's MMAs.
 // A launch may hold several problems (a grouped GEMM): the operand tensor maps cover whole
 // planes and every problem only moves the tile origins.
-// Every mbarrier wait is bounded; on expiry the status word gets BAKRON_ERR_TIMEOUT, in-flight
-// copies and MMAs are drained (with a bound) and the TMEM is released before returning.
+// Every mbarrier wait is bounded and also gives up when another role has raised the CTA's
+// abort word; on expiry the status word gets BAKRON_ERR_TIMEOUT, in-flight copies and MMAs are
+// drained (with a bound) and the TMEM is released before returning.
 #pragma once
 
 #include "sm100.cuh"
@@ -29,7 +33,8 @@ namespace tc {
 constexpr int BM = 128;
 constexpr int BK = 32;
 constexpr int kMaxProblems = 48;
-constexpr int kThreads = 128;
+constexpr int kThreads = 192;
+constexpr int kEpiWarp0 = 2;       // first of the 4 epilogue warps
 
 struct Problem {
     int a_row0, a_k0;   // origin of the A tile rows (M) and of K in the A planes
@@ -54,12 +59,32 @@ struct Cfg {
     static constexpr uint32_t kABytes = BM * BK * 4;          // one A plane k-block
     static constexpr uint32_t kBBytes = BN * BK * 4;          // one B plane k-block
     static constexpr uint32_t kStageBytes = 2 * kABytes + 2 * kBBytes;
-    static constexpr uint32_t kTmemCols = BN < 32 ? 32 : BN;  // power of two >= 32
+    static constexpr uint32_t kTmemCols = 2 * BN;             // two accumulators
+    static constexpr uint32_t kEpiBytes = 4 * 32 * 33 * 4;    // per-warp 32 x 33 staging
+    static_assert(kTmemCols >= 32 && kTmemCols <= 512 && (kTmemCols & (kTmemCols - 1)) == 0,
+                  "TMEM allocation must be a power of two in [32, 512]");
 };
 
 template <int BN, int STAGES>
 constexpr size_t gemm_smem_bytes() {
-    return 1024 /*alignment slack*/ + (size_t)STAGES * Cfg<BN>::kStageBytes + 256;
+    return 1024 /*alignment slack*/ + (size_t)STAGES * Cfg<BN>::kStageBytes + Cfg<BN>::kEpiBytes +
+           256;
+}
+
+// Bounded wait that also gives up once *abort is set (by any role of the CTA).
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, int* status,
+                                              uint64_t limit_ns, volatile int* abort) {
+    if (sm100::mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (!sm100::mbar_try_wait(bar, parity)) {
+        if (*abort) return false;
+        if (globaltimer_ns() - t0 > limit_ns) {
+            set_status(status, BAKRON_ERR_TIMEOUT);
+            *abort = 1;
+            return false;
+        }
+    }
+    return true;
 }
 
 // Maps a linear tile index of the launch to (problem, m0, n0). Returns false if out of range.
@@ -99,31 +124,32 @@ gemm3x_kernel(const __grid_constant__ CUtensorMap a_hi, const __grid_constant__ 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * C::kStageBytes);
+    float* epi_stage = reinterpret_cast<float*>(smem + STAGES * C::kStageBytes);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * C::kStageBytes + C::kEpiBytes);
     uint64_t* empty = full + STAGES;
-    uint64_t* done = empty + STAGES;       // accumulator complete
-    uint64_t* drain = done + 1;            // error path: all MMAs retired
+    uint64_t* acc_full = empty + STAGES;   // [2] accumulator ready for the epilogue
+    uint64_t* acc_empty = acc_full + 2;    // [2] accumulator read out (4 epilogue warps)
+    uint64_t* drain = acc_empty + 2;       // error path: all MMAs retired
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
-    int* s_abort = reinterpret_cast<int*>(tmem_slot + 1);
+    volatile int* s_abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    Epi e = epi;
-    int pi, m0, n0;
-    if (!decode_tile(probs, BN, blockIdx.x, pi, m0, n0)) return;
-    const Problem& P = probs.p[pi];
-    const int nkb = (P.K + BK - 1) / BK;
+    const int total = probs.total_tiles;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             sm100::mbar_init(&full[s], 1);
             sm100::mbar_init(&empty[s], 1);
         }
-        sm100::mbar_init(done, 1);
+        for (int b = 0; b < 2; ++b) {
+            sm100::mbar_init(&acc_full[b], 1);
+            sm100::mbar_init(&acc_empty[b], 4);
+        }
         sm100::mbar_init(drain, 1);
         *s_abort = 0;
         sm100::fence_mbar_init();
     }
-    if (warp == 0) {
+    if (warp == 1) {
         sm100::tmem_alloc(tmem_slot, C::kTmemCols);
         sm100::tmem_relinquish();
     }
@@ -138,112 +164,132 @@ gemm3x_kernel(const __grid_constant__ CUtensorMap a_hi, const __grid_constant__ 
         return which < 2 ? base + which * C::kABytes : base + 2 * C::kABytes + (which - 2) * C::kBBytes;
     };
 
-    if (warp == 0 && lane == 0 && nkb > 0) {
+    if (warp == 0) {
         // ---------------- TMA producer
-        sm100::prefetch_tmap(&a_hi);
-        sm100::prefetch_tmap(&a_lo);
-        sm100::prefetch_tmap(&b_hi);
-        sm100::prefetch_tmap(&b_lo);
-        int issued = 0;
-        for (int kb = 0; kb < nkb; ++kb) {
-            const int s = kb % STAGES;
-            const uint32_t ph = (kb / STAGES) & 1;
-            if (kb >= STAGES) {
-                if (!sm100::mbar_wait(&empty[s], ph ^ 1, status, limit_ns)) {
-                    atomicExch(s_abort, 1);
-                    break;
+        if (lane == 0) {
+            sm100::prefetch_tmap(&a_hi);
+            sm100::prefetch_tmap(&a_lo);
+            sm100::prefetch_tmap(&b_hi);
+            sm100::prefetch_tmap(&b_lo);
+            uint32_t g = 0;   // k-blocks issued by this CTA
+            for (int t = blockIdx.x; t < total && !*s_abort; t += gridDim.x) {
+                int pi, m0, n0;
+                if (!decode_tile(probs, BN, t, pi, m0, n0)) break;
+                const Problem& P = probs.p[pi];
+                const int nkb = (P.K + BK - 1) / BK;
+                for (int kb = 0; kb < nkb; ++kb, ++g) {
+                    const int s = g % STAGES;
+                    if (g >= STAGES &&
+                        !wait_or_abort(&empty[s], ((g / STAGES) & 1) ^ 1, status, limit_ns, s_abort))
+                        break;
+                    sm100::mbar_arrive_expect_tx(&full[s], C::kStageBytes);
+                    const int ka = P.a_k0 + kb * BK, kbb = P.b_k0 + kb * BK;
+                    sm100::tma_load_2d(stage_ptr(s, 0), &a_hi, ka, P.a_row0 + m0, &full[s]);
+                    sm100::tma_load_2d(stage_ptr(s, 1), &a_lo, ka, P.a_row0 + m0, &full[s]);
+                    sm100::tma_load_2d(stage_ptr(s, 2), &b_hi, kbb, P.b_row0 + n0, &full[s]);
+                    sm100::tma_load_2d(stage_ptr(s, 3), &b_lo, kbb, P.b_row0 + n0, &full[s]);
                 }
             }
-            if (*(volatile int*)s_abort) break;
-            sm100::mbar_arrive_expect_tx(&full[s], C::kStageBytes);
-            const int ka = P.a_k0 + kb * BK, kbb = P.b_k0 + kb * BK;
-            sm100::tma_load_2d(stage_ptr(s, 0), &a_hi, ka, P.a_row0 + m0, &full[s]);
-            sm100::tma_load_2d(stage_ptr(s, 1), &a_lo, ka, P.a_row0 + m0, &full[s]);
-            sm100::tma_load_2d(stage_ptr(s, 2), &b_hi, kbb, P.b_row0 + n0, &full[s]);
-            sm100::tma_load_2d(stage_ptr(s, 3), &b_lo, kbb, P.b_row0 + n0, &full[s]);
-            issued = kb + 1;
+            // Error path: let every issued copy land before the CTA can exit.
+            if (*s_abort) {
+                for (uint32_t q = (g > (uint32_t)STAGES ? g - STAGES : 0); q < g; ++q)
+                    sm100::mbar_wait(&full[q % STAGES], (q / STAGES) & 1, status, limit_ns);
+            }
         }
-        // Error path: let every issued copy land before the CTA can exit.
-        if (*(volatile int*)s_abort) {
-            for (int kb = (issued > STAGES ? issued - STAGES : 0); kb < issued; ++kb)
-                sm100::mbar_wait(&full[kb % STAGES], (kb / STAGES) & 1, status, limit_ns);
-        }
-    } else if (warp == 1 && lane == 0 && nkb > 0) {
+    } else if (warp == 1) {
         // ---------------- MMA issuer
-        constexpr uint32_t idesc = sm100::idesc_tf32(BM, BN);
-        for (int kb = 0; kb < nkb; ++kb) {
-            const int s = kb % STAGES;
-            const uint32_t ph = (kb / STAGES) & 1;
-            if (!sm100::mbar_wait(&full[s], ph, status, limit_ns)) {
-                atomicExch(s_abort, 1);
-                break;
+        if (lane == 0) {
+            constexpr uint32_t idesc = sm100::idesc_tf32(BM, BN);
+            uint32_t g = 0;   // k-blocks consumed
+            int i = 0;        // tiles of this CTA
+            for (int t = blockIdx.x; t < total && !*s_abort; t += gridDim.x, ++i) {
+                int pi, m0, n0;
+                if (!decode_tile(probs, BN, t, pi, m0, n0)) break;
+                const int nkb = (probs.p[pi].K + BK - 1) / BK;
+                const int b = i & 1;
+                if (i >= 2 &&
+                    !wait_or_abort(&acc_empty[b], ((i >> 1) & 1) ^ 1, status, limit_ns, s_abort))
+                    break;
+                sm100::tc_fence_after();
+                const uint32_t acc = tmem + (uint32_t)(b * BN);
+                bool ok = true;
+                for (int kb = 0; kb < nkb; ++kb, ++g) {
+                    const int s = g % STAGES;
+                    if (!wait_or_abort(&full[s], (g / STAGES) & 1, status, limit_ns, s_abort)) {
+                        ok = false;
+                        break;
+                    }
+                    sm100::tc_fence_after();
+                    const uint32_t ah = sm100::smem_u32(stage_ptr(s, 0));
+                    const uint32_t al = sm100::smem_u32(stage_ptr(s, 1));
+                    const uint32_t bh = sm100::smem_u32(stage_ptr(s, 2));
+                    const uint32_t bl = sm100::smem_u32(stage_ptr(s, 3));
+#pragma unroll
+                    for (int kk = 0; kk < BK / 8; ++kk) {
+                        const uint32_t off = kk * 32;  // 8 tf32 = 32 bytes along the swizzled row
+                        const uint64_t dah = sm100::desc_kmajor_sw128(ah + off);
+                        const uint64_t dal = sm100::desc_kmajor_sw128(al + off);
+                        const uint64_t dbh = sm100::desc_kmajor_sw128(bh + off);
+                        const uint64_t dbl = sm100::desc_kmajor_sw128(bl + off);
+                        const uint32_t acc0 = (kb > 0 || kk > 0) ? 1u : 0u;
+                        sm100::mma_tf32(acc, dah, dbh, idesc, acc0);
+                        sm100::mma_tf32(acc, dah, dbl, idesc, 1u);
+                        sm100::mma_tf32(acc, dal, dbh, idesc, 1u);
+                    }
+                    sm100::mma_commit(&empty[s]);
+                }
+                if (!ok) break;
+                if (nkb > 0) sm100::mma_commit(&acc_full[b]);
+                else sm100::mbar_arrive(&acc_full[b]);   // K = 0: the epilogue writes zeros
             }
-            if (*(volatile int*)s_abort) break;
+            if (*s_abort) {
+                sm100::mma_commit(drain);
+                sm100::mbar_wait(drain, 0, status, limit_ns);
+            }
+        }
+    } else {
+        // ---------------- epilogue (warps 2 .. 5)
+        Epi e = epi;
+        const int quarter = warp & 3;   // TMEM lanes this warp may read
+        float* stage = epi_stage + (warp - kEpiWarp0) * (32 * 33);
+        int i = 0;
+        for (int t = blockIdx.x; t < total; t += gridDim.x, ++i) {
+            int pi, m0, n0;
+            if (!decode_tile(probs, BN, t, pi, m0, n0)) break;
+            const Problem& P = probs.p[pi];
+            const int b = i & 1;
+            bool ok = true;
+            if (lane == 0) ok = wait_or_abort(&acc_full[b], (i >> 1) & 1, status, limit_ns, s_abort);
+            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+            if (!ok) break;
             sm100::tc_fence_after();
-            const uint32_t ah = sm100::smem_u32(stage_ptr(s, 0));
-            const uint32_t al = sm100::smem_u32(stage_ptr(s, 1));
-            const uint32_t bh = sm100::smem_u32(stage_ptr(s, 2));
-            const uint32_t bl = sm100::smem_u32(stage_ptr(s, 3));
-#pragma unroll
-            for (int kk = 0; kk < BK / 8; ++kk) {
-                const uint32_t off = kk * 32;  // 8 tf32 = 32 bytes along the swizzled row
-                const uint64_t dah = sm100::desc_kmajor_sw128(ah + off);
-                const uint64_t dal = sm100::desc_kmajor_sw128(al + off);
-                const uint64_t dbh = sm100::desc_kmajor_sw128(bh + off);
-                const uint64_t dbl = sm100::desc_kmajor_sw128(bl + off);
-                const uint32_t acc0 = (kb > 0 || kk > 0) ? 1u : 0u;
-                sm100::mma_tf32(tmem, dah, dbh, idesc, acc0);
-                sm100::mma_tf32(tmem, dah, dbl, idesc, 1u);
-                sm100::mma_tf32(tmem, dal, dbh, idesc, 1u);
-            }
-            sm100::mma_commit(&empty[s]);
-        }
-        if (*(volatile int*)s_abort) {
-            sm100::mma_commit(drain);
-            sm100::mbar_wait(drain, 0, status, limit_ns);
-        } else {
-            sm100::mma_commit(done);
-        }
-    }
-    __syncwarp();
-
-    // ---------------- epilogue (all 4 warps)
-    bool have = nkb > 0;
-    if (have) {
-        // every thread polls the completion barrier (bounded)
-        if (!sm100::mbar_wait(done, 0, status, limit_ns)) have = false;
-        if (*(volatile int*)s_abort) have = false;
-    }
-    have = __all_sync(0xffffffffu, have);
-    const bool aborted = __any_sync(0xffffffffu, *(volatile int*)s_abort != 0);
-    sm100::tc_fence_after();
-    // Each warp moves its 32 x 32 accumulator chunks through a private, padded shared-memory
-    // tile (the operand ring is idle once the last MMA has completed) so that the epilogue
-    // sees one row per warp-wide step with lanes on consecutive columns: coalesced global
-    // accesses.
-    float* stage = reinterpret_cast<float*>(smem) + warp * (32 * 33);
-    if (!aborted) {
+            const bool have = P.K > 0;
 #pragma unroll 1
-        for (int c0 = 0; c0 < BN; c0 += 32) {
-            float v[32];
-            if (have) {
-                sm100::tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0, v);
-            } else {
+            for (int c0 = 0; c0 < BN; c0 += 32) {
+                float v[32];
+                if (have) {
+                    sm100::tmem_ld32(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(b * BN + c0), v);
+                } else {
 #pragma unroll
-                for (int i = 0; i < 32; ++i) v[i] = 0.f;
+                    for (int q = 0; q < 32; ++q) v[q] = 0.f;
+                }
+#pragma unroll
+                for (int q = 0; q < 32; ++q) stage[lane * 33 + q] = v[q];
+                __syncwarp();
+                // lane = column n0 + c0 + lane, element rr of the chunk at stage[rr * 33 + lane]
+                e.chunk(P, m0 + quarter * 32, n0 + c0 + lane, m0, n0, stage + lane);
+                __syncwarp();
             }
-#pragma unroll
-            for (int i = 0; i < 32; ++i) stage[lane * 33 + i] = v[i];
+            e.tile_done(P, t, quarter);
+            sm100::tc_fence_before();
             __syncwarp();
-            // lane = column n0 + c0 + lane, element rr of the chunk at stage[rr * 33 + lane]
-            e.chunk(P, m0 + warp * 32, n0 + c0 + lane, m0, n0, stage + lane);
-            __syncwarp();
+            if (lane == 0) sm100::mbar_arrive(&acc_empty[b]);
         }
     }
-    e.finish(P, blockIdx.x);
+    __syncwarp();   // the producer and MMA warps reconverge with their idle lanes
     sm100::tc_fence_before();
     __syncthreads();
-    if (warp == 0) sm100::tmem_dealloc(tmem, C::kTmemCols);
+    if (warp == 1) sm100::tmem_dealloc(tmem, C::kTmemCols);
 }
 
 }  // namespace tc

@@ -29,7 +29,8 @@ void split_planes(const float* src, int rows, int cols, int ld_src, float* hi, f
 // row0 is the chunk's first row, col = this lane's column (both relative to the problem
 // origin), element rr of the lane's column is v[rr * 33]; m0, n0 give the tile origin.
 // Global loads of a chunk are all issued before its stores (32 in flight per thread).
-// finish() runs once per CTA, by all threads.
+// tile_done(P, tile, quarter) runs after a tile's chunks, once per epilogue warp (all lanes);
+// quarter (0..3) says which 32 rows of the tile the warp held.
 
 // out = weight * acc, written as hi/lo planes at (c_row0 + r, c_col0 + c).
 struct EpiStoreSplit {
@@ -49,7 +50,7 @@ struct EpiStoreSplit {
             }
         }
     }
-    __device__ void finish(const Problem&, int) {}
+    __device__ void tile_done(const Problem&, int, int) {}
 };
 
 // C (+)= weight * acc at (c_row0 + r, c_col0 + c); `accumulate` selects += over =; with
@@ -76,11 +77,12 @@ struct EpiStore {
             if (ok) C[(size_t)gr * ldc + gc] = old[rr] + P.weight * v[rr * 33];
         }
     }
-    __device__ void finish(const Problem&, int) {}
+    __device__ void tile_done(const Problem&, int, int) {}
 };
 
-// partial[tile] = w * sum_{r,c in tile} acc[r][c] * G[r][c] in fp64, w = 1 on diagonal tiles
-// (m0 == n0) and `offdiag_weight` elsewhere (symmetric products computed on one triangle).
+// partial[4 tile + quarter] = w * sum over the warp's 32 rows of the tile of acc[r][c] G[r][c]
+// in fp64, w = 1 on diagonal tiles (m0 == n0) and `offdiag_weight` elsewhere (symmetric
+// products computed on one triangle). The partials are summed in a fixed order afterwards.
 struct EpiDot {
     const float* G;
     int ldg;
@@ -98,18 +100,12 @@ struct EpiDot {
         for (int rr = 0; rr < 32; ++rr) s += (double)v[rr * 33] * (double)g[rr];
         acc += (m0 == n0) ? s : (double)offdiag_weight * s;
     }
-    __device__ void finish(const Problem&, int tile) {
-        __shared__ double red[kThreads / 32];
+    __device__ void tile_done(const Problem&, int tile, int quarter) {
         double s = acc;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) s += __shfl_down_sync(0xffffffffu, s, o);
-        if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = s;
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            double t = 0.0;
-            for (int w = 0; w < kThreads / 32; ++w) t += red[w];
-            partial[tile] = t;
-        }
+        if ((threadIdx.x & 31) == 0) partial[(size_t)tile * 4 + quarter] = s;
+        acc = 0.0;
     }
 };
 
@@ -138,25 +134,30 @@ struct ProblemList {
     bool empty() const { return P.total_tiles == 0; }
 };
 
+// Number of SMs of the current device (cached per device).
+int sm_count();
+
+// Launches the grouped GEMM with min(tiles, max_ctas) persistent CTAs (max_ctas <= 0: one per
+// SM). A smaller max_ctas leaves SMs free for work on other streams.
 template <int BN, int STAGES, class Epi>
 int launch_gemm3x(const CUtensorMap& ah, const CUtensorMap& al, const CUtensorMap& bh,
                   const CUtensorMap& bl, const ProblemList& L, const Epi& epi, int* status,
-                  cudaStream_t st) {
+                  cudaStream_t st, int max_ctas = 0) {
     if (L.empty()) return BAKRON_OK;
     // A TMA tile load must start on a 16-byte boundary: every K origin a multiple of 4 fp32.
     for (int i = 0; i < L.P.count; ++i)
         if ((L.P.p[i].a_k0 & 3) || (L.P.p[i].b_k0 & 3)) return BAKRON_ERR_INVALID_ARG;
     constexpr size_t smem = gemm_smem_bytes<BN, STAGES>();
+    static_assert(smem <= 227 * 1024, "GEMM shared memory above the per-CTA limit");
     auto kern = gemm3x_kernel<BN, STAGES, Epi>;
-    static bool configured = false;   // per template instance
-    if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)smem);
-        if (e != cudaSuccess) return BAKRON_ERR_CUDA;
-        configured = true;
-    }
-    kern<<<L.P.total_tiles, kThreads, smem, st>>>(ah, al, bh, bl, L.P, epi, status,
-                                                  spin_limit_ns());
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess)
+        return BAKRON_ERR_CUDA;
+    const int nsm = sm_count();
+    if (nsm <= 0) return BAKRON_ERR_CUDA;
+    int grid = (max_ctas > 0 && max_ctas < nsm) ? max_ctas : nsm;
+    if (grid > L.P.total_tiles) grid = L.P.total_tiles;
+    kern<<<grid, kThreads, smem, st>>>(ah, al, bh, bl, L.P, epi, status, spin_limit_ns());
     count_launches(1);
     return cuda_err(cudaGetLastError());
 }
