@@ -29,13 +29,13 @@
 //    block products.
 #include <algorithm>
 
+#include "round_leaf.cuh"
 #include "tcgemm_host.cuh"
 
 namespace bakron {
 namespace {
 
-constexpr int LB = 32;          // leaf edge
-constexpr int NSLOT = 2 * LB - 1;
+using leaf::LB;
 constexpr int SB = 256;         // super-block edge
 constexpr int LPB = SB / LB;    // leaves per super-block edge
 constexpr int BN = 128;
@@ -78,25 +78,11 @@ __device__ __forceinline__ int diag_len(int d, int lm, int ln) {
     return hi >= lo ? hi - lo + 1 : 0;
 }
 
-constexpr int UW = 4;            // wavefront steps per unrolled group
-constexpr int WIN = LB + UW;     // register window of slots
-constexpr int LS = LB + 4;       // row stride of the skewed diagonal blocks (16-byte rows)
 constexpr int NLOAD = 128;       // loader threads (warps 0-3)
 constexpr int NTHW = NLOAD + 32; // + the solver warp (warp 4)
-
-// One staging buffer: a leaf's inputs and outputs (shared memory, floats).
-struct LeafBuf {
-    float W[LB * LB];            // W* of the leaf, row stride LB
-    float T[LB * LB];            // vertical sums (everything above the leaf)
-    float R[LB * LB];            // horizontal sums (everything left of the leaf)
-    float LOr[LB * LS];          // LOr[r*LS + d] = L_O[i0+r][i0+r+d]
-    float LIc[LB * LS];          // LIc[c*LS + d] = L_I[j0+c-d][j0+c]
-    float S[2 * LB];             // s_r and its reciprocal
-    float oW[LB * LB], oE[LB * LB], oU[LB * LB];
-    float oEt[LB * LB];          // E transposed (for the transposed planes)
-    int8_t oC[LB * LB];
-    int meta[4];                 // I, J, rows, cols
-};
+using leaf::LS;
+using leaf::LeafBuf;
+using leaf::solve_leaf;
 
 struct LeafSmem {
     LeafBuf buf[2];
@@ -105,105 +91,6 @@ struct LeafSmem {
     uint64_t full[2], empty[2];
     int stop;
 };
-
-// The in-leaf wavefront, run by the solver warp; lane j owns column j and the element of row
-// r is handled at step s = r + j. Leaf arrays use row stride LB, element (r, c) at r*LB + c,
-// so an anti-diagonal and a row both touch 32 distinct banks. Per lane, slot s of wT / wR
-// holds the vertical / horizontal sum of its element of step s. A step reads slot s, then
-// pushes E down its column into slots s+1..s+31 (in-lane) and U along its row into slot s+d
-// of lane j+d (warp shuffles); the d = 1 pushes, the only ones the next step needs, go
-// first. The step loop stays rolled (4 steps per iteration) over a sliding window of 36
-// slot registers: every register index is static and the code stays small.
-// Q divides by s_r as one correctly rounded fp32 division; the quotient is formed as
-// pre * (1/s_r), whose distance to the division's result is below 2e-7 |x|, and the exact
-// division is taken instead whenever that quotient lies within 1e-6 max(1,|x|) of a rounding
-// boundary, so the decision always equals the division's.
-__device__ __forceinline__ void solve_leaf(int lane, int rows, int cols, float qlo, float qhi,
-                                           LeafBuf& B, int* status) {
-    const int j = lane;
-    const bool colok = j < cols;
-    float li[LB];
-#pragma unroll
-    for (int q = 0; q < LB / 4; ++q) {
-        const float4 v = *reinterpret_cast<const float4*>(&B.LIc[j * LS + 4 * q]);
-        li[4 * q] = v.x; li[4 * q + 1] = v.y; li[4 * q + 2] = v.z; li[4 * q + 3] = v.w;
-    }
-    float wT[WIN], wR[WIN];
-#pragma unroll
-    for (int t = 0; t < WIN; ++t) {
-        const int r = t - j;
-        const bool ok = (r >= 0) && (r < LB);
-        const int rr = ok ? r : 0;
-        wT[t] = ok ? B.T[rr * LB + j] : 0.f;
-        wR[t] = ok ? B.R[rr * LB + j] : 0.f;
-    }
-    bool bad = false;
-#pragma unroll 1
-    for (int s0 = 0; s0 < NSLOT; s0 += UW) {
-#pragma unroll
-        for (int k = 0; k < UW; ++k) {
-            const int r = s0 + k - j;
-            const bool inleaf = (r >= 0) && (r < LB);
-            const int rr = inleaf ? r : 0;
-            const bool act = inleaf && (r < rows) && colok;
-            float lo[LB];
-#pragma unroll
-            for (int q = 0; q < LB / 4; ++q) {
-                const float4 v = *reinterpret_cast<const float4*>(&B.LOr[rr * LS + 4 * q]);
-                lo[4 * q] = v.x; lo[4 * q + 1] = v.y; lo[4 * q + 2] = v.z; lo[4 * q + 3] = v.w;
-            }
-            const float w_star = B.W[rr * LB + j];
-            const float sr = B.S[rr], inv = B.S[LB + rr];
-            float e = 0.f, u = 0.f;
-            if (act) {
-                const float pre = w_star + wT[k] + wR[k];
-                float q = 0.f;
-                if (sr > 0.f) {
-                    float x = pre * inv;
-                    const float t = fabsf(x - rintf(x));
-                    if (0.5f - t < 1e-6f * fmaxf(1.f, fabsf(x))) x = __fdiv_rn(pre, sr);
-                    q = fminf(fmaxf(rintf(x), qlo), qhi);
-                }
-                bad |= !isfinite(pre);
-                const float w = sr * q;
-                e = w_star - w;
-                u = wT[k] + e;
-                B.oC[rr * LB + j] = (int8_t)q;
-                B.oW[rr * LB + j] = w;
-                B.oE[rr * LB + j] = e;
-                B.oEt[j * LB + rr] = e;
-                B.oU[rr * LB + j] = u;
-            }
-            wT[k + 1] = fmaf(lo[1], e, wT[k + 1]);
-            {
-                const float v = __shfl_up_sync(0xffffffffu, u, 1);
-                if (j >= 1) wR[k + 1] = fmaf(v, li[1], wR[k + 1]);
-            }
-#pragma unroll
-            for (int d = 2; d < LB; ++d) wT[k + d] = fmaf(lo[d], e, wT[k + d]);
-#pragma unroll
-            for (int d = 2; d < LB; ++d) {
-                const float v = __shfl_up_sync(0xffffffffu, u, d);
-                if (j >= d) wR[k + d] = fmaf(v, li[d], wR[k + d]);
-            }
-        }
-        // slide the window by UW slots
-#pragma unroll
-        for (int t = 0; t < WIN - UW; ++t) {
-            wT[t] = wT[t + UW];
-            wR[t] = wR[t + UW];
-        }
-#pragma unroll
-        for (int t = WIN - UW; t < WIN; ++t) {
-            const int r = s0 + UW + t - j;
-            const bool ok = (r >= 0) && (r < LB);
-            const int rr = ok ? r : 0;
-            wT[t] = ok ? B.T[rr * LB + j] : 0.f;
-            wR[t] = ok ? B.R[rr * LB + j] : 0.f;
-        }
-    }
-    if (bad) set_status(status, BAKRON_ERR_NONFINITE);
-}
 
 __device__ __forceinline__ void loader_sync() {
     asm volatile("bar.sync 1, %0;" ::"n"(NLOAD) : "memory");
@@ -231,10 +118,34 @@ struct TaskWalker {
     }
 };
 
-// Warps 0-3 stage leaf k into buffer k&1 (far sums, the in-block contributions of the leaves
-// above / left after a bounded wait on each one's ready flag, the diagonal blocks of L_O and
-// L_I) while warp 4 solves leaf k-1 from the other buffer and publishes it (outputs, planes,
-// release flag). The solver warp never runs the staging code and the loaders never run the
+// Codes, W and the E^T planes of the leaf solved from B (its E and U went out with its flag);
+// run by the 128 loader threads before they stage a new leaf into B.
+__device__ __forceinline__ void publish_rest(const PhaseArgs& a, const LeafBuf& B, int tid) {
+    const int I = B.meta[0], J = B.meta[1], rows = B.meta[2], cols = B.meta[3];
+    const int i0 = I * LB, j0 = J * LB;
+#pragma unroll
+    for (int q = 0; q < (LB * LB) / NLOAD; ++q) {
+        const int e = tid + q * NLOAD, r = e >> 5, c = e & 31;
+        if (r < rows && c < cols) {
+            const size_t o = (size_t)(i0 + r) * a.n + j0 + c;
+            a.codes[o] = B.oC[r * LB + c];
+            a.Wq[o] = B.oW[r * LB + c];
+        }
+        // E^T: element (c, r) of the transposed planes, lane = row for coalescing
+        if (c < rows && r < cols) {
+            const float x = B.oEt[r * LB + c], xh = sm100::tf32_hi(x);
+            const size_t ot = (size_t)(j0 + r) * a.ldm + i0 + c;
+            a.et_hi[ot] = xh;
+            a.et_lo[ot] = x - xh;
+        }
+    }
+}
+
+// Warps 0-3 stage leaf k into buffer k&1 (W*, the diagonal blocks of L_O and L_I, then the far
+// sums plus the in-block contributions of the leaves above / left, each after a bounded wait
+// on that leaf's ready flag) while warp 4 solves leaf k-1 from the other buffer and publishes
+// what other leaves read (E, U) followed by its release flag; before restaging a buffer the
+// loaders publish the rest of the leaf solved from it (codes, W, E^T planes). The solver warp never runs the staging code and the loaders never run the
 // solver, so each keeps its own instruction stream.
 __global__ void __launch_bounds__(NTHW, 1) phase_leaves_kernel(PhaseArgs a) {
     extern __shared__ __align__(16) uint8_t leaf_smem_raw[];
@@ -267,6 +178,8 @@ __global__ void __launch_bounds__(NTHW, 1) phase_leaves_kernel(PhaseArgs a) {
                 }
                 loader_sync();
                 if (*(volatile int*)&sm.stop) break;
+                publish_rest(a, B, tid);   // leaf k - 2, solved from this buffer
+                loader_sync();             // its meta is read before it is overwritten
             }
             int I, J;
             wk.find(a, g, I, J);
@@ -283,6 +196,28 @@ __global__ void __launch_bounds__(NTHW, 1) phase_leaves_kernel(PhaseArgs a) {
                 accT[t] = ok ? __ldcg(&a.Tf[o]) : 0.f;
                 accR[t] = ok ? __ldcg(&a.Rf[o]) : 0.f;
             }
+            // what does not depend on other leaves first: W*, the diagonal blocks of L_O and
+            // L_I, the scales (sA / sB are free again after the skew below)
+#pragma unroll
+            for (int q = 0; q < (LB * LB) / NLOAD; ++q) {
+                const int e = tid + q * NLOAD, r = e >> 5, c = e & 31;
+                B.W[e] = (r < rows && c < cols) ? __ldg(&a.Ws[(size_t)(i0 + r) * n + j0 + c]) : 0.f;
+                sm.sA[r][c] = (r < rows && c < rows) ? __ldg(&a.LO[(size_t)(i0 + r) * m + i0 + c]) : 0.f;
+                sm.sB[r][c] = (r < cols && c < cols) ? __ldg(&a.LI[(size_t)(j0 + r) * n + j0 + c]) : 0.f;
+            }
+            if (tid < LB) {
+                const float sv = (tid < rows) ? __ldg(&a.sc[i0 + tid]) : 0.f;
+                B.S[tid] = sv;
+                B.S[LB + tid] = sv > 0.f ? __frcp_rn(sv) : 0.f;
+            }
+            if (tid == 0) { B.meta[0] = I; B.meta[1] = J; B.meta[2] = rows; B.meta[3] = cols; }
+            loader_sync();
+            for (int e = tid; e < LB * LS; e += NLOAD) {
+                const int x = e / LS, dd = e % LS;
+                B.LOr[e] = (dd >= 1 && dd < LB && x + dd < LB) ? sm.sA[x][x + dd] : 0.f;
+                B.LIc[e] = (dd >= 1 && dd < LB && x - dd >= 0) ? sm.sB[x - dd][x] : 0.f;
+            }
+            loader_sync();
             bool stop = false;
             // In-block sources: the leaves above (vertical, via E) and to the left (horizontal,
             // via U). The two most recent ones, (la-1, lc) and (la, lc-1), finish last, so every
@@ -339,30 +274,11 @@ __global__ void __launch_bounds__(NTHW, 1) phase_leaves_kernel(PhaseArgs a) {
                 loader_sync();
             }
             if (stop) break;
-            // stage the leaf into buffer b
+            // the far and in-block sums
 #pragma unroll
             for (int t = 0; t < 8; ++t) {
                 B.T[(warp * 8 + t) * LB + lane] = accT[t];
                 B.R[(warp * 8 + t) * LB + lane] = accR[t];
-            }
-#pragma unroll
-            for (int q = 0; q < (LB * LB) / NLOAD; ++q) {
-                const int e = tid + q * NLOAD, r = e >> 5, c = e & 31;
-                B.W[e] = (r < rows && c < cols) ? __ldg(&a.Ws[(size_t)(i0 + r) * n + j0 + c]) : 0.f;
-                sm.sA[r][c] = (r < rows && c < rows) ? __ldg(&a.LO[(size_t)(i0 + r) * m + i0 + c]) : 0.f;
-                sm.sB[r][c] = (r < cols && c < cols) ? __ldg(&a.LI[(size_t)(j0 + r) * n + j0 + c]) : 0.f;
-            }
-            if (tid < LB) {
-                const float sv = (tid < rows) ? __ldg(&a.sc[i0 + tid]) : 0.f;
-                B.S[tid] = sv;
-                B.S[LB + tid] = sv > 0.f ? __frcp_rn(sv) : 0.f;
-            }
-            if (tid == 0) { B.meta[0] = I; B.meta[1] = J; B.meta[2] = rows; B.meta[3] = cols; }
-            loader_sync();
-            for (int e = tid; e < LB * LS; e += NLOAD) {
-                const int x = e / LS, dd = e % LS;
-                B.LOr[e] = (dd >= 1 && dd < LB && x + dd < LB) ? sm.sA[x][x + dd] : 0.f;
-                B.LIc[e] = (dd >= 1 && dd < LB && x - dd >= 0) ? sm.sB[x - dd][x] : 0.f;
             }
             loader_sync();
             if (tid == 0) {
@@ -373,6 +289,20 @@ __global__ void __launch_bounds__(NTHW, 1) phase_leaves_kernel(PhaseArgs a) {
         if (tid == 0) {
             // loaders ended early: let the solver warp see it
             if (*(volatile int*)&sm.stop) atomicExch(a.abort_word, 1);
+        }
+        // the last (up to) two leaves: wait until they are solved, then publish the rest
+        if (!*(volatile int*)&sm.stop) {
+            for (int kk = (k >= 2 ? k - 2 : 0); kk < k; ++kk) {
+                const int b = kk & 1;
+                if (tid == 0 && !sm100::mbar_wait(&sm.empty[b], (kk >> 1) & 1, a.status,
+                                                  a.limit_ns)) {
+                    atomicExch(a.abort_word, 1);
+                    sm.stop = 1;
+                }
+                loader_sync();
+                if (*(volatile int*)&sm.stop) break;
+                publish_rest(a, sm.buf[b], tid);
+            }
         }
     } else {
         // ------------------------------------------------------------ solver warp
@@ -391,25 +321,16 @@ __global__ void __launch_bounds__(NTHW, 1) phase_leaves_kernel(PhaseArgs a) {
             const int i0 = I * LB, j0 = J * LB;
             solve_leaf(lane, rows, cols, a.qlo, a.qhi, B, a.status);
             __syncwarp();
-            // publish: lane = column for row-major outputs, lane = row for the E^T planes
+            // publish what other leaves read (E for the vertical pulls, U for the horizontal
+            // ones), then the flag; codes, W and the E^T planes follow from the loader warps
             if (lane < cols) {
                 for (int r = 0; r < rows; ++r) {
                     const size_t o = (size_t)(i0 + r) * n + j0 + lane;
-                    a.codes[o] = B.oC[r * LB + lane];
-                    a.Wq[o] = B.oW[r * LB + lane];
                     __stcg(&a.E[o], B.oE[r * LB + lane]);
                     const float u = B.oU[r * LB + lane], uh = sm100::tf32_hi(u);
                     const size_t ou = (size_t)(i0 + r) * a.ldn + j0 + lane;
                     __stcg(&a.u_hi[ou], uh);
                     __stcg(&a.u_lo[ou], u - uh);
-                }
-            }
-            if (lane < rows) {
-                for (int c = 0; c < cols; ++c) {
-                    const float x = B.oEt[c * LB + lane], xh = sm100::tf32_hi(x);
-                    const size_t ot = (size_t)(j0 + c) * a.ldm + i0 + lane;
-                    a.et_hi[ot] = xh;
-                    a.et_lo[ot] = x - xh;
                 }
             }
             __threadfence();

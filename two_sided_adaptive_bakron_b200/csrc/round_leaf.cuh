@@ -1,0 +1,131 @@
+// round_leaf.cuh -- the in-leaf wavefront of the BaKron solve (one warp, 32 x 32 leaf).
+//
+// YAQA article, section 4, rounding rule, with U = (I + L_O)^T E:
+//   pre_ij = W*_ij + T_ij + R_ij,  T_ij = sum_{k<i} L_O[k,i] E_kj,  R_ij = sum_{l<j} U_il L_I[l,j],
+//   W_ij = s_i clamp(rint(pre_ij / s_i)),  E_ij = W*_ij - W_ij,  U_ij = T_ij + E_ij.
+// T and R arrive holding everything from outside the leaf; the wavefront adds the in-leaf part.
+#pragma once
+
+#include "sm100.cuh"
+
+namespace bakron {
+namespace leaf {
+
+constexpr int LB = 32;          // leaf edge
+constexpr int NSLOT = 2 * LB - 1;
+constexpr int UW = 4;            // wavefront steps per unrolled group
+constexpr int WIN = LB + UW;     // register window of slots
+constexpr int LS = LB + 4;       // row stride of the skewed diagonal blocks (16-byte rows)
+
+// One staging buffer: a leaf's inputs and outputs (shared memory, floats).
+struct LeafBuf {
+    float W[LB * LB];            // W* of the leaf, row stride LB
+    float T[LB * LB];            // vertical sums (everything above the leaf)
+    float R[LB * LB];            // horizontal sums (everything left of the leaf)
+    float LOr[LB * LS];          // LOr[r*LS + d] = L_O[i0+r][i0+r+d]
+    float LIc[LB * LS];          // LIc[c*LS + d] = L_I[j0+c-d][j0+c]
+    float S[2 * LB];             // s_r and its reciprocal
+    float oW[LB * LB], oE[LB * LB], oU[LB * LB];
+    float oEt[LB * LB];          // E transposed (for the transposed planes)
+    int8_t oC[LB * LB];
+    int meta[4];                 // I, J, rows, cols
+};
+
+
+// The in-leaf wavefront, run by the solver warp; lane j owns column j and the element of row
+// r is handled at step s = r + j. Leaf arrays use row stride LB, element (r, c) at r*LB + c,
+// so an anti-diagonal and a row both touch 32 distinct banks. Per lane, slot s of wT / wR
+// holds the vertical / horizontal sum of its element of step s. A step reads slot s, then
+// pushes E down its column into slots s+1..s+31 (in-lane) and U along its row into slot s+d
+// of lane j+d (warp shuffles); the d = 1 pushes, the only ones the next step needs, go
+// first. LIc is zero for d > j and LOr for r + d >= 32, so no push needs a guard: a lane
+// j < d gets its own u back from the shuffle and multiplies it by zero. The step loop stays rolled (4 steps per iteration) over a sliding window of 36
+// slot registers: every register index is static and the code stays small.
+// Q divides by s_r as one correctly rounded fp32 division; the quotient is formed as
+// pre * (1/s_r), whose distance to the division's result is below 2e-7 |x|, and the exact
+// division is taken instead whenever that quotient lies within 1e-6 max(1,|x|) of a rounding
+// boundary, so the decision always equals the division's.
+__device__ __forceinline__ void solve_leaf(int lane, int rows, int cols, float qlo, float qhi,
+                                           LeafBuf& B, int* status) {
+    const int j = lane;
+    const bool colok = j < cols;
+    float li[LB];
+#pragma unroll
+    for (int q = 0; q < LB / 4; ++q) {
+        const float4 v = *reinterpret_cast<const float4*>(&B.LIc[j * LS + 4 * q]);
+        li[4 * q] = v.x; li[4 * q + 1] = v.y; li[4 * q + 2] = v.z; li[4 * q + 3] = v.w;
+    }
+    float wT[WIN], wR[WIN];
+#pragma unroll
+    for (int t = 0; t < WIN; ++t) {
+        const int r = t - j;
+        const bool ok = (r >= 0) && (r < LB);
+        const int rr = ok ? r : 0;
+        wT[t] = ok ? B.T[rr * LB + j] : 0.f;
+        wR[t] = ok ? B.R[rr * LB + j] : 0.f;
+    }
+    bool bad = false;
+#pragma unroll 1
+    for (int s0 = 0; s0 < NSLOT; s0 += UW) {
+#pragma unroll
+        for (int k = 0; k < UW; ++k) {
+            const int r = s0 + k - j;
+            const bool inleaf = (r >= 0) && (r < LB);
+            const int rr = inleaf ? r : 0;
+            const bool act = inleaf && (r < rows) && colok;
+            float lo[LB];
+#pragma unroll
+            for (int q = 0; q < LB / 4; ++q) {
+                const float4 v = *reinterpret_cast<const float4*>(&B.LOr[rr * LS + 4 * q]);
+                lo[4 * q] = v.x; lo[4 * q + 1] = v.y; lo[4 * q + 2] = v.z; lo[4 * q + 3] = v.w;
+            }
+            const float w_star = B.W[rr * LB + j];
+            const float sr = B.S[rr], inv = B.S[LB + rr];
+            float e = 0.f, u = 0.f;
+            if (act) {
+                const float pre = w_star + wT[k] + wR[k];
+                float q = 0.f;
+                if (sr > 0.f) {
+                    float x = pre * inv;
+                    const float t = fabsf(x - rintf(x));
+                    if (0.5f - t < 1e-6f * fmaxf(1.f, fabsf(x))) x = __fdiv_rn(pre, sr);
+                    q = fminf(fmaxf(rintf(x), qlo), qhi);
+                }
+                bad |= !isfinite(pre);
+                const float w = sr * q;
+                e = w_star - w;
+                u = wT[k] + e;
+                B.oC[rr * LB + j] = (int8_t)q;
+                B.oW[rr * LB + j] = w;
+                B.oE[rr * LB + j] = e;
+                B.oEt[j * LB + rr] = e;
+                B.oU[rr * LB + j] = u;
+            }
+            wT[k + 1] = fmaf(lo[1], e, wT[k + 1]);
+            wR[k + 1] = fmaf(__shfl_up_sync(0xffffffffu, u, 1), li[1], wR[k + 1]);
+#pragma unroll
+            for (int d = 2; d < LB; ++d) wT[k + d] = fmaf(lo[d], e, wT[k + d]);
+#pragma unroll
+            for (int d = 2; d < LB; ++d)
+                wR[k + d] = fmaf(__shfl_up_sync(0xffffffffu, u, d), li[d], wR[k + d]);
+        }
+        // slide the window by UW slots
+#pragma unroll
+        for (int t = 0; t < WIN - UW; ++t) {
+            wT[t] = wT[t + UW];
+            wR[t] = wR[t + UW];
+        }
+#pragma unroll
+        for (int t = WIN - UW; t < WIN; ++t) {
+            const int r = s0 + UW + t - j;
+            const bool ok = (r >= 0) && (r < LB);
+            const int rr = ok ? r : 0;
+            wT[t] = ok ? B.T[rr * LB + j] : 0.f;
+            wR[t] = ok ? B.R[rr * LB + j] : 0.f;
+        }
+    }
+    if (bad) set_status(status, BAKRON_ERR_NONFINITE);
+}
+
+}  // namespace leaf
+}  // namespace bakron
