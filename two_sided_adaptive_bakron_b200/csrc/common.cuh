@@ -81,6 +81,29 @@ __device__ __forceinline__ bool wait_flag(const int* flag, int* abort_word, int*
     }
 }
 
+// Bounded wait until *counter >= target; same give-up rules as wait_flag.
+__device__ __forceinline__ bool wait_geq(const int* counter, int target, int* abort_word,
+                                         int* status, uint64_t limit_ns) {
+    if (ld_acquire_gpu(counter) >= target) return true;
+    const uint64_t t0 = globaltimer_ns();
+    unsigned ns = 32;
+    while (true) {
+        if (ld_acquire_gpu(counter) >= target) return true;
+        if (ld_acquire_gpu(abort_word) != 0) return false;
+        if (globaltimer_ns() - t0 > limit_ns) {
+            set_status(status, BAKRON_ERR_TIMEOUT);
+            atomicExch(abort_word, 1);
+            return false;
+        }
+        __nanosleep(ns);
+        if (ns < 256) ns <<= 1;
+    }
+}
+
+__device__ __forceinline__ void red_add_release_gpu(int* p, int v) {
+    asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
 // Default limit of one dependency wait; BAKRON_SPIN_LIMIT_NS in the environment overrides it
 // (used by the tests to exercise the timeout path without hanging anything).
 uint64_t spin_limit_ns();

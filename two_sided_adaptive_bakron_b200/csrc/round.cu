@@ -13,21 +13,31 @@
 // a vertical sum over E (rows above) and a horizontal sum over U (columns to the left); the
 // bilinear term a_i^T E[:i,:j] b_j is carried by U.
 //
-// Structure. The matrix is cut into 256 x 256 super-blocks, processed one super-block
-// anti-diagonal ("phase") at a time; the blocks of a phase are independent of each other.
-//  * Leaf launch (persistent, cooperative, one CTA per SM): every block of the phase is cut
-//    into 32 x 32 leaves, taken in anti-diagonal order across all blocks of the phase, round
-//    robin over the CTAs. In each CTA four loader warps stage a leaf: the far sums T_far,
-//    R_far (everything outside its block, already accumulated) plus the contributions of the
-//    leaves above / to the left inside its block (CUDA-core dot products, after a bounded wait
-//    on each source leaf's ready flag). A fifth, solver warp runs the in-leaf wavefront of the
-//    previous leaf meanwhile (two staging buffers, mbarrier handoff) and publishes it: codes,
-//    W, E (row-major), E^T and U as hi/lo planes, then the leaf's release flag.
-//  * Push launches (3xTF32 tcgen05 GEMMs, one grouped launch per direction): every block of
-//    the phase pushes its E into T_far of all rows below it and its U into R_far of all
-//    columns to its right (K = 256), i.e. the divide-and-conquer off-diagonal updates as dense
-//    block products.
+// Structure: one persistent cooperative launch over the whole matrix, cut into 32 x 32 leaves
+// and 256 x 256 super-blocks, with two kinds of CTAs.
+//  * Leaf CTAs take the leaves in anti-diagonal order (round robin over two groups per CTA:
+//    two loader warps and one solver warp each). A leaf's sums come in two parts. The near
+//    field, the leaves above / to the left inside its own super-block and the adjacent one, is
+//    pulled by the loaders on CUDA cores after a bounded wait on each source leaf's flag. The
+//    far field, everything at least two super-blocks away, is read from T_far / R_far once the
+//    leaf's 128 x 128 tile counters say that every far source has been added. The solver warp
+//    runs the in-leaf wavefront (round_leaf.cuh), publishes E and U, releases the leaf's flag,
+//    then publishes the E^T planes and counts the leaf into its super-block.
+//  * GEMM CTAs run the far-field pushes as 3xTF32 tcgen05 tile tasks (128 x 128, K = one
+//    super-block): E of super-block (A', C) into T_far of a target (A, C) with A >= A' + 2, and
+//    U of (A, C') into R_far of (A, C) with C >= C' + 2, i.e. the divide-and-conquer
+//    off-diagonal products as dense block products. Tasks are ordered by their source
+//    super-block in the order the sources finish (anti-diagonal, then row), nearest targets
+//    first; each output tile takes its sources in increasing order (a per-tile counter), so
+//    sums are deterministic, and a tile's successive sources are one super-block apart in
+//    time, so that order rarely has to wait.
+// Every task depends only on tasks that come earlier in one global order (leaves by
+// anti-diagonal, the pushes of a super-block right after its last leaf and before the first
+// leaf two super-blocks on), so the persistent CTAs always make progress; every wait is
+// bounded and ends the launch through a shared abort word when it expires.
 #include <algorithm>
+#include <cstddef>
+#include <cstring>
 
 #include "round_leaf.cuh"
 #include "tcgemm_host.cuh"
@@ -36,20 +46,27 @@ namespace bakron {
 namespace {
 
 using leaf::LB;
-constexpr int SB = 256;         // super-block edge
-constexpr int LPB = SB / LB;    // leaves per super-block edge
+using leaf::LeafBuf;
+using leaf::LS;
+using leaf::solve_leaf;
+
+constexpr int SB = 256;              // super-block edge
+constexpr int LPB = SB / LB;         // leaves per super-block edge
+constexpr int TB = tc::BM;           // push tile edge (128)
 constexpr int BN = 128;
 constexpr int STAGES = 3;
+constexpr int NTH = 192;             // 6 warps in both roles
+constexpr int NLOAD = 64;            // loader threads of one leaf group
+constexpr int LPAD = LB + 4;         // staging row stride (16-byte rows)
+constexpr int kMaxLeafCtas = 96;
+static_assert(TB % LB == 0 && SB % TB == 0, "tile nesting");
 
-struct PhaseArgs {
+struct FusedArgs {
     const float* Ws;
     const float* LO;
     const float* LI;
     const float* sc;
-    const float* Tf;
-    const float* Rf;
-    int m, n, Nt;
-    int delta, p_lo, p_hi, maxd;
+    int m, n;
     float qlo, qhi;
     int8_t* codes;
     float* Wq;
@@ -60,291 +77,785 @@ struct PhaseArgs {
     float* u_hi;
     float* u_lo;
     int ldn;
-    int* flags;
+    float* Tf;
+    float* Rf;
+    float* Ut;           // U^T in full precision (n x ldm), read by the horizontal pulls
+    int box_loads;       // 1: the leaf loaders read through the LeafMaps box maps
+    int* flags;          // [Mt * Nt] leaf solved (E and U published)
+    int* sb_done;        // [MS * NS] leaves of the super-block with E^T published
+    int* cntT;           // [TM * TN] far sources added into the T_far tile
+    int* cntR;           // [TM * TN] far sources added into the R_far tile
     int* abort_word;
     int* status;
+    const int* task_pre; // [nsb + 1] first push task of each source super-block (in order)
+    const int2* task_sb; // [nsb] (A, C) of the source super-blocks, anti-diagonal order
+    int nsb;
+    int Mt, Nt, MS, NS, TN;
+    int leaf_ctas;
     uint64_t limit_ns;
-    int total;
 };
 
-__device__ __forceinline__ int leaves_of(int extent, int blk) {
-    const int e = min(SB, extent - blk * SB);
-    return (e + LB - 1) / LB;
-}
+// 32 x 32 fp32 box maps (no swizzle) of the matrices a leaf reads; only valid when m and n are
+// multiples of 4 (16-byte row strides), otherwise the loaders use plain loads.
+struct LeafMaps {
+    CUtensorMap lo;   // L_O (m x m)
+    CUtensorMap li;   // L_I (n x n)
+    CUtensorMap e;    // E (m x n)
+    CUtensorMap ut;   // U^T (n x m, row stride ldm)
+    CUtensorMap ws;   // W* (m x n)
+    CUtensorMap tf;   // T_far (m x n)
+    CUtensorMap rf;   // R_far (m x n)
+};
 
-// number of leaves (a, c) with a + c = d in a block of lm x ln leaves
-__device__ __forceinline__ int diag_len(int d, int lm, int ln) {
-    const int lo = max(0, d - ln + 1), hi = min(d, lm - 1);
-    return hi >= lo ? hi - lo + 1 : 0;
-}
+constexpr int NRING = 4;             // sources in flight per leaf group (box-load path)
+constexpr int kBox = LB * LB;        // floats of one 32 x 32 box
 
-constexpr int NLOAD = 128;       // loader threads (warps 0-3)
-constexpr int NTHW = NLOAD + 32; // + the solver warp (warp 4)
-using leaf::LS;
-using leaf::LeafBuf;
-using leaf::solve_leaf;
-
-struct LeafSmem {
+struct alignas(128) LeafGroupSmem {
     LeafBuf buf[2];
-    float sA[LB][LB + 1];        // pull staging
-    float sB[LB][LB + 1];
+    // box-load path: NRING stages of two boxes; plain path: sA, sB with row stride LPAD
+    alignas(128) float ring[NRING][2][kBox];
+    uint64_t rfull[NRING];       // box loads of a ring stage landed
+    uint64_t sbar;               // W* and the diagonal blocks landed
+    uint64_t tbar;               // T_far and R_far landed
     uint64_t full[2], empty[2];
     int stop;
 };
+struct LeafCtaSmem {
+    LeafGroupSmem g[2];
+};
+static_assert(sizeof(LeafGroupSmem) % 128 == 0 && offsetof(LeafGroupSmem, buf) % 128 == 0 &&
+                  offsetof(LeafGroupSmem, ring) % 128 == 0 && (LPAD * 4) % 16 == 0 &&
+                  2 * LB * LPAD <= NRING * 2 * kBox,
+              "leaf group layout: 16-byte staging rows, 128-byte box destinations");
 
-__device__ __forceinline__ void loader_sync() {
-    asm volatile("bar.sync 1, %0;" ::"n"(NLOAD) : "memory");
+constexpr size_t kGemmSmem = tc::gemm_smem_bytes<BN, STAGES>();
+constexpr size_t kLeafSmem = sizeof(LeafCtaSmem) + 128;   // + alignment slack
+constexpr size_t kSmem = kLeafSmem > kGemmSmem ? kLeafSmem : kGemmSmem;
+static_assert(kSmem <= 227 * 1024, "shared memory above the per-CTA limit");
+
+__device__ __forceinline__ int leaves_in(int extent_leaves, int blk) {
+    return min(LPB, extent_leaves - blk * LPB);
 }
 
-// Walks the phase's tasks: (local anti-diagonal d, block row P) in order, counting leaves.
-struct TaskWalker {
-    int d, P;
+// Walks the leaves in anti-diagonal order (d = I + J, then I); g must not decrease.
+struct LeafWalker {
+    int d;
     long long base;
-    __device__ void init(int p_lo) { d = 0; P = p_lo; base = 0; }
-    __device__ void find(const PhaseArgs& a, int g, int& I, int& J) {
-        int ln;
+    __device__ void init() { d = 0; base = 0; }
+    __device__ void find(int Mt, int Nt, long long g, int& I, int& J) {
         while (true) {
-            const int Q = a.delta - P;
-            const int lm = leaves_of(a.m, P);
-            ln = leaves_of(a.n, Q);
-            const int cnt = diag_len(d, lm, ln);
-            if (g < base + cnt) break;
+            const int lo = max(0, d - Nt + 1), hi = min(d, Mt - 1);
+            const int cnt = hi - lo + 1;
+            if (g < base + cnt) {
+                I = lo + (int)(g - base);
+                J = d - I;
+                return;
+            }
             base += cnt;
-            if (++P > a.p_hi) { P = a.p_lo; ++d; }
+            ++d;
         }
-        const int la = max(0, d - ln + 1) + (int)(g - base);
-        I = P * LPB + la;
-        J = (a.delta - P) * LPB + (d - la);
     }
 };
 
-// Codes, W and the E^T planes of the leaf solved from B (its E and U went out with its flag);
-// run by the 128 loader threads before they stage a new leaf into B.
-__device__ __forceinline__ void publish_rest(const PhaseArgs& a, const LeafBuf& B, int tid) {
+__device__ __forceinline__ void group_sync(int g) {
+    asm volatile("bar.sync %0, %1;" ::"r"(1 + g), "n"(NLOAD) : "memory");
+}
+
+// Codes and W of the leaf solved from B (W = s_r q, formed as in the solver); run by the
+// group's loader threads before they stage a new leaf into B.
+__device__ __forceinline__ void publish_rest(const FusedArgs& a, const LeafBuf& B, int lt) {
     const int I = B.meta[0], J = B.meta[1], rows = B.meta[2], cols = B.meta[3];
     const int i0 = I * LB, j0 = J * LB;
-#pragma unroll
+#pragma unroll 4
     for (int q = 0; q < (LB * LB) / NLOAD; ++q) {
-        const int e = tid + q * NLOAD, r = e >> 5, c = e & 31;
+        const int e = lt + q * NLOAD, r = e >> 5, c = e & 31;
         if (r < rows && c < cols) {
             const size_t o = (size_t)(i0 + r) * a.n + j0 + c;
-            a.codes[o] = B.oC[r * LB + c];
-            a.Wq[o] = B.oW[r * LB + c];
-        }
-        // E^T: element (c, r) of the transposed planes, lane = row for coalescing
-        if (c < rows && r < cols) {
-            const float x = B.oEt[r * LB + c], xh = sm100::tf32_hi(x);
-            const size_t ot = (size_t)(j0 + r) * a.ldm + i0 + c;
-            a.et_hi[ot] = xh;
-            a.et_lo[ot] = x - xh;
+            const int8_t q = B.oC[r * LB + c];
+            a.codes[o] = q;
+            a.Wq[o] = B.S[r] * (float)q;
         }
     }
 }
 
-// Warps 0-3 stage leaf k into buffer k&1 (W*, the diagonal blocks of L_O and L_I, then the far
-// sums plus the in-block contributions of the leaves above / left, each after a bounded wait
-// on that leaf's ready flag) while warp 4 solves leaf k-1 from the other buffer and publishes
-// what other leaves read (E, U) followed by its release flag; before restaging a buffer the
-// loaders publish the rest of the leaf solved from it (codes, W, E^T planes). The solver warp never runs the staging code and the loaders never run the
-// solver, so each keeps its own instruction stream.
-__global__ void __launch_bounds__(NTHW, 1) phase_leaves_kernel(PhaseArgs a) {
-    extern __shared__ __align__(16) uint8_t leaf_smem_raw[];
-    LeafSmem& sm = *reinterpret_cast<LeafSmem*>(leaf_smem_raw);
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+// acc[i][j] += sum_k X[k][r0 + i] Y[k][c0 + j]: one source's contribution to a 4 x 4 block
+// (X, Y with row stride LD floats)
+template <int LD>
+__device__ __forceinline__ void product_4x4(const float* X, const float* Y, int r0, int c0,
+                                            float (&acc)[4][4]) {
+#pragma unroll 8
+    for (int kk = 0; kk < LB; ++kk) {
+        const float4 x = *reinterpret_cast<const float4*>(&X[kk * LD + r0]);
+        const float4 y = *reinterpret_cast<const float4*>(&Y[kk * LD + c0]);
+        const float xa[4] = {x.x, x.y, x.z, x.w}, ya[4] = {y.x, y.y, y.z, y.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(xa[i], ya[j], acc[i][j]);
+    }
+}
+
+// The near-field sources of leaf (I, J) in super-block (A, C): the leaves above in this and the
+// adjacent super-block (vertical, via E) and to the left (horizontal, via U); the older ones
+// first, (I-1, J) and (I, J-1), which finish last, close the list.
+struct NearField {
+    int I, J, va, ha, nvs, nhs, nv, nh, nold, nsrc;
+    __device__ NearField(int I_, int J_, int A, int C) : I(I_), J(J_) {
+        va = max(0, (A - 1) * LPB);
+        ha = max(0, (C - 1) * LPB);
+        nvs = I - va;
+        nhs = J - ha;
+        nv = max(nvs - 1, 0);
+        nh = max(nhs - 1, 0);
+        nold = nv + nh;
+        nsrc = nvs + nhs;
+    }
+    __device__ bool source(int idx, int& Is, int& Js) const {   // true: vertical
+        if (idx < nv) { Is = va + idx; Js = J; return true; }
+        if (idx < nold) { Is = I; Js = ha + (idx - nv); return false; }
+        if (idx == nold && nvs > 0) { Is = I - 1; Js = J; return true; }
+        Is = I; Js = J - 1;
+        return false;
+    }
+};
+
+// ------------------------------------------------------------------------------ leaf loaders
+// The two loader warps of group g stage leaf k into buffer k & 1: W*, the diagonal blocks of
+// L_O and L_I and the scales first, then (after the far-field counters) T_far / R_far plus the
+// near-field contributions (one 32 x 32 x 32 product per source on CUDA cores). With box
+// loads, one thread keeps NRING sources in flight through a ring of shared-memory stages.
+__device__ void leaf_loaders(const FusedArgs& a, const LeafMaps* maps, LeafGroupSmem& sm, int g,
+                             int lw, int lane, int slot, int nslots) {
+    const int lt = lw * 32 + lane;
+    const bool lead = lt == 0;
     const int m = a.m, n = a.n;
-    if (tid == 0) {
-        for (int b = 0; b < 2; ++b) {
-            sm100::mbar_init(&sm.full[b], 1);
-            sm100::mbar_init(&sm.empty[b], 1);
+    const long long total = (long long)a.Mt * a.Nt;
+    const bool box = a.box_loads != 0;
+    float* sA = &sm.ring[0][0][0];              // plain path staging
+    float* sB = sA + LB * LPAD;
+    LeafWalker wk;
+    wk.init();
+    uint32_t rq = 0;                             // ring stages used so far (box path)
+    int k = 0;
+    for (long long gi = slot; gi < total; gi += nslots, ++k) {
+        const int b = k & 1;
+        LeafBuf& B = sm.buf[b];
+        if (k >= 2) {
+            if (lead && !sm100::mbar_wait(&sm.empty[b], ((k >> 1) - 1) & 1, a.status, a.limit_ns)) {
+                atomicExch(a.abort_word, 1);
+                sm.stop = 1;
+            }
+            group_sync(g);
+            if (*(volatile int*)&sm.stop) break;
+            publish_rest(a, B, lt);   // leaf k - 2, solved from this buffer
+            group_sync(g);            // its meta is read before it is overwritten
         }
-        sm.stop = 0;
+        int I, J;
+        wk.find(a.Mt, a.Nt, gi, I, J);
+        const int A = I / LPB, C = J / LPB;
+        const int i0 = I * LB, j0 = J * LB;
+        const int rows = min(LB, m - i0), cols = min(LB, n - j0);
+        // what does not depend on other leaves: W*, the diagonal blocks, the scales
+        const float* dLO;                        // diagonal blocks, row stride dld
+        const float* dLI;
+        int dld;
+        if (box) {
+            if (lead) {
+                sm100::mbar_arrive_expect_tx(&sm.sbar, 3 * kBox * 4);
+                sm100::tma_load_2d(B.W, &maps->ws, j0, i0, &sm.sbar);
+                sm100::tma_load_2d(sm.ring[0][0], &maps->lo, i0, i0, &sm.sbar);
+                sm100::tma_load_2d(sm.ring[0][1], &maps->li, j0, j0, &sm.sbar);
+            }
+            dLO = sm.ring[0][0];
+            dLI = sm.ring[0][1];
+            dld = LB;
+        } else {
+#pragma unroll 4
+            for (int q = 0; q < (LB * LB) / NLOAD; ++q) {
+                const int e = lt + q * NLOAD, r = e >> 5, c = e & 31;
+                B.W[e] = (r < rows && c < cols) ? __ldg(&a.Ws[(size_t)(i0 + r) * n + j0 + c]) : 0.f;
+                sA[r * LPAD + c] = (r < rows && c < rows) ? __ldg(&a.LO[(size_t)(i0 + r) * m + i0 + c]) : 0.f;
+                sB[r * LPAD + c] = (r < cols && c < cols) ? __ldg(&a.LI[(size_t)(j0 + r) * n + j0 + c]) : 0.f;
+            }
+            dLO = sA;
+            dLI = sB;
+            dld = LPAD;
+        }
+        if (lt < LB) {
+            const float sv = (lt < rows) ? __ldg(&a.sc[i0 + lt]) : 0.f;
+            B.S[lt] = sv;
+            B.S[LB + lt] = sv > 0.f ? __frcp_rn(sv) : 0.f;
+        }
+        if (lead) { B.meta[0] = I; B.meta[1] = J; B.meta[2] = rows; B.meta[3] = cols; }
+        // far field: every super-block at least two steps above / to the left has been added
+        if (lead) {
+            const int tile = (I * LB / TB) * a.TN + (J * LB / TB);
+            bool ok = true;
+            if (A >= 2) ok = wait_geq(&a.cntT[tile], A - 1, a.abort_word, a.status, a.limit_ns);
+            if (ok && C >= 2) ok = wait_geq(&a.cntR[tile], C - 1, a.abort_word, a.status, a.limit_ns);
+            if (ok && box) {
+                // T_far / R_far were written through the generic proxy on other SMs
+                asm volatile("fence.proxy.async.global;" ::: "memory");
+                sm100::mbar_arrive_expect_tx(&sm.tbar, 2 * kBox * 4);
+                sm100::tma_load_2d(B.T, &maps->tf, j0, i0, &sm.tbar);
+                sm100::tma_load_2d(B.R, &maps->rf, j0, i0, &sm.tbar);
+            }
+            if (ok && box && !sm100::mbar_wait(&sm.sbar, k & 1, a.status, a.limit_ns)) ok = false;
+            sm.stop = ok ? 0 : 1;
+        }
+        group_sync(g);
+        if (*(volatile int*)&sm.stop) break;
+        for (int e = lt; e < LB * LS; e += NLOAD) {
+            const int x = e / LS, dd = e % LS;
+            B.LOr[e] = (dd >= 1 && dd < LB && x + dd < LB) ? dLO[x * dld + x + dd] : 0.f;
+            B.LIc[e] = (dd >= 1 && dd < LB && x - dd >= 0) ? dLI[(x - dd) * dld + x] : 0.f;
+        }
+        // this thread's 4 x 4 block of the leaf's sums
+        const int r0 = (lt >> 3) * 4, c0 = (lt & 7) * 4;
+        float accT[4][4], accR[4][4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                float t = 0.f, r = 0.f;
+                if (!box) {
+                    const bool ok = r0 + i < rows && c0 + j < cols;
+                    const size_t o = (size_t)(i0 + r0 + i) * n + j0 + c0 + j;
+                    t = ok ? __ldcg(&a.Tf[o]) : 0.f;
+                    r = ok ? __ldcg(&a.Rf[o]) : 0.f;
+                }
+                accT[i][j] = t;
+                accR[i][j] = r;
+            }
+        const NearField nf(I, J, A, C);
+        // the older sources finished at least a diagonal ago: warp 0's lanes check their flags
+        if (lw == 0) {
+            bool ok = true;
+            for (int idx = lane; idx < nf.nold && ok; idx += 32) {
+                int Is, Js;
+                nf.source(idx, Is, Js);
+                ok = wait_flag(&a.flags[(size_t)Is * a.Nt + Js], a.abort_word, a.status, a.limit_ns);
+            }
+            ok = __all_sync(0xffffffffu, ok);
+            if (lane == 0) sm.stop = ok ? 0 : 1;
+        }
+        group_sync(g);   // also: the skew is done with the diagonal blocks in ring stage 0
+        if (*(volatile int*)&sm.stop) break;
+        bool stop = false;
+        if (box) {
+            // ring: source idx lives in stage (rq + idx) % NRING
+            auto issue = [&](int idx) {
+                int Is, Js;
+                const bool vert = nf.source(idx, Is, Js);
+                const uint32_t q = rq + idx, st = q % NRING;
+                sm100::mbar_arrive_expect_tx(&sm.rfull[st], 2 * kBox * 4);
+                if (vert) {   // L_O[Is rows][leaf rows], E[Is rows][leaf cols]
+                    sm100::tma_load_2d(sm.ring[st][0], &maps->lo, i0, Is * LB, &sm.rfull[st]);
+                    sm100::tma_load_2d(sm.ring[st][1], &maps->e, j0, Is * LB, &sm.rfull[st]);
+                } else {      // U^T[Js cols][leaf rows], L_I[Js cols][leaf cols]
+                    sm100::tma_load_2d(sm.ring[st][0], &maps->ut, i0, Js * LB, &sm.rfull[st]);
+                    sm100::tma_load_2d(sm.ring[st][1], &maps->li, j0, Js * LB, &sm.rfull[st]);
+                }
+            };
+            if (lead) {
+                // the flags were acquired by warp 0's lanes before the barrier above
+                asm volatile("fence.proxy.async.global;" ::: "memory");
+                for (int idx = 0; idx < min(NRING, nf.nold); ++idx) issue(idx);
+            }
+            for (int idx = 0; idx < nf.nsrc; ++idx) {
+                if (idx >= nf.nold && lead) {    // a recent source: its flag first
+                    int Is, Js;
+                    nf.source(idx, Is, Js);
+                    if (wait_flag(&a.flags[(size_t)Is * a.Nt + Js], a.abort_word, a.status, a.limit_ns)) {
+                        asm volatile("fence.proxy.async.global;" ::: "memory");
+                        issue(idx);
+                    } else {
+                        sm.stop = 1;
+                    }
+                }
+                if (idx >= nf.nold) {
+                    group_sync(g);
+                    if (*(volatile int*)&sm.stop) { stop = true; break; }
+                }
+                const uint32_t q = rq + idx, st = q % NRING;
+                if (!sm100::mbar_wait(&sm.rfull[st], (q / NRING) & 1, a.status, a.limit_ns)) {
+                    atomicExch(a.abort_word, 1);
+                    stop = true;
+                }
+                if (__any_sync(0xffffffffu, stop)) { sm.stop = 1; }
+                int Is, Js;
+                const bool vert = nf.source(idx, Is, Js);
+                if (!stop) {
+                    if (vert) product_4x4<LB>(sm.ring[st][0], sm.ring[st][1], r0, c0, accT);
+                    else product_4x4<LB>(sm.ring[st][0], sm.ring[st][1], r0, c0, accR);
+                }
+                group_sync(g);   // the stage is free again
+                if (*(volatile int*)&sm.stop) { stop = true; break; }
+                if (lead && idx + NRING < nf.nold) issue(idx + NRING);
+            }
+            rq += nf.nsrc;
+        } else {
+            // plain loads: the next source's blocks are fetched into registers while the
+            // current one is multiplied; element e = lt + 64 q sits at (e >> 5, e & 31)
+            float pf[32];
+            auto fetch = [&](int idx) {
+                int Is, Js;
+                const bool vert = nf.source(idx, Is, Js);
+#pragma unroll
+                for (int q = 0; q < 16; ++q) {
+                    const int e = lt + q * NLOAD, r = e >> 5, c = e & 31;
+                    if (vert) {
+                        const size_t kr = (size_t)Is * LB + r;
+                        pf[q] = (c < rows) ? __ldg(&a.LO[kr * m + i0 + c]) : 0.f;
+                        pf[16 + q] = (c < cols) ? __ldcg(&a.E[kr * n + j0 + c]) : 0.f;
+                    } else {   // r = source column, c = leaf row (U^T) / leaf column (L_I)
+                        const size_t l = (size_t)Js * LB;
+                        pf[q] = (c < rows) ? __ldcg(&a.Ut[(l + r) * a.ldm + i0 + c]) : 0.f;
+                        pf[16 + q] = (c < cols) ? __ldg(&a.LI[(l + r) * n + j0 + c]) : 0.f;
+                    }
+                }
+            };
+            auto wait_recent = [&](int idx) -> bool {
+                if (idx < nf.nold) return true;
+                if (lead) {
+                    int Is, Js;
+                    nf.source(idx, Is, Js);
+                    sm.stop = wait_flag(&a.flags[(size_t)Is * a.Nt + Js], a.abort_word, a.status,
+                                        a.limit_ns) ? 0 : 1;
+                }
+                group_sync(g);
+                return !*(volatile int*)&sm.stop;
+            };
+            if (nf.nsrc > 0) {
+                if (!wait_recent(0)) stop = true;
+                else fetch(0);
+            }
+            for (int idx = 0; idx < nf.nsrc && !stop; ++idx) {
+                int Is, Js;
+                const bool vert = nf.source(idx, Is, Js);
+                group_sync(g);   // the previous product is done with sA / sB
+#pragma unroll
+                for (int q = 0; q < 16; ++q) {
+                    const int e = lt + q * NLOAD, r = e >> 5, c = e & 31;
+                    sA[r * LPAD + c] = pf[q];        // sA[k = source row / column][leaf row]
+                    sB[r * LPAD + c] = pf[16 + q];   // sB[k][leaf col]
+                }
+                if (idx + 1 < nf.nsrc) {
+                    if (!wait_recent(idx + 1)) { stop = true; break; }
+                    fetch(idx + 1);
+                }
+                group_sync(g);   // sA / sB complete
+                if (vert) product_4x4<LPAD>(sA, sB, r0, c0, accT);
+                else product_4x4<LPAD>(sA, sB, r0, c0, accR);
+            }
+        }
+        if (stop) break;
+        if (box && lead && !sm100::mbar_wait(&sm.tbar, k & 1, a.status, a.limit_ns)) {
+            atomicExch(a.abort_word, 1);
+            sm.stop = 1;
+        }
+        group_sync(g);
+        if (*(volatile int*)&sm.stop) break;
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int o = (r0 + i) * LB + c0 + j;
+                const bool ok = r0 + i < rows && c0 + j < cols;
+                // the box path already holds the far sums in B.T / B.R
+                B.T[o] = ok ? (box ? B.T[o] : 0.f) + accT[i][j] : 0.f;
+                B.R[o] = ok ? (box ? B.R[o] : 0.f) + accR[i][j] : 0.f;
+            }
+        group_sync(g);
+        if (lead) sm100::mbar_arrive(&sm.full[b]);
+    }
+    if (lead && *(volatile int*)&sm.stop) atomicExch(a.abort_word, 1);
+    // the last (up to) two leaves: wait until they are solved, then publish the rest
+    if (!*(volatile int*)&sm.stop) {
+        for (int kk = (k >= 2 ? k - 2 : 0); kk < k; ++kk) {
+            const int b = kk & 1;
+            if (lead && !sm100::mbar_wait(&sm.empty[b], (kk >> 1) & 1, a.status, a.limit_ns)) {
+                atomicExch(a.abort_word, 1);
+                sm.stop = 1;
+            }
+            group_sync(g);
+            if (*(volatile int*)&sm.stop) break;
+            publish_rest(a, sm.buf[b], lt);
+        }
+    }
+}
+
+// ------------------------------------------------------------------------------ leaf solver
+__device__ void leaf_solver(const FusedArgs& a, LeafGroupSmem& sm, int lane, int slot,
+                            int nslots) {
+    const int n = a.n;
+    const long long total = (long long)a.Mt * a.Nt;
+    int k = 0;
+    for (long long gi = slot; gi < total; gi += nslots, ++k) {
+        const int b = k & 1;
+        LeafBuf& B = sm.buf[b];
+        bool ok = true;
+        if (lane == 0) ok = sm100::mbar_wait(&sm.full[b], (k >> 1) & 1, a.status, a.limit_ns);
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        if (!ok || ld_acquire_gpu(a.abort_word) != 0) {
+            if (lane == 0) atomicExch(a.abort_word, 1);
+            break;
+        }
+        const int I = B.meta[0], J = B.meta[1], rows = B.meta[2], cols = B.meta[3];
+        const int i0 = I * LB, j0 = J * LB;
+        solve_leaf(lane, rows, cols, a.qlo, a.qhi, B, a.status);
+        __syncwarp();
+        // what the next leaves read: E (vertical pulls, lane = column) and U^T (horizontal pulls,
+        // lane = row), then the flag
+        if (lane < cols) {
+            for (int r = 0; r < rows; ++r)
+                __stcg(&a.E[(size_t)(i0 + r) * n + j0 + lane], B.oE[r * LB + lane]);
+        }
+        if (lane < rows) {
+            for (int c = 0; c < cols; ++c)
+                __stcg(&a.Ut[(size_t)(j0 + c) * a.ldm + i0 + lane], B.oUt[c * LB + lane]);
+        }
+        __threadfence();
+        __syncwarp();
+        if (lane == 0) st_release_gpu(&a.flags[(size_t)I * a.Nt + J], 1);
+        // what the pushes read: the U planes (lane = column) and the E^T planes (lane = row),
+        // then the super-block count
+        if (lane < cols) {
+            for (int r = 0; r < rows; ++r) {
+                const float u = B.oU[r * LB + lane], uh = sm100::tf32_hi(u);
+                const size_t ou = (size_t)(i0 + r) * a.ldn + j0 + lane;
+                __stcg(&a.u_hi[ou], uh);
+                __stcg(&a.u_lo[ou], u - uh);
+            }
+        }
+        if (lane < rows) {
+            for (int c = 0; c < cols; ++c) {
+                const float x = B.oEt[c * LB + lane], xh = sm100::tf32_hi(x);
+                const size_t ot = (size_t)(j0 + c) * a.ldm + i0 + lane;
+                __stcg(&a.et_hi[ot], xh);
+                __stcg(&a.et_lo[ot], x - xh);
+            }
+        }
+        __threadfence();
+        __syncwarp();
+        if (lane == 0) {
+            red_add_release_gpu(&a.sb_done[(I / LPB) * a.NS + (J / LPB)], 1);
+            sm100::mbar_arrive(&sm.empty[b]);
+        }
+    }
+}
+
+__device__ void leaf_role(const FusedArgs& a, const LeafMaps* maps, uint8_t* smem) {
+    LeafCtaSmem& cs = *reinterpret_cast<LeafCtaSmem*>(smem);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int g = 0; g < 2; ++g) {
+            for (int b = 0; b < 2; ++b) {
+                sm100::mbar_init(&cs.g[g].full[b], 1);
+                sm100::mbar_init(&cs.g[g].empty[b], 1);
+            }
+            for (int r = 0; r < NRING; ++r) sm100::mbar_init(&cs.g[g].rfull[r], 1);
+            sm100::mbar_init(&cs.g[g].sbar, 1);
+            sm100::mbar_init(&cs.g[g].tbar, 1);
+            cs.g[g].stop = 0;
+        }
         sm100::fence_mbar_init();
     }
     __syncthreads();
-    TaskWalker wk;
-    wk.init(a.p_lo);
+    // group g: loader warps 2g and 2g + 1, solver warp 4 + g
+    const int g = warp < 4 ? (warp >> 1) : (warp - 4);
+    const int slot = blockIdx.x * 2 + g, nslots = a.leaf_ctas * 2;
+    if (warp < 4) leaf_loaders(a, maps, cs.g[g], g, warp & 1, lane, slot, nslots);
+    else leaf_solver(a, cs.g[g], lane, slot, nslots);
+}
 
-    if (warp < 4) {
-        // ------------------------------------------------------------ loaders
-        int k = 0;
-        for (int g = blockIdx.x; g < a.total; g += gridDim.x, ++k) {
-            const int b = k & 1;
-            LeafBuf& B = sm.buf[b];
-            if (k >= 2) {
-                if (tid == 0 && !sm100::mbar_wait(&sm.empty[b], ((k >> 1) - 1) & 1, a.status,
-                                                  a.limit_ns)) {
-                    atomicExch(a.abort_word, 1);
-                    sm.stop = 1;
+// ------------------------------------------------------------------------------ push tasks
+struct PushTask {
+    bool valid;
+    bool vert;      // E into T_far (else U into R_far)
+    int src;        // source super-block index along the column (vert) / row
+    int A, C;       // target super-block
+    int tr, tc;     // target 128 x 128 tile
+    int nkb;        // k-blocks of 32
+};
+
+// Task t: source super-block (A', C') by binary search over the prefix, then (target, tile)
+// inside it. Its targets are (A'+2+d, C') for the vertical push (d < nvt) and (A', C'+2+d) for
+// the horizontal one (d < nht), nearest first (vertical, horizontal, then the next distance),
+// 4 tiles each.
+__device__ __forceinline__ PushTask decode_task(const FusedArgs& a, int t) {
+    int lo = 0, hi = a.nsb - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (__ldg(&a.task_pre[mid]) <= t) lo = mid;
+        else hi = mid - 1;
+    }
+    const int2 sc = __ldg(&a.task_sb[lo]);
+    const int local = t - __ldg(&a.task_pre[lo]);
+    const int nvt = max(a.MS - sc.x - 2, 0), nht = max(a.NS - sc.y - 2, 0);
+    const int mn = min(nvt, nht);
+    const int u = local >> 2, q = local & 3;
+    int d;
+    bool vert;
+    if (u < 2 * mn) { d = u >> 1; vert = (u & 1) == 0; }
+    else { d = mn + (u - 2 * mn); vert = nvt > nht; }
+    PushTask p;
+    p.vert = vert;
+    p.A = vert ? sc.x + 2 + d : sc.x;
+    p.C = vert ? sc.y : sc.y + 2 + d;
+    p.src = vert ? sc.x : sc.y;
+    p.tr = 2 * p.A + (q >> 1);
+    p.tc = 2 * p.C + (q & 1);
+    p.valid = p.tr * TB < a.m && p.tc * TB < a.n;
+    const int kext = vert ? min(SB, a.m - p.src * SB) : min(SB, a.n - p.src * SB);
+    p.nkb = (kext + tc::BK - 1) / tc::BK;
+    return p;
+}
+
+__device__ __forceinline__ void epi_sync() {
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+}
+
+// Tensor-core far-field pushes (same warp roles as the GEMM engine: warp 0 TMA, warp 1 MMA,
+// warps 2-5 epilogue). The producer waits until the task's source super-block is complete; the
+// epilogue waits until the output tile has taken every earlier source, adds the tile, and
+// advances the tile's counter.
+__device__ void gemm_role(const CUtensorMap* loth, const CUtensorMap* lotl, const CUtensorMap* eth,
+                          const CUtensorMap* etl, const CUtensorMap* uh, const CUtensorMap* ul,
+                          const CUtensorMap* lith, const CUtensorMap* litl, const FusedArgs& a,
+                          uint8_t* smem_raw) {
+    using Cf = tc::Cfg<BN>;
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    float* epi_stage = reinterpret_cast<float*>(smem + STAGES * Cf::kStageBytes);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * Cf::kStageBytes + Cf::kEpiBytes);
+    uint64_t* empty = full + STAGES;
+    uint64_t* acc_full = empty + STAGES;
+    uint64_t* acc_empty = acc_full + 2;
+    uint64_t* drain = acc_empty + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    volatile int* s_abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    volatile int* s_go = s_abort + 1;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int gid = blockIdx.x - a.leaf_ctas, ng = gridDim.x - a.leaf_ctas;
+    const int total = __ldg(&a.task_pre[a.nsb]);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            sm100::mbar_init(&full[s], 1);
+            sm100::mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            sm100::mbar_init(&acc_full[b], 1);
+            sm100::mbar_init(&acc_empty[b], 4);
+        }
+        sm100::mbar_init(drain, 1);
+        *s_abort = 0;
+        *s_go = 0;
+        sm100::fence_mbar_init();
+    }
+    if (warp == 1) {
+        sm100::tmem_alloc(tmem_slot, Cf::kTmemCols);
+        sm100::tmem_relinquish();
+    }
+    sm100::tc_fence_before();
+    __syncthreads();
+    sm100::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    auto stage_ptr = [&](int s, int which) -> uint8_t* {
+        uint8_t* base = smem + (size_t)s * Cf::kStageBytes;
+        return which < 2 ? base + which * Cf::kABytes : base + 2 * Cf::kABytes + (which - 2) * Cf::kBBytes;
+    };
+
+    if (warp == 0) {
+        // ---------------- TMA producer
+        if (lane == 0) {
+            sm100::prefetch_tmap(loth); sm100::prefetch_tmap(lotl);
+            sm100::prefetch_tmap(eth);  sm100::prefetch_tmap(etl);
+            sm100::prefetch_tmap(uh);   sm100::prefetch_tmap(ul);
+            sm100::prefetch_tmap(lith); sm100::prefetch_tmap(litl);
+            uint32_t g = 0;
+            for (int t = gid; t < total && !*s_abort; t += ng) {
+                const PushTask p = decode_task(a, t);
+                if (!p.valid) continue;
+                const int sA = p.vert ? p.src : p.A, sC = p.vert ? p.C : p.src;
+                const int need = leaves_in(a.Mt, sA) * leaves_in(a.Nt, sC);
+                if (!wait_geq(&a.sb_done[sA * a.NS + sC], need, a.abort_word, a.status, a.limit_ns)) {
+                    *s_abort = 1;
+                    break;
                 }
-                loader_sync();
-                if (*(volatile int*)&sm.stop) break;
-                publish_rest(a, B, tid);   // leaf k - 2, solved from this buffer
-                loader_sync();             // its meta is read before it is overwritten
-            }
-            int I, J;
-            wk.find(a, g, I, J);
-            const int P = wk.P, Q = a.delta - P;
-            const int la = I - P * LPB, lc = J - Q * LPB;
-            const int i0 = I * LB, j0 = J * LB;
-            const int rows = min(LB, m - i0), cols = min(LB, n - j0);
-            float accT[8], accR[8];
-#pragma unroll
-            for (int t = 0; t < 8; ++t) {
-                const int r = warp * 8 + t;
-                const bool ok = r < rows && lane < cols;
-                const size_t o = (size_t)(i0 + r) * n + j0 + lane;
-                accT[t] = ok ? __ldcg(&a.Tf[o]) : 0.f;
-                accR[t] = ok ? __ldcg(&a.Rf[o]) : 0.f;
-            }
-            // what does not depend on other leaves first: W*, the diagonal blocks of L_O and
-            // L_I, the scales (sA / sB are free again after the skew below)
-#pragma unroll
-            for (int q = 0; q < (LB * LB) / NLOAD; ++q) {
-                const int e = tid + q * NLOAD, r = e >> 5, c = e & 31;
-                B.W[e] = (r < rows && c < cols) ? __ldg(&a.Ws[(size_t)(i0 + r) * n + j0 + c]) : 0.f;
-                sm.sA[r][c] = (r < rows && c < rows) ? __ldg(&a.LO[(size_t)(i0 + r) * m + i0 + c]) : 0.f;
-                sm.sB[r][c] = (r < cols && c < cols) ? __ldg(&a.LI[(size_t)(j0 + r) * n + j0 + c]) : 0.f;
-            }
-            if (tid < LB) {
-                const float sv = (tid < rows) ? __ldg(&a.sc[i0 + tid]) : 0.f;
-                B.S[tid] = sv;
-                B.S[LB + tid] = sv > 0.f ? __frcp_rn(sv) : 0.f;
-            }
-            if (tid == 0) { B.meta[0] = I; B.meta[1] = J; B.meta[2] = rows; B.meta[3] = cols; }
-            loader_sync();
-            for (int e = tid; e < LB * LS; e += NLOAD) {
-                const int x = e / LS, dd = e % LS;
-                B.LOr[e] = (dd >= 1 && dd < LB && x + dd < LB) ? sm.sA[x][x + dd] : 0.f;
-                B.LIc[e] = (dd >= 1 && dd < LB && x - dd >= 0) ? sm.sB[x - dd][x] : 0.f;
-            }
-            loader_sync();
-            bool stop = false;
-            // In-block sources: the leaves above (vertical, via E) and to the left (horizontal,
-            // via U). The two most recent ones, (la-1, lc) and (la, lc-1), finish last, so every
-            // older source is pulled first and those two close the list.
-            const int nv = max(la - 1, 0), nh = max(lc - 1, 0);
-            const int nsrc = la + lc;
-            for (int idx = 0; idx < nsrc && !stop; ++idx) {
-                bool vert;
-                int src;
-                if (idx < nv) { vert = true; src = idx; }
-                else if (idx < nv + nh) { vert = false; src = idx - nv; }
-                else if (idx == nv + nh && la > 0) { vert = true; src = la - 1; }
-                else { vert = false; src = lc - 1; }
-                const int Is = vert ? P * LPB + src : I, Js = vert ? J : Q * LPB + src;
-                if (tid == 0)
-                    sm.stop = wait_flag(&a.flags[(size_t)Is * a.Nt + Js], a.abort_word, a.status,
-                                        a.limit_ns) ? 0 : 1;
-                loader_sync();
-                if (*(volatile int*)&sm.stop) { stop = true; break; }
-                if (vert) {
-#pragma unroll
-                    for (int q = 0; q < (LB * LB) / NLOAD; ++q) {
-                        const int e = tid + q * NLOAD, kk = e >> 5, c = e & 31;
-                        const size_t kr = (size_t)Is * LB + kk;
-                        sm.sA[kk][c] = (c < rows) ? __ldg(&a.LO[kr * m + i0 + c]) : 0.f;
-                        sm.sB[kk][c] = (c < cols) ? __ldcg(&a.E[kr * n + j0 + c]) : 0.f;
+                // the source planes were written through the generic proxy on other SMs
+                asm volatile("fence.proxy.async.global;" ::: "memory");
+                const CUtensorMap* ma_h = p.vert ? loth : uh;
+                const CUtensorMap* ma_l = p.vert ? lotl : ul;
+                const CUtensorMap* mb_h = p.vert ? eth : lith;
+                const CUtensorMap* mb_l = p.vert ? etl : litl;
+                bool ok = true;
+                for (int kb = 0; kb < p.nkb; ++kb, ++g) {
+                    const int s = g % STAGES;
+                    if (g >= STAGES &&
+                        !tc::wait_or_abort(&empty[s], ((g / STAGES) & 1) ^ 1, a.status, a.limit_ns, s_abort)) {
+                        ok = false;
+                        break;
                     }
-                    loader_sync();
-#pragma unroll 8
-                    for (int kk = 0; kk < LB; ++kk) {
-                        const float bv = sm.sB[kk][lane];
-#pragma unroll
-                        for (int t = 0; t < 8; ++t)
-                            accT[t] = fmaf(sm.sA[kk][warp * 8 + t], bv, accT[t]);
-                    }
-                } else {
-#pragma unroll
-                    for (int q = 0; q < (LB * LB) / NLOAD; ++q) {
-                        const int e = tid + q * NLOAD, rr = e >> 5, c = e & 31;
-                        const size_t l = (size_t)Js * LB;
-                        const size_t o = (size_t)(i0 + rr) * a.ldn + l + c;
-                        sm.sA[rr][c] = (rr < rows) ? (__ldcg(&a.u_hi[o]) + __ldcg(&a.u_lo[o])) : 0.f;
-                        sm.sB[rr][c] = (c < cols) ? __ldg(&a.LI[(l + rr) * n + j0 + c]) : 0.f;
-                    }
-                    loader_sync();
-#pragma unroll 8
-                    for (int ll = 0; ll < LB; ++ll) {
-                        const float bv = sm.sB[ll][lane];
-#pragma unroll
-                        for (int t = 0; t < 8; ++t)
-                            accR[t] = fmaf(sm.sA[warp * 8 + t][ll], bv, accR[t]);
-                    }
+                    sm100::mbar_arrive_expect_tx(&full[s], Cf::kStageBytes);
+                    const int kx = p.src * SB + kb * tc::BK;
+                    sm100::tma_load_2d(stage_ptr(s, 0), ma_h, kx, p.tr * TB, &full[s]);
+                    sm100::tma_load_2d(stage_ptr(s, 1), ma_l, kx, p.tr * TB, &full[s]);
+                    sm100::tma_load_2d(stage_ptr(s, 2), mb_h, kx, p.tc * TB, &full[s]);
+                    sm100::tma_load_2d(stage_ptr(s, 3), mb_l, kx, p.tc * TB, &full[s]);
                 }
-                loader_sync();
+                if (!ok) break;
             }
-            if (stop) break;
-            // the far and in-block sums
-#pragma unroll
-            for (int t = 0; t < 8; ++t) {
-                B.T[(warp * 8 + t) * LB + lane] = accT[t];
-                B.R[(warp * 8 + t) * LB + lane] = accR[t];
-            }
-            loader_sync();
-            if (tid == 0) {
-                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(sm100::smem_u32(&sm.full[b])) : "memory");
+            if (*s_abort) {
+                atomicExch(a.abort_word, 1);
+                for (uint32_t q = (g > (uint32_t)STAGES ? g - STAGES : 0); q < g; ++q)
+                    sm100::mbar_wait(&full[q % STAGES], (q / STAGES) & 1, a.status, a.limit_ns);
             }
         }
-        if (tid == 0) {
-            // loaders ended early: let the solver warp see it
-            if (*(volatile int*)&sm.stop) atomicExch(a.abort_word, 1);
-        }
-        // the last (up to) two leaves: wait until they are solved, then publish the rest
-        if (!*(volatile int*)&sm.stop) {
-            for (int kk = (k >= 2 ? k - 2 : 0); kk < k; ++kk) {
-                const int b = kk & 1;
-                if (tid == 0 && !sm100::mbar_wait(&sm.empty[b], (kk >> 1) & 1, a.status,
-                                                  a.limit_ns)) {
-                    atomicExch(a.abort_word, 1);
-                    sm.stop = 1;
+    } else if (warp == 1) {
+        // ---------------- MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc = sm100::idesc_tf32(tc::BM, BN);
+            uint32_t g = 0;
+            int i = 0;
+            for (int t = gid; t < total && !*s_abort; t += ng) {
+                const PushTask p = decode_task(a, t);
+                if (!p.valid) continue;
+                const int b = i & 1;
+                if (i >= 2 &&
+                    !tc::wait_or_abort(&acc_empty[b], ((i >> 1) & 1) ^ 1, a.status, a.limit_ns, s_abort))
+                    break;
+                sm100::tc_fence_after();
+                const uint32_t acc = tmem + (uint32_t)(b * BN);
+                bool ok = true;
+                for (int kb = 0; kb < p.nkb; ++kb, ++g) {
+                    const int s = g % STAGES;
+                    if (!tc::wait_or_abort(&full[s], (g / STAGES) & 1, a.status, a.limit_ns, s_abort)) {
+                        ok = false;
+                        break;
+                    }
+                    sm100::tc_fence_after();
+                    const uint32_t ah = sm100::smem_u32(stage_ptr(s, 0));
+                    const uint32_t al = sm100::smem_u32(stage_ptr(s, 1));
+                    const uint32_t bh = sm100::smem_u32(stage_ptr(s, 2));
+                    const uint32_t bl = sm100::smem_u32(stage_ptr(s, 3));
+#pragma unroll
+                    for (int kk = 0; kk < tc::BK / 8; ++kk) {
+                        const uint32_t off = kk * 32;
+                        const uint64_t dah = sm100::desc_kmajor_sw128(ah + off);
+                        const uint64_t dal = sm100::desc_kmajor_sw128(al + off);
+                        const uint64_t dbh = sm100::desc_kmajor_sw128(bh + off);
+                        const uint64_t dbl = sm100::desc_kmajor_sw128(bl + off);
+                        const uint32_t acc0 = (kb > 0 || kk > 0) ? 1u : 0u;
+                        sm100::mma_tf32(acc, dah, dbh, idesc, acc0);
+                        sm100::mma_tf32(acc, dah, dbl, idesc, 1u);
+                        sm100::mma_tf32(acc, dal, dbh, idesc, 1u);
+                    }
+                    sm100::mma_commit(&empty[s]);
                 }
-                loader_sync();
-                if (*(volatile int*)&sm.stop) break;
-                publish_rest(a, sm.buf[b], tid);
+                if (!ok) break;
+                sm100::mma_commit(&acc_full[b]);
+                ++i;
+            }
+            if (*s_abort) {
+                sm100::mma_commit(drain);
+                sm100::mbar_wait(drain, 0, a.status, a.limit_ns);
             }
         }
     } else {
-        // ------------------------------------------------------------ solver warp
-        int k = 0;
-        for (int g = blockIdx.x; g < a.total; g += gridDim.x, ++k) {
-            const int b = k & 1;
-            LeafBuf& B = sm.buf[b];
-            bool ok = true;
-            if (lane == 0) ok = sm100::mbar_wait(&sm.full[b], (k >> 1) & 1, a.status, a.limit_ns);
-            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-            if (!ok || ld_acquire_gpu(a.abort_word) != 0) {
-                if (lane == 0) atomicExch(a.abort_word, 1);
-                break;
+        // ---------------- epilogue (warps 2 .. 5): T_far / R_far tile += accumulator
+        const int quarter = warp & 3;
+        float* stage = epi_stage + (warp - tc::kEpiWarp0) * (32 * 33);
+        int i = 0;
+        for (int t = gid; t < total; t += ng) {
+            const PushTask p = decode_task(a, t);
+            if (!p.valid) continue;
+            const int b = i & 1;
+            int* cnt = (p.vert ? a.cntT : a.cntR) + (size_t)p.tr * a.TN + p.tc;
+            if (threadIdx.x == tc::kEpiWarp0 * 32) {
+                bool ok = tc::wait_or_abort(&acc_full[b], (i >> 1) & 1, a.status, a.limit_ns, s_abort);
+                // the tile takes its sources in order
+                if (ok) ok = wait_geq(cnt, p.src, a.abort_word, a.status, a.limit_ns);
+                if (!ok) { *s_abort = 1; atomicExch(a.abort_word, 1); }
+                *s_go = ok ? 1 : 0;
             }
-            const int I = B.meta[0], J = B.meta[1], rows = B.meta[2], cols = B.meta[3];
-            const int i0 = I * LB, j0 = J * LB;
-            solve_leaf(lane, rows, cols, a.qlo, a.qhi, B, a.status);
-            __syncwarp();
-            // publish what other leaves read (E for the vertical pulls, U for the horizontal
-            // ones), then the flag; codes, W and the E^T planes follow from the loader warps
-            if (lane < cols) {
-                for (int r = 0; r < rows; ++r) {
-                    const size_t o = (size_t)(i0 + r) * n + j0 + lane;
-                    __stcg(&a.E[o], B.oE[r * LB + lane]);
-                    const float u = B.oU[r * LB + lane], uh = sm100::tf32_hi(u);
-                    const size_t ou = (size_t)(i0 + r) * a.ldn + j0 + lane;
-                    __stcg(&a.u_hi[ou], uh);
-                    __stcg(&a.u_lo[ou], u - uh);
+            epi_sync();
+            if (!*s_go) break;
+            sm100::tc_fence_after();
+            float* Cm = p.vert ? a.Tf : a.Rf;
+            const int row0 = p.tr * TB + quarter * 32;
+#pragma unroll 1
+            for (int c0 = 0; c0 < BN; c0 += 32) {
+                float v[32];
+                sm100::tmem_ld32(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(b * BN + c0), v);
+#pragma unroll
+                for (int q = 0; q < 32; ++q) stage[lane * 33 + q] = v[q];
+                __syncwarp();
+                const int gc = p.tc * TB + c0 + lane;
+                if (gc < a.n) {
+                    float old[32];
+#pragma unroll
+                    for (int rr = 0; rr < 32; ++rr)
+                        old[rr] = (row0 + rr < a.m) ? __ldcg(&Cm[(size_t)(row0 + rr) * a.n + gc]) : 0.f;
+#pragma unroll
+                    for (int rr = 0; rr < 32; ++rr)
+                        if (row0 + rr < a.m)
+                            __stcg(&Cm[(size_t)(row0 + rr) * a.n + gc], old[rr] + stage[rr * 33 + lane]);
                 }
+                __syncwarp();
             }
             __threadfence();
-            __syncwarp();
-            if (lane == 0) {
-                st_release_gpu(&a.flags[(size_t)I * a.Nt + J], 1);
-                asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(sm100::smem_u32(&sm.empty[b])) : "memory");
-            }
+            sm100::tc_fence_before();
+            epi_sync();
+            if (threadIdx.x == tc::kEpiWarp0 * 32) st_release_gpu(cnt, p.src + 1);
+            if (lane == 0) sm100::mbar_arrive(&acc_empty[b]);
+            ++i;
         }
     }
+    __syncwarp();
+    sm100::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) sm100::tmem_dealloc(tmem, Cf::kTmemCols);
+}
+
+__global__ void __launch_bounds__(NTH, 1)
+round_kernel(const __grid_constant__ CUtensorMap loth, const __grid_constant__ CUtensorMap lotl,
+             const __grid_constant__ CUtensorMap eth, const __grid_constant__ CUtensorMap etl,
+             const __grid_constant__ CUtensorMap uh, const __grid_constant__ CUtensorMap ul,
+             const __grid_constant__ CUtensorMap lith, const __grid_constant__ CUtensorMap litl,
+             const __grid_constant__ LeafMaps lmaps, const __grid_constant__ FusedArgs a) {
+    extern __shared__ __align__(1024) uint8_t round_smem[];
+    if ((int)blockIdx.x < a.leaf_ctas) {
+        // box-copy destinations need 128-byte alignment of the leaf layout's base
+        uint8_t* base = reinterpret_cast<uint8_t*>(
+            (reinterpret_cast<uintptr_t>(round_smem) + 127) & ~uintptr_t(127));
+        leaf_role(a, &lmaps, base);
+        return;
+    }
+    gemm_role(&loth, &lotl, &eth, &etl, &uh, &ul, &lith, &litl, a, round_smem);
+}
+
+// Push tasks per source super-block, in the order the sources finish (anti-diagonal, then row).
+__global__ void task_prefix_kernel(int MS, int NS, int* pre, int2* sb) {
+    if (threadIdx.x != 0 || blockIdx.x != 0) return;
+    int idx = 0, acc = 0;
+    for (int d = 0; d < MS + NS - 1; ++d) {
+        for (int A = max(0, d - NS + 1); A <= min(d, MS - 1); ++A) {
+            const int C = d - A;
+            pre[idx] = acc;
+            sb[idx] = make_int2(A, C);
+            acc += 4 * (max(MS - A - 2, 0) + max(NS - C - 2, 0));
+            ++idx;
+        }
+    }
+    pre[idx] = acc;
 }
 
 struct Layout {
-    int Mt, Nt, MS, NS, ldm, ldn;
+    int Mt, Nt, MS, NS, TM, TN, ldm, ldn, nsb;
     size_t mn;
 };
 
@@ -354,10 +865,18 @@ Layout layout(int m, int n) {
     L.Nt = (n + LB - 1) / LB;
     L.MS = (m + SB - 1) / SB;
     L.NS = (n + SB - 1) / SB;
+    L.TM = (m + TB - 1) / TB;
+    L.TN = (n + TB - 1) / TB;
     L.ldm = tc::plane_ld(m);
     L.ldn = tc::plane_ld(n);
+    L.nsb = L.MS * L.NS;
     L.mn = (size_t)m * n;
     return L;
+}
+
+// the int region: leaf flags, super-block counts, tile counters, abort word (zeroed per call)
+size_t sync_ints(const Layout& L) {
+    return (size_t)L.Mt * L.Nt + (size_t)L.nsb + 2 * (size_t)L.TM * L.TN + 64;
 }
 
 template <class F>
@@ -367,28 +886,12 @@ void round_ws_layout(const Layout& L, int m, int n, F&& take) {
     take((size_t)n * L.ldn * 4); take((size_t)n * L.ldn * 4);   // L_I^T planes
     take((size_t)n * L.ldm * 4); take((size_t)n * L.ldm * 4);   // E^T planes
     take((size_t)m * L.ldn * 4); take((size_t)m * L.ldn * 4);   // U planes
+    take((size_t)n * L.ldm * 4);                    // U^T (full precision)
     take((size_t)L.mn * 4);                         // T_far
     take((size_t)L.mn * 4);                         // R_far
-    take(((size_t)L.Mt * L.Nt + 64) * 4);           // leaf flags + abort word
-}
-
-int leaf_grid(int tasks) {
-    static int cached = 0;
-    if (!cached) {
-        int dev = 0, nsm = 0, per_sm = 0;
-        if (cudaGetDevice(&dev) != cudaSuccess) return -1;
-        if (cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-            return -1;
-        if (cudaFuncSetAttribute(phase_leaves_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)sizeof(LeafSmem)) != cudaSuccess)
-            return -1;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, phase_leaves_kernel, NTHW,
-                                                          sizeof(LeafSmem)) != cudaSuccess)
-            return -1;
-        if (per_sm < 1) return -1;
-        cached = per_sm * nsm;
-    }
-    return std::min(tasks, cached);
+    take(sync_ints(L) * 4);                         // flags and counters
+    take(((size_t)L.nsb + 1) * 4);                  // push-task prefix
+    take((size_t)L.nsb * 8);                        // target super-blocks
 }
 
 }  // namespace
@@ -414,7 +917,7 @@ extern "C" int bakron_round(const float* Wstar, int m, int n, const float* L_O, 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const Layout L = layout(m, n);
     WsCarver c(ws);
-    char* p[12];
+    char* p[15];
     int k = 0;
     round_ws_layout(L, m, n, [&](size_t bytes) { p[k++] = c.take<char>(bytes); });
     float* E = (float*)p[0];
@@ -422,15 +925,21 @@ extern "C" int bakron_round(const float* Wstar, int m, int n, const float* L_O, 
     float *lit_hi = (float*)p[3], *lit_lo = (float*)p[4];
     float *et_hi = (float*)p[5], *et_lo = (float*)p[6];
     float *u_hi = (float*)p[7], *u_lo = (float*)p[8];
-    float *Tf = (float*)p[9], *Rf = (float*)p[10];
-    int* flags = (int*)p[11];
+    float* Ut = (float*)p[9];
+    float *Tf = (float*)p[10], *Rf = (float*)p[11];
+    int* ints = (int*)p[12];
+    int* task_pre = (int*)p[13];
+    int2* task_sb = (int2*)p[14];
+
     int e;
-    if ((e = cuda_err(cudaMemsetAsync(flags, 0, ((size_t)L.Mt * L.Nt + 64) * 4, st)))) return e;
+    if ((e = cuda_err(cudaMemsetAsync(ints, 0, sync_ints(L) * 4, st)))) return e;
     if ((e = cuda_err(cudaMemsetAsync(Tf, 0, L.mn * 4, st)))) return e;
     if ((e = cuda_err(cudaMemsetAsync(Rf, 0, L.mn * 4, st)))) return e;
     // static operands of the pushes: L_O^T and L_I^T as hi/lo planes
     tc::split_planes(L_O, m, m, m, lot_hi, lot_lo, L.ldm, 1, st);
     tc::split_planes(L_I, n, n, n, lit_hi, lit_lo, L.ldn, 1, st);
+    task_prefix_kernel<<<1, 32, 0, st>>>(L.MS, L.NS, task_pre, task_sb);
+    count_launches(1);
 
     CUtensorMap m_loth, m_lotl, m_eth, m_etl, m_uh, m_ul, m_lith, m_litl;
     if ((e = tc::make_kmajor_map(&m_loth, lot_hi, m, m, L.ldm, tc::BM))) return e;
@@ -442,73 +951,58 @@ extern "C" int bakron_round(const float* Wstar, int m, int n, const float* L_O, 
     if ((e = tc::make_kmajor_map(&m_lith, lit_hi, n, n, L.ldn, BN))) return e;
     if ((e = tc::make_kmajor_map(&m_litl, lit_lo, n, n, L.ldn, BN))) return e;
 
-    PhaseArgs a;
-    a.Ws = Wstar; a.LO = L_O; a.LI = L_I; a.sc = scales; a.Tf = Tf; a.Rf = Rf;
-    a.m = m; a.n = n; a.Nt = L.Nt;
+    FusedArgs a;
+    a.Ws = Wstar; a.LO = L_O; a.LI = L_I; a.sc = scales;
+    a.m = m; a.n = n;
     a.qlo = (float)(-(1 << (bits - 1)));
     a.qhi = (float)((1 << (bits - 1)) - 1);
     a.codes = codes; a.Wq = W; a.E = E;
     a.et_hi = et_hi; a.et_lo = et_lo; a.ldm = L.ldm;
     a.u_hi = u_hi; a.u_lo = u_lo; a.ldn = L.ldn;
-    a.flags = flags;
-    a.abort_word = flags + (size_t)L.Mt * L.Nt;
+    a.Tf = Tf; a.Rf = Rf; a.Ut = Ut;
+    a.flags = ints;
+    a.sb_done = a.flags + (size_t)L.Mt * L.Nt;
+    a.cntT = a.sb_done + L.nsb;
+    a.cntR = a.cntT + (size_t)L.TM * L.TN;
+    a.abort_word = a.cntR + (size_t)L.TM * L.TN;
     a.status = dev_status;
+    a.task_pre = task_pre;
+    a.task_sb = task_sb;
+    a.nsb = L.nsb;
+    a.Mt = L.Mt; a.Nt = L.Nt; a.MS = L.MS; a.NS = L.NS; a.TN = L.TN;
     a.limit_ns = spin_limit_ns();
 
-    for (int delta = 0; delta < L.MS + L.NS - 1; ++delta) {
-        const int p_lo = std::max(0, delta - (L.NS - 1)), p_hi = std::min(delta, L.MS - 1);
-        int total = 0, maxd = 0;
-        for (int P = p_lo; P <= p_hi; ++P) {
-            const int lm = (std::min(SB, m - P * SB) + LB - 1) / LB;
-            const int ln = (std::min(SB, n - (delta - P) * SB) + LB - 1) / LB;
-            total += lm * ln;
-            maxd = std::max(maxd, lm + ln - 2);
-        }
-        a.delta = delta; a.p_lo = p_lo; a.p_hi = p_hi; a.maxd = maxd; a.total = total;
-        const int grid = leaf_grid(total);
-        if (grid < 1) return BAKRON_ERR_CUDA;
-        void* params[] = {&a};
-        count_launches(1);
-        if ((e = cuda_err(cudaLaunchCooperativeKernel((const void*)phase_leaves_kernel,
-                                                      dim3(grid), dim3(NTHW), params,
-                                                      sizeof(LeafSmem), st))))
-            return e;
-
-        // pushes of the phase's blocks: E down into T_far, U right into R_far
-        tc::ProblemList pv(BN), ph(BN);
-        auto flush_v = [&]() -> int {
-            tc::EpiStore epi{Tf, n, 1, 0};
-            int r = tc::launch_gemm3x<BN, STAGES>(m_loth, m_lotl, m_eth, m_etl, pv, epi,
-                                                   dev_status, st);
-            pv = tc::ProblemList(BN);
-            return r;
-        };
-        auto flush_h = [&]() -> int {
-            tc::EpiStore epi{Rf, n, 1, 0};
-            int r = tc::launch_gemm3x<BN, STAGES>(m_uh, m_ul, m_lith, m_litl, ph, epi,
-                                                   dev_status, st);
-            ph = tc::ProblemList(BN);
-            return r;
-        };
-        for (int P = p_lo; P <= p_hi; ++P) {
-            const int Q = delta - P;
-            const int r0 = P * SB, c0 = Q * SB;
-            const int br = std::min(SB, m - r0), bc = std::min(SB, n - c0);
-            if (r0 + br < m) {
-                if (!pv.add(r0 + br, r0, c0, r0, m - (r0 + br), bc, br, r0 + br, c0)) {
-                    if ((e = flush_v())) return e;
-                    pv.add(r0 + br, r0, c0, r0, m - (r0 + br), bc, br, r0 + br, c0);
-                }
-            }
-            if (c0 + bc < n) {
-                if (!ph.add(r0, c0, c0 + bc, c0, br, n - (c0 + bc), bc, r0, c0 + bc)) {
-                    if ((e = flush_h())) return e;
-                    ph.add(r0, c0, c0 + bc, c0, br, n - (c0 + bc), bc, r0, c0 + bc);
-                }
-            }
-        }
-        if (!pv.empty() && (e = flush_v())) return e;
-        if (!ph.empty() && (e = flush_h())) return e;
+    // box loads for the leaves when every row stride is a multiple of 16 bytes
+    LeafMaps lm;
+    memset(&lm, 0, sizeof(lm));
+    auto al16 = [](const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15) == 0; };
+    a.box_loads = (m % 4 == 0 && n % 4 == 0 && al16(Wstar) && al16(L_O) && al16(L_I)) ? 1 : 0;
+    if (a.box_loads) {
+        if ((e = tc::make_box_map(&lm.lo, L_O, m, m, m, LB))) return e;
+        if ((e = tc::make_box_map(&lm.li, L_I, n, n, n, LB))) return e;
+        if ((e = tc::make_box_map(&lm.e, E, m, n, n, LB))) return e;
+        if ((e = tc::make_box_map(&lm.ut, Ut, n, m, L.ldm, LB))) return e;
+        if ((e = tc::make_box_map(&lm.ws, Wstar, m, n, n, LB))) return e;
+        if ((e = tc::make_box_map(&lm.tf, Tf, m, n, n, LB))) return e;
+        if ((e = tc::make_box_map(&lm.rf, Rf, m, n, n, LB))) return e;
     }
+
+    if (cudaFuncSetAttribute(round_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kSmem) != cudaSuccess)
+        return BAKRON_ERR_CUDA;
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, round_kernel, NTH, kSmem) !=
+            cudaSuccess || per_sm < 1)
+        return BAKRON_ERR_CUDA;
+    const int resident = per_sm * tc::sm_count();
+    if (resident < 2) return BAKRON_ERR_CUDA;
+    // two solver slots per leaf CTA, enough for one leaf anti-diagonal; the rest push
+    const int diag = std::min(L.Mt, L.Nt);
+    a.leaf_ctas = std::min({(diag + 1) / 2, kMaxLeafCtas, resident - 1});
+    void* params[] = {&m_loth, &m_lotl, &m_eth, &m_etl, &m_uh, &m_ul, &m_lith, &m_litl, &lm, &a};
+    count_launches(1);
+    if ((e = cuda_err(cudaLaunchCooperativeKernel((const void*)round_kernel, dim3(resident),
+                                                  dim3(NTH), params, kSmem, st))))
+        return e;
     return cuda_err(cudaGetLastError());
 }

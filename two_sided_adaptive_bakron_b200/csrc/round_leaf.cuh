@@ -6,6 +6,8 @@
 // T and R arrive holding everything from outside the leaf; the wavefront adds the in-leaf part.
 #pragma once
 
+#include <cstddef>
+
 #include "sm100.cuh"
 
 namespace bakron {
@@ -17,19 +19,27 @@ constexpr int UW = 4;            // wavefront steps per unrolled group
 constexpr int WIN = LB + UW;     // register window of slots
 constexpr int LS = LB + 4;       // row stride of the skewed diagonal blocks (16-byte rows)
 
-// One staging buffer: a leaf's inputs and outputs (shared memory, floats).
-struct LeafBuf {
+// One staging buffer: a leaf's inputs and outputs (shared memory, floats). LOr and LIc rows
+// are read as float4 (16-byte rows); W, T and R may be filled by tensor (box) copies, whose
+// shared-memory destination must sit on a 128-byte boundary.
+struct alignas(128) LeafBuf {
     float W[LB * LB];            // W* of the leaf, row stride LB
     float T[LB * LB];            // vertical sums (everything above the leaf)
     float R[LB * LB];            // horizontal sums (everything left of the leaf)
     float LOr[LB * LS];          // LOr[r*LS + d] = L_O[i0+r][i0+r+d]
     float LIc[LB * LS];          // LIc[c*LS + d] = L_I[j0+c-d][j0+c]
     float S[2 * LB];             // s_r and its reciprocal
-    float oW[LB * LB], oE[LB * LB], oU[LB * LB];
+    float oE[LB * LB], oU[LB * LB];
     float oEt[LB * LB];          // E transposed (for the transposed planes)
+    float oUt[LB * LB];          // U transposed
     int8_t oC[LB * LB];
     int meta[4];                 // I, J, rows, cols
 };
+static_assert(offsetof(LeafBuf, LOr) % 16 == 0 && offsetof(LeafBuf, LIc) % 16 == 0 &&
+                  (LS * 4) % 16 == 0 && offsetof(LeafBuf, W) % 128 == 0 &&
+                  offsetof(LeafBuf, T) % 128 == 0 && offsetof(LeafBuf, R) % 128 == 0 &&
+                  sizeof(LeafBuf) % 128 == 0,
+              "staging buffer: 16-byte float4 rows, 128-byte box destinations");
 
 
 // The in-leaf wavefront, run by the solver warp; lane j owns column j and the element of row
@@ -96,10 +106,10 @@ __device__ __forceinline__ void solve_leaf(int lane, int rows, int cols, float q
                 e = w_star - w;
                 u = wT[k] + e;
                 B.oC[rr * LB + j] = (int8_t)q;
-                B.oW[rr * LB + j] = w;
                 B.oE[rr * LB + j] = e;
                 B.oEt[j * LB + rr] = e;
                 B.oU[rr * LB + j] = u;
+                B.oUt[j * LB + rr] = u;
             }
             wT[k + 1] = fmaf(lo[1], e, wT[k + 1]);
             wR[k + 1] = fmaf(__shfl_up_sync(0xffffffffu, u, 1), li[1], wR[k + 1]);

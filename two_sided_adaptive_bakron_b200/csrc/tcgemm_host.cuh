@@ -19,6 +19,11 @@ inline int plane_ld(int cols) { return (cols + 31) / 32 * 32; }
 int make_kmajor_map(CUtensorMap* map, const float* base, int rows, int kcols, int ld,
                     int box_rows);
 
+// 2-D fp32 tensor map of a row-major matrix (rows x cols, row stride ld elements, ld % 4 == 0,
+// base 16-byte aligned) with a box x box box, no swizzle (the box lands as a dense row-major
+// tile), out-of-range elements read as zero.
+int make_box_map(CUtensorMap* map, const float* base, int rows, int cols, int ld, int box);
+
 // Splits an fp32 matrix (rows x cols, row stride ld_src) into hi/lo planes (row stride
 // ld_dst). transpose = 1 writes the planes of the transposed matrix (cols x rows).
 void split_planes(const float* src, int rows, int cols, int ld_src, float* hi, float* lo,
