@@ -104,6 +104,10 @@ __device__ __forceinline__ void red_add_release_gpu(int* p, int v) {
     asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
+__device__ __forceinline__ void red_add_f32(float* p, float v) {
+    asm volatile("red.relaxed.gpu.global.add.f32 [%0], %1;" ::"l"(p), "f"(v) : "memory");
+}
+
 // Default limit of one dependency wait; BAKRON_SPIN_LIMIT_NS in the environment overrides it
 // (used by the tests to exercise the timeout path without hanging anything).
 uint64_t spin_limit_ns();

@@ -55,9 +55,8 @@ constexpr int LPB = SB / LB;         // leaves per super-block edge
 constexpr int TB = tc::BM;           // push tile edge (128)
 constexpr int BN = 128;
 constexpr int STAGES = 3;
-constexpr int NTH = 192;             // 6 warps in both roles
+constexpr int NTH = 256;             // 8 warps; each role uses 6 of them (see leaf_role, gemm_role)
 constexpr int NLOAD = 64;            // loader threads of one leaf group
-constexpr int LPAD = LB + 4;         // staging row stride (16-byte rows)
 constexpr int kMaxLeafCtas = 96;
 static_assert(TB % LB == 0 && SB % TB == 0, "tile nesting");
 
@@ -112,7 +111,7 @@ constexpr int kBox = LB * LB;        // floats of one 32 x 32 box
 
 struct alignas(128) LeafGroupSmem {
     LeafBuf buf[2];
-    // box-load path: NRING stages of two boxes; plain path: sA, sB with row stride LPAD
+    // box-load path: NRING stages of two boxes; plain path: sA, sB in stage 0
     alignas(128) float ring[NRING][2][kBox];
     uint64_t rfull[NRING];       // box loads of a ring stage landed
     uint64_t sbar;               // W* and the diagonal blocks landed
@@ -124,8 +123,7 @@ struct LeafCtaSmem {
     LeafGroupSmem g[2];
 };
 static_assert(sizeof(LeafGroupSmem) % 128 == 0 && offsetof(LeafGroupSmem, buf) % 128 == 0 &&
-                  offsetof(LeafGroupSmem, ring) % 128 == 0 && (LPAD * 4) % 16 == 0 &&
-                  2 * LB * LPAD <= NRING * 2 * kBox,
+                  offsetof(LeafGroupSmem, ring) % 128 == 0,
               "leaf group layout: 16-byte staging rows, 128-byte box destinations");
 
 constexpr size_t kGemmSmem = tc::gemm_smem_bytes<BN, STAGES>();
@@ -178,20 +176,48 @@ __device__ __forceinline__ void publish_rest(const FusedArgs& a, const LeafBuf& 
     }
 }
 
-// acc[i][j] += sum_k X[k][r0 + i] Y[k][c0 + j]: one source's contribution to a 4 x 4 block
-// (X, Y with row stride LD floats)
-template <int LD>
-__device__ __forceinline__ void product_4x4(const float* X, const float* Y, int r0, int c0,
+__device__ __forceinline__ void mma_16x8x8_tf32(float (&d)[4], const uint32_t (&a)[4],
+                                                const uint32_t (&b)[2]) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+// One source's contribution D[m][n] += sum_k X[k][m] Y[k][n] (X, Y: 32 x 32, row stride 32) on
+// the tensor cores, 3xTF32 as in the GEMM engine (hi = tf32 truncation, lo = x - hi,
+// hi*hi + hi*lo + lo*hi). Warp w of the group holds rows 16w .. 16w + 15, all 32 columns:
+// acc[nt] is the m16n8 accumulator of columns 8nt .. 8nt + 7 (element q at row
+// 16w + g + 8 (q >> 1), column 8nt + 2t + (q & 1), g = lane / 4, t = lane % 4).
+__device__ __forceinline__ void product_mma(const float* X, const float* Y, int w, int lane,
                                             float (&acc)[4][4]) {
-#pragma unroll 8
-    for (int kk = 0; kk < LB; ++kk) {
-        const float4 x = *reinterpret_cast<const float4*>(&X[kk * LD + r0]);
-        const float4 y = *reinterpret_cast<const float4*>(&Y[kk * LD + c0]);
-        const float xa[4] = {x.x, x.y, x.z, x.w}, ya[4] = {y.x, y.y, y.z, y.w};
+    const int g = lane >> 2, t = lane & 3;
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
+    for (int k0 = 0; k0 < LB; k0 += 8) {
+        const float a[4] = {X[(k0 + t) * LB + 16 * w + g], X[(k0 + t) * LB + 16 * w + g + 8],
+                            X[(k0 + t + 4) * LB + 16 * w + g], X[(k0 + t + 4) * LB + 16 * w + g + 8]};
+        uint32_t ah[4], al[4];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(xa[i], ya[j], acc[i][j]);
+        for (int i = 0; i < 4; ++i) {
+            const float h = sm100::tf32_hi(a[i]);
+            ah[i] = __float_as_uint(h);
+            al[i] = __float_as_uint(a[i] - h);
+        }
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt) {
+            const float b[2] = {Y[(k0 + t) * LB + 8 * nt + g], Y[(k0 + t + 4) * LB + 8 * nt + g]};
+            uint32_t bh[2], bl[2];
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                const float h = sm100::tf32_hi(b[i]);
+                bh[i] = __float_as_uint(h);
+                bl[i] = __float_as_uint(b[i] - h);
+            }
+            mma_16x8x8_tf32(acc[nt], ah, bh);
+            mma_16x8x8_tf32(acc[nt], ah, bl);
+            mma_16x8x8_tf32(acc[nt], al, bh);
+        }
     }
 }
 
@@ -231,8 +257,8 @@ __device__ void leaf_loaders(const FusedArgs& a, const LeafMaps* maps, LeafGroup
     const int m = a.m, n = a.n;
     const long long total = (long long)a.Mt * a.Nt;
     const bool box = a.box_loads != 0;
-    float* sA = &sm.ring[0][0][0];              // plain path staging
-    float* sB = sA + LB * LPAD;
+    float* sA = &sm.ring[0][0][0];              // plain path staging (row stride LB)
+    float* sB = sA + LB * LB;
     LeafWalker wk;
     wk.init();
     uint32_t rq = 0;                             // ring stages used so far (box path)
@@ -274,12 +300,12 @@ __device__ void leaf_loaders(const FusedArgs& a, const LeafMaps* maps, LeafGroup
             for (int q = 0; q < (LB * LB) / NLOAD; ++q) {
                 const int e = lt + q * NLOAD, r = e >> 5, c = e & 31;
                 B.W[e] = (r < rows && c < cols) ? __ldg(&a.Ws[(size_t)(i0 + r) * n + j0 + c]) : 0.f;
-                sA[r * LPAD + c] = (r < rows && c < rows) ? __ldg(&a.LO[(size_t)(i0 + r) * m + i0 + c]) : 0.f;
-                sB[r * LPAD + c] = (r < cols && c < cols) ? __ldg(&a.LI[(size_t)(j0 + r) * n + j0 + c]) : 0.f;
+                sA[r * LB + c] = (r < rows && c < rows) ? __ldg(&a.LO[(size_t)(i0 + r) * m + i0 + c]) : 0.f;
+                sB[r * LB + c] = (r < cols && c < cols) ? __ldg(&a.LI[(size_t)(j0 + r) * n + j0 + c]) : 0.f;
             }
             dLO = sA;
             dLI = sB;
-            dld = LPAD;
+            dld = LB;
         }
         if (lt < LB) {
             const float sv = (lt < rows) ? __ldg(&a.sc[i0 + lt]) : 0.f;
@@ -310,22 +336,23 @@ __device__ void leaf_loaders(const FusedArgs& a, const LeafMaps* maps, LeafGroup
             B.LOr[e] = (dd >= 1 && dd < LB && x + dd < LB) ? dLO[x * dld + x + dd] : 0.f;
             B.LIc[e] = (dd >= 1 && dd < LB && x - dd >= 0) ? dLI[(x - dd) * dld + x] : 0.f;
         }
-        // this thread's 4 x 4 block of the leaf's sums
-        const int r0 = (lt >> 3) * 4, c0 = (lt & 7) * 4;
+        // this thread's accumulator elements (m16n8 layout, see product_mma)
+        const int eg = lane >> 2, et = lane & 3;
         float accT[4][4], accR[4][4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
+        for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                float t = 0.f, r = 0.f;
+            for (int q = 0; q < 4; ++q) {
+                const int r = 16 * lw + eg + 8 * (q >> 1), c = 8 * nt + 2 * et + (q & 1);
+                float tv = 0.f, rv = 0.f;
                 if (!box) {
-                    const bool ok = r0 + i < rows && c0 + j < cols;
-                    const size_t o = (size_t)(i0 + r0 + i) * n + j0 + c0 + j;
-                    t = ok ? __ldcg(&a.Tf[o]) : 0.f;
-                    r = ok ? __ldcg(&a.Rf[o]) : 0.f;
+                    const bool ok = r < rows && c < cols;
+                    const size_t o = (size_t)(i0 + r) * n + j0 + c;
+                    tv = ok ? __ldcg(&a.Tf[o]) : 0.f;
+                    rv = ok ? __ldcg(&a.Rf[o]) : 0.f;
                 }
-                accT[i][j] = t;
-                accR[i][j] = r;
+                accT[nt][q] = tv;
+                accR[nt][q] = rv;
             }
         const NearField nf(I, J, A, C);
         // the older sources finished at least a diagonal ago: warp 0's lanes check their flags
@@ -363,17 +390,22 @@ __device__ void leaf_loaders(const FusedArgs& a, const LeafMaps* maps, LeafGroup
                 for (int idx = 0; idx < min(NRING, nf.nold); ++idx) issue(idx);
             }
             for (int idx = 0; idx < nf.nsrc; ++idx) {
-                if (idx >= nf.nold && lead) {    // a recent source: its flag first
-                    int Is, Js;
-                    nf.source(idx, Is, Js);
-                    if (wait_flag(&a.flags[(size_t)Is * a.Nt + Js], a.abort_word, a.status, a.limit_ns)) {
-                        asm volatile("fence.proxy.async.global;" ::: "memory");
-                        issue(idx);
-                    } else {
-                        sm.stop = 1;
+                if (idx == nf.nold) {
+                    // the recent sources (at most two, finishing about together): each one's
+                    // boxes go out as soon as its flag is up
+                    if (lead) {
+                        for (int r = idx; r < nf.nsrc; ++r) {
+                            int Is, Js;
+                            nf.source(r, Is, Js);
+                            if (!wait_flag(&a.flags[(size_t)Is * a.Nt + Js], a.abort_word,
+                                           a.status, a.limit_ns)) {
+                                sm.stop = 1;
+                                break;
+                            }
+                            asm volatile("fence.proxy.async.global;" ::: "memory");
+                            issue(r);
+                        }
                     }
-                }
-                if (idx >= nf.nold) {
                     group_sync(g);
                     if (*(volatile int*)&sm.stop) { stop = true; break; }
                 }
@@ -386,8 +418,8 @@ __device__ void leaf_loaders(const FusedArgs& a, const LeafMaps* maps, LeafGroup
                 int Is, Js;
                 const bool vert = nf.source(idx, Is, Js);
                 if (!stop) {
-                    if (vert) product_4x4<LB>(sm.ring[st][0], sm.ring[st][1], r0, c0, accT);
-                    else product_4x4<LB>(sm.ring[st][0], sm.ring[st][1], r0, c0, accR);
+                    if (vert) product_mma(sm.ring[st][0], sm.ring[st][1], lw, lane, accT);
+                    else product_mma(sm.ring[st][0], sm.ring[st][1], lw, lane, accR);
                 }
                 group_sync(g);   // the stage is free again
                 if (*(volatile int*)&sm.stop) { stop = true; break; }
@@ -437,16 +469,16 @@ __device__ void leaf_loaders(const FusedArgs& a, const LeafMaps* maps, LeafGroup
 #pragma unroll
                 for (int q = 0; q < 16; ++q) {
                     const int e = lt + q * NLOAD, r = e >> 5, c = e & 31;
-                    sA[r * LPAD + c] = pf[q];        // sA[k = source row / column][leaf row]
-                    sB[r * LPAD + c] = pf[16 + q];   // sB[k][leaf col]
+                    sA[r * LB + c] = pf[q];        // sA[k = source row / column][leaf row]
+                    sB[r * LB + c] = pf[16 + q];   // sB[k][leaf col]
                 }
                 if (idx + 1 < nf.nsrc) {
                     if (!wait_recent(idx + 1)) { stop = true; break; }
                     fetch(idx + 1);
                 }
                 group_sync(g);   // sA / sB complete
-                if (vert) product_4x4<LPAD>(sA, sB, r0, c0, accT);
-                else product_4x4<LPAD>(sA, sB, r0, c0, accR);
+                if (vert) product_mma(sA, sB, lw, lane, accT);
+                else product_mma(sA, sB, lw, lane, accR);
             }
         }
         if (stop) break;
@@ -457,14 +489,15 @@ __device__ void leaf_loaders(const FusedArgs& a, const LeafMaps* maps, LeafGroup
         group_sync(g);
         if (*(volatile int*)&sm.stop) break;
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
+        for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int o = (r0 + i) * LB + c0 + j;
-                const bool ok = r0 + i < rows && c0 + j < cols;
+            for (int q = 0; q < 4; ++q) {
+                const int r = 16 * lw + eg + 8 * (q >> 1), c = 8 * nt + 2 * et + (q & 1);
+                const int o = r * LB + c;
+                const bool ok = r < rows && c < cols;
                 // the box path already holds the far sums in B.T / B.R
-                B.T[o] = ok ? (box ? B.T[o] : 0.f) + accT[i][j] : 0.f;
-                B.R[o] = ok ? (box ? B.R[o] : 0.f) + accR[i][j] : 0.f;
+                B.T[o] = ok ? (box ? B.T[o] : 0.f) + accT[nt][q] : 0.f;
+                B.R[o] = ok ? (box ? B.R[o] : 0.f) + accR[nt][q] : 0.f;
             }
         group_sync(g);
         if (lead) sm100::mbar_arrive(&sm.full[b]);
@@ -562,11 +595,14 @@ __device__ void leaf_role(const FusedArgs& a, const LeafMaps* maps, uint8_t* sme
         sm100::fence_mbar_init();
     }
     __syncthreads();
-    // group g: loader warps 2g and 2g + 1, solver warp 4 + g
-    const int g = warp < 4 ? (warp >> 1) : (warp - 4);
+    // warp w runs on SM sub-partition w % 4: the two solver warps (0, 1) get sub-partitions 0
+    // and 1 to themselves, the loader warps of group g are 2 + g and 6 + g (sub-partition
+    // 2 + g), warps 4 and 5 have nothing to do
+    if (warp == 4 || warp == 5) return;
+    const int g = warp < 2 ? warp : (warp & 1);
     const int slot = blockIdx.x * 2 + g, nslots = a.leaf_ctas * 2;
-    if (warp < 4) leaf_loaders(a, maps, cs.g[g], g, warp & 1, lane, slot, nslots);
-    else leaf_solver(a, cs.g[g], lane, slot, nslots);
+    if (warp < 2) leaf_solver(a, cs.g[g], lane, slot, nslots);
+    else leaf_loaders(a, maps, cs.g[g], g, warp >> 2, lane, slot, nslots);
 }
 
 // ------------------------------------------------------------------------------ push tasks
@@ -612,6 +648,10 @@ __device__ __forceinline__ PushTask decode_task(const FusedArgs& a, int t) {
     return p;
 }
 
+__device__ __forceinline__ void gemm_sync() {   // the six warps of the push pipeline
+    asm volatile("bar.sync 2, 192;" ::: "memory");
+}
+
 __device__ __forceinline__ void epi_sync() {
     asm volatile("bar.sync 1, 128;" ::: "memory");
 }
@@ -638,6 +678,7 @@ __device__ void gemm_role(const CUtensorMap* loth, const CUtensorMap* lotl, cons
     volatile int* s_go = s_abort + 1;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (warp >= 6) return;   // the push pipeline uses warps 0 .. 5
     const int gid = blockIdx.x - a.leaf_ctas, ng = gridDim.x - a.leaf_ctas;
     const int total = __ldg(&a.task_pre[a.nsb]);
 
@@ -660,7 +701,7 @@ __device__ void gemm_role(const CUtensorMap* loth, const CUtensorMap* lotl, cons
         sm100::tmem_relinquish();
     }
     sm100::tc_fence_before();
-    __syncthreads();
+    gemm_sync();
     sm100::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
@@ -796,14 +837,12 @@ __device__ void gemm_role(const CUtensorMap* loth, const CUtensorMap* lotl, cons
                 __syncwarp();
                 const int gc = p.tc * TB + c0 + lane;
                 if (gc < a.n) {
-                    float old[32];
-#pragma unroll
-                    for (int rr = 0; rr < 32; ++rr)
-                        old[rr] = (row0 + rr < a.m) ? __ldcg(&Cm[(size_t)(row0 + rr) * a.n + gc]) : 0.f;
+                    // one fp32 add per element and source, in source order (the tile counter):
+                    // the same sums as a load-add-store, without waiting for the loads
 #pragma unroll
                     for (int rr = 0; rr < 32; ++rr)
                         if (row0 + rr < a.m)
-                            __stcg(&Cm[(size_t)(row0 + rr) * a.n + gc], old[rr] + stage[rr * 33 + lane]);
+                            red_add_f32(&Cm[(size_t)(row0 + rr) * a.n + gc], stage[rr * 33 + lane]);
                 }
                 __syncwarp();
             }
@@ -817,7 +856,7 @@ __device__ void gemm_role(const CUtensorMap* loth, const CUtensorMap* lotl, cons
     }
     __syncwarp();
     sm100::tc_fence_before();
-    __syncthreads();
+    gemm_sync();
     if (warp == 1) sm100::tmem_dealloc(tmem, Cf::kTmemCols);
 }
 
