@@ -48,7 +48,9 @@ namespace {
 using leaf::LB;
 using leaf::LeafBuf;
 using leaf::LS;
-using leaf::solve_leaf;
+using leaf::LeafXchg;
+using leaf::solve_leaf_chain;
+using leaf::solve_leaf_pushes;
 
 constexpr int SB = 256;              // super-block edge
 constexpr int LPB = SB / LB;         // leaves per super-block edge
@@ -117,6 +119,8 @@ struct alignas(128) LeafGroupSmem {
     uint64_t sbar;               // W* and the diagonal blocks landed
     uint64_t tbar;               // T_far and R_far landed
     uint64_t full[2], empty[2];
+    LeafXchg xch;                // solver / helper exchange
+    int go;                      // solver -> helper: this leaf is on
     int stop;
 };
 struct LeafCtaSmem {
@@ -520,7 +524,7 @@ __device__ void leaf_loaders(const FusedArgs& a, const LeafMaps* maps, LeafGroup
 
 // ------------------------------------------------------------------------------ leaf solver
 __device__ void leaf_solver(const FusedArgs& a, LeafGroupSmem& sm, int lane, int slot,
-                            int nslots) {
+                            int nslots, int bar) {
     const int n = a.n;
     const long long total = (long long)a.Mt * a.Nt;
     int k = 0;
@@ -530,13 +534,17 @@ __device__ void leaf_solver(const FusedArgs& a, LeafGroupSmem& sm, int lane, int
         bool ok = true;
         if (lane == 0) ok = sm100::mbar_wait(&sm.full[b], (k >> 1) & 1, a.status, a.limit_ns);
         ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-        if (!ok || ld_acquire_gpu(a.abort_word) != 0) {
+        if (ok && ld_acquire_gpu(a.abort_word) != 0) ok = false;
+        // the helper follows this decision (it never waits on anything but the pair barrier)
+        if (lane == 0) sm.go = ok ? 1 : 0;
+        leaf::pair_sync(bar);
+        if (!ok) {
             if (lane == 0) atomicExch(a.abort_word, 1);
             break;
         }
         const int I = B.meta[0], J = B.meta[1], rows = B.meta[2], cols = B.meta[3];
         const int i0 = I * LB, j0 = J * LB;
-        solve_leaf(lane, rows, cols, a.qlo, a.qhi, B, a.status);
+        solve_leaf_chain(lane, rows, cols, a.qlo, a.qhi, B, sm.xch, bar, a.status);
         __syncwarp();
         // what the next leaves read: E (vertical pulls, lane = column) and U^T (horizontal pulls,
         // lane = row), then the flag
@@ -578,6 +586,18 @@ __device__ void leaf_solver(const FusedArgs& a, LeafGroupSmem& sm, int lane, int
     }
 }
 
+// The helper warp of a solver: the distance >= 2 pushes of every leaf the solver takes.
+__device__ void leaf_helper(const FusedArgs& a, LeafGroupSmem& sm, int lane, int slot, int nslots,
+                            int bar) {
+    const long long total = (long long)a.Mt * a.Nt;
+    int k = 0;
+    for (long long gi = slot; gi < total; gi += nslots, ++k) {
+        leaf::pair_sync(bar);             // the solver has decided (and seen the buffer full)
+        if (!*(volatile int*)&sm.go) break;
+        solve_leaf_pushes(lane, sm.buf[k & 1], sm.xch, bar);
+    }
+}
+
 __device__ void leaf_role(const FusedArgs& a, const LeafMaps* maps, uint8_t* smem) {
     LeafCtaSmem& cs = *reinterpret_cast<LeafCtaSmem*>(smem);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -595,13 +615,13 @@ __device__ void leaf_role(const FusedArgs& a, const LeafMaps* maps, uint8_t* sme
         sm100::fence_mbar_init();
     }
     __syncthreads();
-    // warp w runs on SM sub-partition w % 4: the two solver warps (0, 1) get sub-partitions 0
-    // and 1 to themselves, the loader warps of group g are 2 + g and 6 + g (sub-partition
-    // 2 + g), warps 4 and 5 have nothing to do
-    if (warp == 4 || warp == 5) return;
-    const int g = warp < 2 ? warp : (warp & 1);
+    // warp w runs on SM sub-partition w % 4: group g's solver warp (g) and its helper (4 + g)
+    // share sub-partition g, its loader warps are 2 + g and 6 + g (sub-partition 2 + g).
+    // Named barriers: 1 + g for the loaders of group g, 3 + g for its solver and helper.
+    const int g = warp & 1;
     const int slot = blockIdx.x * 2 + g, nslots = a.leaf_ctas * 2;
-    if (warp < 2) leaf_solver(a, cs.g[g], lane, slot, nslots);
+    if (warp < 2) leaf_solver(a, cs.g[g], lane, slot, nslots, 3 + g);
+    else if (warp == 4 || warp == 5) leaf_helper(a, cs.g[g], lane, slot, nslots, 3 + g);
     else leaf_loaders(a, maps, cs.g[g], g, warp >> 2, lane, slot, nslots);
 }
 

@@ -137,5 +137,139 @@ __device__ __forceinline__ void solve_leaf(int lane, int rows, int cols, float q
     if (bad) set_status(status, BAKRON_ERR_NONFINITE);
 }
 
+// ------------------------------------------------------------------------------ two warps
+// The same wavefront split over two warps of one SM sub-partition, with the same additions in
+// the same order (so the same results): the solver warp runs the element chain (the slot's
+// sum, Q, e, u and the distance-1 terms), the helper warp the distance >= 2 pushes one step
+// behind. Round rho: the solver computes step rho from the helper's partial sums of slot rho
+// (everything from steps <= rho - 2 on top of T, R) plus its own distance-1 terms of step
+// rho - 1; the helper pushes step rho - 1 and publishes slot rho + 1. One named barrier of the
+// two warps closes each round.
+struct LeafXchg {
+    float part[2][2][LB];        // [slot & 1][T, R][lane]: the helper's partial sums
+    float eu[2][2][LB];          // [step & 1][e, u][lane]: the solver's step results
+};
+
+__device__ __forceinline__ void pair_sync(int id) {
+    asm volatile("bar.sync %0, 64;" ::"r"(id) : "memory");
+}
+
+__device__ __forceinline__ void solve_leaf_chain(int lane, int rows, int cols, float qlo,
+                                                 float qhi, LeafBuf& B, LeafXchg& X, int bar,
+                                                 int* status) {
+    const int j = lane;
+    const bool colok = j < cols;
+    const float li1 = B.LIc[j * LS + 1];
+    float lo1p = 0.f, ep = 0.f, usp = 0.f;   // distance-1 terms of the previous step
+    bool bad = false;
+    pair_sync(bar);                          // the helper's slots 0 and 1 are in place
+#pragma unroll 1
+    for (int s = 0; s < NSLOT; ++s) {
+        const int r = s - j;
+        const bool inleaf = (r >= 0) && (r < LB);
+        const int rr = inleaf ? r : 0;
+        const bool act = inleaf && (r < rows) && colok;
+        const float tT = fmaf(lo1p, ep, X.part[s & 1][0][j]);
+        const float tR = fmaf(usp, li1, X.part[s & 1][1][j]);
+        const float lo1 = B.LOr[rr * LS + 1];
+        const float w_star = B.W[rr * LB + j];
+        const float sr = B.S[rr], inv = B.S[LB + rr];
+        float e = 0.f, u = 0.f;
+        if (act) {
+            const float pre = w_star + tT + tR;
+            float q = 0.f;
+            if (sr > 0.f) {
+                float x = pre * inv;
+                const float t = fabsf(x - rintf(x));
+                if (0.5f - t < 1e-6f * fmaxf(1.f, fabsf(x))) x = __fdiv_rn(pre, sr);
+                q = fminf(fmaxf(rintf(x), qlo), qhi);
+            }
+            bad |= !isfinite(pre);
+            const float w = sr * q;
+            e = w_star - w;
+            u = tT + e;
+            B.oC[rr * LB + j] = (int8_t)q;
+            B.oE[rr * LB + j] = e;
+            B.oEt[j * LB + rr] = e;
+            B.oU[rr * LB + j] = u;
+            B.oUt[j * LB + rr] = u;
+        }
+        X.eu[s & 1][0][j] = e;
+        X.eu[s & 1][1][j] = u;
+        lo1p = lo1;
+        ep = e;
+        usp = __shfl_up_sync(0xffffffffu, u, 1);
+        pair_sync(bar);
+    }
+    pair_sync(bar);                          // the helper's last round
+    if (bad) set_status(status, BAKRON_ERR_NONFINITE);
+}
+
+__device__ __forceinline__ void solve_leaf_pushes(int lane, LeafBuf& B, LeafXchg& X, int bar) {
+    const int j = lane;
+    float li[LB];
+#pragma unroll
+    for (int q = 0; q < LB / 4; ++q) {
+        const float4 v = *reinterpret_cast<const float4*>(&B.LIc[j * LS + 4 * q]);
+        li[4 * q] = v.x; li[4 * q + 1] = v.y; li[4 * q + 2] = v.z; li[4 * q + 3] = v.w;
+    }
+    float wT[WIN], wR[WIN];
+#pragma unroll
+    for (int t = 0; t < WIN; ++t) {
+        const int r = t - j;
+        const bool ok = (r >= 0) && (r < LB);
+        const int rr = ok ? r : 0;
+        wT[t] = ok ? B.T[rr * LB + j] : 0.f;
+        wR[t] = ok ? B.R[rr * LB + j] : 0.f;
+    }
+    X.part[0][0][j] = wT[0];
+    X.part[0][1][j] = wR[0];
+    X.part[1][0][j] = wT[1];
+    X.part[1][1][j] = wR[1];
+    pair_sync(bar);                          // slots 0 and 1 are in place
+    pair_sync(bar);                          // round 0: step 0 is being computed
+#pragma unroll 1
+    for (int s0 = 0; s0 < NSLOT; s0 += UW) {
+#pragma unroll
+        for (int k = 0; k < UW; ++k) {
+            const int s = s0 + k;            // step pushed in round s + 1
+            if (s < NSLOT) {
+                const int r = s - j;
+                const bool inleaf = (r >= 0) && (r < LB);
+                const int rr = inleaf ? r : 0;
+                float lo[LB];
+#pragma unroll
+                for (int q = 0; q < LB / 4; ++q) {
+                    const float4 v = *reinterpret_cast<const float4*>(&B.LOr[rr * LS + 4 * q]);
+                    lo[4 * q] = v.x; lo[4 * q + 1] = v.y; lo[4 * q + 2] = v.z; lo[4 * q + 3] = v.w;
+                }
+                const float e = X.eu[s & 1][0][j], u = X.eu[s & 1][1][j];
+#pragma unroll
+                for (int d = 2; d < LB; ++d) wT[k + d] = fmaf(lo[d], e, wT[k + d]);
+#pragma unroll
+                for (int d = 2; d < LB; ++d)
+                    wR[k + d] = fmaf(__shfl_up_sync(0xffffffffu, u, d), li[d], wR[k + d]);
+                // slot s + 2 has all its distance >= 2 terms now
+                X.part[(s + 2) & 1][0][j] = wT[k + 2];
+                X.part[(s + 2) & 1][1][j] = wR[k + 2];
+                pair_sync(bar);
+            }
+        }
+#pragma unroll
+        for (int t = 0; t < WIN - UW; ++t) {
+            wT[t] = wT[t + UW];
+            wR[t] = wR[t + UW];
+        }
+#pragma unroll
+        for (int t = WIN - UW; t < WIN; ++t) {
+            const int r = s0 + UW + t - j;
+            const bool ok = (r >= 0) && (r < LB);
+            const int rr = ok ? r : 0;
+            wT[t] = ok ? B.T[rr * LB + j] : 0.f;
+            wR[t] = ok ? B.R[rr * LB + j] : 0.f;
+        }
+    }
+}
+
 }  // namespace leaf
 }  // namespace bakron
