@@ -119,6 +119,7 @@ struct alignas(128) LeafGroupSmem {
     uint64_t sbar;               // W* and the diagonal blocks landed
     uint64_t tbar;               // T_far and R_far landed
     uint64_t full[2], empty[2];
+    uint64_t solved[2];          // the solver is done with the leaf's wavefront (outputs in B)
     LeafXchg xch;                // solver / helper exchange
     int go;                      // solver -> helper: this leaf is on
     int stop;
@@ -164,7 +165,7 @@ __device__ __forceinline__ void group_sync(int g) {
 }
 
 // Codes and W of the leaf solved from B (W = s_r q, formed as in the solver); run by the
-// group's loader threads before they stage a new leaf into B.
+// group's loader threads before they restage B.
 __device__ __forceinline__ void publish_rest(const FusedArgs& a, const LeafBuf& B, int lt) {
     const int I = B.meta[0], J = B.meta[1], rows = B.meta[2], cols = B.meta[3];
     const int i0 = I * LB, j0 = J * LB;
@@ -173,9 +174,9 @@ __device__ __forceinline__ void publish_rest(const FusedArgs& a, const LeafBuf& 
         const int e = lt + q * NLOAD, r = e >> 5, c = e & 31;
         if (r < rows && c < cols) {
             const size_t o = (size_t)(i0 + r) * a.n + j0 + c;
-            const int8_t q = B.oC[r * LB + c];
-            a.codes[o] = q;
-            a.Wq[o] = B.S[r] * (float)q;
+            const int8_t q8 = B.oC[r * LB + c];
+            a.codes[o] = q8;
+            a.Wq[o] = B.S[r] * (float)q8;
         }
     }
 }
@@ -266,6 +267,7 @@ __device__ void leaf_loaders(const FusedArgs& a, const LeafMaps* maps, LeafGroup
     LeafWalker wk;
     wk.init();
     uint32_t rq = 0;                             // ring stages used so far (box path)
+    int prevI = -1, prevJ = -1;                  // the group's previous leaf
     int k = 0;
     for (long long gi = slot; gi < total; gi += nslots, ++k) {
         const int b = k & 1;
@@ -359,6 +361,11 @@ __device__ void leaf_loaders(const FusedArgs& a, const LeafMaps* maps, LeafGroup
                 accR[nt][q] = rv;
             }
         const NearField nf(I, J, A, C);
+        // the recent horizontal source (I, J-1) is usually this group's previous leaf: its U is
+        // still in the other buffer, so it needs no global round trip (box path only)
+        const bool local_h = box && nf.nhs > 0 && prevI == I && prevJ == J - 1;
+        const int hloc = nf.nsrc - 1;            // its index in the source list
+        const LeafBuf& P = sm.buf[b ^ 1];        // the previous leaf's buffer
         // the older sources finished at least a diagonal ago: warp 0's lanes check their flags
         if (lw == 0) {
             bool ok = true;
@@ -379,6 +386,11 @@ __device__ void leaf_loaders(const FusedArgs& a, const LeafMaps* maps, LeafGroup
                 int Is, Js;
                 const bool vert = nf.source(idx, Is, Js);
                 const uint32_t q = rq + idx, st = q % NRING;
+                if (local_h && idx == hloc) {   // only L_I[Js cols][leaf cols]; U is in P
+                    sm100::mbar_arrive_expect_tx(&sm.rfull[st], kBox * 4);
+                    sm100::tma_load_2d(sm.ring[st][1], &maps->li, j0, Js * LB, &sm.rfull[st]);
+                    return;
+                }
                 sm100::mbar_arrive_expect_tx(&sm.rfull[st], 2 * kBox * 4);
                 if (vert) {   // L_O[Is rows][leaf rows], E[Is rows][leaf cols]
                     sm100::tma_load_2d(sm.ring[st][0], &maps->lo, i0, Is * LB, &sm.rfull[st]);
@@ -398,7 +410,9 @@ __device__ void leaf_loaders(const FusedArgs& a, const LeafMaps* maps, LeafGroup
                     // the recent sources (at most two, finishing about together): each one's
                     // boxes go out as soon as its flag is up
                     if (lead) {
+                        if (local_h) issue(hloc);
                         for (int r = idx; r < nf.nsrc; ++r) {
+                            if (local_h && r == hloc) continue;
                             int Is, Js;
                             nf.source(r, Is, Js);
                             if (!wait_flag(&a.flags[(size_t)Is * a.Nt + Js], a.abort_word,
@@ -421,9 +435,19 @@ __device__ void leaf_loaders(const FusedArgs& a, const LeafMaps* maps, LeafGroup
                 if (__any_sync(0xffffffffu, stop)) { sm.stop = 1; }
                 int Is, Js;
                 const bool vert = nf.source(idx, Is, Js);
+                const bool loc = local_h && idx == hloc;
+                if (loc) {   // the previous leaf's wavefront is done: its U^T is P.oUt
+                    if (lead && !sm100::mbar_wait(&sm.solved[b ^ 1], ((k - 1) >> 1) & 1, a.status,
+                                                  a.limit_ns)) {
+                        atomicExch(a.abort_word, 1);
+                        sm.stop = 1;
+                    }
+                    group_sync(g);
+                    if (*(volatile int*)&sm.stop) stop = true;
+                }
                 if (!stop) {
                     if (vert) product_mma(sm.ring[st][0], sm.ring[st][1], lw, lane, accT);
-                    else product_mma(sm.ring[st][0], sm.ring[st][1], lw, lane, accR);
+                    else product_mma(loc ? P.oUt : sm.ring[st][0], sm.ring[st][1], lw, lane, accR);
                 }
                 group_sync(g);   // the stage is free again
                 if (*(volatile int*)&sm.stop) { stop = true; break; }
@@ -505,9 +529,11 @@ __device__ void leaf_loaders(const FusedArgs& a, const LeafMaps* maps, LeafGroup
             }
         group_sync(g);
         if (lead) sm100::mbar_arrive(&sm.full[b]);
+        prevI = I;
+        prevJ = J;
     }
     if (lead && *(volatile int*)&sm.stop) atomicExch(a.abort_word, 1);
-    // the last (up to) two leaves: wait until they are solved, then publish the rest
+    // the last (up to) two leaves: wait until they are done with, then publish the rest
     if (!*(volatile int*)&sm.stop) {
         for (int kk = (k >= 2 ? k - 2 : 0); kk < k; ++kk) {
             const int b = kk & 1;
@@ -546,8 +572,9 @@ __device__ void leaf_solver(const FusedArgs& a, LeafGroupSmem& sm, int lane, int
         const int i0 = I * LB, j0 = J * LB;
         solve_leaf_chain(lane, rows, cols, a.qlo, a.qhi, B, sm.xch, bar, a.status);
         __syncwarp();
+        if (lane == 0) sm100::mbar_arrive(&sm.solved[b]);
         // what the next leaves read: E (vertical pulls, lane = column) and U^T (horizontal pulls,
-        // lane = row), then the flag
+        // lane = row), then the flag; the loaders publish the rest
         if (lane < cols) {
             for (int r = 0; r < rows; ++r)
                 __stcg(&a.E[(size_t)(i0 + r) * n + j0 + lane], B.oE[r * LB + lane]);
@@ -558,9 +585,27 @@ __device__ void leaf_solver(const FusedArgs& a, LeafGroupSmem& sm, int lane, int
         }
         __threadfence();
         __syncwarp();
-        if (lane == 0) st_release_gpu(&a.flags[(size_t)I * a.Nt + J], 1);
+        if (lane == 0) {
+            st_release_gpu(&a.flags[(size_t)I * a.Nt + J], 1);
+            sm100::mbar_arrive(&sm.empty[b]);
+        }
+    }
+}
+
+__device__ void leaf_helper(const FusedArgs& a, LeafGroupSmem& sm, int lane, int slot, int nslots,
+                            int bar) {
+    const long long total = (long long)a.Mt * a.Nt;
+    int k = 0;
+    for (long long gi = slot; gi < total; gi += nslots, ++k) {
+        leaf::pair_sync(bar);             // the solver has decided (and seen the buffer full)
+        if (!*(volatile int*)&sm.go) break;
+        const int b = k & 1;
+        LeafBuf& B = sm.buf[b];
+        solve_leaf_pushes(lane, B, sm.xch, bar);
         // what the pushes read: the U planes (lane = column) and the E^T planes (lane = row),
-        // then the super-block count
+        // then the leaf counts into its super-block; this depends on the leaf's own solve only
+        const int I = B.meta[0], J = B.meta[1], rows = B.meta[2], cols = B.meta[3];
+        const int i0 = I * LB, j0 = J * LB;
         if (lane < cols) {
             for (int r = 0; r < rows; ++r) {
                 const float u = B.oU[r * LB + lane], uh = sm100::tf32_hi(u);
@@ -586,18 +631,6 @@ __device__ void leaf_solver(const FusedArgs& a, LeafGroupSmem& sm, int lane, int
     }
 }
 
-// The helper warp of a solver: the distance >= 2 pushes of every leaf the solver takes.
-__device__ void leaf_helper(const FusedArgs& a, LeafGroupSmem& sm, int lane, int slot, int nslots,
-                            int bar) {
-    const long long total = (long long)a.Mt * a.Nt;
-    int k = 0;
-    for (long long gi = slot; gi < total; gi += nslots, ++k) {
-        leaf::pair_sync(bar);             // the solver has decided (and seen the buffer full)
-        if (!*(volatile int*)&sm.go) break;
-        solve_leaf_pushes(lane, sm.buf[k & 1], sm.xch, bar);
-    }
-}
-
 __device__ void leaf_role(const FusedArgs& a, const LeafMaps* maps, uint8_t* smem) {
     LeafCtaSmem& cs = *reinterpret_cast<LeafCtaSmem*>(smem);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -605,7 +638,8 @@ __device__ void leaf_role(const FusedArgs& a, const LeafMaps* maps, uint8_t* sme
         for (int g = 0; g < 2; ++g) {
             for (int b = 0; b < 2; ++b) {
                 sm100::mbar_init(&cs.g[g].full[b], 1);
-                sm100::mbar_init(&cs.g[g].empty[b], 1);
+                sm100::mbar_init(&cs.g[g].empty[b], 2);   // solver and helper
+                sm100::mbar_init(&cs.g[g].solved[b], 1);
             }
             for (int r = 0; r < NRING; ++r) sm100::mbar_init(&cs.g[g].rfull[r], 1);
             sm100::mbar_init(&cs.g[g].sbar, 1);
@@ -616,13 +650,14 @@ __device__ void leaf_role(const FusedArgs& a, const LeafMaps* maps, uint8_t* sme
     }
     __syncthreads();
     // warp w runs on SM sub-partition w % 4: group g's solver warp (g) and its helper (4 + g)
-    // share sub-partition g, its loader warps are 2 + g and 6 + g (sub-partition 2 + g).
-    // Named barriers: 1 + g for the loaders of group g, 3 + g for its solver and helper.
-    const int g = warp & 1;
+    // share sub-partition g; its two loader warps (2, 3 for group 0, 6, 7 for group 1) sit on
+    // sub-partitions 2 and 3, one each. Named barriers: 1 + g for the loaders of group g,
+    // 3 + g for its solver and helper.
+    const int g = (warp == 1 || warp == 5 || warp >= 6) ? 1 : 0;
     const int slot = blockIdx.x * 2 + g, nslots = a.leaf_ctas * 2;
     if (warp < 2) leaf_solver(a, cs.g[g], lane, slot, nslots, 3 + g);
     else if (warp == 4 || warp == 5) leaf_helper(a, cs.g[g], lane, slot, nslots, 3 + g);
-    else leaf_loaders(a, maps, cs.g[g], g, warp >> 2, lane, slot, nslots);
+    else leaf_loaders(a, maps, cs.g[g], g, warp & 1, lane, slot, nslots);
 }
 
 // ------------------------------------------------------------------------------ push tasks
