@@ -68,7 +68,11 @@ def test_round_codes_identical_to_oracle_small(bk, name):
 
 @pytest.mark.parametrize("m,n,bits,seed", [(1, 1, 2, 0), (1, 70, 3, 1), (70, 1, 2, 2),
                                            (7, 300, 2, 3), (33, 65, 4, 4), (64, 31, 2, 5),
-                                           (100, 37, 3, 6), (31, 33, 8, 7), (96, 96, 2, 8)])
+                                           (100, 37, 3, 6), (31, 33, 8, 7), (96, 96, 2, 8),
+                                           # several super-blocks (far-field pushes) with partial
+                                           # leaves and tiles: row strides that allow tensor box
+                                           # loads (multiples of 4) and ones that do not
+                                           (520, 780, 3, 9), (515, 777, 3, 10)])
 def test_round_codes_identical_ragged(bk, m, n, bits, seed):
     Ws, HO, HI, s, _ = random_problem(m, n, bits, seed)
     LO32, LI32 = _oracle_factors32(HO, HI)

@@ -380,80 +380,83 @@ __device__ void leaf_loaders(const FusedArgs& a, const LeafMaps* maps, LeafGroup
         group_sync(g);   // also: the skew is done with the diagonal blocks in ring stage 0
         if (*(volatile int*)&sm.stop) break;
         bool stop = false;
+        float acc[2][4][4];                      // box path: this warp's direction, all 32 rows
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                for (int q = 0; q < 4; ++q) acc[mt][nt][q] = 0.f;
         if (box) {
-            // ring: source idx lives in stage (rq + idx) % NRING
-            auto issue = [&](int idx) {
-                int Is, Js;
-                const bool vert = nf.source(idx, Is, Js);
-                const uint32_t q = rq + idx, st = q % NRING;
-                if (local_h && idx == hloc) {   // only L_I[Js cols][leaf cols]; U is in P
+            // loader warp lw takes one direction with its own two ring stages (2 lw, 2 lw + 1):
+            // lw = 0 the vertical sources (E, into T), lw = 1 the horizontal ones (U, into R);
+            // each source's product covers all 32 rows, so the warps never wait for each other
+            const bool vdir = lw == 0;
+            const int nold_d = vdir ? nf.nv : nf.nh;
+            const int ns = nold_d + ((vdir ? nf.nvs : nf.nhs) > 0 ? 1 : 0);
+            const bool loc = !vdir && local_h;   // the recent horizontal source is local
+            auto srcd = [&](int i) -> int {      // the source's leaf index along the direction
+                return i < nold_d ? (vdir ? nf.va : nf.ha) + i : (vdir ? I : J) - 1;
+            };
+            auto issue = [&](int i) {
+                const uint32_t q = rq + i, st = 2 * lw + (q & 1);
+                const int sl = srcd(i);
+                if (loc && i == nold_d) {        // only L_I[sl cols][leaf cols]; U is in P
                     sm100::mbar_arrive_expect_tx(&sm.rfull[st], kBox * 4);
-                    sm100::tma_load_2d(sm.ring[st][1], &maps->li, j0, Js * LB, &sm.rfull[st]);
+                    sm100::tma_load_2d(sm.ring[st][1], &maps->li, j0, sl * LB, &sm.rfull[st]);
                     return;
                 }
                 sm100::mbar_arrive_expect_tx(&sm.rfull[st], 2 * kBox * 4);
-                if (vert) {   // L_O[Is rows][leaf rows], E[Is rows][leaf cols]
-                    sm100::tma_load_2d(sm.ring[st][0], &maps->lo, i0, Is * LB, &sm.rfull[st]);
-                    sm100::tma_load_2d(sm.ring[st][1], &maps->e, j0, Is * LB, &sm.rfull[st]);
-                } else {      // U^T[Js cols][leaf rows], L_I[Js cols][leaf cols]
-                    sm100::tma_load_2d(sm.ring[st][0], &maps->ut, i0, Js * LB, &sm.rfull[st]);
-                    sm100::tma_load_2d(sm.ring[st][1], &maps->li, j0, Js * LB, &sm.rfull[st]);
+                if (vdir) {   // L_O[sl rows][leaf rows], E[sl rows][leaf cols]
+                    sm100::tma_load_2d(sm.ring[st][0], &maps->lo, i0, sl * LB, &sm.rfull[st]);
+                    sm100::tma_load_2d(sm.ring[st][1], &maps->e, j0, sl * LB, &sm.rfull[st]);
+                } else {      // U^T[sl cols][leaf rows], L_I[sl cols][leaf cols]
+                    sm100::tma_load_2d(sm.ring[st][0], &maps->ut, i0, sl * LB, &sm.rfull[st]);
+                    sm100::tma_load_2d(sm.ring[st][1], &maps->li, j0, sl * LB, &sm.rfull[st]);
                 }
             };
-            if (lead) {
-                // the flags were acquired by warp 0's lanes before the barrier above
+            if (lane == 0) {
+                // the older sources' flags were acquired before the group barrier above
                 asm volatile("fence.proxy.async.global;" ::: "memory");
-                for (int idx = 0; idx < min(NRING, nf.nold); ++idx) issue(idx);
+                for (int i = 0; i < min(2, nold_d); ++i) issue(i);
             }
-            for (int idx = 0; idx < nf.nsrc; ++idx) {
-                if (idx == nf.nold) {
-                    // the recent sources (at most two, finishing about together): each one's
-                    // boxes go out as soon as its flag is up
-                    if (lead) {
-                        if (local_h) issue(hloc);
-                        for (int r = idx; r < nf.nsrc; ++r) {
-                            if (local_h && r == hloc) continue;
-                            int Is, Js;
-                            nf.source(r, Is, Js);
-                            if (!wait_flag(&a.flags[(size_t)Is * a.Nt + Js], a.abort_word,
-                                           a.status, a.limit_ns)) {
-                                sm.stop = 1;
-                                break;
+            for (int i = 0; i < ns; ++i) {
+                const bool recent = i == nold_d;
+                if (recent) {   // its flag first (the local one needs none)
+                    int okr = 1;
+                    if (lane == 0) {
+                        if (loc) {
+                            issue(i);
+                        } else {
+                            const int sl = srcd(i);
+                            const int* f = vdir ? &a.flags[(size_t)sl * a.Nt + J]
+                                                : &a.flags[(size_t)I * a.Nt + sl];
+                            okr = wait_flag(f, a.abort_word, a.status, a.limit_ns) ? 1 : 0;
+                            if (okr) {
+                                asm volatile("fence.proxy.async.global;" ::: "memory");
+                                issue(i);
                             }
-                            asm volatile("fence.proxy.async.global;" ::: "memory");
-                            issue(r);
                         }
                     }
-                    group_sync(g);
-                    if (*(volatile int*)&sm.stop) { stop = true; break; }
+                    if (!__shfl_sync(0xffffffffu, okr, 0)) { stop = true; break; }
                 }
-                const uint32_t q = rq + idx, st = q % NRING;
-                if (!sm100::mbar_wait(&sm.rfull[st], (q / NRING) & 1, a.status, a.limit_ns)) {
-                    atomicExch(a.abort_word, 1);
-                    stop = true;
-                }
-                if (__any_sync(0xffffffffu, stop)) { sm.stop = 1; }
-                int Is, Js;
-                const bool vert = nf.source(idx, Is, Js);
-                const bool loc = local_h && idx == hloc;
-                if (loc) {   // the previous leaf's wavefront is done: its U^T is P.oUt
-                    if (lead && !sm100::mbar_wait(&sm.solved[b ^ 1], ((k - 1) >> 1) & 1, a.status,
-                                                  a.limit_ns)) {
-                        atomicExch(a.abort_word, 1);
-                        sm.stop = 1;
-                    }
-                    group_sync(g);
-                    if (*(volatile int*)&sm.stop) stop = true;
-                }
-                if (!stop) {
-                    if (vert) product_mma(sm.ring[st][0], sm.ring[st][1], lw, lane, accT);
-                    else product_mma(loc ? P.oUt : sm.ring[st][0], sm.ring[st][1], lw, lane, accR);
-                }
-                group_sync(g);   // the stage is free again
-                if (*(volatile int*)&sm.stop) { stop = true; break; }
-                if (lead && idx + NRING < nf.nold) issue(idx + NRING);
+                const uint32_t q = rq + i, st = 2 * lw + (q & 1);
+                bool okw = sm100::mbar_wait(&sm.rfull[st], (q >> 1) & 1, a.status, a.limit_ns);
+                if (okw && loc && recent)   // the previous leaf's wavefront is done
+                    okw = sm100::mbar_wait(&sm.solved[b ^ 1], ((k - 1) >> 1) & 1, a.status,
+                                           a.limit_ns);
+                if (!__all_sync(0xffffffffu, okw)) { stop = true; break; }
+                const float* X = (loc && recent) ? P.oUt : sm.ring[st][0];
+                product_mma(X, sm.ring[st][1], 0, lane, acc[0]);
+                product_mma(X, sm.ring[st][1], 1, lane, acc[1]);
+                __syncwarp();   // the stage is free again
+                if (lane == 0 && i + 2 < nold_d) issue(i + 2);
             }
-            rq += nf.nsrc;
+            rq += ns;
+            if (stop && lane == 0) {
+                atomicExch(a.abort_word, 1);
+                sm.stop = 1;
+            }
         } else {
             // plain loads: the next source's blocks are fetched into registers while the
             // current one is multiplied; element e = lt + 64 q sits at (e >> 5, e & 31)
@@ -509,24 +512,40 @@ __device__ void leaf_loaders(const FusedArgs& a, const LeafMaps* maps, LeafGroup
                 else product_mma(sA, sB, lw, lane, accR);
             }
         }
-        if (stop) break;
+        // box path: the two warps may stop independently; they agree through sm.stop after the
+        // barrier below (a warp leaving alone would strand the other at a named barrier)
+        if (stop && !box) break;
         if (box && lead && !sm100::mbar_wait(&sm.tbar, k & 1, a.status, a.limit_ns)) {
             atomicExch(a.abort_word, 1);
             sm.stop = 1;
         }
         group_sync(g);
         if (*(volatile int*)&sm.stop) break;
+        if (box) {
+            // B.T / B.R hold the far sums; warp lw adds its direction's near field
+            float* dst = lw == 0 ? B.T : B.R;
 #pragma unroll
-        for (int nt = 0; nt < 4; ++nt)
+            for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const int r = 16 * lw + eg + 8 * (q >> 1), c = 8 * nt + 2 * et + (q & 1);
-                const int o = r * LB + c;
-                const bool ok = r < rows && c < cols;
-                // the box path already holds the far sums in B.T / B.R
-                B.T[o] = ok ? (box ? B.T[o] : 0.f) + accT[nt][q] : 0.f;
-                B.R[o] = ok ? (box ? B.R[o] : 0.f) + accR[nt][q] : 0.f;
-            }
+                for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const int r = 16 * mt + eg + 8 * (q >> 1), c = 8 * nt + 2 * et + (q & 1);
+                        const int o = r * LB + c;
+                        dst[o] = (r < rows && c < cols) ? dst[o] + acc[mt][nt][q] : 0.f;
+                    }
+        } else {
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int r = 16 * lw + eg + 8 * (q >> 1), c = 8 * nt + 2 * et + (q & 1);
+                    const int o = r * LB + c;
+                    const bool ok = r < rows && c < cols;
+                    B.T[o] = ok ? accT[nt][q] : 0.f;
+                    B.R[o] = ok ? accR[nt][q] : 0.f;
+                }
+        }
         group_sync(g);
         if (lead) sm100::mbar_arrive(&sm.full[b]);
         prevI = I;
