@@ -290,6 +290,12 @@ def _e2e(args, torch, bk, solver, stream, dev, ws, m, n, bits, Ws, HO, HI, sc,
             "d2h_bytes_per_step": d2h}
 
 
+# DRAM bytes (read + written) of one round_kernel launch on down_4096x14336, from one ncu
+# capture of this kernel version (dram__bytes_read.sum + dram__bytes_write.sum, 1 pass):
+# 27.30 GB + 9.37 GB. Reported as the roofline's traffic for that workload only.
+ROUND_TRAFFIC_BYTES = {(4096, 14336): 36.67e9}
+
+
 def _roofline(per, m, n):
     """Roofline of the dominant call of the step, on its algorithmic work.
 
@@ -314,6 +320,7 @@ def _roofline(per, m, n):
                            "/ 3 (3xTF32), fp32-equivalent flops"),
            "work_flops": work[dom]}
     if dom == "round":
+        out["traffic"] = ROUND_TRAFFIC_BYTES.get((m, n))
         # the solver benchmark's own definition: nominal dense-equivalent 2 m n (m + n)
         out["nominal_frac"] = 2.0 * work["round"] / (per["round"] * 1e-3) / 1e12 / peak
     return out
