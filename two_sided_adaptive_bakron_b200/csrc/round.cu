@@ -668,15 +668,15 @@ __device__ void leaf_role(const FusedArgs& a, const LeafMaps* maps, uint8_t* sme
         sm100::fence_mbar_init();
     }
     __syncthreads();
-    // warp w runs on SM sub-partition w % 4: group g's solver warp (g) and its helper (4 + g)
-    // share sub-partition g; its two loader warps (2, 3 for group 0, 6, 7 for group 1) sit on
-    // sub-partitions 2 and 3, one each. Named barriers: 1 + g for the loaders of group g,
-    // 3 + g for its solver and helper.
-    const int g = (warp == 1 || warp == 5 || warp >= 6) ? 1 : 0;
+    // warp w runs on SM sub-partition w % 4. Group g: helper warp g, solver warp 2 + g, loader
+    // warps 4 + g and 6 + g, so the solver and its helper issue from different
+    // sub-partitions and each sub-partition holds one of them plus one loader warp.
+    // Named barriers: 1 + g for the loaders of group g, 3 + g for its solver and helper.
+    const int g = warp & 1;
     const int slot = blockIdx.x * 2 + g, nslots = a.leaf_ctas * 2;
-    if (warp < 2) leaf_solver(a, cs.g[g], lane, slot, nslots, 3 + g);
-    else if (warp == 4 || warp == 5) leaf_helper(a, cs.g[g], lane, slot, nslots, 3 + g);
-    else leaf_loaders(a, maps, cs.g[g], g, warp & 1, lane, slot, nslots);
+    if (warp < 2) leaf_helper(a, cs.g[g], lane, slot, nslots, 3 + g);
+    else if (warp < 4) leaf_solver(a, cs.g[g], lane, slot, nslots, 3 + g);
+    else leaf_loaders(a, maps, cs.g[g], g, (warp - 4) >> 1, lane, slot, nslots);
 }
 
 // ------------------------------------------------------------------------------ push tasks
