@@ -42,106 +42,22 @@ static_assert(offsetof(LeafBuf, LOr) % 16 == 0 && offsetof(LeafBuf, LIc) % 16 ==
               "staging buffer: 16-byte float4 rows, 128-byte box destinations");
 
 
-// The in-leaf wavefront, run by the solver warp; lane j owns column j and the element of row
-// r is handled at step s = r + j. Leaf arrays use row stride LB, element (r, c) at r*LB + c,
-// so an anti-diagonal and a row both touch 32 distinct banks. Per lane, slot s of wT / wR
-// holds the vertical / horizontal sum of its element of step s. A step reads slot s, then
-// pushes E down its column into slots s+1..s+31 (in-lane) and U along its row into slot s+d
-// of lane j+d (warp shuffles); the d = 1 pushes, the only ones the next step needs, go
-// first. LIc is zero for d > j and LOr for r + d >= 32, so no push needs a guard: a lane
-// j < d gets its own u back from the shuffle and multiplies it by zero. The step loop stays rolled (4 steps per iteration) over a sliding window of 36
-// slot registers: every register index is static and the code stays small.
-// Q divides by s_r as one correctly rounded fp32 division; the quotient is formed as
+// ------------------------------------------------------------------------------ the wavefront
+// The in-leaf wavefront: lane j owns column j and the element of row r is handled at step
+// s = r + j. Leaf arrays use row stride LB, element (r, c) at r*LB + c, so an anti-diagonal and a
+// row both touch 32 distinct banks. Per lane, slot s of a window holds the vertical / horizontal
+// sum of its element of step s; a step reads slot s, then pushes E down its column into slots
+// s+1..s+31 (in-lane) and U along its row into slot s+d of lane j+d (warp shuffles). LIc is
+// zero for d > j and LOr for r + d >= 32, so no push needs a guard (a lane j < d gets its own
+// u back from the shuffle and multiplies it by zero). The step loop stays rolled (4 steps per
+// iteration) over a sliding window of 36 slot registers, so every register index is static.
+// Q divides by s_r as one correctly rounded fp32 division: the quotient is formed as
 // pre * (1/s_r), whose distance to the division's result is below 2e-7 |x|, and the exact
 // division is taken instead whenever that quotient lies within 1e-6 max(1,|x|) of a rounding
 // boundary, so the decision always equals the division's.
-__device__ __forceinline__ void solve_leaf(int lane, int rows, int cols, float qlo, float qhi,
-                                           LeafBuf& B, int* status) {
-    const int j = lane;
-    const bool colok = j < cols;
-    float li[LB];
-#pragma unroll
-    for (int q = 0; q < LB / 4; ++q) {
-        const float4 v = *reinterpret_cast<const float4*>(&B.LIc[j * LS + 4 * q]);
-        li[4 * q] = v.x; li[4 * q + 1] = v.y; li[4 * q + 2] = v.z; li[4 * q + 3] = v.w;
-    }
-    float wT[WIN], wR[WIN];
-#pragma unroll
-    for (int t = 0; t < WIN; ++t) {
-        const int r = t - j;
-        const bool ok = (r >= 0) && (r < LB);
-        const int rr = ok ? r : 0;
-        wT[t] = ok ? B.T[rr * LB + j] : 0.f;
-        wR[t] = ok ? B.R[rr * LB + j] : 0.f;
-    }
-    bool bad = false;
-#pragma unroll 1
-    for (int s0 = 0; s0 < NSLOT; s0 += UW) {
-#pragma unroll
-        for (int k = 0; k < UW; ++k) {
-            const int r = s0 + k - j;
-            const bool inleaf = (r >= 0) && (r < LB);
-            const int rr = inleaf ? r : 0;
-            const bool act = inleaf && (r < rows) && colok;
-            float lo[LB];
-#pragma unroll
-            for (int q = 0; q < LB / 4; ++q) {
-                const float4 v = *reinterpret_cast<const float4*>(&B.LOr[rr * LS + 4 * q]);
-                lo[4 * q] = v.x; lo[4 * q + 1] = v.y; lo[4 * q + 2] = v.z; lo[4 * q + 3] = v.w;
-            }
-            const float w_star = B.W[rr * LB + j];
-            const float sr = B.S[rr], inv = B.S[LB + rr];
-            float e = 0.f, u = 0.f;
-            if (act) {
-                const float pre = w_star + wT[k] + wR[k];
-                float q = 0.f;
-                if (sr > 0.f) {
-                    float x = pre * inv;
-                    const float t = fabsf(x - rintf(x));
-                    if (0.5f - t < 1e-6f * fmaxf(1.f, fabsf(x))) x = __fdiv_rn(pre, sr);
-                    q = fminf(fmaxf(rintf(x), qlo), qhi);
-                }
-                bad |= !isfinite(pre);
-                const float w = sr * q;
-                e = w_star - w;
-                u = wT[k] + e;
-                B.oC[rr * LB + j] = (int8_t)q;
-                B.oE[rr * LB + j] = e;
-                B.oEt[j * LB + rr] = e;
-                B.oU[rr * LB + j] = u;
-                B.oUt[j * LB + rr] = u;
-            }
-            wT[k + 1] = fmaf(lo[1], e, wT[k + 1]);
-            wR[k + 1] = fmaf(__shfl_up_sync(0xffffffffu, u, 1), li[1], wR[k + 1]);
-#pragma unroll
-            for (int d = 2; d < LB; ++d) wT[k + d] = fmaf(lo[d], e, wT[k + d]);
-#pragma unroll
-            for (int d = 2; d < LB; ++d)
-                wR[k + d] = fmaf(__shfl_up_sync(0xffffffffu, u, d), li[d], wR[k + d]);
-        }
-        // slide the window by UW slots
-#pragma unroll
-        for (int t = 0; t < WIN - UW; ++t) {
-            wT[t] = wT[t + UW];
-            wR[t] = wR[t + UW];
-        }
-#pragma unroll
-        for (int t = WIN - UW; t < WIN; ++t) {
-            const int r = s0 + UW + t - j;
-            const bool ok = (r >= 0) && (r < LB);
-            const int rr = ok ? r : 0;
-            wT[t] = ok ? B.T[rr * LB + j] : 0.f;
-            wR[t] = ok ? B.R[rr * LB + j] : 0.f;
-        }
-    }
-    if (bad) set_status(status, BAKRON_ERR_NONFINITE);
-}
-
-// ------------------------------------------------------------------------------ two warps
-// The same wavefront split over two warps of one SM sub-partition, with the same additions in
-// the same order (so the same results): the solver warp runs the element chain (the slot's
-// sum, Q, e, u and the distance-1 terms), the helper warp the distance >= 2 pushes one step
-// behind. Round rho: the solver computes step rho from the helper's partial sums of slot rho
+//
+// The wavefront runs on two warps: the solver warp runs the element chain (the slot's sum, Q,
+// e, u and the distance-1 terms), the helper warp the distance >= 2 pushes one step behind. Round rho: the solver computes step rho from the helper's partial sums of slot rho
 // (everything from steps <= rho - 2 on top of T, R) plus its own distance-1 terms of step
 // rho - 1; the helper pushes step rho - 1 and publishes slot rho + 1. One named barrier of the
 // two warps closes each round.
