@@ -29,7 +29,14 @@ Readings taken where the pages are garbled or silent (each one is listed in the 
   it is taken in the precision of the CUDA kernels: pre is rounded to fp32 and divided by s_i
   with one correctly rounded fp32 division before round-half-even (pre itself stays fp64);
 * E = W* - W always includes the clamp error;
-* the proxy loss is tr(H_O dW H_I dW^T) with no factor 1/2.
+* the proxy loss is tr(H_O dW H_I dW^T) with no factor 1/2;
+* stochastic Q (the section-4 alternative to nearest rounding) rounds x = pre/s_i up with
+  probability frac(x): code = clamp(floor(x + u)) with u uniform on (0, 1). The pages name no
+  generator, so u is drawn by Philox4x64-10 (Salmon, Moraes, Dror, Shaw, "Parallel random
+  numbers: as easy as 1, 2, 3", SC 2011), keyed by (seed, 0) with counter (j // 16, i, 0, 0);
+  entry (i, j) takes the 16-bit field j % 16 of the 256-bit block (word (j % 16) // 4, bits
+  16 (j % 4) and up), u = (field + 1/2) / 2^16. x is the fp32 quotient as for nearest rounding,
+  and x + u is one fp32 addition.
 
 Parity status: every function below is pinned by ``tests/test_oracle.py`` against closed
 forms, textbook routines (numpy Cholesky, the GPTQ/OBS update on the vectorised problem),
@@ -46,6 +53,7 @@ __all__ = [
     "udu", "quantize", "round_naive", "round_row_sweep", "fixed_point_pre",
     "proxy_loss", "proxy_loss_kron", "brute_force_fixed_points", "gptq_obs",
     "code_range", "fixed_point_pre_rows", "band_check", "grid_quotient",
+    "philox4x64_10", "dither", "quantize_stochastic",
 ]
 
 
@@ -102,14 +110,68 @@ def quantize(pre: float, s: float, bits: int) -> int:
 
 
 # ---------------------------------------------------------------------------------------------
+# Stochastic Q ([YAQA] section 4 allows stochastic rounding in place of nearest rounding).
+# ---------------------------------------------------------------------------------------------
+_M64 = (1 << 64) - 1
+_PHILOX_M = (0xD2E7470EE14C6C93, 0xCA5A826395121157)   # round multipliers of Philox4x64
+_PHILOX_W = (0x9E3779B97F4A7C15, 0xBB67AE8584CAA73B)   # key increments (Weyl sequence)
+
+
+def philox4x64_10(counter, key):
+    """Philox4x64 with 10 rounds (Salmon et al., SC 2011, section 4): per round the two
+    64 x 64 -> 128-bit products of words 0 and 2 with the round multipliers, the high halves
+    xored with words 1 and 3 and the round key, the words permuted; the key advances by the
+    Weyl increments between rounds. counter: 4 ints < 2^64, key: 2 ints < 2^64. Returns the
+    4 output words."""
+    x0, x1, x2, x3 = (int(v) & _M64 for v in counter)
+    k0, k1 = (int(v) & _M64 for v in key)
+    for _ in range(10):
+        p0 = _PHILOX_M[0] * x0
+        p1 = _PHILOX_M[1] * x2
+        x0, x1, x2, x3 = (p1 >> 64) ^ x1 ^ k0, p1 & _M64, (p0 >> 64) ^ x3 ^ k1, p0 & _M64
+        k0 = (k0 + _PHILOX_W[0]) & _M64
+        k1 = (k1 + _PHILOX_W[1]) & _M64
+    return x0, x1, x2, x3
+
+
+def dither(rows, n: int, seed: int) -> np.ndarray:
+    """The uniform variates u_ij of stochastic Q for the given rows (an int m gives rows
+    0..m-1), all n columns: len(rows) x n fp64, each (k + 1/2) / 2^16 for a 16-bit k."""
+    rows = np.arange(rows) if np.isscalar(rows) else np.asarray(rows)
+    out = np.empty((rows.size, n))
+    for a, i in enumerate(rows):
+        for cb in range((n + 15) // 16):
+            words = philox4x64_10((cb, int(i), 0, 0), (seed, 0))
+            for t in range(min(16, n - 16 * cb)):
+                k = (words[t // 4] >> (16 * (t % 4))) & 0xFFFF
+                out[a, 16 * cb + t] = (k + 0.5) / 65536.0
+    return out
+
+
+def quantize_stochastic(pre: float, s: float, bits: int, u: float) -> int:
+    """Stochastic code for one entry: clamp(floor(x + u)), x the fp32 quotient pre / s and
+    x + u one fp32 addition; s == 0 gives 0."""
+    lo, hi = code_range(bits)
+    if s == 0.0:
+        return 0
+    y = np.float32(grid_quotient(pre, s)) + np.float32(u)
+    return int(min(max(float(np.floor(y)), lo), hi))
+
+
+def _q(pre, s, bits, U, i, j):
+    return quantize(pre, s, bits) if U is None else quantize_stochastic(pre, s, bits, U[i, j])
+
+
+# ---------------------------------------------------------------------------------------------
 # The rule, entry by entry, in raster order ([YAQA] section 4). Raster order is a valid order
 # because entry (i, j) reads only entries (k, l) with k <= i and l <= j, (k, l) != (i, j).
 # ---------------------------------------------------------------------------------------------
-def round_naive(Wstar, L_O, L_I, scales, bits, return_pre=False):
+def round_naive(Wstar, L_O, L_I, scales, bits, return_pre=False, dither=None):
     """Plain definition, O(m^2 n^2 / 4) multiply-adds.
 
     pre_ij = W*_ij + a_i^T E[:i,:j] b_j + a_i^T E[:i,j] + E[i,:j] b_j,   E = W* - W
-    with a_i = L_O[:i, i] and b_j = L_I[:j, j].
+    with a_i = L_O[:i, i] and b_j = L_I[:j, j]. ``dither`` (m x n variates u_ij) selects
+    stochastic Q; None selects nearest rounding.
     Returns (codes int64 m x n, W fp64 m x n[, pre fp64 m x n]).
     """
     Ws = np.asarray(Wstar, dtype=np.float64)
@@ -132,7 +194,7 @@ def round_naive(Wstar, L_O, L_I, scales, bits, return_pre=False):
                 pre += a @ E[:i, j]
             if j > 0:
                 pre += E[i, :j] @ b
-            c = quantize(pre, s[i], bits)
+            c = _q(pre, s[i], bits, dither, i, j)
             C[i, j] = c
             W[i, j] = s[i] * c
             E[i, j] = Ws[i, j] - W[i, j]
@@ -140,7 +202,7 @@ def round_naive(Wstar, L_O, L_I, scales, bits, return_pre=False):
     return (C, W, P) if return_pre else (C, W)
 
 
-def round_row_sweep(Wstar, L_O, L_I, scales, bits, return_pre=False):
+def round_row_sweep(Wstar, L_O, L_I, scales, bits, return_pre=False, dither=None):
     """Same result as ``round_naive`` in O(mn(m+n)) work (the row-by-row reading).
 
     Row i sees every earlier row only through T_i = sum_{k<i} L_O[k,i] E_k (a row vector).
@@ -161,7 +223,7 @@ def round_row_sweep(Wstar, L_O, L_I, scales, bits, return_pre=False):
         r = Ws[i] + T + T @ LI
         for j in range(n):
             pre = r[j] + E[i, :j] @ LI[:j, j]
-            c = quantize(pre, s[i], bits)
+            c = _q(pre, s[i], bits, dither, i, j)
             C[i, j] = c
             W[i, j] = s[i] * c
             E[i, j] = Ws[i, j] - W[i, j]
@@ -201,11 +263,12 @@ def fixed_point_pre_rows(Wstar, W, L_O, L_I, rows):
     return Ws[rows] + T + T @ LI - E[rows]
 
 
-def band_check(pre, codes, scales, bits, band=1e-3):
+def band_check(pre, codes, scales, bits, band=1e-3, dither=None):
     """Compare codes with Q(pre) under the exemption band of the tolerance rule.
 
     An entry may disagree only if pre/s lies within ``band`` grid steps of a rounding boundary
-    (a half-integer). Returns (n_mismatch, n_mismatch_outside_band, n_in_band).
+    (a half-integer for nearest rounding; for stochastic Q with variates ``dither``, an
+    integer value of pre/s + u). Returns (n_mismatch, n_mismatch_outside_band, n_in_band).
     """
     s = np.asarray(scales, dtype=np.float64)[:, None]
     lo, hi = code_range(bits)
@@ -213,9 +276,14 @@ def band_check(pre, codes, scales, bits, band=1e-3):
     with np.errstate(divide="ignore", invalid="ignore"):
         x = np.where(s > 0, pre / s_safe, 0.0)
     xq = np.where(s > 0, grid_quotient(pre, np.broadcast_to(s_safe, pre.shape)), 0.0)
-    q = np.clip(np.rint(xq), lo, hi)
+    if dither is None:
+        q = np.clip(np.rint(xq), lo, hi)
+        frac = np.abs(x - np.floor(x) - 0.5)
+    else:
+        u = np.asarray(dither, dtype=np.float64)
+        q = np.clip(np.floor(xq.astype(np.float32) + u.astype(np.float32)), lo, hi)
+        frac = np.abs(x + u - np.rint(x + u))
     q = np.where(s > 0, q, 0.0)
-    frac = np.abs(x - np.floor(x) - 0.5)
     in_band = frac < band
     mism = q != np.asarray(codes, dtype=np.float64)
     return int(mism.sum()), int((mism & ~in_band).sum()), int(in_band.sum())
@@ -238,20 +306,22 @@ def proxy_loss_kron(dW, H_O, H_I) -> float:
 # ---------------------------------------------------------------------------------------------
 # Independent algorithms used only to pin the rule.
 # ---------------------------------------------------------------------------------------------
-def gptq_obs(w_star: np.ndarray, H: np.ndarray, scales: np.ndarray, bits: int):
+def gptq_obs(w_star: np.ndarray, H: np.ndarray, scales: np.ndarray, bits: int, dither=None):
     """GPTQ in its optimal-brain-surgeon form on a vector w (length N) with Hessian H.
 
     Coordinates are fixed in index order. After fixing coordinate q to its quantised value,
     every still-free coordinate f moves by  -(w_q - Q(w_q)) [H_F^{-1}]_{f q} / [H_F^{-1}]_{q q},
     where H_F is H restricted to the free set (q included). ``scales[q]`` is the grid step of
-    coordinate q. Returns integer codes. Uses an explicit inverse per step: tiny N only.
+    coordinate q; ``dither`` (length N) selects stochastic Q. Returns integer codes. Uses an
+    explicit inverse per step: tiny N only.
     """
     w = np.asarray(w_star, dtype=np.float64).copy()
     H = np.asarray(H, dtype=np.float64)
     N = w.shape[0]
     codes = np.zeros(N, dtype=np.int64)
     for q in range(N):
-        c = quantize(w[q], float(scales[q]), bits)
+        c = quantize(w[q], float(scales[q]), bits) if dither is None else \
+            quantize_stochastic(w[q], float(scales[q]), bits, float(dither[q]))
         codes[q] = c
         wq = float(scales[q]) * c
         F = np.arange(q, N)
@@ -262,12 +332,13 @@ def gptq_obs(w_star: np.ndarray, H: np.ndarray, scales: np.ndarray, bits: int):
     return codes
 
 
-def brute_force_fixed_points(Wstar, L_O, L_I, scales, bits, chunk=4096):
+def brute_force_fixed_points(Wstar, L_O, L_I, scales, bits, chunk=4096, dither=None):
     """All code matrices C with C = Q(pre(C)) under the closed form, by enumeration.
 
     Every candidate C in [lo, hi]^(m x n) is tried: W = s * C, pre is the closed form of
     ``fixed_point_pre`` (evaluated for a batch of candidates at once with the same fp64
-    products), and C is kept when clamp(rint(pre / s)) == C at every entry. Tiny shapes only
+    products), and C is kept when Q(pre) == C at every entry (nearest, or stochastic with the
+    variates ``dither``). Tiny shapes only
     ((2^bits)^(mn) candidates). Rows with s_i = 0 are not supported here.
     """
     Ws = np.asarray(Wstar, dtype=np.float64)
@@ -289,8 +360,12 @@ def brute_force_fixed_points(Wstar, L_O, L_I, scales, bits, chunk=4096):
         C = digits.reshape(-1, m, n)
         E = Ws[None] - s[None, :, None] * C
         pre = Ws[None] + np.einsum("ki,bkl,lj->bij", Ao, E, Ai) - E
-        Q = np.clip(np.rint(grid_quotient(pre, np.broadcast_to(s[None, :, None], pre.shape))),
-                    lo, hi)
+        xq = grid_quotient(pre, np.broadcast_to(s[None, :, None], pre.shape))
+        if dither is None:
+            Q = np.clip(np.rint(xq), lo, hi)
+        else:
+            u = np.asarray(dither, dtype=np.float32)[None]
+            Q = np.clip(np.floor(xq.astype(np.float32) + u), lo, hi)
         ok = np.all(Q == C, axis=(1, 2))
         found.extend(C[ok])
     return found
