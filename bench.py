@@ -1,11 +1,13 @@
 """Benchmark of the BaKron solve path on synthetic LLM-layer workloads.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+                    [--rounding nearest|stochastic]
 
 One step = the whole path on one layer with inputs resident in HBM:
     bakron_ldl(H_O), bakron_ldl(H_I), bakron_round(W*, L_O, L_I, scales, bits),
     bakron_proxy_loss(W* - W, H_O, H_I).
-Metric: quantized weights per second, m*n / step time (whole job: summed over replicas, one
+--rounding stochastic times bakron_round_stochastic (stochastic Q, a fixed seed per step) in
+place of bakron_round. Metric: quantized weights per second, m*n / step time (whole job: summed over replicas, one
 independent layer per GPU, no collective on the data path; timed as the max over ranks).
 
 --impl reference times the fp64 CPU oracle (the deliberately slow reference) on a bounded
@@ -198,9 +200,11 @@ def run(args):
     # ---- per-call timing events on the launching stream (device-timed breakdown)
     names = ["ldl_O", "ldl_I", "round", "loss"]
 
+    seed = 0x5EED if args.rounding == "stochastic" else None
+
     def step(evs=None):
         timing = None if evs is None else dict(zip(names, evs))
-        solver.run(Ws, HO, HI, sc, bits, stream, timing=timing)
+        solver.run(Ws, HO, HI, sc, bits, stream, timing=timing, seed=seed)
 
     for _ in range(args.warmup):
         step()
@@ -240,13 +244,13 @@ def run(args):
     e2e = None
     if not args.no_e2e:
         e2e = _e2e(args, torch, bk, solver, stream, dev, ws, m, n, bits, Ws, HO, HI, sc,
-                   Ws_np, HO_np, HI_np, s_np)
+                   Ws_np, HO_np, HI_np, s_np, seed)
     return _report(args, torch, bk, wl, ws, rank, m, n, bits, per, ms_step, value, launches,
                    clk, e2e, (Ws_np, HO_np, HI_np, s_np, bits))
 
 
 def _e2e(args, torch, bk, solver, stream, dev, ws, m, n, bits, Ws, HO, HI, sc,
-         Ws_np, HO_np, HI_np, s_np):
+         Ws_np, HO_np, HI_np, s_np, seed):
     """Same metric through the public API with host buffers: pinned host -> device copies of
     the step's inputs, the whole path, device -> host copies of the codes and the loss."""
     hW = torch.from_numpy(Ws_np).pin_memory()
@@ -265,7 +269,7 @@ def _e2e(args, torch, bk, solver, stream, dev, ws, m, n, bits, Ws, HO, HI, sc,
         dO2.copy_(hO, non_blocking=True)
         dI2.copy_(hI, non_blocking=True)
         ds2.copy_(hs, non_blocking=True)
-        solver.run(dW2, dO2, dI2, ds2, bits, stream)
+        solver.run(dW2, dO2, dI2, ds2, bits, stream, seed=seed)
         hcodes.copy_(solver.codes, non_blocking=True)
         hloss.copy_(solver.loss, non_blocking=True)
 
@@ -290,14 +294,17 @@ def _e2e(args, torch, bk, solver, stream, dev, ws, m, n, bits, Ws, HO, HI, sc,
             "d2h_bytes_per_step": d2h}
 
 
-# DRAM bytes (read + written) of one round_kernel launch on down_4096x14336, from one ncu
-# capture of this kernel version (dram__bytes_read.sum + dram__bytes_write.sum, 1 pass):
-# 27.30 GB + 9.37 GB. Reported as the roofline's traffic for that workload only.
-ROUND_TRAFFIC_BYTES = {(4096, 14336): 36.67e9}
+# DRAM bytes (read + written) of one round_kernel launch on down_4096x14336 with nearest Q,
+# from one ncu capture of this kernel version (dram__bytes_read.sum + dram__bytes_write.sum,
+# 1 pass): 26.98 GB + 9.37 GB. Reported as the roofline's traffic for that workload only.
+ROUND_TRAFFIC_BYTES = {(4096, 14336): 36.35e9}
 
 
-def _roofline(per, m, n):
-    """Roofline of the dominant call of the step, on its algorithmic work.
+def _roofline(per, m, n, rounding="nearest"):
+    """Roofline of the step's dominant kernel, round_kernel (one launch per step that runs the
+    whole rounding solve: the largest single kernel and the largest share of the launch
+    list), on its algorithmic work. The factorisation of H_I takes about as long, but as
+    hundreds of short launches (diagonal blocks, panel and trailing-update GEMMs).
 
     The contractions run as 3xTF32 on the tensor cores (three tf32 MMAs per fp32-accurate
     product), so their peak is the measured dense bf16 rate x the nominal tf32/bf16 ratio
@@ -312,23 +319,22 @@ def _roofline(per, m, n):
         "round": float(m) * n * (m + n),                       # triangular pushes, 2 flop/MAC
         "loss": 2.0 * min(m, n) ** 2 * max(m, n) + float(m) * n * max(m, n),
     }
-    dom = max(per, key=lambda k: per[k])
-    achieved = work[dom] / (per[dom] * 1e-3) / 1e12
-    out = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak,
-           "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
-           "peak_source": (f"{kind} sustained bf16 {bf16:.1f} TFLOP/s x 0.5 (tf32/bf16 nominal) "
-                           "/ 3 (3xTF32), fp32-equivalent flops"),
-           "work_flops": work[dom]}
-    if dom == "round":
-        out["traffic"] = ROUND_TRAFFIC_BYTES.get((m, n))
-        # the solver benchmark's own definition: nominal dense-equivalent 2 m n (m + n)
-        out["nominal_frac"] = 2.0 * work["round"] / (per["round"] * 1e-3) / 1e12 / peak
-    return out
+    t = per["round"] * 1e-3
+    achieved = work["round"] / t / 1e12
+    return {"bound": "tensor", "kernel": "round_kernel", "achieved": achieved, "peak": peak,
+            "unit": "TFLOP/s", "frac": achieved / peak,
+            "traffic": ROUND_TRAFFIC_BYTES.get((m, n)) if rounding == "nearest" else None,
+            "peak_source": (f"{kind} sustained bf16 {bf16:.1f} TFLOP/s x 0.5 (tf32/bf16 "
+                            "nominal) / 3 (3xTF32), fp32-equivalent flops"),
+            "work_flops": work["round"],
+            # the solver benchmark's own definition: nominal dense-equivalent 2 m n (m + n)
+            "nominal_frac": 2.0 * work["round"] / t / 1e12 / peak,
+            "others_tflops": {k: work[k] / (per[k] * 1e-3) / 1e12 for k in per if k != "round"}}
 
 
 def _report(args, torch, bk, wl, ws, rank, m, n, bits, per, ms_step, value, launches, clk,
             e2e, arrays):
-    roofline = _roofline(per, m, n)
+    roofline = _roofline(per, m, n, args.rounding)
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         rr, c, dt = oracle_sample(wl, arrays)
@@ -340,6 +346,7 @@ def _report(args, torch, bk, wl, ws, rank, m, n, bits, per, ms_step, value, laun
                 "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
                 "config": {"workload": wl.name, "m": m, "n": n, "bits": bits,
+                           "rounding": args.rounding,
                            "parallelism": f"replicas x{ws}" if ws > 1 else "single",
                            "l2": "inputs larger than L2 (H_I alone is "
                                  f"{4 * n * n / 2**20:.0f} MiB), no flush"},
@@ -364,6 +371,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--ref-seconds", type=float, default=12.0)
+    ap.add_argument("--rounding", default="nearest", choices=["nearest", "stochastic"])
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)

@@ -117,6 +117,28 @@ int bakron_round(const float* Wstar, int m, int n, const float* L_O, const float
                  void* ws, size_t ws_bytes, int* dev_status, void* stream);
 
 /* ------------------------------------------------------------------------------------------
+ * bakron_round_stochastic -- bakron_round with stochastic Q in place of nearest rounding (the
+ * YAQA article's rounding rule, section 4, takes Q as nearest or stochastic rounding).
+ *
+ *   code_ij = clamp(floor(x_ij + u_ij), -2^(bits-1), 2^(bits-1) - 1),   x_ij = pre_ij / s_i,
+ *
+ * so that, away from the clamp, s_i code_ij is an unbiased rounding of pre_ij: it takes the
+ * grid point above with probability frac(x_ij). x_ij is the correctly rounded fp32 quotient
+ * and x_ij + u_ij one fp32 addition. The variate u_ij = (k_ij + 1/2) / 2^16, where k_ij is the
+ * 16-bit field (j mod 16) (least significant first: word (j mod 16) / 4, bits 16 (j mod 4)
+ * and up) of the Philox4x64-10 block (Salmon, Moraes, Dror, Shaw, "Parallel random numbers:
+ * as easy as 1, 2, 3", SC 2011) with key (seed, 0) and counter (j / 16, i, 0, 0).
+ *
+ *   seed     [in]  64-bit key of the variates; the same seed gives bitwise the same result.
+ * Every other argument, the workspace (bakron_round_workspace_bytes) and the error behaviour
+ * are those of bakron_round.
+ * ---------------------------------------------------------------------------------------- */
+int bakron_round_stochastic(const float* Wstar, int m, int n, const float* L_O,
+                            const float* L_I, const float* scales, int bits, uint64_t seed,
+                            int8_t* codes, float* W, void* ws, size_t ws_bytes, int* dev_status,
+                            void* stream);
+
+/* ------------------------------------------------------------------------------------------
  * bakron_proxy_loss -- tr(H_O dW H_I dW^T) = vec(dW)^T (H_O (x) H_I) vec(dW).
  *
  * The layer proxy of the YAQA article (section 4 error bound, section 2 second-order

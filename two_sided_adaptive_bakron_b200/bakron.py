@@ -1,9 +1,9 @@
 """Python binding of libbakron.so (ctypes): argument marshalling only.
 
-The functions named like the C ABI (``bakron_ldl``, ``bakron_round``, ``bakron_proxy_loss``,
-``bakron_read_status``, ``bakron_status_string`` and the ``*_workspace_bytes`` queries) take
-torch CUDA tensors, pass their device pointers and the current CUDA stream to the library and
-return its status code. ``ldl``, ``round_weights``, ``proxy_loss`` and ``solve`` additionally
+The functions named like the C ABI (``bakron_ldl``, ``bakron_round``,
+``bakron_round_stochastic``, ``bakron_proxy_loss``, ``bakron_read_status``,
+``bakron_status_string`` and the ``*_workspace_bytes`` queries) take torch CUDA tensors, pass
+their device pointers and the current CUDA stream to the library and return its status code. ``ldl``, ``round_weights``, ``proxy_loss`` and ``solve`` additionally
 allocate outputs and workspaces with torch and raise on any error.
 
 Every step of the computation runs in the library's CUDA kernels; there is no CPU path. If
@@ -37,6 +37,8 @@ _SIGNATURES = {
     "bakron_round_workspace_bytes": (_c_size_t, [_c_int, _c_int]),
     "bakron_round": (_c_int, [_vp, _c_int, _c_int, _vp, _vp, _vp, _c_int, _vp, _vp, _vp,
                               _c_size_t, _vp, _vp]),
+    "bakron_round_stochastic": (_c_int, [_vp, _c_int, _c_int, _vp, _vp, _vp, _c_int,
+                                         ctypes.c_uint64, _vp, _vp, _vp, _c_size_t, _vp, _vp]),
     "bakron_proxy_loss_workspace_bytes": (_c_size_t, [_c_int, _c_int]),
     "bakron_proxy_loss": (_c_int, [_vp, _c_int, _c_int, _vp, _vp, _vp, _vp, _c_size_t, _vp]),
     "bakron_read_status": (_c_int, [_vp, _vp]),
@@ -146,6 +148,21 @@ def bakron_round(Wstar, L_O, L_I, scales, bits, codes, W, ws, dev_status, stream
                               _ptr(dev_status), _stream(stream))
 
 
+def bakron_round_stochastic(Wstar, L_O, L_I, scales, bits, seed, codes, W, ws, dev_status,
+                            stream=None) -> int:
+    m, n = Wstar.shape
+    _check_cuda(Wstar, torch.float32, (m, n), "Wstar")
+    _check_cuda(L_O, torch.float32, (m, m), "L_O")
+    _check_cuda(L_I, torch.float32, (n, n), "L_I")
+    _check_cuda(scales, torch.float32, (m,), "scales")
+    _check_cuda(codes, torch.int8, (m, n), "codes")
+    _check_cuda(W, torch.float32, (m, n), "W")
+    return lib().bakron_round_stochastic(_ptr(Wstar), m, n, _ptr(L_O), _ptr(L_I), _ptr(scales),
+                                         int(bits), int(seed) & ((1 << 64) - 1), _ptr(codes),
+                                         _ptr(W), _ptr(ws), ws.numel() * ws.element_size(),
+                                         _ptr(dev_status), _stream(stream))
+
+
 def bakron_proxy_loss(dW, H_O, H_I, loss, ws, stream=None) -> int:
     m, n = dW.shape
     _check_cuda(dW, torch.float32, (m, n), "dW")
@@ -235,14 +252,19 @@ def ldl(H: torch.Tensor, stream=None, check: bool = True):
     return L, D
 
 
-def round_weights(Wstar, L_O, L_I, scales, bits, stream=None, check: bool = True):
-    """(codes int8, W fp32) of the BaKron solve."""
+def round_weights(Wstar, L_O, L_I, scales, bits, stream=None, check: bool = True, seed=None):
+    """(codes int8, W fp32) of the BaKron solve; a seed selects stochastic Q."""
     m, n = Wstar.shape
     codes = torch.empty((m, n), dtype=torch.int8, device=Wstar.device)
     W = torch.empty((m, n), dtype=torch.float32, device=Wstar.device)
     ws = workspace(bakron_round_workspace_bytes(m, n), Wstar.device)
     st = new_status(Wstar.device)
-    _raise(bakron_round(Wstar, L_O, L_I, scales, bits, codes, W, ws, st, stream), "bakron_round")
+    if seed is None:
+        _raise(bakron_round(Wstar, L_O, L_I, scales, bits, codes, W, ws, st, stream),
+               "bakron_round")
+    else:
+        _raise(bakron_round_stochastic(Wstar, L_O, L_I, scales, bits, seed, codes, W, ws, st,
+                                       stream), "bakron_round_stochastic")
     if check:
         _raise(bakron_read_status(st, stream), "bakron_round (device)")
     return codes, W
@@ -286,8 +308,10 @@ class Solver:
         self._fork = torch.cuda.Event()
         self._join = torch.cuda.Event()
 
-    def run(self, Wstar, H_O, H_I, scales, bits, stream=None, with_loss=True, timing=None):
-        """Enqueues the whole path (reads: self.codes, self.W, self.E, self.loss).
+    def run(self, Wstar, H_O, H_I, scales, bits, stream=None, with_loss=True, timing=None,
+            seed=None):
+        """Enqueues the whole path (reads: self.codes, self.W, self.E, self.loss); a seed
+        selects stochastic Q for the round.
 
         timing: optional {name: (start_event, end_event)} for any of "ldl_O", "ldl_I", "round",
         "loss"; each pair is recorded around its call on the stream that runs it.
@@ -310,8 +334,12 @@ class Solver:
         call("ldl_I", stream, bakron_ldl, H_I, self.L_I, self.D_I, self.ws, self.status)
         self._join.record(self.side)
         stream.wait_event(self._join)
-        call("round", stream, bakron_round, Wstar, self.L_O, self.L_I, scales, bits, self.codes,
-             self.W, self.ws_round, self.status)
+        if seed is None:
+            call("round", stream, bakron_round, Wstar, self.L_O, self.L_I, scales, bits,
+                 self.codes, self.W, self.ws_round, self.status)
+        else:
+            call("round", stream, bakron_round_stochastic, Wstar, self.L_O, self.L_I, scales,
+                 bits, seed, self.codes, self.W, self.ws_round, self.status)
         if with_loss:
             call("loss", stream, bakron_proxy_loss, self.E, H_O, H_I, self.loss, self.ws)
 
@@ -319,9 +347,10 @@ class Solver:
         _raise(bakron_read_status(self.status, stream), "bakron (device)")
 
 
-def solve(Wstar, H_O, H_I, scales, bits, stream=None):
-    """Whole path on device tensors: returns (codes, W, loss, (L_O, D_O), (L_I, D_I))."""
+def solve(Wstar, H_O, H_I, scales, bits, stream=None, seed=None):
+    """Whole path on device tensors: returns (codes, W, loss, (L_O, D_O), (L_I, D_I)); a seed
+    selects stochastic Q."""
     s = Solver(Wstar.shape[0], Wstar.shape[1], Wstar.device)
-    s.run(Wstar, H_O, H_I, scales, bits, stream)
+    s.run(Wstar, H_O, H_I, scales, bits, stream, seed=seed)
     s.check(stream)
     return s.codes, s.W, s.loss, (s.L_O, s.D_O), (s.L_I, s.D_I)

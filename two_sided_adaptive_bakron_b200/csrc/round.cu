@@ -39,6 +39,7 @@
 #include <cstddef>
 #include <cstring>
 
+#include "philox.cuh"
 #include "round_leaf.cuh"
 #include "tcgemm_host.cuh"
 
@@ -94,6 +95,8 @@ struct FusedArgs {
     int Mt, Nt, MS, NS, TN;
     int leaf_ctas;
     uint64_t limit_ns;
+    int stoch;           // 1: stochastic Q with the variates of `seed`
+    unsigned long long seed;
 };
 
 // 32 x 32 fp32 box maps (no swizzle) of the matrices a leaf reads; only valid when m and n are
@@ -174,9 +177,9 @@ __device__ __forceinline__ void publish_rest(const FusedArgs& a, const LeafBuf& 
         const int e = lt + q * NLOAD, r = e >> 5, c = e & 31;
         if (r < rows && c < cols) {
             const size_t o = (size_t)(i0 + r) * a.n + j0 + c;
-            const int8_t q8 = B.oC[r * LB + c];
-            a.codes[o] = q8;
-            a.Wq[o] = B.S[r] * (float)q8;
+            const int q = B.oC[r * LB + c];
+            a.codes[o] = (int8_t)q;
+            a.Wq[o] = B.S[r] * (float)q;
         }
     }
 }
@@ -319,6 +322,17 @@ __device__ void leaf_loaders(const FusedArgs& a, const LeafMaps* maps, LeafGroup
             B.S[LB + lt] = sv > 0.f ? __frcp_rn(sv) : 0.f;
         }
         if (lead) { B.meta[0] = I; B.meta[1] = J; B.meta[2] = rows; B.meta[3] = cols; }
+        if (a.stoch) {
+            // the variates: thread lt takes row lt / 2 and the 16 columns from 16 (lt % 2), one
+            // Philox block keyed (seed, 0) at counter (column / 16, row, 0, 0); the block's four
+            // words, little-endian, are the 16 fields of those columns in order
+            const int r = lt >> 1, cb = lt & 1;
+            uint64_t w[4];
+            philox4x64_10((uint64_t)((j0 >> 4) + cb), (uint64_t)(i0 + r), 0, 0, a.seed, 0, w);
+            ulonglong2* dst = reinterpret_cast<ulonglong2*>(&B.oC[r * LB + 16 * cb]);
+            dst[0] = make_ulonglong2(w[0], w[1]);
+            dst[1] = make_ulonglong2(w[2], w[3]);
+        }
         // far field: every super-block at least two steps above / to the left has been added
         if (lead) {
             const int tile = (I * LB / TB) * a.TN + (J * LB / TB);
@@ -589,7 +603,8 @@ __device__ void leaf_solver(const FusedArgs& a, LeafGroupSmem& sm, int lane, int
         }
         const int I = B.meta[0], J = B.meta[1], rows = B.meta[2], cols = B.meta[3];
         const int i0 = I * LB, j0 = J * LB;
-        solve_leaf_chain(lane, rows, cols, a.qlo, a.qhi, B, sm.xch, bar, a.status);
+        if (a.stoch) solve_leaf_chain<true>(lane, rows, cols, a.qlo, a.qhi, B, sm.xch, bar, a.status);
+        else solve_leaf_chain<false>(lane, rows, cols, a.qlo, a.qhi, B, sm.xch, bar, a.status);
         __syncwarp();
         if (lane == 0) sm100::mbar_arrive(&sm.solved[b]);
         // what the next leaves read: E (vertical pulls, lane = column) and U^T (horizontal pulls,
@@ -1020,9 +1035,11 @@ extern "C" size_t bakron_round_workspace_bytes(int m, int n) {
     return z.bytes();
 }
 
-extern "C" int bakron_round(const float* Wstar, int m, int n, const float* L_O, const float* L_I,
-                            const float* scales, int bits, int8_t* codes, float* W, void* ws,
-                            size_t ws_bytes, int* dev_status, void* stream) {
+namespace {
+
+int round_impl(const float* Wstar, int m, int n, const float* L_O, const float* L_I,
+               const float* scales, int bits, int stoch, unsigned long long seed, int8_t* codes,
+               float* W, void* ws, size_t ws_bytes, int* dev_status, void* stream) {
     if (m < 1 || n < 1 || (long long)m * n >= (1LL << 31) || bits < 2 || bits > 8 ||
         !Wstar || !L_O || !L_I || !scales || !codes || !W || !dev_status)
         return BAKRON_ERR_INVALID_ARG;
@@ -1084,6 +1101,8 @@ extern "C" int bakron_round(const float* Wstar, int m, int n, const float* L_O, 
     a.nsb = L.nsb;
     a.Mt = L.Mt; a.Nt = L.Nt; a.MS = L.MS; a.NS = L.NS; a.TN = L.TN;
     a.limit_ns = spin_limit_ns();
+    a.stoch = stoch;
+    a.seed = seed;
 
     // box loads for the leaves when every row stride is a multiple of 16 bytes
     LeafMaps lm;
@@ -1118,4 +1137,21 @@ extern "C" int bakron_round(const float* Wstar, int m, int n, const float* L_O, 
                                                   dim3(NTH), params, kSmem, st))))
         return e;
     return cuda_err(cudaGetLastError());
+}
+
+}  // namespace
+
+extern "C" int bakron_round(const float* Wstar, int m, int n, const float* L_O, const float* L_I,
+                            const float* scales, int bits, int8_t* codes, float* W, void* ws,
+                            size_t ws_bytes, int* dev_status, void* stream) {
+    return round_impl(Wstar, m, n, L_O, L_I, scales, bits, 0, 0ull, codes, W, ws, ws_bytes,
+                      dev_status, stream);
+}
+
+extern "C" int bakron_round_stochastic(const float* Wstar, int m, int n, const float* L_O,
+                                       const float* L_I, const float* scales, int bits,
+                                       uint64_t seed, int8_t* codes, float* W, void* ws,
+                                       size_t ws_bytes, int* dev_status, void* stream) {
+    return round_impl(Wstar, m, n, L_O, L_I, scales, bits, 1, (unsigned long long)seed, codes,
+                      W, ws, ws_bytes, dev_status, stream);
 }

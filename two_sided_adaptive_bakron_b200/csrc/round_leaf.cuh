@@ -1,8 +1,10 @@
-// round_leaf.cuh -- the in-leaf wavefront of the BaKron solve (one warp, 32 x 32 leaf).
+// round_leaf.cuh -- the in-leaf wavefront of the BaKron solve (32 x 32 leaf, a warp pair).
 //
 // YAQA article, section 4, rounding rule, with U = (I + L_O)^T E:
 //   pre_ij = W*_ij + T_ij + R_ij,  T_ij = sum_{k<i} L_O[k,i] E_kj,  R_ij = sum_{l<j} U_il L_I[l,j],
-//   W_ij = s_i clamp(rint(pre_ij / s_i)),  E_ij = W*_ij - W_ij,  U_ij = T_ij + E_ij.
+//   W_ij = s_i clamp(rint(pre_ij / s_i)),  E_ij = W*_ij - W_ij,  U_ij = T_ij + E_ij,
+// or, with stochastic Q (the same section's alternative),
+//   W_ij = s_i clamp(floor(pre_ij / s_i + u_ij)),  u_ij uniform on (0, 1).
 // T and R arrive holding everything from outside the leaf; the wavefront adds the in-leaf part.
 #pragma once
 
@@ -32,11 +34,14 @@ struct alignas(128) LeafBuf {
     float oE[LB * LB], oU[LB * LB];
     float oEt[LB * LB];          // E transposed (for the transposed planes)
     float oUt[LB * LB];          // U transposed
-    int8_t oC[LB * LB];
+    // the codes; before the wavefront, with stochastic Q, the 16-bit fields k of the leaf's
+    // variates u = (k + 1/2) / 2^16 (each is read by the lane that then writes the code there)
+    alignas(16) int16_t oC[LB * LB];
     int meta[4];                 // I, J, rows, cols
 };
 static_assert(offsetof(LeafBuf, LOr) % 16 == 0 && offsetof(LeafBuf, LIc) % 16 == 0 &&
                   (LS * 4) % 16 == 0 && offsetof(LeafBuf, W) % 128 == 0 &&
+                  offsetof(LeafBuf, oC) % 16 == 0 &&
                   offsetof(LeafBuf, T) % 128 == 0 && offsetof(LeafBuf, R) % 128 == 0 &&
                   sizeof(LeafBuf) % 128 == 0,
               "staging buffer: 16-byte float4 rows, 128-byte box destinations");
@@ -54,10 +59,15 @@ static_assert(offsetof(LeafBuf, LOr) % 16 == 0 && offsetof(LeafBuf, LIc) % 16 ==
 // Q divides by s_r as one correctly rounded fp32 division: the quotient is formed as
 // pre * (1/s_r), whose distance to the division's result is below 2e-7 |x|, and the exact
 // division is taken instead whenever that quotient lies within 1e-6 max(1,|x|) of a rounding
-// boundary, so the decision always equals the division's.
+// boundary, so the decision always equals the division's. Stochastic Q (kStoch) decides on
+// y = x + u (one fp32 addition) with floor: its boundaries are the integers, and the exact
+// division is taken whenever y lies within 1e-6 max(1,|y|) of one; the two y differ by at most
+// 2e-7 |x| + 2^-24 (|y| + |y'|) <= 5.2e-7 max(1,|y|) since |x| <= |y| + 1, so outside that
+// zone both lie between the same integers.
 //
 // The wavefront runs on two warps: the solver warp runs the element chain (the slot's sum, Q,
-// e, u and the distance-1 terms), the helper warp the distance >= 2 pushes one step behind. Round rho: the solver computes step rho from the helper's partial sums of slot rho
+// e, u and the distance-1 terms), the helper warp the distance >= 2 pushes one step behind.
+// Round rho: the solver computes step rho from the helper's partial sums of slot rho
 // (everything from steps <= rho - 2 on top of T, R) plus its own distance-1 terms of step
 // rho - 1; the helper pushes step rho - 1 and publishes slot rho + 1. One named barrier of the
 // two warps closes each round.
@@ -70,6 +80,7 @@ __device__ __forceinline__ void pair_sync(int id) {
     asm volatile("bar.sync %0, 64;" ::"r"(id) : "memory");
 }
 
+template <bool kStoch>
 __device__ __forceinline__ void solve_leaf_chain(int lane, int rows, int cols, float qlo,
                                                  float qhi, LeafBuf& B, LeafXchg& X, int bar,
                                                  int* status) {
@@ -95,16 +106,24 @@ __device__ __forceinline__ void solve_leaf_chain(int lane, int rows, int cols, f
             const float pre = w_star + tT + tR;
             float q = 0.f;
             if (sr > 0.f) {
-                float x = pre * inv;
-                const float t = fabsf(x - rintf(x));
-                if (0.5f - t < 1e-6f * fmaxf(1.f, fabsf(x))) x = __fdiv_rn(pre, sr);
-                q = fminf(fmaxf(rintf(x), qlo), qhi);
+                if constexpr (kStoch) {
+                    const float uv = ((float)(uint16_t)B.oC[rr * LB + j] + 0.5f) * (1.f / 65536.f);
+                    float y = __fadd_rn(__fmul_rn(pre, inv), uv);
+                    const float t = fabsf(y - rintf(y));
+                    if (t < 1e-6f * fmaxf(1.f, fabsf(y))) y = __fadd_rn(__fdiv_rn(pre, sr), uv);
+                    q = fminf(fmaxf(floorf(y), qlo), qhi);
+                } else {
+                    float x = pre * inv;
+                    const float t = fabsf(x - rintf(x));
+                    if (0.5f - t < 1e-6f * fmaxf(1.f, fabsf(x))) x = __fdiv_rn(pre, sr);
+                    q = fminf(fmaxf(rintf(x), qlo), qhi);
+                }
             }
             bad |= !isfinite(pre);
             const float w = sr * q;
             e = w_star - w;
             u = tT + e;
-            B.oC[rr * LB + j] = (int8_t)q;
+            B.oC[rr * LB + j] = (int16_t)q;
             B.oE[rr * LB + j] = e;
             B.oEt[j * LB + rr] = e;
             B.oU[rr * LB + j] = u;
