@@ -17,7 +17,11 @@ Sources (web pages on the method):
     a_i column i of the strictly upper triangular m x m L_O, b_j column j of the strictly upper
     triangular n x n L_I, Q nearest (or stochastic) rounding;
   - section 4: the factorisation H_O = (L_O + I) D_O (L_O + I)^T (likewise H_I) and the bound
-    dW (H_O (x) H_I) dW^T <= tr(D_I) tr(D_O) sigma^2.
+    dW (H_O (x) H_I) dW^T <= tr(D_I) tr(D_O) sigma^2;
+  - section 3: the Kronecker factors themselves: the one-sided input second moment
+    H_1 = E[x^T x] (also Sketch A's starting point) and Sketch B, one power-iteration round from
+    the identity, (H_I)_1 = E_s[G_s^T G_s] / m and (H_O)_1 = E_s[G_s G_s^T] / n over the
+    per-sequence weight gradients G_s (m x n).
 
 Readings taken where the pages are garbled or silent (each one is listed in the design notes):
 * index ranges ``:i`` / ``:j`` are exclusive (rows k < i, columns l < j);
@@ -30,6 +34,8 @@ Readings taken where the pages are garbled or silent (each one is listed in the 
   with one correctly rounded fp32 division before round-half-even (pre itself stays fp64);
 * E = W* - W always includes the clamp error;
 * the proxy loss is tr(H_O dW H_I dW^T) with no factor 1/2;
+* every Kronecker factor is damped like the benchmark's inputs: H + damp * mean(diag(H)) * I,
+  the mean taken over the undamped diagonal;
 * stochastic Q (the section-4 alternative to nearest rounding) rounds x = pre/s_i up with
   probability frac(x): code = clamp(floor(x + u)) with u uniform on (0, 1). The pages name no
   generator, so u is drawn by Philox4x64-10 (Salmon, Moraes, Dror, Shaw, "Parallel random
@@ -53,7 +59,7 @@ __all__ = [
     "udu", "quantize", "round_naive", "round_row_sweep", "fixed_point_pre",
     "proxy_loss", "proxy_loss_kron", "brute_force_fixed_points", "gptq_obs",
     "code_range", "fixed_point_pre_rows", "band_check", "grid_quotient",
-    "philox4x64_10", "dither", "quantize_stochastic",
+    "philox4x64_10", "dither", "quantize_stochastic", "damped_gram", "sketch_b",
 ]
 
 
@@ -301,6 +307,33 @@ def proxy_loss_kron(dW, H_O, H_I) -> float:
     v = np.asarray(dW, dtype=np.float64).reshape(-1)
     K = np.kron(np.asarray(H_O, np.float64), np.asarray(H_I, np.float64))
     return float(v @ K @ v)
+
+
+# ---------------------------------------------------------------------------------------------
+# The Kronecker factors ([YAQA] section 3), damped.
+# ---------------------------------------------------------------------------------------------
+def _damp(G: np.ndarray, damp: float) -> np.ndarray:
+    H = G.copy()
+    H[np.diag_indices_from(H)] += damp * float(np.mean(np.diag(G)))
+    return H
+
+
+def damped_gram(X, damp: float) -> np.ndarray:
+    """E[x^T x] over the N rows x of X (N x d), plus damp * mean(diag) * I, in fp64:
+    H = X^T X / N + damp * mean_i (X^T X / N)_ii * I."""
+    X = np.asarray(X, dtype=np.float64)
+    return _damp(X.T @ X / X.shape[0], damp)
+
+
+def sketch_b(G, damp: float) -> tuple[np.ndarray, np.ndarray]:
+    """Sketch B, one power-iteration round from H_O = H_I = I, for per-sequence gradients
+    G (S x m x n), each factor damped: returns (H_O, H_I) with
+    H_O = (1/S) sum_s G_s G_s^T / n,   H_I = (1/S) sum_s G_s^T G_s / m."""
+    G = np.asarray(G, dtype=np.float64)
+    S, m, n = G.shape
+    HO = sum(G[s] @ G[s].T for s in range(S)) / (S * n)
+    HI = sum(G[s].T @ G[s] for s in range(S)) / (S * m)
+    return _damp(HO, damp), _damp(HI, damp)
 
 
 # ---------------------------------------------------------------------------------------------
