@@ -1,11 +1,13 @@
 """Benchmark of the BaKron solve path on synthetic LLM-layer workloads.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
-                    [--rounding nearest|stochastic]
+                    [--rounding nearest|stochastic] [--hessian]
 
 One step = the whole path on one layer with inputs resident in HBM:
     bakron_ldl(H_O), bakron_ldl(H_I), bakron_round(W*, L_O, L_I, scales, bits),
     bakron_proxy_loss(W* - W, H_O, H_I).
+--hessian adds the two damped Kronecker factors to the step: bakron_damped_gram builds H_I from
+the layer's token matrix X and H_O from its gradient rows G (resident in HBM) before the solve.
 --rounding stochastic times bakron_round_stochastic (stochastic Q, a fixed seed per step) in
 place of bakron_round. Metric: quantized weights per second, m*n / step time (whole job: summed over replicas, one
 independent layer per GPU, no collective on the data path; timed as the max over ranks).
@@ -105,6 +107,24 @@ def _dist():
     return ws, rank, local
 
 
+def max_over_ranks(x: float, device) -> float:
+    """The maximum of x over all ranks, returned on every rank (x itself without a process
+    group): a multi-GPU time is the slowest rank's."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_value(world: int, m: int, n: int, ms_per_step: float) -> float:
+    """Weights per second of the whole job: each of the `world` replicas rounds its own m x n
+    layer per step, and the step takes the slowest rank's time."""
+    return world * m * n / (ms_per_step * 1e-3)
+
+
 def oracle_sample(wl, arrays=None, seconds_target: float = 12.0):
     """Times the oracle's whole path on leading r x 2r sub-layers of the workload, growing r by
     1.25x until one run takes a quarter of ``seconds_target``; returns the last (r, c, s)."""
@@ -186,24 +206,55 @@ def run(args):
     dev = torch.device("cuda", torch.cuda.current_device())
 
     from two_sided_adaptive_bakron_b200 import bakron as bk
-    from two_sided_adaptive_bakron_b200.workloads import WORKLOADS, make_workload
+    from two_sided_adaptive_bakron_b200.workloads import (WORKLOADS, make_layer_samples,
+                                                          make_workload)
     wl = WORKLOADS[args.workload]
     m, n = wl.m, wl.n
-    Ws_np, HO_np, HI_np, s_np, bits = make_workload(wl, device=str(dev))
+    samples = None   # --hessian: (X, G) on the device, their host copies, the Gram shapes
+    if args.hessian:
+        Ws_np, X_np, G_np, s_np, bits = make_layer_samples(wl)
+        if X_np is None or G_np is None:
+            raise SystemExit(f"--hessian needs both sample matrices; {wl.name} has an "
+                             "identity factor")
+        samples = ((torch.from_numpy(X_np).to(dev), torch.from_numpy(G_np).to(dev)),
+                   (X_np, G_np),
+                   {"gram_I": (n, X_np.shape[0]), "gram_O": (m, G_np.shape[0])})
+        HO = torch.empty((m, m), dtype=torch.float32, device=dev)
+        HI = torch.empty((n, n), dtype=torch.float32, device=dev)
+        HO_np = HI_np = None
+        ws_g = bk.workspace(max(bk.bakron_damped_gram_workspace_bytes(X_np.shape[0], n),
+                                bk.bakron_damped_gram_workspace_bytes(G_np.shape[0], m)), dev)
+        del X_np, G_np
+    else:
+        Ws_np, HO_np, HI_np, s_np, bits = make_workload(wl, device=str(dev))
+        HO = torch.from_numpy(HO_np).to(dev)
+        HI = torch.from_numpy(HI_np).to(dev)
     Ws = torch.from_numpy(Ws_np).to(dev)
-    HO = torch.from_numpy(HO_np).to(dev)
-    HI = torch.from_numpy(HI_np).to(dev)
     sc = torch.from_numpy(s_np).to(dev)
     solver = bk.Solver(m, n, dev)
     stream = torch.cuda.current_stream(dev)
 
     # ---- per-call timing events on the launching stream (device-timed breakdown)
-    names = ["ldl_O", "ldl_I", "round", "loss"]
+    names = (["gram_I", "gram_O"] if args.hessian else []) + ["ldl_O", "ldl_I", "round", "loss"]
 
     seed = 0x5EED if args.rounding == "stochastic" else None
 
+    def factors(X, G, timing):
+        # H_I from the tokens, H_O from the gradient rows, into the buffers the solve reads
+        for nm, A, H in (("gram_I", X, HI), ("gram_O", G, HO)):
+            ev = timing.get(nm) if timing else None
+            if ev is not None:
+                ev[0].record(stream)
+            rc = bk.bakron_damped_gram(A, wl.damp, H, ws_g, solver.status, stream)
+            if rc != 0:
+                raise bk.BakronError(rc, "bakron_damped_gram")
+            if ev is not None:
+                ev[1].record(stream)
+
     def step(evs=None):
         timing = None if evs is None else dict(zip(names, evs))
+        if samples is not None:
+            factors(samples[0][0], samples[0][1], timing)
         solver.run(Ws, HO, HI, sc, bits, stream, timing=timing, seed=seed)
 
     for _ in range(args.warmup):
@@ -228,48 +279,55 @@ def run(args):
         t_end.record(stream)
         torch.cuda.synchronize()
     launches = bk.bakron_kernel_launches() - l0
-    ms_total = t_start.elapsed_time(t_end)
-    if ws > 1:
-        t = torch.tensor([ms_total], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms_total = float(t.item())
+    ms_total = max_over_ranks(t_start.elapsed_time(t_end), dev)
     st = bk.bakron_read_status(solver.status, stream)
     if st != 0:
         raise bk.BakronError(st, "timed region")
     ms_step = ms_total / args.steps
-    value = ws * m * n / (ms_step * 1e-3)
+    value = whole_job_value(ws, m, n, ms_step)
     per = {nm: statistics.mean(evs[k][i][0].elapsed_time(evs[k][i][1]) for k in range(args.steps))
            for i, nm in enumerate(names)}
 
     e2e = None
     if not args.no_e2e:
         e2e = _e2e(args, torch, bk, solver, stream, dev, ws, m, n, bits, Ws, HO, HI, sc,
-                   Ws_np, HO_np, HI_np, s_np, seed)
+                   Ws_np, HO_np, HI_np, s_np, seed,
+                   (samples[1], samples[0], factors) if samples is not None else None)
     return _report(args, torch, bk, wl, ws, rank, m, n, bits, per, ms_step, value, launches,
-                   clk, e2e, (Ws_np, HO_np, HI_np, s_np, bits))
+                   clk, e2e, None if samples is not None else (Ws_np, HO_np, HI_np, s_np, bits),
+                   samples[2] if samples is not None else None)
 
 
 def _e2e(args, torch, bk, solver, stream, dev, ws, m, n, bits, Ws, HO, HI, sc,
-         Ws_np, HO_np, HI_np, s_np, seed):
+         Ws_np, HO_np, HI_np, s_np, seed, hess=None):
     """Same metric through the public API with host buffers: pinned host -> device copies of
-    the step's inputs, the whole path, device -> host copies of the codes and the loss."""
+    the step's inputs (W*, the scales and either H_O, H_I or, with --hessian, the samples X and
+    G), the whole path, device -> host copies of the codes and the loss."""
     hW = torch.from_numpy(Ws_np).pin_memory()
-    hO = torch.from_numpy(HO_np).pin_memory()
-    hI = torch.from_numpy(HI_np).pin_memory()
     hs = torch.from_numpy(s_np).pin_memory()
+    if hess is None:
+        h_in = (torch.from_numpy(HO_np).pin_memory(), torch.from_numpy(HI_np).pin_memory())
+        d_in = (torch.empty_like(HO), torch.empty_like(HI))
+    else:
+        (X_np, G_np), (Xd, Gd), factors = hess
+        h_in = (torch.from_numpy(X_np).pin_memory(), torch.from_numpy(G_np).pin_memory())
+        d_in = (torch.empty_like(Xd), torch.empty_like(Gd))
     hcodes = torch.empty((m, n), dtype=torch.int8).pin_memory()
     hloss = torch.empty((1,), dtype=torch.float64).pin_memory()
-    dW2, dO2, dI2, ds2 = (torch.empty_like(Ws), torch.empty_like(HO), torch.empty_like(HI),
-                          torch.empty_like(sc))
-    h2d = sum(x.numel() * x.element_size() for x in (hW, hO, hI, hs))
+    dW2, ds2 = torch.empty_like(Ws), torch.empty_like(sc)
+    h2d = sum(x.numel() * x.element_size() for x in (hW, hs) + h_in)
     d2h = m * n + 8
 
     def e2e_step():
         dW2.copy_(hW, non_blocking=True)
-        dO2.copy_(hO, non_blocking=True)
-        dI2.copy_(hI, non_blocking=True)
         ds2.copy_(hs, non_blocking=True)
-        solver.run(dW2, dO2, dI2, ds2, bits, stream, seed=seed)
+        for d_, h_ in zip(d_in, h_in):
+            d_.copy_(h_, non_blocking=True)
+        if hess is None:
+            solver.run(dW2, d_in[0], d_in[1], ds2, bits, stream, seed=seed)
+        else:
+            factors(d_in[0], d_in[1], None)
+            solver.run(dW2, HO, HI, ds2, bits, stream, seed=seed)
         hcodes.copy_(solver.codes, non_blocking=True)
         hloss.copy_(solver.loss, non_blocking=True)
 
@@ -284,12 +342,8 @@ def _e2e(args, torch, bk, solver, stream, dev, ws, m, n, bits, Ws, HO, HI, sc,
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / args.steps
-    if ws > 1:
-        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = ws * m * n / (e2e_ms * 1e-3)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, dev)
+    e2e_value = whole_job_value(ws, m, n, e2e_ms)
     return {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h}
 
@@ -300,7 +354,7 @@ def _e2e(args, torch, bk, solver, stream, dev, ws, m, n, bits, Ws, HO, HI, sc,
 ROUND_TRAFFIC_BYTES = {(4096, 14336): 36.35e9}
 
 
-def _roofline(per, m, n, rounding="nearest"):
+def _roofline(per, m, n, rounding="nearest", gram_dims=None):
     """Roofline of the step's dominant kernel, round_kernel (one launch per step that runs the
     whole rounding solve: the largest single kernel and the largest share of the launch
     list), on its algorithmic work. The factorisation of H_I takes about as long, but as
@@ -319,6 +373,8 @@ def _roofline(per, m, n, rounding="nearest"):
         "round": float(m) * n * (m + n),                       # triangular pushes, 2 flop/MAC
         "loss": 2.0 * min(m, n) ** 2 * max(m, n) + float(m) * n * max(m, n),
     }
+    for k, (d, K) in (gram_dims or {}).items():       # a Gram: d (d + 1) / 2 K multiply-adds
+        work[k] = float(d) * (d + 1) * K
     t = per["round"] * 1e-3
     achieved = work["round"] / t / 1e12
     return {"bound": "tensor", "kernel": "round_kernel", "achieved": achieved, "peak": peak,
@@ -333,8 +389,8 @@ def _roofline(per, m, n, rounding="nearest"):
 
 
 def _report(args, torch, bk, wl, ws, rank, m, n, bits, per, ms_step, value, launches, clk,
-            e2e, arrays):
-    roofline = _roofline(per, m, n, args.rounding)
+            e2e, arrays, gram_dims=None):
+    roofline = _roofline(per, m, n, args.rounding, gram_dims)
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         rr, c, dt = oracle_sample(wl, arrays)
@@ -346,7 +402,7 @@ def _report(args, torch, bk, wl, ws, rank, m, n, bits, per, ms_step, value, laun
                 "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
                 "config": {"workload": wl.name, "m": m, "n": n, "bits": bits,
-                           "rounding": args.rounding,
+                           "rounding": args.rounding, "hessian": bool(args.hessian),
                            "parallelism": f"replicas x{ws}" if ws > 1 else "single",
                            "l2": "inputs larger than L2 (H_I alone is "
                                  f"{4 * n * n / 2**20:.0f} MiB), no flush"},
@@ -372,6 +428,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--ref-seconds", type=float, default=12.0)
     ap.add_argument("--rounding", default="nearest", choices=["nearest", "stochastic"])
+    ap.add_argument("--hessian", action="store_true")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)

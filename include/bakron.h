@@ -153,6 +153,49 @@ size_t bakron_proxy_loss_workspace_bytes(int m, int n);
 int bakron_proxy_loss(const float* dW, int m, int n, const float* H_O, const float* H_I,
                       double* loss, void* ws, size_t ws_bytes, void* stream);
 
+/* ------------------------------------------------------------------------------------------
+ * bakron_damped_gram -- one damped Kronecker factor from samples: the input second moment.
+ *
+ *   H = X^T X / N + damp * mean_i (X^T X / N)_ii * I
+ *
+ * (YAQA article, section 3: H_1 = E[x^T x] over the input rows x, the one-sided factor and
+ * Sketch A's starting point; the same call gives E[g^T g] over output-gradient rows g. The
+ * relative damping is that of the solver's inputs.) The product runs as 3xTF32 on the tensor
+ * cores over the upper block triangle; H is then made exactly symmetric. Accuracy: each
+ * product is within 3 * 2^-20 of exact, and the fp32 accumulation over the N samples loses
+ * up to about 2^-24 N sqrt(H_aa H_bb) per entry (the tensor core rounds its accumulator
+ * toward zero; 1.6e-4 sqrt(H_aa H_bb) at N = 8192).
+ *
+ *   X        [in]  N x d samples (rows), fp32.
+ *   N, d     [in]  1 <= N <= 2097120, 1 <= d <= 65536.
+ *   damp     [in]  relative damping >= 0 (0.01 for the solver's inputs).
+ *   H        [out] d x d, symmetric, written in full; ready for bakron_ldl.
+ *   ws       [in]  at least bakron_damped_gram_workspace_bytes(N, d) bytes, 256-B aligned.
+ *   dev_status [out] BAKRON_ERR_TIMEOUT if a pipeline wait of the product gave up.
+ * ---------------------------------------------------------------------------------------- */
+size_t bakron_damped_gram_workspace_bytes(int N, int d);
+int bakron_damped_gram(const float* X, int N, int d, float damp, float* H, void* ws,
+                       size_t ws_bytes, int* dev_status, void* stream);
+
+/* ------------------------------------------------------------------------------------------
+ * bakron_sketch_b -- both Kronecker factors from per-sequence weight gradients (YAQA article,
+ * section 3, Sketch B: one power-iteration round on the Fisher from H_O = H_I = I), damped:
+ *
+ *   H_O = (1/S) sum_s G_s G_s^T / n  + damp * mean(diag) * I      (m x m)
+ *   H_I = (1/S) sum_s G_s^T G_s / m  + damp * mean(diag) * I      (n x n)
+ *
+ *   G        [in]  S x m x n: the gradient of the loss of sequence s w.r.t. the m x n weight
+ *                  is G + s*m*n, row-major.
+ *   S, m, n  [in]  1 <= m, n <= 65536, S*m <= 2097120, S*n <= 2^30.
+ *   damp     [in]  relative damping >= 0.
+ *   H_O, H_I [out] symmetric, written in full.
+ *   ws       [in]  at least bakron_sketch_b_workspace_bytes(S, m, n) bytes, 256-B aligned.
+ *   dev_status [out] as for bakron_damped_gram.
+ * ---------------------------------------------------------------------------------------- */
+size_t bakron_sketch_b_workspace_bytes(int S, int m, int n);
+int bakron_sketch_b(const float* G, int S, int m, int n, float damp, float* H_O, float* H_I,
+                    void* ws, size_t ws_bytes, int* dev_status, void* stream);
+
 /* Synchronises `stream`, then returns the device status word (a bakron_status value), or
  * BAKRON_ERR_CUDA if the synchronisation itself failed. */
 int bakron_read_status(const int* dev_status, void* stream);

@@ -60,6 +60,7 @@ __all__ = [
     "proxy_loss", "proxy_loss_kron", "brute_force_fixed_points", "gptq_obs",
     "code_range", "fixed_point_pre_rows", "band_check", "grid_quotient",
     "philox4x64_10", "dither", "quantize_stochastic", "damped_gram", "sketch_b",
+    "damped_gram_rows",
 ]
 
 
@@ -323,6 +324,18 @@ def damped_gram(X, damp: float) -> np.ndarray:
     H = X^T X / N + damp * mean_i (X^T X / N)_ii * I."""
     X = np.asarray(X, dtype=np.float64)
     return _damp(X.T @ X / X.shape[0], damp)
+
+
+def damped_gram_rows(X, damp: float, rows) -> np.ndarray:
+    """``damped_gram`` restricted to the given rows (same definition, fp64): the rows R of
+    X^T X / N, with damp * mean of the full diagonal added at (R[k], R[k])."""
+    X = np.asarray(X, dtype=np.float64)
+    rows = np.asarray(rows)
+    N = X.shape[0]
+    out = X[:, rows].T @ X / N
+    mean_diag = float(np.mean(np.einsum("ti,ti->i", X, X))) / N
+    out[np.arange(rows.size), rows] += damp * mean_diag
+    return out
 
 
 def sketch_b(G, damp: float) -> tuple[np.ndarray, np.ndarray]:

@@ -15,7 +15,7 @@ other than itself:
 import numpy as np
 import pytest
 
-from oracle import damped_gram, sketch_b
+from oracle import damped_gram, damped_gram_rows, sketch_b
 
 
 def _rng(seed):
@@ -100,3 +100,10 @@ def test_sketch_b_kronecker_gradients():
     e = np.mean(c ** 2)
     np.testing.assert_allclose(HO, e * (v @ v) / n * np.outer(u, u), rtol=1e-12, atol=1e-14)
     np.testing.assert_allclose(HI, e * (u @ u) / m * np.outer(v, v), rtol=1e-12, atol=1e-14)
+
+
+def test_gram_rows_is_the_gram_restricted():
+    X = _rng(6).standard_normal((40, 23))
+    rows = np.array([0, 5, 22, 5])
+    np.testing.assert_allclose(damped_gram_rows(X, 0.03, rows), damped_gram(X, 0.03)[rows],
+                               rtol=1e-12, atol=1e-14)

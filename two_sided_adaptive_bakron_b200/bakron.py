@@ -1,10 +1,12 @@
 """Python binding of libbakron.so (ctypes): argument marshalling only.
 
 The functions named like the C ABI (``bakron_ldl``, ``bakron_round``,
-``bakron_round_stochastic``, ``bakron_proxy_loss``, ``bakron_read_status``,
-``bakron_status_string`` and the ``*_workspace_bytes`` queries) take torch CUDA tensors, pass
-their device pointers and the current CUDA stream to the library and return its status code. ``ldl``, ``round_weights``, ``proxy_loss`` and ``solve`` additionally
-allocate outputs and workspaces with torch and raise on any error.
+``bakron_round_stochastic``, ``bakron_proxy_loss``, ``bakron_damped_gram``, ``bakron_sketch_b``,
+``bakron_read_status``, ``bakron_status_string`` and the ``*_workspace_bytes`` queries) take
+torch CUDA tensors, pass their device pointers and the current CUDA stream to the library and
+return its status code. ``ldl``, ``round_weights``, ``proxy_loss``, ``damped_gram``,
+``sketch_b`` and ``solve`` additionally allocate outputs and workspaces with torch and raise on
+any error.
 
 Every step of the computation runs in the library's CUDA kernels; there is no CPU path. If
 the shared library is missing the first call raises.
@@ -41,6 +43,12 @@ _SIGNATURES = {
                                          ctypes.c_uint64, _vp, _vp, _vp, _c_size_t, _vp, _vp]),
     "bakron_proxy_loss_workspace_bytes": (_c_size_t, [_c_int, _c_int]),
     "bakron_proxy_loss": (_c_int, [_vp, _c_int, _c_int, _vp, _vp, _vp, _vp, _c_size_t, _vp]),
+    "bakron_damped_gram_workspace_bytes": (_c_size_t, [_c_int, _c_int]),
+    "bakron_damped_gram": (_c_int, [_vp, _c_int, _c_int, ctypes.c_float, _vp, _vp, _c_size_t,
+                                    _vp, _vp]),
+    "bakron_sketch_b_workspace_bytes": (_c_size_t, [_c_int, _c_int, _c_int]),
+    "bakron_sketch_b": (_c_int, [_vp, _c_int, _c_int, _c_int, ctypes.c_float, _vp, _vp, _vp,
+                                 _c_size_t, _vp, _vp]),
     "bakron_read_status": (_c_int, [_vp, _vp]),
     "bakron_status_string": (ctypes.c_char_p, [_c_int]),
     "bakron_version": (_c_int, []),
@@ -173,6 +181,33 @@ def bakron_proxy_loss(dW, H_O, H_I, loss, ws, stream=None) -> int:
                                    ws.numel() * ws.element_size(), _stream(stream))
 
 
+def bakron_damped_gram_workspace_bytes(N: int, d: int) -> int:
+    return int(lib().bakron_damped_gram_workspace_bytes(int(N), int(d)))
+
+
+def bakron_sketch_b_workspace_bytes(S: int, m: int, n: int) -> int:
+    return int(lib().bakron_sketch_b_workspace_bytes(int(S), int(m), int(n)))
+
+
+def bakron_damped_gram(X, damp, H, ws, dev_status, stream=None) -> int:
+    N, d = X.shape
+    _check_cuda(X, torch.float32, (N, d), "X")
+    _check_cuda(H, torch.float32, (d, d), "H")
+    return lib().bakron_damped_gram(_ptr(X), N, d, float(damp), _ptr(H), _ptr(ws),
+                                    ws.numel() * ws.element_size(), _ptr(dev_status),
+                                    _stream(stream))
+
+
+def bakron_sketch_b(G, damp, H_O, H_I, ws, dev_status, stream=None) -> int:
+    S, m, n = G.shape
+    _check_cuda(G, torch.float32, (S, m, n), "G")
+    _check_cuda(H_O, torch.float32, (m, m), "H_O")
+    _check_cuda(H_I, torch.float32, (n, n), "H_I")
+    return lib().bakron_sketch_b(_ptr(G), S, m, n, float(damp), _ptr(H_O), _ptr(H_I), _ptr(ws),
+                                 ws.numel() * ws.element_size(), _ptr(dev_status),
+                                 _stream(stream))
+
+
 def bakron_ldl_noalloc(H, L, D, dev_status, stream=None) -> int:
     """bakron_ldl with the library's own fixed scratch (no workspace argument)."""
     n = H.shape[0]
@@ -268,6 +303,31 @@ def round_weights(Wstar, L_O, L_I, scales, bits, stream=None, check: bool = True
     if check:
         _raise(bakron_read_status(st, stream), "bakron_round (device)")
     return codes, W
+
+
+def damped_gram(X, damp: float = 0.01, stream=None, check: bool = True) -> torch.Tensor:
+    """X^T X / N + damp * mean(diag) * I for samples X (N x d) on the device."""
+    N, d = X.shape
+    H = torch.empty((d, d), dtype=torch.float32, device=X.device)
+    ws = workspace(bakron_damped_gram_workspace_bytes(N, d), X.device)
+    st = new_status(X.device)
+    _raise(bakron_damped_gram(X, damp, H, ws, st, stream), "bakron_damped_gram")
+    if check:
+        _raise(bakron_read_status(st, stream), "bakron_damped_gram (device)")
+    return H
+
+
+def sketch_b(G, damp: float = 0.01, stream=None, check: bool = True):
+    """(H_O, H_I) of Sketch B from per-sequence gradients G (S x m x n) on the device."""
+    S, m, n = G.shape
+    H_O = torch.empty((m, m), dtype=torch.float32, device=G.device)
+    H_I = torch.empty((n, n), dtype=torch.float32, device=G.device)
+    ws = workspace(bakron_sketch_b_workspace_bytes(S, m, n), G.device)
+    st = new_status(G.device)
+    _raise(bakron_sketch_b(G, damp, H_O, H_I, ws, st, stream), "bakron_sketch_b")
+    if check:
+        _raise(bakron_read_status(st, stream), "bakron_sketch_b (device)")
+    return H_O, H_I
 
 
 def proxy_loss(dW, H_O, H_I, stream=None) -> torch.Tensor:

@@ -31,8 +31,8 @@ from typing import Optional
 
 import numpy as np
 
-__all__ = ["Workload", "WORKLOADS", "make_workload", "row_scales", "damped_gram",
-           "code_range"]
+__all__ = ["Workload", "WORKLOADS", "make_workload", "make_layer_samples", "row_scales",
+           "damped_gram", "code_range"]
 
 
 @dataclasses.dataclass(frozen=True)
@@ -117,11 +117,11 @@ def _token_matrix(rng, N: int, d: int, lognormal: bool, out_idx, out_scale):
     return X
 
 
-def make_workload(w: Workload | str, device: Optional[str] = None, seed: Optional[int] = None):
-    """Draw (W*, H_O, H_I, scales, bits) for a workload, all fp32 numpy arrays.
-
-    ``device`` (e.g. "cuda") only moves the fp64 Gram products onto a GPU for speed; the random
-    draws are always numpy PCG64 on the host.
+def make_layer_samples(w: Workload | str, seed: Optional[int] = None):
+    """Draw (W*, X, G, scales, bits): the layer and the raw samples whose damped second moments
+    are its Kronecker factors, all fp32 numpy arrays. X (tokens x n) gives H_I, G (gradient
+    rows x m) gives H_O; either is None where the workload's factor is the identity. The draws
+    are those of ``make_workload`` (same order), which forms the damped Grams from them.
     """
     if isinstance(w, str):
         w = WORKLOADS[w]
@@ -139,30 +139,40 @@ def make_workload(w: Workload | str, device: Optional[str] = None, seed: Optiona
         Wstar[:, out_idx] *= w.outlier_scale
     Wstar = Wstar.astype(np.float32)
 
-    if w.variant == "identity":
-        H_I = np.eye(n, dtype=np.float32)
-    else:
+    X = None
+    if w.variant != "identity":
         X = _token_matrix(rng, w.tokens, n, w.x_lognormal, out_idx, w.outlier_scale)
-        H_I = damped_gram(X, w.damp, device)
-        del X
 
+    G = None
     if w.variant in ("identity", "ho_identity"):
-        H_O = np.eye(m, dtype=np.float32)
+        pass
     elif w.grad_rank == 0:
         G = _token_matrix(rng, w.grad_rows, m, True, None, 1.0)
-        H_O = damped_gram(G, w.damp, device)
-        del G
     else:
         r = w.grad_rank
         Z = rng.standard_normal((w.grad_rows, r), dtype=np.float32)
         B = rng.standard_normal((r, m), dtype=np.float32)
         G = (Z @ B) * np.float32(1.0 / math.sqrt(r))
         G += np.float32(0.1) * rng.standard_normal((w.grad_rows, m), dtype=np.float32)
-        H_O = damped_gram(G, w.damp, device)
-        del G, Z, B
+        del Z, B
 
-    scales = row_scales(Wstar, w.bits)
-    return Wstar, H_O, H_I, scales, w.bits
+    return Wstar, X, G, row_scales(Wstar, w.bits), w.bits
+
+
+def make_workload(w: Workload | str, device: Optional[str] = None, seed: Optional[int] = None):
+    """Draw (W*, H_O, H_I, scales, bits) for a workload, all fp32 numpy arrays.
+
+    ``device`` (e.g. "cuda") only moves the fp64 Gram products onto a GPU for speed; the random
+    draws are always numpy PCG64 on the host.
+    """
+    if isinstance(w, str):
+        w = WORKLOADS[w]
+    Wstar, X, G, scales, bits = make_layer_samples(w, seed)
+    H_I = np.eye(w.n, dtype=np.float32) if X is None else damped_gram(X, w.damp, device)
+    del X
+    H_O = np.eye(w.m, dtype=np.float32) if G is None else damped_gram(G, w.damp, device)
+    del G
+    return Wstar, H_O, H_I, scales, bits
 
 
 def random_problem(m: int, n: int, bits: int, seed: int, tokens: Optional[int] = None,
