@@ -34,6 +34,12 @@ Readings taken where the pages are garbled or silent (each one is listed in the 
   with one correctly rounded fp32 division before round-half-even (pre itself stays fp64);
 * E = W* - W always includes the clamp error;
 * the proxy loss is tr(H_O dW H_I dW^T) with no factor 1/2;
+* the base quantizer is pluggable ([BaKron] summary: the solver is modular in the base
+  quantizer): the grid step may be per row and column group, s_ij = scales[i, j // group_size],
+  and Q may round to a sorted scalar codebook c_0 < ... < c_{K-1} instead of the integers:
+  the code is the index of the nearest entry to x = pre / s_ij (the fp32 quotient), decided
+  against the fp32 midpoints fl32((c_k + c_{k+1}) / 2), a tie going to the lower entry, and
+  W_ij = s_ij c_code;
 * every Kronecker factor is damped like the benchmark's inputs: H + damp * mean(diag(H)) * I,
   the mean taken over the undamped diagonal;
 * stochastic Q (the section-4 alternative to nearest rounding) rounds x = pre/s_i up with
@@ -60,7 +66,7 @@ __all__ = [
     "proxy_loss", "proxy_loss_kron", "brute_force_fixed_points", "gptq_obs",
     "code_range", "fixed_point_pre_rows", "band_check", "grid_quotient",
     "philox4x64_10", "dither", "quantize_stochastic", "damped_gram", "sketch_b",
-    "damped_gram_rows",
+    "damped_gram_rows", "codebook_midpoints", "quantize_codebook", "scale_of",
 ]
 
 
@@ -165,20 +171,54 @@ def quantize_stochastic(pre: float, s: float, bits: int, u: float) -> int:
     return int(min(max(float(np.floor(y)), lo), hi))
 
 
-def _q(pre, s, bits, U, i, j):
+# ---------------------------------------------------------------------------------------------
+# Pluggable base quantizer ([BaKron] summary): per-group grid steps, scalar codebooks.
+# ---------------------------------------------------------------------------------------------
+def codebook_midpoints(codebook) -> np.ndarray:
+    """The decision thresholds of a sorted codebook: fl32((c_k + c_{k+1}) / 2) (fp32 sum and
+    halving, both exact or correctly rounded), returned as fp64."""
+    c = np.asarray(codebook, dtype=np.float32)
+    return ((c[:-1] + c[1:]) * np.float32(0.5)).astype(np.float64)
+
+
+def quantize_codebook(pre: float, s: float, codebook) -> int:
+    """Index of the nearest codebook entry to the fp32 quotient pre / s: the number of
+    midpoints strictly below it (a tie goes to the lower entry); s == 0 gives index 0."""
+    if s == 0.0:
+        return 0
+    x = float(grid_quotient(pre, s))
+    return int(np.sum(x > codebook_midpoints(codebook)))
+
+
+def scale_of(scales, i: int, j: int, group_size=None) -> float:
+    """The grid step of entry (i, j): scales[i] (one per row) or scales[i, j // group_size]."""
+    sc = np.asarray(scales)
+    return float(sc[i]) if sc.ndim == 1 else float(sc[i, j // group_size])
+
+
+def _q(pre, s, bits, U, i, j, codebook=None):
+    if codebook is not None:
+        return quantize_codebook(pre, s, codebook)
     return quantize(pre, s, bits) if U is None else quantize_stochastic(pre, s, bits, U[i, j])
+
+
+def _value(code, s, codebook=None):
+    return s * (code if codebook is None else float(np.float32(codebook[code])))
 
 
 # ---------------------------------------------------------------------------------------------
 # The rule, entry by entry, in raster order ([YAQA] section 4). Raster order is a valid order
 # because entry (i, j) reads only entries (k, l) with k <= i and l <= j, (k, l) != (i, j).
 # ---------------------------------------------------------------------------------------------
-def round_naive(Wstar, L_O, L_I, scales, bits, return_pre=False, dither=None):
+def round_naive(Wstar, L_O, L_I, scales, bits, return_pre=False, dither=None, codebook=None,
+                group_size=None):
     """Plain definition, O(m^2 n^2 / 4) multiply-adds.
 
     pre_ij = W*_ij + a_i^T E[:i,:j] b_j + a_i^T E[:i,j] + E[i,:j] b_j,   E = W* - W
     with a_i = L_O[:i, i] and b_j = L_I[:j, j]. ``dither`` (m x n variates u_ij) selects
-    stochastic Q; None selects nearest rounding.
+    stochastic Q; None selects nearest rounding. ``codebook`` selects the nearest entry of a
+    sorted codebook (codes are then entry indices); 2-D ``scales`` (m x G) are per row and
+    column group of ``group_size`` columns.
     Returns (codes int64 m x n, W fp64 m x n[, pre fp64 m x n]).
     """
     Ws = np.asarray(Wstar, dtype=np.float64)
@@ -201,15 +241,17 @@ def round_naive(Wstar, L_O, L_I, scales, bits, return_pre=False, dither=None):
                 pre += a @ E[:i, j]
             if j > 0:
                 pre += E[i, :j] @ b
-            c = _q(pre, s[i], bits, dither, i, j)
+            sij = scale_of(s, i, j, group_size)
+            c = _q(pre, sij, bits, dither, i, j, codebook)
             C[i, j] = c
-            W[i, j] = s[i] * c
+            W[i, j] = _value(c, sij, codebook)
             E[i, j] = Ws[i, j] - W[i, j]
             P[i, j] = pre
     return (C, W, P) if return_pre else (C, W)
 
 
-def round_row_sweep(Wstar, L_O, L_I, scales, bits, return_pre=False, dither=None):
+def round_row_sweep(Wstar, L_O, L_I, scales, bits, return_pre=False, dither=None, codebook=None,
+                    group_size=None):
     """Same result as ``round_naive`` in O(mn(m+n)) work (the row-by-row reading).
 
     Row i sees every earlier row only through T_i = sum_{k<i} L_O[k,i] E_k (a row vector).
@@ -230,9 +272,10 @@ def round_row_sweep(Wstar, L_O, L_I, scales, bits, return_pre=False, dither=None
         r = Ws[i] + T + T @ LI
         for j in range(n):
             pre = r[j] + E[i, :j] @ LI[:j, j]
-            c = _q(pre, s[i], bits, dither, i, j)
+            sij = scale_of(s, i, j, group_size)
+            c = _q(pre, sij, bits, dither, i, j, codebook)
             C[i, j] = c
-            W[i, j] = s[i] * c
+            W[i, j] = _value(c, sij, codebook)
             E[i, j] = Ws[i, j] - W[i, j]
             P[i, j] = pre
     return (C, W, P) if return_pre else (C, W)
@@ -270,20 +313,29 @@ def fixed_point_pre_rows(Wstar, W, L_O, L_I, rows):
     return Ws[rows] + T + T @ LI - E[rows]
 
 
-def band_check(pre, codes, scales, bits, band=1e-3, dither=None):
+def band_check(pre, codes, scales, bits, band=1e-3, dither=None, codebook=None, group_size=None):
     """Compare codes with Q(pre) under the exemption band of the tolerance rule.
 
     An entry may disagree only if pre/s lies within ``band`` grid steps of a rounding boundary
     (a half-integer for nearest rounding; for stochastic Q with variates ``dither``, an
-    integer value of pre/s + u). Returns (n_mismatch, n_mismatch_outside_band, n_in_band).
+    integer value of pre/s + u; for a codebook, a midpoint of two entries). 2-D ``scales``
+    are per row and column group. Returns (n_mismatch, n_mismatch_outside_band, n_in_band).
     """
-    s = np.asarray(scales, dtype=np.float64)[:, None]
+    s = np.asarray(scales, dtype=np.float64)
+    if s.ndim == 1:
+        s = s[:, None]
+    else:
+        s = np.repeat(s, group_size, axis=1)[:, :pre.shape[1]]
     lo, hi = code_range(bits)
     s_safe = np.where(s > 0, s, 1.0)
     with np.errstate(divide="ignore", invalid="ignore"):
         x = np.where(s > 0, pre / s_safe, 0.0)
     xq = np.where(s > 0, grid_quotient(pre, np.broadcast_to(s_safe, pre.shape)), 0.0)
-    if dither is None:
+    if codebook is not None:
+        mids = codebook_midpoints(codebook)
+        q = np.sum(xq[..., None] > mids, axis=-1).astype(np.float64)
+        frac = np.min(np.abs(x[..., None] - mids), axis=-1)
+    elif dither is None:
         q = np.clip(np.rint(xq), lo, hi)
         frac = np.abs(x - np.floor(x) - 0.5)
     else:
@@ -352,7 +404,8 @@ def sketch_b(G, damp: float) -> tuple[np.ndarray, np.ndarray]:
 # ---------------------------------------------------------------------------------------------
 # Independent algorithms used only to pin the rule.
 # ---------------------------------------------------------------------------------------------
-def gptq_obs(w_star: np.ndarray, H: np.ndarray, scales: np.ndarray, bits: int, dither=None):
+def gptq_obs(w_star: np.ndarray, H: np.ndarray, scales: np.ndarray, bits: int, dither=None,
+             codebook=None):
     """GPTQ in its optimal-brain-surgeon form on a vector w (length N) with Hessian H.
 
     Coordinates are fixed in index order. After fixing coordinate q to its quantised value,
@@ -366,10 +419,14 @@ def gptq_obs(w_star: np.ndarray, H: np.ndarray, scales: np.ndarray, bits: int, d
     N = w.shape[0]
     codes = np.zeros(N, dtype=np.int64)
     for q in range(N):
-        c = quantize(w[q], float(scales[q]), bits) if dither is None else \
-            quantize_stochastic(w[q], float(scales[q]), bits, float(dither[q]))
+        if codebook is not None:
+            c = quantize_codebook(w[q], float(scales[q]), codebook)
+        elif dither is None:
+            c = quantize(w[q], float(scales[q]), bits)
+        else:
+            c = quantize_stochastic(w[q], float(scales[q]), bits, float(dither[q]))
         codes[q] = c
-        wq = float(scales[q]) * c
+        wq = _value(c, float(scales[q]), codebook)
         F = np.arange(q, N)
         Hinv = np.linalg.inv(H[np.ix_(F, F)])
         delta = (w[q] - wq) / Hinv[0, 0]
@@ -378,13 +435,15 @@ def gptq_obs(w_star: np.ndarray, H: np.ndarray, scales: np.ndarray, bits: int, d
     return codes
 
 
-def brute_force_fixed_points(Wstar, L_O, L_I, scales, bits, chunk=4096, dither=None):
+def brute_force_fixed_points(Wstar, L_O, L_I, scales, bits, chunk=4096, dither=None,
+                             codebook=None):
     """All code matrices C with C = Q(pre(C)) under the closed form, by enumeration.
 
     Every candidate C in [lo, hi]^(m x n) is tried: W = s * C, pre is the closed form of
     ``fixed_point_pre`` (evaluated for a batch of candidates at once with the same fp64
-    products), and C is kept when Q(pre) == C at every entry (nearest, or stochastic with the
-    variates ``dither``). Tiny shapes only
+    products), and C is kept when Q(pre) == C at every entry (nearest, stochastic with the
+    variates ``dither``, or the index of the nearest ``codebook`` entry, when the candidates
+    are the indices 0 .. K-1 and W = s * c_C). Tiny shapes only
     ((2^bits)^(mn) candidates). Rows with s_i = 0 are not supported here.
     """
     Ws = np.asarray(Wstar, dtype=np.float64)
@@ -393,7 +452,8 @@ def brute_force_fixed_points(Wstar, L_O, L_I, scales, bits, chunk=4096, dither=N
     lo, hi = code_range(bits)
     Ao = np.eye(m) + np.asarray(L_O, dtype=np.float64)
     Ai = np.eye(n) + np.asarray(L_I, dtype=np.float64)
-    values = np.arange(lo, hi + 1)
+    values = np.arange(lo, hi + 1) if codebook is None else np.arange(len(codebook))
+    cb32 = None if codebook is None else np.asarray(codebook, dtype=np.float32).astype(np.float64)
     total = len(values) ** (m * n)
     found = []
     for start in range(0, total, chunk):
@@ -404,10 +464,12 @@ def brute_force_fixed_points(Wstar, L_O, L_I, scales, bits, chunk=4096, dither=N
             digits[:, p] = values[rest % len(values)]
             rest //= len(values)
         C = digits.reshape(-1, m, n)
-        E = Ws[None] - s[None, :, None] * C
+        E = Ws[None] - s[None, :, None] * (C if cb32 is None else cb32[C])
         pre = Ws[None] + np.einsum("ki,bkl,lj->bij", Ao, E, Ai) - E
         xq = grid_quotient(pre, np.broadcast_to(s[None, :, None], pre.shape))
-        if dither is None:
+        if codebook is not None:
+            Q = np.sum(xq[..., None] > codebook_midpoints(codebook), axis=-1)
+        elif dither is None:
             Q = np.clip(np.rint(xq), lo, hi)
         else:
             u = np.asarray(dither, dtype=np.float32)[None]
