@@ -2,12 +2,16 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
                     [--rounding nearest|stochastic] [--hessian]
+                    [--group-size G] [--codebook normal]
 
 One step = the whole path on one layer with inputs resident in HBM:
     bakron_ldl(H_O), bakron_ldl(H_I), bakron_round(W*, L_O, L_I, scales, bits),
     bakron_proxy_loss(W* - W, H_O, H_I).
 --hessian adds the two damped Kronecker factors to the step: bakron_damped_gram builds H_I from
 the layer's token matrix X and H_O from its gradient rows G (resident in HBM) before the solve.
+--group-size G / --codebook normal time bakron_round_ex: one grid step per row and group of G
+columns (max |W*| over the group / the grid's top), and/or the 2^bits-entry codebook of normal
+quantiles (k + 1/2) / 2^bits scaled to [-1, 1].
 --rounding stochastic times bakron_round_stochastic (stochastic Q, a fixed seed per step) in
 place of bakron_round. Metric: quantized weights per second, m*n / step time (whole job: summed over replicas, one
 independent layer per GPU, no collective on the data path; timed as the max over ranks).
@@ -105,6 +109,15 @@ def _dist():
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     return ws, rank, local
+
+
+def normal_codebook(bits: int):
+    """2^bits normal quantiles at (k + 1/2) / 2^bits, scaled to [-1, 1] (fp32)."""
+    import numpy as np
+    from statistics import NormalDist
+    K = 1 << bits
+    q = np.array([NormalDist().inv_cdf((k + 0.5) / K) for k in range(K)])
+    return (q / np.abs(q).max()).astype(np.float32)
 
 
 def max_over_ranks(x: float, device) -> float:
@@ -238,6 +251,20 @@ def run(args):
     names = (["gram_I", "gram_O"] if args.hessian else []) + ["ldl_O", "ldl_I", "round", "loss"]
 
     seed = 0x5EED if args.rounding == "stochastic" else None
+    quant = {}
+    s_in = s_np          # the grid steps the step reads (per row, or per row and group)
+    if args.group_size or args.codebook:
+        if seed is not None:
+            raise SystemExit("stochastic Q takes the per-row integer grid")
+        gs = min(args.group_size or n, n)
+        book = normal_codebook(bits) if args.codebook == "normal" else None
+        top = 1.0 if book is not None else (1 << (bits - 1)) - 0.5
+        G = (n + gs - 1) // gs
+        sg = np.stack([np.abs(Ws_np[:, g * gs:(g + 1) * gs]).max(axis=1) for g in range(G)],
+                      axis=1) / np.float32(top)
+        s_in = np.ascontiguousarray(sg, dtype=np.float32)
+        sc = torch.from_numpy(s_in).to(dev)
+        quant = {"group_size": gs, "codebook": book}
 
     def factors(X, G, timing):
         # H_I from the tokens, H_O from the gradient rows, into the buffers the solve reads
@@ -255,7 +282,7 @@ def run(args):
         timing = None if evs is None else dict(zip(names, evs))
         if samples is not None:
             factors(samples[0][0], samples[0][1], timing)
-        solver.run(Ws, HO, HI, sc, bits, stream, timing=timing, seed=seed)
+        solver.run(Ws, HO, HI, sc, bits, stream, timing=timing, seed=seed, **quant)
 
     for _ in range(args.warmup):
         step()
@@ -291,15 +318,15 @@ def run(args):
     e2e = None
     if not args.no_e2e:
         e2e = _e2e(args, torch, bk, solver, stream, dev, ws, m, n, bits, Ws, HO, HI, sc,
-                   Ws_np, HO_np, HI_np, s_np, seed,
-                   (samples[1], samples[0], factors) if samples is not None else None)
+                   Ws_np, HO_np, HI_np, s_in, seed,
+                   (samples[1], samples[0], factors) if samples is not None else None, quant)
     return _report(args, torch, bk, wl, ws, rank, m, n, bits, per, ms_step, value, launches,
                    clk, e2e, None if samples is not None else (Ws_np, HO_np, HI_np, s_np, bits),
                    samples[2] if samples is not None else None)
 
 
 def _e2e(args, torch, bk, solver, stream, dev, ws, m, n, bits, Ws, HO, HI, sc,
-         Ws_np, HO_np, HI_np, s_np, seed, hess=None):
+         Ws_np, HO_np, HI_np, s_np, seed, hess=None, quant=None):
     """Same metric through the public API with host buffers: pinned host -> device copies of
     the step's inputs (W*, the scales and either H_O, H_I or, with --hessian, the samples X and
     G), the whole path, device -> host copies of the codes and the loss."""
@@ -324,10 +351,10 @@ def _e2e(args, torch, bk, solver, stream, dev, ws, m, n, bits, Ws, HO, HI, sc,
         for d_, h_ in zip(d_in, h_in):
             d_.copy_(h_, non_blocking=True)
         if hess is None:
-            solver.run(dW2, d_in[0], d_in[1], ds2, bits, stream, seed=seed)
+            solver.run(dW2, d_in[0], d_in[1], ds2, bits, stream, seed=seed, **(quant or {}))
         else:
             factors(d_in[0], d_in[1], None)
-            solver.run(dW2, HO, HI, ds2, bits, stream, seed=seed)
+            solver.run(dW2, HO, HI, ds2, bits, stream, seed=seed, **(quant or {}))
         hcodes.copy_(solver.codes, non_blocking=True)
         hloss.copy_(solver.loss, non_blocking=True)
 
@@ -403,6 +430,8 @@ def _report(args, torch, bk, wl, ws, rank, m, n, bits, per, ms_step, value, laun
                 "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
                 "config": {"workload": wl.name, "m": m, "n": n, "bits": bits,
                            "rounding": args.rounding, "hessian": bool(args.hessian),
+                           "group_size": args.group_size or None,
+                           "codebook": args.codebook,
                            "parallelism": f"replicas x{ws}" if ws > 1 else "single",
                            "l2": "inputs larger than L2 (H_I alone is "
                                  f"{4 * n * n / 2**20:.0f} MiB), no flush"},
@@ -429,6 +458,8 @@ def main():
     ap.add_argument("--ref-seconds", type=float, default=12.0)
     ap.add_argument("--rounding", default="nearest", choices=["nearest", "stochastic"])
     ap.add_argument("--hessian", action="store_true")
+    ap.add_argument("--group-size", type=int, default=0)
+    ap.add_argument("--codebook", default=None, choices=["normal"])
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)

@@ -139,6 +139,34 @@ int bakron_round_stochastic(const float* Wstar, int m, int n, const float* L_O,
                             void* stream);
 
 /* ------------------------------------------------------------------------------------------
+ * bakron_round_ex -- bakron_round with the base quantizer chosen by the caller (the BaKron
+ * page, summary: the solver is modular in the base quantizer): per-group grid steps and/or a
+ * sorted scalar codebook. The rule and its order are those of bakron_round; only Q changes:
+ *
+ *   s_ij   = scales[i * G + j / group_size],   G = ceil(n / group_size)
+ *   without a codebook: code_ij = clamp(round_half_even(pre_ij / s_ij)), W_ij = s_ij code_ij
+ *   with a codebook c_0 < ... < c_{K-1}, K = 2^bits:
+ *            code_ij = the index k of the entry nearest to x = pre_ij / s_ij, decided against
+ *                      the fp32 midpoints fl32((c_k + c_{k+1}) / 2) (a tie goes to the lower
+ *                      entry; x is the correctly rounded fp32 quotient),
+ *            W_ij    = s_ij c_k.
+ *
+ *   scales   [in]  m x G grid steps (device), s_ij >= 0 (0: code 0 and W 0 on that row part;
+ *                  with a codebook, code 0 is the index of c_0 and W is still 0).
+ *   group_size [in] columns per grid step: a multiple of 32, or >= n (one step per row, the
+ *                  layout of bakron_round).
+ *   codebook [in]  HOST pointer to 2^bits finite, strictly increasing fp32 entries, copied
+ *                  during the call; NULL selects the integer grid.
+ *   bits     [in]  1..4 with a codebook (codes are entry indices 0 .. 2^bits - 1), else 2..8.
+ * Every other argument, the workspace (bakron_round_workspace_bytes) and the error behaviour
+ * are those of bakron_round; an invalid group_size or codebook returns BAKRON_ERR_INVALID_ARG.
+ * ---------------------------------------------------------------------------------------- */
+int bakron_round_ex(const float* Wstar, int m, int n, const float* L_O, const float* L_I,
+                    const float* scales, int group_size, const float* codebook, int bits,
+                    int8_t* codes, float* W, void* ws, size_t ws_bytes, int* dev_status,
+                    void* stream);
+
+/* ------------------------------------------------------------------------------------------
  * bakron_proxy_loss -- tr(H_O dW H_I dW^T) = vec(dW)^T (H_O (x) H_I) vec(dW).
  *
  * The layer proxy of the YAQA article (section 4 error bound, section 2 second-order

@@ -1,12 +1,12 @@
 """Python binding of libbakron.so (ctypes): argument marshalling only.
 
 The functions named like the C ABI (``bakron_ldl``, ``bakron_round``,
-``bakron_round_stochastic``, ``bakron_proxy_loss``, ``bakron_damped_gram``, ``bakron_sketch_b``,
-``bakron_read_status``, ``bakron_status_string`` and the ``*_workspace_bytes`` queries) take
-torch CUDA tensors, pass their device pointers and the current CUDA stream to the library and
-return its status code. ``ldl``, ``round_weights``, ``proxy_loss``, ``damped_gram``,
-``sketch_b`` and ``solve`` additionally allocate outputs and workspaces with torch and raise on
-any error.
+``bakron_round_stochastic``, ``bakron_round_ex``, ``bakron_proxy_loss``, ``bakron_damped_gram``,
+``bakron_sketch_b``, ``bakron_read_status``, ``bakron_status_string`` and the
+``*_workspace_bytes`` queries) take torch CUDA tensors, pass their device pointers and the
+current CUDA stream to the library and return its status code. ``ldl``, ``round_weights``,
+``proxy_loss``, ``damped_gram``, ``sketch_b`` and ``solve`` additionally allocate outputs and
+workspaces with torch and raise on any error.
 
 Every step of the computation runs in the library's CUDA kernels; there is no CPU path. If
 the shared library is missing the first call raises.
@@ -41,6 +41,8 @@ _SIGNATURES = {
                               _c_size_t, _vp, _vp]),
     "bakron_round_stochastic": (_c_int, [_vp, _c_int, _c_int, _vp, _vp, _vp, _c_int,
                                          ctypes.c_uint64, _vp, _vp, _vp, _c_size_t, _vp, _vp]),
+    "bakron_round_ex": (_c_int, [_vp, _c_int, _c_int, _vp, _vp, _vp, _c_int, _vp, _c_int, _vp,
+                                 _vp, _vp, _c_size_t, _vp, _vp]),
     "bakron_proxy_loss_workspace_bytes": (_c_size_t, [_c_int, _c_int]),
     "bakron_proxy_loss": (_c_int, [_vp, _c_int, _c_int, _vp, _vp, _vp, _vp, _c_size_t, _vp]),
     "bakron_damped_gram_workspace_bytes": (_c_size_t, [_c_int, _c_int]),
@@ -171,6 +173,28 @@ def bakron_round_stochastic(Wstar, L_O, L_I, scales, bits, seed, codes, W, ws, d
                                          _ptr(dev_status), _stream(stream))
 
 
+def bakron_round_ex(Wstar, L_O, L_I, scales, group_size, codebook, bits, codes, W, ws,
+                    dev_status, stream=None) -> int:
+    """``scales``: m x G device tensor (G = ceil(n / group_size)); ``codebook``: None or a
+    host sequence of 2^bits increasing floats (copied by the call)."""
+    m, n = Wstar.shape
+    _check_cuda(Wstar, torch.float32, (m, n), "Wstar")
+    _check_cuda(L_O, torch.float32, (m, m), "L_O")
+    _check_cuda(L_I, torch.float32, (n, n), "L_I")
+    gs = min(int(group_size), n)
+    _check_cuda(scales, torch.float32, (m, (n + gs - 1) // gs), "scales")
+    _check_cuda(codes, torch.int8, (m, n), "codes")
+    _check_cuda(W, torch.float32, (m, n), "W")
+    cb = None
+    if codebook is not None:
+        vals = [float(v) for v in codebook]
+        cb = (ctypes.c_float * len(vals))(*vals)
+    return lib().bakron_round_ex(_ptr(Wstar), m, n, _ptr(L_O), _ptr(L_I), _ptr(scales),
+                                 int(group_size), cb, int(bits), _ptr(codes), _ptr(W), _ptr(ws),
+                                 ws.numel() * ws.element_size(), _ptr(dev_status),
+                                 _stream(stream))
+
+
 def bakron_proxy_loss(dW, H_O, H_I, loss, ws, stream=None) -> int:
     m, n = dW.shape
     _check_cuda(dW, torch.float32, (m, n), "dW")
@@ -287,14 +311,21 @@ def ldl(H: torch.Tensor, stream=None, check: bool = True):
     return L, D
 
 
-def round_weights(Wstar, L_O, L_I, scales, bits, stream=None, check: bool = True, seed=None):
-    """(codes int8, W fp32) of the BaKron solve; a seed selects stochastic Q."""
+def round_weights(Wstar, L_O, L_I, scales, bits, stream=None, check: bool = True, seed=None,
+                  group_size=None, codebook=None):
+    """(codes int8, W fp32) of the BaKron solve; a seed selects stochastic Q, a group size
+    (with m x G scales) and/or a host codebook select the base quantizer of bakron_round_ex."""
     m, n = Wstar.shape
     codes = torch.empty((m, n), dtype=torch.int8, device=Wstar.device)
     W = torch.empty((m, n), dtype=torch.float32, device=Wstar.device)
     ws = workspace(bakron_round_workspace_bytes(m, n), Wstar.device)
     st = new_status(Wstar.device)
-    if seed is None:
+    if group_size is not None or codebook is not None:
+        if seed is not None:
+            raise ValueError("stochastic Q takes the per-row integer grid")
+        _raise(bakron_round_ex(Wstar, L_O, L_I, scales, n if group_size is None else group_size,
+                               codebook, bits, codes, W, ws, st, stream), "bakron_round_ex")
+    elif seed is None:
         _raise(bakron_round(Wstar, L_O, L_I, scales, bits, codes, W, ws, st, stream),
                "bakron_round")
     else:
@@ -369,9 +400,10 @@ class Solver:
         self._join = torch.cuda.Event()
 
     def run(self, Wstar, H_O, H_I, scales, bits, stream=None, with_loss=True, timing=None,
-            seed=None):
+            seed=None, group_size=None, codebook=None):
         """Enqueues the whole path (reads: self.codes, self.W, self.E, self.loss); a seed
-        selects stochastic Q for the round.
+        selects stochastic Q for the round, a group size (with m x G scales) and/or a host
+        codebook the base quantizer of bakron_round_ex.
 
         timing: optional {name: (start_event, end_event)} for any of "ldl_O", "ldl_I", "round",
         "loss"; each pair is recorded around its call on the stream that runs it.
@@ -394,7 +426,11 @@ class Solver:
         call("ldl_I", stream, bakron_ldl, H_I, self.L_I, self.D_I, self.ws, self.status)
         self._join.record(self.side)
         stream.wait_event(self._join)
-        if seed is None:
+        if group_size is not None or codebook is not None:
+            call("round", stream, bakron_round_ex, Wstar, self.L_O, self.L_I, scales,
+                 self.n if group_size is None else group_size, codebook, bits, self.codes,
+                 self.W, self.ws_round, self.status)
+        elif seed is None:
             call("round", stream, bakron_round, Wstar, self.L_O, self.L_I, scales, bits,
                  self.codes, self.W, self.ws_round, self.status)
         else:

@@ -38,6 +38,7 @@
 #include <algorithm>
 #include <cstddef>
 #include <cstring>
+#include <limits>
 
 #include "philox.cuh"
 #include "round_leaf.cuh"
@@ -50,6 +51,8 @@ using leaf::LB;
 using leaf::LeafBuf;
 using leaf::LS;
 using leaf::LeafXchg;
+using leaf::QKind;
+using leaf::kMaxCodebook;
 using leaf::solve_leaf_chain;
 using leaf::solve_leaf_pushes;
 
@@ -97,6 +100,11 @@ struct FusedArgs {
     uint64_t limit_ns;
     int stoch;           // 1: stochastic Q with the variates of `seed`
     unsigned long long seed;
+    int n_groups;        // grid steps per row (scales is m x n_groups)
+    int group_size;      // columns per grid step: a multiple of the leaf width, or n
+    int ncb;             // codebook entries (0: the integer grid)
+    float cb[kMaxCodebook];       // the sorted codebook, last entry repeated
+    float cbmid[kMaxCodebook];    // fl32((c_k + c_{k+1}) / 2), +inf past the last threshold
 };
 
 // 32 x 32 fp32 box maps (no swizzle) of the matrices a leaf reads; only valid when m and n are
@@ -129,6 +137,7 @@ struct alignas(128) LeafGroupSmem {
 };
 struct LeafCtaSmem {
     LeafGroupSmem g[2];
+    float qcb[kMaxCodebook];     // the codebook (read with a per-lane index)
 };
 static_assert(sizeof(LeafGroupSmem) % 128 == 0 && offsetof(LeafGroupSmem, buf) % 128 == 0 &&
                   offsetof(LeafGroupSmem, ring) % 128 == 0,
@@ -167,9 +176,10 @@ __device__ __forceinline__ void group_sync(int g) {
     asm volatile("bar.sync %0, %1;" ::"r"(1 + g), "n"(NLOAD) : "memory");
 }
 
-// Codes and W of the leaf solved from B (W = s_r q, formed as in the solver); run by the
-// group's loader threads before they restage B.
-__device__ __forceinline__ void publish_rest(const FusedArgs& a, const LeafBuf& B, int lt) {
+// Codes and W of the leaf solved from B (W = s_r q, or s_r c_q with a codebook, formed as in
+// the solver); run by the group's loader threads before they restage B.
+__device__ __forceinline__ void publish_rest(const FusedArgs& a, const LeafBuf& B, int lt,
+                                             const float* qcb) {
     const int I = B.meta[0], J = B.meta[1], rows = B.meta[2], cols = B.meta[3];
     const int i0 = I * LB, j0 = J * LB;
 #pragma unroll 4
@@ -179,7 +189,7 @@ __device__ __forceinline__ void publish_rest(const FusedArgs& a, const LeafBuf& 
             const size_t o = (size_t)(i0 + r) * a.n + j0 + c;
             const int q = B.oC[r * LB + c];
             a.codes[o] = (int8_t)q;
-            a.Wq[o] = B.S[r] * (float)q;
+            a.Wq[o] = B.S[r] * (a.ncb > 0 ? qcb[q] : (float)q);
         }
     }
 }
@@ -259,7 +269,7 @@ struct NearField {
 // near-field contributions (one 32 x 32 x 32 product per source on CUDA cores). With box
 // loads, one thread keeps NRING sources in flight through a ring of shared-memory stages.
 __device__ void leaf_loaders(const FusedArgs& a, const LeafMaps* maps, LeafGroupSmem& sm, int g,
-                             int lw, int lane, int slot, int nslots) {
+                             int lw, int lane, int slot, int nslots, const float* qcb) {
     const int lt = lw * 32 + lane;
     const bool lead = lt == 0;
     const int m = a.m, n = a.n;
@@ -282,7 +292,7 @@ __device__ void leaf_loaders(const FusedArgs& a, const LeafMaps* maps, LeafGroup
             }
             group_sync(g);
             if (*(volatile int*)&sm.stop) break;
-            publish_rest(a, B, lt);   // leaf k - 2, solved from this buffer
+            publish_rest(a, B, lt, qcb);   // leaf k - 2, solved from this buffer
             group_sync(g);            // its meta is read before it is overwritten
         }
         int I, J;
@@ -317,7 +327,9 @@ __device__ void leaf_loaders(const FusedArgs& a, const LeafMaps* maps, LeafGroup
             dld = LB;
         }
         if (lt < LB) {
-            const float sv = (lt < rows) ? __ldg(&a.sc[i0 + lt]) : 0.f;
+            // the leaf's grid step: per row, or per row and column group (one group per leaf)
+            const float sv = (lt < rows)
+                ? __ldg(&a.sc[(size_t)(i0 + lt) * a.n_groups + j0 / a.group_size]) : 0.f;
             B.S[lt] = sv;
             B.S[LB + lt] = sv > 0.f ? __frcp_rn(sv) : 0.f;
         }
@@ -576,14 +588,14 @@ __device__ void leaf_loaders(const FusedArgs& a, const LeafMaps* maps, LeafGroup
             }
             group_sync(g);
             if (*(volatile int*)&sm.stop) break;
-            publish_rest(a, sm.buf[b], lt);
+            publish_rest(a, sm.buf[b], lt, qcb);
         }
     }
 }
 
 // ------------------------------------------------------------------------------ leaf solver
 __device__ void leaf_solver(const FusedArgs& a, LeafGroupSmem& sm, int lane, int slot,
-                            int nslots, int bar) {
+                            int nslots, int bar, const float* qcb) {
     const int n = a.n;
     const long long total = (long long)a.Mt * a.Nt;
     int k = 0;
@@ -603,8 +615,15 @@ __device__ void leaf_solver(const FusedArgs& a, LeafGroupSmem& sm, int lane, int
         }
         const int I = B.meta[0], J = B.meta[1], rows = B.meta[2], cols = B.meta[3];
         const int i0 = I * LB, j0 = J * LB;
-        if (a.stoch) solve_leaf_chain<true>(lane, rows, cols, a.qlo, a.qhi, B, sm.xch, bar, a.status);
-        else solve_leaf_chain<false>(lane, rows, cols, a.qlo, a.qhi, B, sm.xch, bar, a.status);
+        if (a.ncb > 0)
+            solve_leaf_chain<QKind::kCodebook>(lane, rows, cols, a.qlo, a.qhi, B, sm.xch, bar,
+                                               a.status, qcb, a.cbmid);
+        else if (a.stoch)
+            solve_leaf_chain<QKind::kStochastic>(lane, rows, cols, a.qlo, a.qhi, B, sm.xch, bar,
+                                                 a.status);
+        else
+            solve_leaf_chain<QKind::kNearest>(lane, rows, cols, a.qlo, a.qhi, B, sm.xch, bar,
+                                              a.status);
         __syncwarp();
         if (lane == 0) sm100::mbar_arrive(&sm.solved[b]);
         // what the next leaves read: E (vertical pulls, lane = column) and U^T (horizontal pulls,
@@ -682,6 +701,7 @@ __device__ void leaf_role(const FusedArgs& a, const LeafMaps* maps, uint8_t* sme
         }
         sm100::fence_mbar_init();
     }
+    if (threadIdx.x < kMaxCodebook) cs.qcb[threadIdx.x] = a.cb[threadIdx.x];
     __syncthreads();
     // warp w runs on SM sub-partition w % 4. Group g: helper warp g, solver warp 2 + g, loader
     // warps 4 + g and 6 + g, so the solver and its helper issue from different
@@ -690,8 +710,8 @@ __device__ void leaf_role(const FusedArgs& a, const LeafMaps* maps, uint8_t* sme
     const int g = warp & 1;
     const int slot = blockIdx.x * 2 + g, nslots = a.leaf_ctas * 2;
     if (warp < 2) leaf_helper(a, cs.g[g], lane, slot, nslots, 3 + g);
-    else if (warp < 4) leaf_solver(a, cs.g[g], lane, slot, nslots, 3 + g);
-    else leaf_loaders(a, maps, cs.g[g], g, (warp - 4) >> 1, lane, slot, nslots);
+    else if (warp < 4) leaf_solver(a, cs.g[g], lane, slot, nslots, 3 + g, cs.qcb);
+    else leaf_loaders(a, maps, cs.g[g], g, (warp - 4) >> 1, lane, slot, nslots, cs.qcb);
 }
 
 // ------------------------------------------------------------------------------ push tasks
@@ -1037,12 +1057,40 @@ extern "C" size_t bakron_round_workspace_bytes(int m, int n) {
 
 namespace {
 
+// The base quantizer of one call: the grid-step layout and the optional codebook.
+struct QuantSpec {
+    int group_size;              // columns per grid step (>= n: one per row)
+    const float* codebook;       // host, 2^bits sorted entries, or nullptr (integer grid)
+};
+
 int round_impl(const float* Wstar, int m, int n, const float* L_O, const float* L_I,
-               const float* scales, int bits, int stoch, unsigned long long seed, int8_t* codes,
-               float* W, void* ws, size_t ws_bytes, int* dev_status, void* stream) {
-    if (m < 1 || n < 1 || (long long)m * n >= (1LL << 31) || bits < 2 || bits > 8 ||
-        !Wstar || !L_O || !L_I || !scales || !codes || !W || !dev_status)
+               const float* scales, int bits, int stoch, unsigned long long seed,
+               QuantSpec qs, int8_t* codes, float* W, void* ws, size_t ws_bytes,
+               int* dev_status, void* stream) {
+    if (m < 1 || n < 1 || (long long)m * n >= (1LL << 31) || !Wstar || !L_O || !L_I ||
+        !scales || !codes || !W || !dev_status)
         return BAKRON_ERR_INVALID_ARG;
+    if (qs.codebook ? (bits < 1 || bits > 4 || stoch) : (bits < 2 || bits > 8))
+        return BAKRON_ERR_INVALID_ARG;
+    if (qs.group_size < 1 || (qs.group_size < n && qs.group_size % LB != 0))
+        return BAKRON_ERR_INVALID_ARG;
+    const int group_size = std::min(qs.group_size, n);
+    const int n_groups = (n + group_size - 1) / group_size;
+    int ncb = 0;
+    float cb[kMaxCodebook], cbmid[kMaxCodebook];
+    if (qs.codebook) {
+        ncb = 1 << bits;
+        for (int k = 0; k < ncb; ++k) {
+            const float c = qs.codebook[k];
+            if (!(c > -3.0e38f && c < 3.0e38f) || (k > 0 && !(c > qs.codebook[k - 1])))
+                return BAKRON_ERR_INVALID_ARG;   // non-finite or not strictly increasing
+        }
+    }
+    for (int k = 0; k < kMaxCodebook; ++k) {
+        cb[k] = ncb ? qs.codebook[std::min(k, ncb - 1)] : 0.f;
+        const float sum = (k + 1 < ncb) ? qs.codebook[k] + qs.codebook[k + 1] : 0.f;
+        cbmid[k] = (k + 1 < ncb) ? sum * 0.5f : std::numeric_limits<float>::infinity();
+    }
     if (!ws_ok(ws, ws_bytes, bakron_round_workspace_bytes(m, n))) return BAKRON_ERR_WORKSPACE;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const Layout L = layout(m, n);
@@ -1103,6 +1151,13 @@ int round_impl(const float* Wstar, int m, int n, const float* L_O, const float* 
     a.limit_ns = spin_limit_ns();
     a.stoch = stoch;
     a.seed = seed;
+    a.n_groups = n_groups;
+    a.group_size = group_size;
+    a.ncb = ncb;
+    for (int k = 0; k < kMaxCodebook; ++k) {
+        a.cb[k] = cb[k];
+        a.cbmid[k] = cbmid[k];
+    }
 
     // box loads for the leaves when every row stride is a multiple of 16 bytes
     LeafMaps lm;
@@ -1144,14 +1199,23 @@ int round_impl(const float* Wstar, int m, int n, const float* L_O, const float* 
 extern "C" int bakron_round(const float* Wstar, int m, int n, const float* L_O, const float* L_I,
                             const float* scales, int bits, int8_t* codes, float* W, void* ws,
                             size_t ws_bytes, int* dev_status, void* stream) {
-    return round_impl(Wstar, m, n, L_O, L_I, scales, bits, 0, 0ull, codes, W, ws, ws_bytes,
-                      dev_status, stream);
+    return round_impl(Wstar, m, n, L_O, L_I, scales, bits, 0, 0ull, QuantSpec{n, nullptr},
+                      codes, W, ws, ws_bytes, dev_status, stream);
+}
+
+extern "C" int bakron_round_ex(const float* Wstar, int m, int n, const float* L_O,
+                               const float* L_I, const float* scales, int group_size,
+                               const float* codebook, int bits, int8_t* codes, float* W,
+                               void* ws, size_t ws_bytes, int* dev_status, void* stream) {
+    return round_impl(Wstar, m, n, L_O, L_I, scales, bits, 0, 0ull,
+                      QuantSpec{group_size, codebook}, codes, W, ws, ws_bytes, dev_status,
+                      stream);
 }
 
 extern "C" int bakron_round_stochastic(const float* Wstar, int m, int n, const float* L_O,
                                        const float* L_I, const float* scales, int bits,
                                        uint64_t seed, int8_t* codes, float* W, void* ws,
                                        size_t ws_bytes, int* dev_status, void* stream) {
-    return round_impl(Wstar, m, n, L_O, L_I, scales, bits, 1, (unsigned long long)seed, codes,
-                      W, ws, ws_bytes, dev_status, stream);
+    return round_impl(Wstar, m, n, L_O, L_I, scales, bits, 1, (unsigned long long)seed,
+                      QuantSpec{n, nullptr}, codes, W, ws, ws_bytes, dev_status, stream);
 }

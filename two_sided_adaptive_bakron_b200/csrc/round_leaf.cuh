@@ -4,7 +4,10 @@
 //   pre_ij = W*_ij + T_ij + R_ij,  T_ij = sum_{k<i} L_O[k,i] E_kj,  R_ij = sum_{l<j} U_il L_I[l,j],
 //   W_ij = s_i clamp(rint(pre_ij / s_i)),  E_ij = W*_ij - W_ij,  U_ij = T_ij + E_ij,
 // or, with stochastic Q (the same section's alternative),
-//   W_ij = s_i clamp(floor(pre_ij / s_i + u_ij)),  u_ij uniform on (0, 1).
+//   W_ij = s_i clamp(floor(pre_ij / s_i + u_ij)),  u_ij uniform on (0, 1),
+// or, with a scalar codebook c_0 < ... < c_{K-1} (the BaKron page, summary: the solver is
+// modular in the base quantizer), W_ij = s_ij c_k for the entry k nearest to pre_ij / s_ij.
+// The grid step s may be per row or per row and column group (one group per leaf).
 // T and R arrive holding everything from outside the leaf; the wavefront adds the in-leaf part.
 #pragma once
 
@@ -59,7 +62,7 @@ static_assert(offsetof(LeafBuf, LOr) % 16 == 0 && offsetof(LeafBuf, LIc) % 16 ==
 // Q divides by s_r as one correctly rounded fp32 division: the quotient is formed as
 // pre * (1/s_r), whose distance to the division's result is below 2e-7 |x|, and the exact
 // division is taken instead whenever that quotient lies within 1e-6 max(1,|x|) of a rounding
-// boundary, so the decision always equals the division's. Stochastic Q (kStoch) decides on
+// boundary, so the decision always equals the division's. Stochastic Q (kStochastic) decides on
 // y = x + u (one fp32 addition) with floor: its boundaries are the integers, and the exact
 // division is taken whenever y lies within 1e-6 max(1,|y|) of one; the two y differ by at most
 // 2e-7 |x| + 2^-24 (|y| + |y'|) <= 5.2e-7 max(1,|y|) since |x| <= |y| + 1, so outside that
@@ -71,6 +74,10 @@ static_assert(offsetof(LeafBuf, LOr) % 16 == 0 && offsetof(LeafBuf, LIc) % 16 ==
 // (everything from steps <= rho - 2 on top of T, R) plus its own distance-1 terms of step
 // rho - 1; the helper pushes step rho - 1 and publishes slot rho + 1. One named barrier of the
 // two warps closes each round.
+// The base quantizer of the wavefront.
+enum class QKind { kNearest, kStochastic, kCodebook };
+constexpr int kMaxCodebook = 16;
+
 struct LeafXchg {
     float part[2][2][LB];        // [slot & 1][T, R][lane]: the helper's partial sums
     float eu[2][2][LB];          // [step & 1][e, u][lane]: the solver's step results
@@ -80,15 +87,25 @@ __device__ __forceinline__ void pair_sync(int id) {
     asm volatile("bar.sync %0, 64;" ::"r"(id) : "memory");
 }
 
-template <bool kStoch>
+// Codebook Q: cb (shared memory) holds the entries, mid (any memory, read once per leaf) the
+// decision thresholds fl32((c_k + c_{k+1}) / 2), +inf past the last one; the code is the number
+// of thresholds below x (a tie goes to the lower entry), found by independent compares that
+// also give the distance to the nearest threshold for the exact-division guard.
+template <QKind kQ>
 __device__ __forceinline__ void solve_leaf_chain(int lane, int rows, int cols, float qlo,
                                                  float qhi, LeafBuf& B, LeafXchg& X, int bar,
-                                                 int* status) {
+                                                 int* status, const float* cb = nullptr,
+                                                 const float* mid = nullptr) {
     const int j = lane;
     const bool colok = j < cols;
     const float li1 = B.LIc[j * LS + 1];
     float lo1p = 0.f, ep = 0.f, usp = 0.f;   // distance-1 terms of the previous step
     bool bad = false;
+    float md[kMaxCodebook - 1];
+    if constexpr (kQ == QKind::kCodebook) {
+#pragma unroll
+        for (int t = 0; t < kMaxCodebook - 1; ++t) md[t] = mid[t];
+    }
     pair_sync(bar);                          // the helper's slots 0 and 1 are in place
 #pragma unroll 1
     for (int s = 0; s < NSLOT; ++s) {
@@ -104,23 +121,42 @@ __device__ __forceinline__ void solve_leaf_chain(int lane, int rows, int cols, f
         float e = 0.f, u = 0.f;
         if (act) {
             const float pre = w_star + tT + tR;
-            float q = 0.f;
+            float q = 0.f, qv = 0.f;         // the code and its grid value
             if (sr > 0.f) {
-                if constexpr (kStoch) {
+                if constexpr (kQ == QKind::kCodebook) {
+                    float x = pre * inv;
+                    int k = 0;
+                    float dmin = __int_as_float(0x7f800000);
+#pragma unroll
+                    for (int t = 0; t < kMaxCodebook - 1; ++t) {
+                        k += (x > md[t]) ? 1 : 0;
+                        dmin = fminf(dmin, fabsf(x - md[t]));
+                    }
+                    if (dmin < 1e-6f * fmaxf(1.f, fabsf(x))) {
+                        x = __fdiv_rn(pre, sr);
+                        k = 0;
+#pragma unroll
+                        for (int t = 0; t < kMaxCodebook - 1; ++t) k += (x > md[t]) ? 1 : 0;
+                    }
+                    q = (float)k;
+                    qv = cb[k];
+                } else if constexpr (kQ == QKind::kStochastic) {
                     const float uv = ((float)(uint16_t)B.oC[rr * LB + j] + 0.5f) * (1.f / 65536.f);
                     float y = __fadd_rn(__fmul_rn(pre, inv), uv);
                     const float t = fabsf(y - rintf(y));
                     if (t < 1e-6f * fmaxf(1.f, fabsf(y))) y = __fadd_rn(__fdiv_rn(pre, sr), uv);
                     q = fminf(fmaxf(floorf(y), qlo), qhi);
+                    qv = q;
                 } else {
                     float x = pre * inv;
                     const float t = fabsf(x - rintf(x));
                     if (0.5f - t < 1e-6f * fmaxf(1.f, fabsf(x))) x = __fdiv_rn(pre, sr);
                     q = fminf(fmaxf(rintf(x), qlo), qhi);
+                    qv = q;
                 }
             }
             bad |= !isfinite(pre);
-            const float w = sr * q;
+            const float w = sr * qv;
             e = w_star - w;
             u = tT + e;
             B.oC[rr * LB + j] = (int16_t)q;
