@@ -57,3 +57,45 @@ def test_invalid_arguments_rejected_on_host(libpath):
     lib.bakron_ldl.restype = ctypes.c_int
     lib.bakron_ldl.argtypes = [vp, ctypes.c_int, vp, vp, vp, ctypes.c_size_t, vp, vp]
     assert lib.bakron_ldl(fake, 0, fake, fake, fake, 1 << 20, fake, None) == -1
+
+
+def test_new_entry_points_reject_bad_arguments_on_host(libpath):
+    """Argument checks of the stochastic, quantizer and Kronecker-factor entry points return
+    before any device work (no GPU needed)."""
+    lib = ctypes.CDLL(libpath)
+    vp, ci, cf = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+    fake, big = vp(0x1000), 1 << 30
+    lib.bakron_round_stochastic.restype = ci
+    lib.bakron_round_stochastic.argtypes = [vp, ci, ci, vp, vp, vp, ci, ctypes.c_uint64, vp, vp,
+                                            vp, ctypes.c_size_t, vp, vp]
+    assert lib.bakron_round_stochastic(fake, 4, 4, fake, fake, fake, 9, 1, fake, fake, fake, big,
+                                       fake, None) == -1
+    lib.bakron_round_ex.restype = ci
+    lib.bakron_round_ex.argtypes = [vp, ci, ci, vp, vp, vp, ci, vp, ci, vp, vp, vp,
+                                    ctypes.c_size_t, vp, vp]
+
+    def ex(n, group, book, bits, ws_bytes=big):
+        cb = None if book is None else (cf * len(book))(*book)
+        return lib.bakron_round_ex(fake, 8, n, fake, fake, fake, group, cb, bits, fake, fake,
+                                   fake, ws_bytes, fake, None)
+    assert ex(64, 48, None, 3) == -1                       # group not a multiple of 32
+    assert ex(64, 0, None, 3) == -1
+    assert ex(64, 32, [0.0, 2.0, 1.0, 3.0], 2) == -1       # not increasing
+    assert ex(64, 32, [0.0, 0.0, 1.0, 3.0], 2) == -1       # not strictly increasing
+    assert ex(64, 32, [0.0, 1.0, float("nan"), 3.0], 2) == -1
+    assert ex(64, 32, [float(k) for k in range(32)], 5) == -1   # more than 16 entries
+    assert ex(64, 32, None, 9) == -1
+    assert ex(64, 32, [0.0, 1.0], 1, ws_bytes=16) == -5    # valid: then the tiny workspace fails
+    lib.bakron_damped_gram.restype = ci
+    lib.bakron_damped_gram.argtypes = [vp, ci, ci, cf, vp, vp, ctypes.c_size_t, vp, vp]
+    assert lib.bakron_damped_gram(fake, 0, 4, 0.01, fake, fake, big, fake, None) == -1
+    assert lib.bakron_damped_gram(fake, 4, 4, -0.5, fake, fake, big, fake, None) == -1
+    assert lib.bakron_damped_gram(fake, 4, 70000, 0.01, fake, fake, big, fake, None) == -1
+    assert lib.bakron_damped_gram(fake, 4, 4, 0.01, fake, vp(0x1001), big, fake, None) == -5
+    lib.bakron_sketch_b.restype = ci
+    lib.bakron_sketch_b.argtypes = [vp, ci, ci, ci, cf, vp, vp, vp, ctypes.c_size_t, vp, vp]
+    assert lib.bakron_sketch_b(fake, 0, 4, 4, 0.01, fake, fake, fake, big, fake, None) == -1
+    assert lib.bakron_sketch_b(fake, 2, 4, 4, 0.01, fake, fake, fake, 16, fake, None) == -5
+    lib.bakron_damped_gram_workspace_bytes.restype = ctypes.c_size_t
+    lib.bakron_damped_gram_workspace_bytes.argtypes = [ci, ci]
+    assert lib.bakron_damped_gram_workspace_bytes(1000, 300) >= 2 * 300 * 1000 * 4

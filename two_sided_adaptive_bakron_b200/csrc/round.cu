@@ -2,7 +2,8 @@
 //
 // What is computed (YAQA article, news.43b.com.cn/a/479517.html, section 4, rounding rule):
 //   pre_ij = W*_ij + a_i^T E[:i,:j] b_j + a_i^T E[:i,j] + E[i,:j] b_j,  E = W* - W,
-//   W_ij   = s_i * clamp(rint(pre_ij / s_i)).
+//   W_ij   = s_i * clamp(rint(pre_ij / s_i))
+// (or stochastic rounding, or a per-group grid step and a scalar codebook: round_leaf.cuh).
 // Entry (i,j) reads only entries (k,l) with k <= i, l <= j, so every anti-diagonal i+j = const
 // is independent (BaKron page, abstract: O(m+n) sequential steps, anti-diagonal parallelism
 // combined with a divide-and-conquer construction that brings the work to O(mn(m+n))).
@@ -15,14 +16,17 @@
 //
 // Structure: one persistent cooperative launch over the whole matrix, cut into 32 x 32 leaves
 // and 256 x 256 super-blocks, with two kinds of CTAs.
-//  * Leaf CTAs take the leaves in anti-diagonal order (round robin over two groups per CTA:
-//    two loader warps and one solver warp each). A leaf's sums come in two parts. The near
-//    field, the leaves above / to the left inside its own super-block and the adjacent one, is
-//    pulled by the loaders on CUDA cores after a bounded wait on each source leaf's flag. The
-//    far field, everything at least two super-blocks away, is read from T_far / R_far once the
-//    leaf's 128 x 128 tile counters say that every far source has been added. The solver warp
-//    runs the in-leaf wavefront (round_leaf.cuh), publishes E and U, releases the leaf's flag,
-//    then publishes the E^T planes and counts the leaf into its super-block.
+//  * Leaf CTAs take the leaves in anti-diagonal order (round robin over two groups per CTA,
+//    each with two loader warps, a solver warp and its helper warp). A leaf's sums come in two
+//    parts. The near field, the leaves above / to the left inside its own super-block and the
+//    adjacent one, is pulled by the loaders (one warp per direction, 32 x 32 x 32 products on
+//    the tensor cores from boxes brought in by TMA) after a bounded wait on each source leaf's
+//    flag; the source to the left is usually the group's previous leaf, read from shared
+//    memory. The far field, everything at least two super-blocks away, is read from T_far /
+//    R_far once the leaf's 128 x 128 tile counters say that every far source has been added.
+//    The solver and helper warps run the in-leaf wavefront (round_leaf.cuh); the solver then
+//    publishes E and U^T and releases the leaf's flag, the helper publishes the U and E^T
+//    planes and counts the leaf into its super-block, and the loaders copy out codes and W.
 //  * GEMM CTAs run the far-field pushes as 3xTF32 tcgen05 tile tasks (128 x 128, K = one
 //    super-block): E of super-block (A', C) into T_far of a target (A, C) with A >= A' + 2, and
 //    U of (A, C') into R_far of (A, C) with C >= C' + 2, i.e. the divide-and-conquer
