@@ -51,14 +51,64 @@ def _peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clock/throttle samples taken while the timed region runs."""
+    """SM clock and clock-event reasons sampled while the timed region runs (reads only).
+
+    NVML is read every 10 ms from a thread; without NVML, nvidia-smi samples every 100 ms,
+    and the timed region starts only after its first line, so a short region still gets
+    samples. Any failure leaves the summary empty; it never stops the benchmark.
+    """
+
+    PERIOD_S = 0.01
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown", 0x8),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown", 0x40),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown", 0x20),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap", 0x4))
 
     def __init__(self, index: int):
         self.index = index
+        self.source = None
         self.proc = None
         self.lines: list[str] = []
+        self.samples: list[tuple[float, int]] = []   # NVML: (SM MHz, reason bits)
+        self.max_mhz = None
+        self.mark = 0
 
     def __enter__(self):
+        if not self._start_nvml():
+            self._start_smi()
+        return self
+
+    def _start_nvml(self) -> bool:
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            reasons = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
+            pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)   # both reads work here
+            reasons(h)
+        except Exception:
+            return False
+        self.nvml, self.bits = pynvml, {nm: int(getattr(pynvml, attr, dflt))
+                                        for nm, attr, dflt in self.REASONS}
+        self.stop = threading.Event()
+
+        def loop():
+            while not self.stop.is_set():
+                try:
+                    self.samples.append((float(pynvml.nvmlDeviceGetClockInfo(
+                        h, pynvml.NVML_CLOCK_SM)), int(reasons(h))))
+                except Exception:
+                    pass
+                self.stop.wait(self.PERIOD_S)
+
+        self.t = threading.Thread(target=loop, daemon=True)
+        self.t.start()
+        self.source = "nvml"
+        return True
+
+    def _start_smi(self):
         q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -67,18 +117,30 @@ class ClockSampler:
                 ["nvidia-smi", f"--id={self.index}", f"--query-gpu={q}",
                  "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.t = threading.Thread(target=self._read, daemon=True)
-            self.t.start()
         except (OSError, FileNotFoundError):
             self.proc = None
-        return self
+            return
+        self.source = "nvidia-smi"
+        self.first = threading.Event()
+        self.t = threading.Thread(target=self._read, daemon=True)
+        self.t.start()
+        self.first.wait(3.0)            # the tool is up; samples from here on
+        self.mark = len(self.lines)
 
     def _read(self):
         for line in self.proc.stdout:
             self.lines.append(line.strip())
+            self.first.set()
 
     def __exit__(self, *exc):
-        if self.proc is not None:
+        if self.source == "nvml":
+            self.stop.set()
+            self.t.join(timeout=1.0)
+            try:
+                self.nvml.nvmlShutdown()
+            except Exception:
+                pass
+        elif self.proc is not None:
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
@@ -86,9 +148,13 @@ class ClockSampler:
                 self.proc.kill()
 
     def summary(self):
-        sm, mx, reasons = [], None, set()
+        sm, mx, reasons = [], self.max_mhz, set()
+        if self.source == "nvml":
+            for mhz, r in self.samples:
+                sm.append(mhz)
+                reasons.update(nm for nm, bit in self.bits.items() if r & bit)
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        for ln in self.lines[self.mark:]:
             parts = [p.strip() for p in ln.split(",")]
             if len(parts) < 9:
                 continue
@@ -101,7 +167,7 @@ class ClockSampler:
                 if v.lower() == "active":
                     reasons.add(nm)
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "reasons": sorted(reasons), "samples": len(sm), "source": self.source}
 
 
 def _dist():
