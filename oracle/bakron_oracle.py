@@ -40,6 +40,16 @@ Readings taken where the pages are garbled or silent (each one is listed in the 
   the code is the index of the nearest entry to x = pre / s_ij (the fp32 quotient), decided
   against the fp32 midpoints fl32((c_k + c_{k+1}) / 2), a tie going to the lower entry, and
   W_ij = s_ij c_code;
+* incoherence processing ([YAQA] section 4: like LDLQ, lower the incoherence of the Hessian
+  factors before quantising) is the randomised Hadamard transform T_d = H_d S_d / sqrt(d) on
+  both sides: W~ = T_m W* T_n^T, H_O~ = T_m H_O T_m^T, H_I~ = T_n H_I T_n^T, and after
+  rounding W = T_m^T W~_q T_n. H_d is Sylvester's for d = 2^k and the Kronecker product
+  H_28 (x) H_{2^k} for d = 28 2^k, with H_28 Paley's skew construction over GF(27) =
+  GF(3)[t] / (t^3 + 2t + 1), element e <-> (e mod 3) + (e div 3 mod 3) t + (e div 9) t^2,
+  H_28[0][*] = 1, H_28[1+x][0] = -1, H_28[1+x][1+y] = chi(x - y) + [x = y] (chi the
+  quadratic character); the signs S_d are bit i mod 256 of the Philox4x64-10 block keyed
+  (seed, 0) at counter (i div 256, 0, 1, 0) (word (i mod 256) div 64, bit i mod 64; set
+  bit = -1);
 * every Kronecker factor is damped like the benchmark's inputs: H + damp * mean(diag(H)) * I,
   the mean taken over the undamped diagonal;
 * stochastic Q (the section-4 alternative to nearest rounding) rounds x = pre/s_i up with
@@ -67,6 +77,7 @@ __all__ = [
     "code_range", "fixed_point_pre_rows", "band_check", "grid_quotient",
     "philox4x64_10", "dither", "quantize_stochastic", "damped_gram", "sketch_b",
     "damped_gram_rows", "codebook_midpoints", "quantize_codebook", "scale_of",
+    "gf27_chi", "hadamard28", "hadamard", "rht_signs", "rht_matrix", "rht",
 ]
 
 
@@ -360,6 +371,79 @@ def proxy_loss_kron(dW, H_O, H_I) -> float:
     v = np.asarray(dW, dtype=np.float64).reshape(-1)
     K = np.kron(np.asarray(H_O, np.float64), np.asarray(H_I, np.float64))
     return float(v @ K @ v)
+
+
+# ---------------------------------------------------------------------------------------------
+# Incoherence processing ([YAQA] section 4): the randomised Hadamard transform.
+# ---------------------------------------------------------------------------------------------
+def _gf27(e: int) -> tuple[int, int, int]:
+    return e % 3, (e // 3) % 3, e // 9
+
+
+def _gf27_mul(a, b):
+    """Product in GF(3)[t] / (t^3 + 2t + 1), i.e. t^3 = t + 2 (coefficients mod 3)."""
+    c = [0] * 5
+    for i in range(3):
+        for j in range(3):
+            c[i + j] += a[i] * b[j]
+    for k in (4, 3):                       # t^k = t^(k-3) (t + 2)
+        c[k - 2] += c[k]
+        c[k - 3] += 2 * c[k]
+        c[k] = 0
+    return tuple(v % 3 for v in c[:3])
+
+
+def gf27_chi() -> np.ndarray:
+    """The quadratic character of GF(27) on the 27 labelled elements: 0, +1 (nonzero square)
+    or -1."""
+    squares = {_gf27_mul(_gf27(e), _gf27(e)) for e in range(1, 27)}
+    return np.array([0] + [1 if _gf27(e) in squares else -1 for e in range(1, 27)])
+
+
+def hadamard28() -> np.ndarray:
+    """Paley's skew Hadamard matrix of order 28 (q = 27), rows/columns 1 + x for x in GF(27)."""
+    chi = gf27_chi()
+    H = np.zeros((28, 28))
+    H[0, :] = 1.0
+    H[1:, 0] = -1.0
+    for x in range(27):
+        for y in range(27):
+            a, b = _gf27(x), _gf27(y)
+            diff = sum(((a[k] - b[k]) % 3) * 3 ** k for k in range(3))
+            H[1 + x, 1 + y] = chi[diff] + (1.0 if x == y else 0.0)
+    return H
+
+
+def hadamard(d: int) -> np.ndarray:
+    """H_d for d = 2^k (Sylvester: (-1)^popcount(i & j)) or d = 28 2^k (H_28 (x) H_{2^k})."""
+    k = d // 28 if d % 28 == 0 and (d // 28) & (d // 28 - 1) == 0 else d
+    if k & (k - 1) != 0:
+        raise ValueError(f"no Hadamard construction here for d = {d}")
+    i = np.arange(k)
+    syl = np.array([[(-1.0) ** bin(a & b).count("1") for b in i] for a in i])
+    return syl if k == d else np.kron(hadamard28(), syl)
+
+
+def rht_signs(d: int, seed: int) -> np.ndarray:
+    """The random signs S_d (+1 / -1) of the transform."""
+    out = np.empty(d)
+    for blk in range((d + 255) // 256):
+        words = philox4x64_10((blk, 0, 1, 0), (seed, 0))
+        for t in range(min(256, d - 256 * blk)):
+            out[256 * blk + t] = -1.0 if (words[t // 64] >> (t % 64)) & 1 else 1.0
+    return out
+
+
+def rht_matrix(d: int, seed: int) -> np.ndarray:
+    """T_d = H_d diag(S_d) / sqrt(d), orthogonal, in fp64."""
+    return hadamard(d) * rht_signs(d, seed)[None, :] / np.sqrt(d)
+
+
+def rht(X, seed_rows: int, seed_cols: int, inverse: bool = False) -> np.ndarray:
+    """T_r X T_c^T (or, inverse, T_r^T X T_c) for X (r x c), in fp64."""
+    X = np.asarray(X, dtype=np.float64)
+    Tr, Tc = rht_matrix(X.shape[0], seed_rows), rht_matrix(X.shape[1], seed_cols)
+    return Tr.T @ X @ Tc if inverse else Tr @ X @ Tc.T
 
 
 # ---------------------------------------------------------------------------------------------
