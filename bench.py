@@ -2,7 +2,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
                     [--rounding nearest|stochastic] [--hessian]
-                    [--group-size G] [--codebook normal]
+                    [--group-size G] [--codebook normal] [--incoherence]
 
 One step = the whole path on one layer with inputs resident in HBM:
     bakron_ldl(H_O), bakron_ldl(H_I), bakron_round(W*, L_O, L_I, scales, bits),
@@ -12,6 +12,9 @@ the layer's token matrix X and H_O from its gradient rows G (resident in HBM) be
 --group-size G / --codebook normal time bakron_round_ex: one grid step per row and group of G
 columns (max |W*| over the group / the grid's top), and/or the 2^bits-entry codebook of normal
 quantiles (k + 1/2) / 2^bits scaled to [-1, 1].
+--incoherence adds the two-sided randomised Hadamard transform (bakron_rht) of W*, H_O and
+H_I, the grid steps of the rotated W* (bakron_row_scales) and the inverse transform of the
+rounded weights to the step.
 --rounding stochastic times bakron_round_stochastic (stochastic Q, a fixed seed per step) in
 place of bakron_round. Metric: quantized weights per second, m*n / step time (whole job: summed over replicas, one
 independent layer per GPU, no collective on the data path; timed as the max over ranks).
@@ -314,14 +317,15 @@ def run(args):
     stream = torch.cuda.current_stream(dev)
 
     # ---- per-call timing events on the launching stream (device-timed breakdown)
-    names = (["gram_I", "gram_O"] if args.hessian else []) + ["ldl_O", "ldl_I", "round", "loss"]
+    names = (["gram_I", "gram_O"] if args.hessian else []) + \
+        (["rotate", "unrotate"] if args.incoherence else []) + ["ldl_O", "ldl_I", "round", "loss"]
 
     seed = 0x5EED if args.rounding == "stochastic" else None
     quant = {}
     s_in = s_np          # the grid steps the step reads (per row, or per row and group)
     if args.group_size or args.codebook:
-        if seed is not None:
-            raise SystemExit("stochastic Q takes the per-row integer grid")
+        if seed is not None or args.incoherence:
+            raise SystemExit("stochastic Q and incoherence processing take the per-row grid")
         gs = min(args.group_size or n, n)
         book = normal_codebook(bits) if args.codebook == "normal" else None
         top = 1.0 if book is not None else (1 << (bits - 1)) - 0.5
@@ -331,6 +335,8 @@ def run(args):
         s_in = np.ascontiguousarray(sg, dtype=np.float32)
         sc = torch.from_numpy(s_in).to(dev)
         quant = {"group_size": gs, "codebook": book}
+    if args.incoherence:
+        quant = {"incoherence": (0x1C0, 0x1C1)}
 
     def factors(X, G, timing):
         # H_I from the tokens, H_O from the gradient rows, into the buffers the solve reads
@@ -478,7 +484,13 @@ def _roofline(per, m, n, rounding="nearest", gram_dims=None):
             "work_flops": work["round"],
             # the solver benchmark's own definition: nominal dense-equivalent 2 m n (m + n)
             "nominal_frac": 2.0 * work["round"] / t / 1e12 / peak,
-            "others_tflops": {k: work[k] / (per[k] * 1e-3) / 1e12 for k in per if k != "round"}}
+            "others_tflops": {k: work[k] / (per[k] * 1e-3) / 1e12 for k in per
+                              if k in work and k != "round"},
+            # the transforms are HBM-bound: 4 passes (read + write) per matrix, plus the grid
+            # steps' read of W~
+            "others_gbs": {k: b / (per[k] * 1e-3) / 1e9 for k, b in
+                           (("rotate", 32.0 * (m * n + m * m + n * n) + 4.0 * m * n),
+                            ("unrotate", 32.0 * m * n)) if k in per}}
 
 
 def _report(args, torch, bk, wl, ws, rank, m, n, bits, per, ms_step, value, launches, clk,
@@ -497,7 +509,7 @@ def _report(args, torch, bk, wl, ws, rank, m, n, bits, per, ms_step, value, laun
                 "config": {"workload": wl.name, "m": m, "n": n, "bits": bits,
                            "rounding": args.rounding, "hessian": bool(args.hessian),
                            "group_size": args.group_size or None,
-                           "codebook": args.codebook,
+                           "codebook": args.codebook, "incoherence": bool(args.incoherence),
                            "parallelism": f"replicas x{ws}" if ws > 1 else "single",
                            "l2": "inputs larger than L2 (H_I alone is "
                                  f"{4 * n * n / 2**20:.0f} MiB), no flush"},
@@ -526,6 +538,7 @@ def main():
     ap.add_argument("--hessian", action="store_true")
     ap.add_argument("--group-size", type=int, default=0)
     ap.add_argument("--codebook", default=None, choices=["normal"])
+    ap.add_argument("--incoherence", action="store_true")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)

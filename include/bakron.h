@@ -224,6 +224,47 @@ size_t bakron_sketch_b_workspace_bytes(int S, int m, int n);
 int bakron_sketch_b(const float* G, int S, int m, int n, float damp, float* H_O, float* H_I,
                     void* ws, size_t ws_bytes, int* dev_status, void* stream);
 
+/* ------------------------------------------------------------------------------------------
+ * bakron_rht -- the randomised Hadamard transform on both sides of a matrix (incoherence
+ * processing; YAQA article, section 4: the bound on the rounding error grows with the
+ * incoherence of H_O and H_I, which is lowered before quantising, as for LDLQ).
+ *
+ *   T_d = H_d S_d / sqrt(d),  S_d = diag(+-1),
+ *   H_d = Sylvester's Hadamard matrix ((-1)^popcount(i & j)) for d = 2^k, and
+ *         H_28 (x) H_{2^k} for d = 28 * 2^k, H_28 Paley's skew Hadamard matrix from the
+ *         quadratic character chi of GF(27) = GF(3)[t] / (t^3 + 2t + 1) (element e <->
+ *         (e mod 3) + (e/3 mod 3) t + (e/9) t^2; H_28[0][*] = 1, H_28[1+x][0] = -1,
+ *         H_28[1+x][1+y] = chi(x - y) + [x = y]);
+ *   S_d[i] = -1 when bit (i mod 256) of the Philox4x64-10 block keyed (seed, 0) at counter
+ *         (i / 256, 0, 1, 0) is set (word (i mod 256) / 64, bit i mod 64), else +1;
+ *   Y = T_rows X T_cols^T   (inverse = 0),    Y = T_rows^T X T_cols   (inverse = 1).
+ *
+ * The layer is processed as W~ = rht(W*, seed_o, seed_i), H_O~ = rht(H_O, seed_o, seed_o),
+ * H_I~ = rht(H_I, seed_i, seed_i); after rounding W~, W = rht(W~_q, seed_o, seed_i, inverse).
+ *
+ *   X        [in]  rows x cols; may be the same buffer as Y.
+ *   rows, cols [in] each 2^k or 28 * 2^k, at most 32768 (bakron_rht_supported tells).
+ *   Y        [out] rows x cols.
+ *   ws       [in]  at least bakron_rht_workspace_bytes(rows, cols) bytes, 256-B aligned.
+ * Returns BAKRON_ERR_INVALID_ARG for an unsupported size. Four passes over the matrix: the
+ * signs, butterflies and order-28 stage along rows in shared memory, then the same along
+ * columns through two tiled transposes.
+ * ---------------------------------------------------------------------------------------- */
+int bakron_rht_supported(int d);
+size_t bakron_rht_workspace_bytes(int rows, int cols);
+int bakron_rht(const float* X, int rows, int cols, uint64_t seed_rows, uint64_t seed_cols,
+               int inverse, float* Y, void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------------------------
+ * bakron_row_scales -- grid steps from a matrix: scales[i * G + g] = max over the columns j of
+ * group g of |W[i][j]|, divided by `divisor` (one correctly rounded fp32 division);
+ * G = ceil(n / group_size), group_size >= n gives one step per row. With divisor
+ * 2^(bits-1) - 0.5 these are the per-row max-abs grid steps of the integer grid.
+ *   W [in] m x n; scales [out] m x G (device); divisor > 0.
+ * ---------------------------------------------------------------------------------------- */
+int bakron_row_scales(const float* W, int m, int n, int group_size, float divisor,
+                      float* scales, void* stream);
+
 /* Synchronises `stream`, then returns the device status word (a bakron_status value), or
  * BAKRON_ERR_CUDA if the synchronisation itself failed. */
 int bakron_read_status(const int* dev_status, void* stream);

@@ -27,6 +27,10 @@ int bakron_internal_proxy_loss_simt(const float* dW, int m, int n, const float* 
                                     const float* H_I, double* loss, void* ws, size_t ws_bytes,
                                     void* stream);
 
+/* Writes the order-28 Hadamard matrix the transform of bakron_rht uses (row-major, 784 HOST
+ * bytes of +1 / -1). Host only; no device work. */
+void bakron_internal_hadamard28(signed char* out);
+
 #ifdef __cplusplus
 }
 #endif

@@ -77,7 +77,7 @@ __all__ = [
     "code_range", "fixed_point_pre_rows", "band_check", "grid_quotient",
     "philox4x64_10", "dither", "quantize_stochastic", "damped_gram", "sketch_b",
     "damped_gram_rows", "codebook_midpoints", "quantize_codebook", "scale_of",
-    "gf27_chi", "hadamard28", "hadamard", "rht_signs", "rht_matrix", "rht",
+    "gf27_chi", "hadamard28", "hadamard", "rht_signs", "rht_matrix", "rht", "hadamard_rows",
 ]
 
 
@@ -422,6 +422,22 @@ def hadamard(d: int) -> np.ndarray:
     i = np.arange(k)
     syl = np.array([[(-1.0) ** bin(a & b).count("1") for b in i] for a in i])
     return syl if k == d else np.kron(hadamard28(), syl)
+
+
+def hadamard_rows(d: int, rows) -> np.ndarray:
+    """Rows ``rows`` of H_d without forming H_d (the same definitions: Sylvester's
+    (-1)^popcount(i & j), times H_28[i div 2^k][j div 2^k] for d = 28 2^k)."""
+    rows = np.asarray(rows)
+    k = d // 28 if d % 28 == 0 and (d // 28) & (d // 28 - 1) == 0 else d
+    if k & (k - 1) != 0:
+        raise ValueError(f"no Hadamard construction here for d = {d}")
+    j = np.arange(d)
+    b_i, b_j = (rows % k)[:, None], (j % k)[None, :]
+    par = np.vectorize(lambda v: bin(int(v)).count("1") & 1)(b_i & b_j)
+    out = np.where(par == 1, -1.0, 1.0)
+    if k != d:
+        out = out * hadamard28()[(rows // k)[:, None], (j // k)[None, :]]
+    return out
 
 
 def rht_signs(d: int, seed: int) -> np.ndarray:

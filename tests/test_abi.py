@@ -99,3 +99,31 @@ def test_new_entry_points_reject_bad_arguments_on_host(libpath):
     lib.bakron_damped_gram_workspace_bytes.restype = ctypes.c_size_t
     lib.bakron_damped_gram_workspace_bytes.argtypes = [ci, ci]
     assert lib.bakron_damped_gram_workspace_bytes(1000, 300) >= 2 * 300 * 1000 * 4
+
+
+def test_library_hadamard28_equals_the_oracle(libpath):
+    """The library builds H_28 on the host from its own GF(27) arithmetic; it must be the
+    oracle's matrix (checked here, without a GPU)."""
+    import numpy as np
+
+    import oracle
+    from two_sided_adaptive_bakron_b200 import bakron
+    np.testing.assert_array_equal(bakron.internal_hadamard28().astype(np.float64),
+                                  oracle.hadamard28())
+    assert all(bakron.bakron_rht_supported(d) for d in (1, 2, 28, 56, 4096, 14336, 28672, 32768))
+    assert not any(bakron.bakron_rht_supported(d) for d in (0, 3, 12, 20, 84, 65536, 57344))
+
+
+def test_rht_rejects_bad_arguments_on_host(libpath):
+    lib = ctypes.CDLL(libpath)
+    vp, ci = ctypes.c_void_p, ctypes.c_int
+    lib.bakron_rht.restype = ci
+    lib.bakron_rht.argtypes = [vp, ci, ci, ctypes.c_uint64, ctypes.c_uint64, ci, vp, vp,
+                               ctypes.c_size_t, vp]
+    fake = vp(0x1000)
+    assert lib.bakron_rht(fake, 12, 28, 1, 2, 0, fake, fake, 1 << 30, None) == -1
+    assert lib.bakron_rht(fake, 28, 28, 1, 2, 2, fake, fake, 1 << 30, None) == -1
+    assert lib.bakron_rht(fake, 28, 28, 1, 2, 0, fake, fake, 16, None) == -5
+    lib.bakron_row_scales.restype = ci
+    lib.bakron_row_scales.argtypes = [vp, ci, ci, ci, ctypes.c_float, vp, vp]
+    assert lib.bakron_row_scales(fake, 4, 4, 4, 0.0, fake, None) == -1

@@ -14,8 +14,8 @@ import numpy as np
 import pytest
 import scipy.linalg
 
-from oracle import (gf27_chi, hadamard, hadamard28, philox4x64_10, proxy_loss, rht, rht_matrix,
-                    rht_signs)
+from oracle import (gf27_chi, hadamard, hadamard28, hadamard_rows, philox4x64_10, proxy_loss, rht,
+                    rht_matrix, rht_signs)
 from oracle.bakron_oracle import _gf27, _gf27_mul
 
 
@@ -89,3 +89,9 @@ def test_proxy_loss_is_invariant():
     so, si = 21, 22
     dWt, HOt, HIt = rht(dW, so, si), rht(HO, so, so), rht(HI, si, si)
     assert abs(proxy_loss(dWt, HOt, HIt) - proxy_loss(dW, HO, HI)) < 1e-10 * proxy_loss(dW, HO, HI)
+
+
+@pytest.mark.parametrize("d", [1, 8, 28, 112])
+def test_hadamard_rows_are_rows_of_hadamard(d):
+    rows = np.array([0, d - 1, d // 2, d // 3])
+    np.testing.assert_array_equal(hadamard_rows(d, rows), hadamard(d)[rows])

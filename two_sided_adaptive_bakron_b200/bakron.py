@@ -2,11 +2,12 @@
 
 The functions named like the C ABI (``bakron_ldl``, ``bakron_round``,
 ``bakron_round_stochastic``, ``bakron_round_ex``, ``bakron_proxy_loss``, ``bakron_damped_gram``,
-``bakron_sketch_b``, ``bakron_read_status``, ``bakron_status_string`` and the
-``*_workspace_bytes`` queries) take torch CUDA tensors, pass their device pointers and the
-current CUDA stream to the library and return its status code. ``ldl``, ``round_weights``,
-``proxy_loss``, ``damped_gram``, ``sketch_b`` and ``solve`` additionally allocate outputs and
-workspaces with torch and raise on any error.
+``bakron_sketch_b``, ``bakron_rht``, ``bakron_row_scales``, ``bakron_read_status``,
+``bakron_status_string`` and the ``*_workspace_bytes`` queries) take torch CUDA tensors, pass
+their device pointers and the current CUDA stream to the library and return its status code.
+``ldl``, ``round_weights``, ``proxy_loss``, ``damped_gram``, ``sketch_b``, ``rht``,
+``row_scales`` and ``solve`` additionally allocate outputs and workspaces with torch and raise
+on any error.
 
 Every step of the computation runs in the library's CUDA kernels; there is no CPU path. If
 the shared library is missing the first call raises.
@@ -51,6 +52,11 @@ _SIGNATURES = {
     "bakron_sketch_b_workspace_bytes": (_c_size_t, [_c_int, _c_int, _c_int]),
     "bakron_sketch_b": (_c_int, [_vp, _c_int, _c_int, _c_int, ctypes.c_float, _vp, _vp, _vp,
                                  _c_size_t, _vp, _vp]),
+    "bakron_rht_supported": (_c_int, [_c_int]),
+    "bakron_rht_workspace_bytes": (_c_size_t, [_c_int, _c_int]),
+    "bakron_rht": (_c_int, [_vp, _c_int, _c_int, ctypes.c_uint64, ctypes.c_uint64, _c_int, _vp,
+                            _vp, _c_size_t, _vp]),
+    "bakron_row_scales": (_c_int, [_vp, _c_int, _c_int, _c_int, ctypes.c_float, _vp, _vp]),
     "bakron_read_status": (_c_int, [_vp, _vp]),
     "bakron_status_string": (ctypes.c_char_p, [_c_int]),
     "bakron_version": (_c_int, []),
@@ -62,6 +68,7 @@ _SIGNATURES = {
     "bakron_internal_gemm3x": (_c_int, [_vp, _c_int, _c_int, _c_int, _vp, _c_int, _c_int, _vp,
                                         _c_int, _vp, _c_size_t, _vp, _vp]),
     "bakron_internal_proxy_loss_simt_workspace_bytes": (_c_size_t, [_c_int, _c_int]),
+    "bakron_internal_hadamard28": (None, [_vp]),
     "bakron_internal_proxy_loss_simt": (_c_int, [_vp, _c_int, _c_int, _vp, _vp, _vp, _vp,
                                                  _c_size_t, _vp]),
 }
@@ -232,6 +239,41 @@ def bakron_sketch_b(G, damp, H_O, H_I, ws, dev_status, stream=None) -> int:
                                  _stream(stream))
 
 
+def bakron_rht_supported(d: int) -> bool:
+    return bool(lib().bakron_rht_supported(int(d)))
+
+
+def bakron_rht_workspace_bytes(rows: int, cols: int) -> int:
+    return int(lib().bakron_rht_workspace_bytes(int(rows), int(cols)))
+
+
+def bakron_rht(X, seed_rows, seed_cols, inverse, Y, ws, stream=None) -> int:
+    r, c = X.shape
+    _check_cuda(X, torch.float32, (r, c), "X")
+    _check_cuda(Y, torch.float32, (r, c), "Y")
+    m64 = (1 << 64) - 1
+    return lib().bakron_rht(_ptr(X), r, c, int(seed_rows) & m64, int(seed_cols) & m64,
+                            int(bool(inverse)), _ptr(Y), _ptr(ws), ws.numel() * ws.element_size(),
+                            _stream(stream))
+
+
+def bakron_row_scales(W, group_size, divisor, scales, stream=None) -> int:
+    m, n = W.shape
+    _check_cuda(W, torch.float32, (m, n), "W")
+    g = min(int(group_size), n)
+    _check_cuda(scales, torch.float32, (m, (n + g - 1) // g), "scales")
+    return lib().bakron_row_scales(_ptr(W), m, n, int(group_size), float(divisor), _ptr(scales),
+                                   _stream(stream))
+
+
+def internal_hadamard28():
+    """The order-28 Hadamard matrix the library's transform uses (host construction)."""
+    import numpy as np
+    buf = (ctypes.c_byte * 784)()
+    lib().bakron_internal_hadamard28(buf)
+    return np.frombuffer(bytes(buf), dtype=np.int8).reshape(28, 28).copy()
+
+
 def bakron_ldl_noalloc(H, L, D, dev_status, stream=None) -> int:
     """bakron_ldl with the library's own fixed scratch (no workspace argument)."""
     n = H.shape[0]
@@ -361,6 +403,23 @@ def sketch_b(G, damp: float = 0.01, stream=None, check: bool = True):
     return H_O, H_I
 
 
+def rht(X, seed_rows: int, seed_cols: int, inverse: bool = False, stream=None) -> torch.Tensor:
+    """T_rows X T_cols^T (inverse: T_rows^T X T_cols) on the device (a new tensor)."""
+    Y = torch.empty_like(X)
+    ws = workspace(bakron_rht_workspace_bytes(*X.shape), X.device)
+    _raise(bakron_rht(X, seed_rows, seed_cols, inverse, Y, ws, stream), "bakron_rht")
+    return Y
+
+
+def row_scales(W, divisor: float, group_size=None, stream=None) -> torch.Tensor:
+    """max |W| over each row (and group of columns) / divisor, on the device."""
+    m, n = W.shape
+    g = n if group_size is None else min(int(group_size), n)
+    out = torch.empty((m, (n + g - 1) // g), dtype=torch.float32, device=W.device)
+    _raise(bakron_row_scales(W, g, divisor, out, stream), "bakron_row_scales")
+    return out if group_size is not None else out.view(m)
+
+
 def proxy_loss(dW, H_O, H_I, stream=None) -> torch.Tensor:
     """tr(H_O dW H_I dW^T) as a one-element float64 CUDA tensor."""
     m, n = dW.shape
@@ -392,6 +451,7 @@ class Solver:
         self.ws = workspace(max(bakron_ldl_workspace_bytes(n),
                                 bakron_proxy_loss_workspace_bytes(m, n)), self.device)
         self.E = self.ws_round[: 4 * m * n].view(torch.float32).view(m, n)
+        self._rot = None     # incoherence buffers, made on first use
         self.status = new_status(self.device)
         # the two factorisations are independent: ldl(H_O) runs on a side stream while
         # ldl(H_I) runs on the caller's stream
@@ -399,11 +459,28 @@ class Solver:
         self._fork = torch.cuda.Event()
         self._join = torch.cuda.Event()
 
+    def _rotated(self):
+        if self._rot is None:
+            m, n, dev = self.m, self.n, self.device
+            f32 = dict(dtype=torch.float32, device=dev)
+            self._rot = dict(W=torch.empty((m, n), **f32), HO=torch.empty((m, m), **f32),
+                             HI=torch.empty((n, n), **f32), s=torch.empty((m, 1), **f32),
+                             W_orig=torch.empty((m, n), **f32),
+                             ws=workspace(max(bakron_rht_workspace_bytes(m, n),
+                                              bakron_rht_workspace_bytes(m, m),
+                                              bakron_rht_workspace_bytes(n, n)), dev))
+        return self._rot
+
     def run(self, Wstar, H_O, H_I, scales, bits, stream=None, with_loss=True, timing=None,
-            seed=None, group_size=None, codebook=None):
+            seed=None, group_size=None, codebook=None, incoherence=None):
         """Enqueues the whole path (reads: self.codes, self.W, self.E, self.loss); a seed
         selects stochastic Q for the round, a group size (with m x G scales) and/or a host
         codebook the base quantizer of bakron_round_ex.
+
+        incoherence=(seed_o, seed_i) runs the path on the rotated layer (bakron_rht):
+        W~ = T_m W* T_n^T, H_O~ = T_m H_O T_m^T, H_I~ = T_n H_I T_n^T, per-row grid steps of
+        W~ (``scales`` is then ignored), and writes self.W_orig = T_m^T W~_q T_n. self.codes,
+        self.W and self.E stay in the rotated basis, where the proxy loss is the same.
 
         timing: optional {name: (start_event, end_event)} for any of "ldl_O", "ldl_I", "round",
         "loss"; each pair is recorded around its call on the stream that runs it.
@@ -411,6 +488,22 @@ class Solver:
         if stream is None:
             stream = torch.cuda.current_stream(self.device)
         timing = timing or {}
+        if incoherence is not None:
+            if group_size is not None or codebook is not None:
+                raise ValueError("incoherence processing takes per-row integer-grid steps")
+            so, si = incoherence
+            R = self._rotated()
+            ev = timing.get("rotate")
+            if ev is not None:
+                ev[0].record(stream)
+            for X, Y, a, b in ((Wstar, R["W"], so, si), (H_O, R["HO"], so, so),
+                               (H_I, R["HI"], si, si)):
+                _raise(bakron_rht(X, a, b, False, Y, R["ws"], stream), "bakron_rht")
+            _raise(bakron_row_scales(R["W"], self.n, (1 << (bits - 1)) - 0.5, R["s"], stream),
+                   "bakron_row_scales")
+            if ev is not None:
+                ev[1].record(stream)
+            Wstar, H_O, H_I, scales = R["W"], R["HO"], R["HI"], R["s"].view(self.m)
 
         def call(name, st, fn, *a):
             ev = timing.get(name)
@@ -438,6 +531,15 @@ class Solver:
                  bits, seed, self.codes, self.W, self.ws_round, self.status)
         if with_loss:
             call("loss", stream, bakron_proxy_loss, self.E, H_O, H_I, self.loss, self.ws)
+        if incoherence is not None:
+            R = self._rotated()
+            ev = timing.get("unrotate")
+            if ev is not None:
+                ev[0].record(stream)
+            _raise(bakron_rht(self.W, so, si, True, R["W_orig"], R["ws"], stream), "bakron_rht")
+            if ev is not None:
+                ev[1].record(stream)
+            self.W_orig = R["W_orig"]
 
     def check(self, stream=None):
         _raise(bakron_read_status(self.status, stream), "bakron (device)")

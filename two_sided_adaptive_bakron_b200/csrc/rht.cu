@@ -1,0 +1,254 @@
+// rht.cu -- incoherence processing: the randomised Hadamard transform on both sides of a
+// matrix (bakron_rht) and the grid steps of a matrix (bakron_row_scales).
+//
+// YAQA article (news.43b.com.cn/a/479517.html), section 4: the error bound of the rounding
+// rule grows with the incoherence of H_O and H_I, so, as with LDLQ, the factors' incoherence is
+// lowered before quantising. The transform is T_d = H_d S_d / sqrt(d): S_d random signs, H_d
+// Sylvester's Hadamard matrix for d = 2^k, or H_28 (x) H_{2^k} for d = 28 2^k with H_28
+// Paley's skew Hadamard matrix of order 28 (from the quadratic character of GF(27)). Applied
+// as W~ = T_m W T_n^T, H_O~ = T_m H_O T_m^T, H_I~ = T_n H_I T_n^T, and W = T_m^T W~_q T_n after
+// rounding; the proxy loss is the same in both bases.
+//
+// One CTA transforms one row in shared memory: the signs (one Philox4x64-10 block per 256
+// indices, keyed (seed, 0) at counter (i / 256, 0, 1, 0), bit i % 256, set = -1), the
+// Sylvester butterflies over each 2^k segment (the standard in-place fast Walsh-Hadamard
+// transform over the whole row: a pair (i, i + h) with 2h <= 2^k never leaves its segment),
+// then the order-28 stage across segments, and the 1/sqrt(d) scale. The column transform is a
+// row transform of the transpose (tiled 32 x 32 transposes through shared memory). Every pass
+// reads and writes the matrix once: HBM-bound.
+#include <cmath>
+#include <cstring>
+
+#include "bakron_internal.h"
+#include "common.cuh"
+#include "philox.cuh"
+
+namespace bakron {
+namespace {
+
+constexpr int kRowThreads = 512;
+constexpr int kMaxLen = 32768;        // 2^15, or 28 * 2^10 = 28672
+
+struct H28 {
+    signed char h[28][28];
+};
+
+// Paley's construction over GF(27) = GF(3)[t] / (t^3 + 2t + 1): element e has coefficients
+// (e mod 3, e / 3 mod 3, e / 9) of 1, t, t^2; H[0][*] = 1, H[1+x][0] = -1,
+// H[1+x][1+y] = chi(x - y) + [x == y], chi the quadratic character (0, +1 square, -1 not).
+H28 make_h28() {
+    auto mul = [](const int* a, const int* b, int* out) {
+        int c[5] = {0, 0, 0, 0, 0};
+        for (int i = 0; i < 3; ++i)
+            for (int j = 0; j < 3; ++j) c[i + j] += a[i] * b[j];
+        for (int k = 4; k >= 3; --k) {   // t^3 = t + 2
+            c[k - 2] += c[k];
+            c[k - 3] += 2 * c[k];
+            c[k] = 0;
+        }
+        for (int i = 0; i < 3; ++i) out[i] = c[i] % 3;
+    };
+    int el[27][3];
+    for (int e = 0; e < 27; ++e) {
+        el[e][0] = e % 3;
+        el[e][1] = (e / 3) % 3;
+        el[e][2] = e / 9;
+    }
+    bool square[27] = {};
+    for (int e = 1; e < 27; ++e) {
+        int sq[3];
+        mul(el[e], el[e], sq);
+        square[sq[0] + 3 * sq[1] + 9 * sq[2]] = true;
+    }
+    H28 H;
+    for (int y = 0; y < 28; ++y) H.h[0][y] = 1;
+    for (int x = 0; x < 27; ++x) {
+        H.h[1 + x][0] = -1;
+        for (int y = 0; y < 27; ++y) {
+            int d = 0, p = 1;
+            for (int k = 0; k < 3; ++k, p *= 3) d += ((el[x][k] - el[y][k] + 3) % 3) * p;
+            const int chi = d == 0 ? 0 : (square[d] ? 1 : -1);
+            H.h[1 + x][1 + y] = (signed char)(chi + (x == y ? 1 : 0));
+        }
+    }
+    return H;
+}
+
+// d = 28 * 2^k (returns 28, sets seg = 2^k) or 2^k (returns 1, seg = d); 0 otherwise.
+int factor(int d, int& seg) {
+    const bool pow2 = d > 0 && (d & (d - 1)) == 0;
+    if (pow2 && d <= kMaxLen) { seg = d; return 1; }
+    if (d > 0 && d % 28 == 0) {
+        const int k = d / 28;
+        if ((k & (k - 1)) == 0 && d <= kMaxLen) { seg = k; return 28; }
+    }
+    return 0;
+}
+
+// Row r of Y = T X_r (inverse: T^T X_r) for rows of length d = outer * seg, in place allowed.
+__global__ void __launch_bounds__(kRowThreads)
+rht_rows_kernel(const float* __restrict__ X, float* __restrict__ Y, int d, int seg, int outer,
+                unsigned long long seed, int inverse, float scale, const __grid_constant__ H28 H) {
+    extern __shared__ __align__(16) uint8_t rht_smem[];
+    float* v = reinterpret_cast<float*>(rht_smem);
+    uint64_t* sw = reinterpret_cast<uint64_t*>(v + ((d + 3) & ~3));   // sign words, 4 per block
+    const size_t row = blockIdx.x;
+    const float* x = X + row * (size_t)d;
+    const int tid = threadIdx.x;
+    const int nblk = (d + 255) / 256;
+    for (int b = tid; b < nblk; b += kRowThreads) {
+        uint64_t w[4];
+        philox4x64_10((uint64_t)b, 0, 1, 0, seed, 0, w);
+        for (int q = 0; q < 4; ++q) sw[4 * b + q] = w[q];
+    }
+    for (int j = tid; j < d; j += kRowThreads) v[j] = x[j];
+    __syncthreads();
+    auto sign = [&](int j) { return ((sw[j >> 6] >> (j & 63)) & 1ull) ? -1.f : 1.f; };
+    if (!inverse) {
+        for (int j = tid; j < d; j += kRowThreads) v[j] *= sign(j);
+        __syncthreads();
+    }
+    // Sylvester butterflies on every segment of length seg
+    for (int h = 1; h < seg; h <<= 1) {
+        for (int p = tid; p < d / 2; p += kRowThreads) {
+            const int i = (p / h) * 2 * h + (p % h);
+            const float a = v[i], b = v[i + h];
+            v[i] = a + b;
+            v[i + h] = a - b;
+        }
+        __syncthreads();
+    }
+    // the order-28 stage across segments: v[a seg + b] <- sum_a' H[a][a'] v[a' seg + b]
+    // (inverse: H^T)
+    if (outer == 28) {
+        for (int b = tid; b < seg; b += kRowThreads) {
+            float in[28], out[28];
+#pragma unroll
+            for (int a = 0; a < 28; ++a) in[a] = v[a * seg + b];
+#pragma unroll
+            for (int a = 0; a < 28; ++a) {
+                float acc = 0.f;
+#pragma unroll
+                for (int c = 0; c < 28; ++c) {
+                    const int hv = inverse ? H.h[c][a] : H.h[a][c];
+                    acc = hv > 0 ? acc + in[c] : acc - in[c];
+                }
+                out[a] = acc;
+            }
+#pragma unroll
+            for (int a = 0; a < 28; ++a) v[a * seg + b] = out[a];
+        }
+        __syncthreads();
+    }
+    float* y = Y + row * (size_t)d;
+    for (int j = tid; j < d; j += kRowThreads) y[j] = (inverse ? v[j] * sign(j) : v[j]) * scale;
+}
+
+// Y (c x r) = X^T for X (r x c), 32 x 32 tiles.
+__global__ void transpose_kernel(const float* __restrict__ X, float* __restrict__ Y, int r,
+                                 int c) {
+    __shared__ float t[32][33];
+    const int r0 = blockIdx.y * 32, c0 = blockIdx.x * 32;
+    for (int k = threadIdx.y; k < 32; k += 8) {
+        const int rr = r0 + k, cc = c0 + threadIdx.x;
+        if (rr < r && cc < c) t[k][threadIdx.x] = X[(size_t)rr * c + cc];
+    }
+    __syncthreads();
+    for (int k = threadIdx.y; k < 32; k += 8) {
+        const int cc = c0 + k, rr = r0 + threadIdx.x;
+        if (rr < r && cc < c) Y[(size_t)cc * r + rr] = t[threadIdx.x][k];
+    }
+}
+
+// scales[i * G + g] = max_{j in group g} |W[i][j]| / divisor; one CTA per row, one warp per
+// group at a time.
+__global__ void row_scales_kernel(const float* __restrict__ W, int n, int group, int G,
+                                  float divisor, float* __restrict__ scales) {
+    const size_t i = blockIdx.x;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    for (int g = warp; g < G; g += nw) {
+        const int j0 = g * group, j1 = min(n, j0 + group);
+        float mx = 0.f;
+        for (int j = j0 + lane; j < j1; j += 32) mx = fmaxf(mx, fabsf(W[i * n + j]));
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        if (lane == 0) scales[i * G + g] = mx / divisor;
+    }
+}
+
+int rows_pass(const float* X, float* Y, int rows, int d, unsigned long long seed, int inverse,
+              const H28& H, cudaStream_t st) {
+    int seg = 0;
+    const int outer = factor(d, seg);
+    const size_t smem = (size_t)((d + 3) & ~3) * sizeof(float) +
+                        (size_t)4 * ((d + 255) / 256) * sizeof(uint64_t);
+    if (cudaFuncSetAttribute(rht_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem) != cudaSuccess)
+        return BAKRON_ERR_CUDA;
+    const float scale = 1.0f / sqrtf((float)d);
+    rht_rows_kernel<<<rows, kRowThreads, smem, st>>>(X, Y, d, seg, outer, seed, inverse, scale, H);
+    count_launches(1);
+    return cuda_err(cudaGetLastError());
+}
+
+void transpose(const float* X, float* Y, int r, int c, cudaStream_t st) {
+    transpose_kernel<<<dim3((c + 31) / 32, (r + 31) / 32), dim3(32, 8), 0, st>>>(X, Y, r, c);
+    count_launches(1);
+}
+
+}  // namespace
+}  // namespace bakron
+
+using namespace bakron;
+
+extern "C" void bakron_internal_hadamard28(signed char* out) {
+    const H28 H = make_h28();
+    memcpy(out, H.h, sizeof(H.h));
+}
+
+extern "C" int bakron_rht_supported(int d) {
+    int seg = 0;
+    return factor(d, seg) != 0 ? 1 : 0;
+}
+
+extern "C" size_t bakron_rht_workspace_bytes(int rows, int cols) {
+    if (rows < 1 || cols < 1) return 0;
+    WsSizer z;
+    z.take<float>((size_t)rows * cols);
+    return z.bytes();
+}
+
+extern "C" int bakron_rht(const float* X, int rows, int cols, uint64_t seed_rows,
+                          uint64_t seed_cols, int inverse, float* Y, void* ws, size_t ws_bytes,
+                          void* stream) {
+    int seg = 0;
+    if (rows < 1 || cols < 1 || !factor(rows, seg) || !factor(cols, seg) || !X || !Y ||
+        (inverse != 0 && inverse != 1) || (long long)rows * cols >= (1LL << 31))
+        return BAKRON_ERR_INVALID_ARG;
+    if (!ws_ok(ws, ws_bytes, bakron_rht_workspace_bytes(rows, cols))) return BAKRON_ERR_WORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    static const H28 H = make_h28();
+    WsCarver c(ws);
+    float* t = c.take<float>((size_t)rows * cols);
+    int e;
+    // Y = X T_c^T (inverse: X T_c): each row x -> T_c x (inverse: T_c^T x)
+    if ((e = rows_pass(X, Y, rows, cols, seed_cols, inverse, H, st))) return e;
+    // then T_r Y (inverse: T_r^T Y) as a row pass over Y^T
+    transpose(Y, t, rows, cols, st);
+    if ((e = rows_pass(t, t, cols, rows, seed_rows, inverse, H, st))) return e;
+    transpose(t, Y, cols, rows, st);
+    return cuda_err(cudaGetLastError());
+}
+
+extern "C" int bakron_row_scales(const float* W, int m, int n, int group_size, float divisor,
+                                 float* scales, void* stream) {
+    if (m < 1 || n < 1 || group_size < 1 || !(divisor > 0.f && divisor < 3.0e38f) || !W ||
+        !scales)
+        return BAKRON_ERR_INVALID_ARG;
+    const int group = group_size < n ? group_size : n;
+    const int G = (n + group - 1) / group;
+    row_scales_kernel<<<m, 256, 0, static_cast<cudaStream_t>(stream)>>>(W, n, group, G, divisor,
+                                                                       scales);
+    count_launches(1);
+    return cuda_err(cudaGetLastError());
+}
