@@ -9,13 +9,13 @@
 // as W~ = T_m W T_n^T, H_O~ = T_m H_O T_m^T, H_I~ = T_n H_I T_n^T, and W = T_m^T W~_q T_n after
 // rounding; the proxy loss is the same in both bases.
 //
-// One CTA transforms one row in shared memory: the signs (one Philox4x64-10 block per 256
-// indices, keyed (seed, 0) at counter (i / 256, 0, 1, 0), bit i % 256, set = -1), the
-// Sylvester butterflies over each 2^k segment (the standard in-place fast Walsh-Hadamard
-// transform over the whole row: a pair (i, i + h) with 2h <= 2^k never leaves its segment),
-// then the order-28 stage across segments, and the 1/sqrt(d) scale. The column transform is a
-// row transform of the transpose (tiled 32 x 32 transposes through shared memory). Every pass
-// reads and writes the matrix once: HBM-bound.
+// One CTA transforms one row with the row in registers: the signs (one Philox4x64-10 block per
+// 256 indices, keyed (seed, 0) at counter (i / 256, 0, 1, 0), bit i % 256, set = -1), the
+// Sylvester butterflies over each 2^k segment (the fast Walsh-Hadamard transform: a pair
+// (i, i ^ h) with 2h <= 2^k never leaves its segment), by warp shuffles, shared memory or
+// inside a thread depending on the stride, then the order-28 stage across segments, and the
+// 1/sqrt(d) scale. The column transform is a row transform of the transpose (tiled 32 x 32
+// transposes through shared memory). Every pass reads and writes the matrix once: HBM-bound.
 #include <cmath>
 #include <cstring>
 
@@ -26,7 +26,6 @@
 namespace bakron {
 namespace {
 
-constexpr int kRowThreads = 512;
 constexpr int kMaxLen = 32768;        // 2^15, or 28 * 2^10 = 28672
 
 struct H28 {
@@ -85,63 +84,101 @@ int factor(int d, int& seg) {
     return 0;
 }
 
-// Row r of Y = T X_r (inverse: T^T X_r) for rows of length d = outer * seg, in place allowed.
+// H_28 as +-1.0f for the order-28 stage (fmaf(+-1, x, acc) rounds exactly like acc +- x).
+struct H28f {
+    float h[28][28];
+};
+
+// Row r of Y = T X_r (inverse: T^T X_r), rows of length d = OUTER * seg, in place allowed.
+// Thread t of T threads holds the E = OUTER * U elements j = t + T e in registers, T = seg / U:
+// e = a U + u is element t + T u of segment a. A butterfly of stride h pairs j with j ^ h: for
+// h < T the partner is thread t ^ h with the same e (a warp shuffle for h < 32, shared memory
+// above); for T <= h < seg it is element e ^ (h / T) of the same thread (same segment). The
+// order-28 stage then mixes the 28 segments in registers. The additions are those of the
+// textbook order (strides 1, 2, 4, ..., then the order-28 sums in index order).
+constexpr int kRowThreads = 512;
+
+template <int U, int OUTER, bool kInverse>
 __global__ void __launch_bounds__(kRowThreads)
-rht_rows_kernel(const float* __restrict__ X, float* __restrict__ Y, int d, int seg, int outer,
-                unsigned long long seed, int inverse, float scale, const __grid_constant__ H28 H) {
+rht_rows_kernel(const float* __restrict__ X, float* __restrict__ Y, int d, int T,
+                unsigned long long seed, float scale, const __grid_constant__ H28f H) {
+    constexpr int E = OUTER * U;
     extern __shared__ __align__(16) uint8_t rht_smem[];
-    float* v = reinterpret_cast<float*>(rht_smem);
-    uint64_t* sw = reinterpret_cast<uint64_t*>(v + ((d + 3) & ~3));   // sign words, 4 per block
+    float* buf = reinterpret_cast<float*>(rht_smem);                    // d floats (exchange)
+    uint64_t* sw = reinterpret_cast<uint64_t*>(buf + ((d + 3) & ~3));   // sign words
     const size_t row = blockIdx.x;
-    const float* x = X + row * (size_t)d;
-    const int tid = threadIdx.x;
+    const int t = threadIdx.x;
+    const bool own = t < T;                   // blockDim.x = max(T, 32)
     const int nblk = (d + 255) / 256;
-    for (int b = tid; b < nblk; b += kRowThreads) {
+    for (int b = t; b < nblk; b += blockDim.x) {
         uint64_t w[4];
         philox4x64_10((uint64_t)b, 0, 1, 0, seed, 0, w);
         for (int q = 0; q < 4; ++q) sw[4 * b + q] = w[q];
     }
-    for (int j = tid; j < d; j += kRowThreads) v[j] = x[j];
-    __syncthreads();
-    auto sign = [&](int j) { return ((sw[j >> 6] >> (j & 63)) & 1ull) ? -1.f : 1.f; };
-    if (!inverse) {
-        for (int j = tid; j < d; j += kRowThreads) v[j] *= sign(j);
-        __syncthreads();
+    const float* x = X + row * (size_t)d;
+    float v[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) v[e] = own ? x[t + T * e] : 0.f;
+    __syncthreads();                          // the sign words are in place
+    auto sgn = [&](int j) { return ((sw[j >> 6] >> (j & 63)) & 1ull) ? -1.f : 1.f; };
+    if (!kInverse && own) {
+#pragma unroll
+        for (int e = 0; e < E; ++e) v[e] *= sgn(t + T * e);
     }
-    // Sylvester butterflies on every segment of length seg
-    for (int h = 1; h < seg; h <<= 1) {
-        for (int p = tid; p < d / 2; p += kRowThreads) {
-            const int i = (p / h) * 2 * h + (p % h);
-            const float a = v[i], b = v[i + h];
-            v[i] = a + b;
-            v[i + h] = a - b;
+    for (int h = 1; h < T && h < 32; h <<= 1) {
+        const bool hi = (t & h) != 0;
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+            const float p = __shfl_xor_sync(0xffffffffu, v[e], h);
+            v[e] = hi ? p - v[e] : v[e] + p;
+        }
+    }
+    for (int h = 32; h < T; h <<= 1) {        // T >= 64 here, every thread owns elements
+        const bool hi = (t & h) != 0;
+#pragma unroll
+        for (int e = 0; e < E; ++e) buf[t + T * e] = v[e];
+        __syncthreads();
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+            const float p = buf[(t ^ h) + T * e];
+            v[e] = hi ? p - v[e] : v[e] + p;
         }
         __syncthreads();
     }
-    // the order-28 stage across segments: v[a seg + b] <- sum_a' H[a][a'] v[a' seg + b]
-    // (inverse: H^T)
-    if (outer == 28) {
-        for (int b = tid; b < seg; b += kRowThreads) {
-            float in[28], out[28];
 #pragma unroll
-            for (int a = 0; a < 28; ++a) in[a] = v[a * seg + b];
+    for (int q = 1; q < U; q <<= 1) {         // strides T, 2T, ... < seg: inside the thread
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+            if ((e & q) == 0) {
+                const float a = v[e], b = v[e | q];
+                v[e] = a + b;
+                v[e | q] = a - b;
+            }
+        }
+    }
+    if (OUTER == 28) {                        // v[a U + u] <- sum_c H[a][c] v[c U + u] (or H^T)
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            float out[28];
 #pragma unroll
             for (int a = 0; a < 28; ++a) {
                 float acc = 0.f;
 #pragma unroll
-                for (int c = 0; c < 28; ++c) {
-                    const int hv = inverse ? H.h[c][a] : H.h[a][c];
-                    acc = hv > 0 ? acc + in[c] : acc - in[c];
-                }
+                for (int c = 0; c < 28; ++c)
+                    acc = fmaf(kInverse ? H.h[c][a] : H.h[a][c], v[c * U + u], acc);
                 out[a] = acc;
             }
 #pragma unroll
-            for (int a = 0; a < 28; ++a) v[a * seg + b] = out[a];
+            for (int a = 0; a < 28; ++a) v[a * U + u] = out[a];
         }
-        __syncthreads();
     }
+    if (!own) return;
     float* y = Y + row * (size_t)d;
-    for (int j = tid; j < d; j += kRowThreads) y[j] = (inverse ? v[j] * sign(j) : v[j]) * scale;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+        const int j = t + T * e;
+        y[j] = (kInverse ? v[e] * sgn(j) : v[e]) * scale;
+    }
 }
 
 // Y (c x r) = X^T for X (r x c), 32 x 32 tiles.
@@ -176,19 +213,52 @@ __global__ void row_scales_kernel(const float* __restrict__ W, int n, int group,
     }
 }
 
-int rows_pass(const float* X, float* Y, int rows, int d, unsigned long long seed, int inverse,
-              const H28& H, cudaStream_t st) {
-    int seg = 0;
-    const int outer = factor(d, seg);
+template <int U, int OUTER, bool kInverse>
+int launch_rows(const float* X, float* Y, int rows, int d, unsigned long long seed,
+                const H28f& H, cudaStream_t st) {
+    const int T = d / (OUTER * U);
     const size_t smem = (size_t)((d + 3) & ~3) * sizeof(float) +
                         (size_t)4 * ((d + 255) / 256) * sizeof(uint64_t);
-    if (cudaFuncSetAttribute(rht_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem) != cudaSuccess)
+    auto kern = rht_rows_kernel<U, OUTER, kInverse>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess)
         return BAKRON_ERR_CUDA;
     const float scale = 1.0f / sqrtf((float)d);
-    rht_rows_kernel<<<rows, kRowThreads, smem, st>>>(X, Y, d, seg, outer, seed, inverse, scale, H);
+    kern<<<rows, T < 32 ? 32 : T, smem, st>>>(X, Y, d, T, seed, scale, H);
     count_launches(1);
     return cuda_err(cudaGetLastError());
+}
+
+// T = min(seg, 512) threads, U = seg / T columns of each segment per thread.
+template <bool kInverse>
+int rows_pass_dir(const float* X, float* Y, int rows, int d, unsigned long long seed,
+                  const H28f& H, cudaStream_t st) {
+    int seg = 0;
+    const int outer = factor(d, seg);
+    const int U = seg <= kRowThreads ? 1 : seg / kRowThreads;
+    if (outer == 28) {
+        switch (U) {
+            case 1: return launch_rows<1, 28, kInverse>(X, Y, rows, d, seed, H, st);
+            case 2: return launch_rows<2, 28, kInverse>(X, Y, rows, d, seed, H, st);
+            default: return BAKRON_ERR_INVALID_ARG;
+        }
+    }
+    switch (U) {
+        case 1: return launch_rows<1, 1, kInverse>(X, Y, rows, d, seed, H, st);
+        case 2: return launch_rows<2, 1, kInverse>(X, Y, rows, d, seed, H, st);
+        case 4: return launch_rows<4, 1, kInverse>(X, Y, rows, d, seed, H, st);
+        case 8: return launch_rows<8, 1, kInverse>(X, Y, rows, d, seed, H, st);
+        case 16: return launch_rows<16, 1, kInverse>(X, Y, rows, d, seed, H, st);
+        case 32: return launch_rows<32, 1, kInverse>(X, Y, rows, d, seed, H, st);
+        case 64: return launch_rows<64, 1, kInverse>(X, Y, rows, d, seed, H, st);
+        default: return BAKRON_ERR_INVALID_ARG;
+    }
+}
+
+int rows_pass(const float* X, float* Y, int rows, int d, unsigned long long seed, int inverse,
+              const H28f& H, cudaStream_t st) {
+    return inverse ? rows_pass_dir<true>(X, Y, rows, d, seed, H, st)
+                   : rows_pass_dir<false>(X, Y, rows, d, seed, H, st);
 }
 
 void transpose(const float* X, float* Y, int r, int c, cudaStream_t st) {
@@ -227,7 +297,13 @@ extern "C" int bakron_rht(const float* X, int rows, int cols, uint64_t seed_rows
         return BAKRON_ERR_INVALID_ARG;
     if (!ws_ok(ws, ws_bytes, bakron_rht_workspace_bytes(rows, cols))) return BAKRON_ERR_WORKSPACE;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    static const H28 H = make_h28();
+    static const H28f H = [] {
+        const H28 h = make_h28();
+        H28f f;
+        for (int a = 0; a < 28; ++a)
+            for (int c = 0; c < 28; ++c) f.h[a][c] = (float)h.h[a][c];
+        return f;
+    }();
     WsCarver c(ws);
     float* t = c.take<float>((size_t)rows * cols);
     int e;
