@@ -447,10 +447,12 @@ def _e2e(args, torch, bk, solver, stream, dev, ws, m, n, bits, Ws, HO, HI, sc,
             "d2h_bytes_per_step": d2h}
 
 
-# DRAM bytes (read + written) of one round_kernel launch on down_4096x14336 with nearest Q,
-# from one ncu capture of this kernel version (dram__bytes_read.sum + dram__bytes_write.sum,
-# 1 pass): 26.98 GB + 9.37 GB. Reported as the roofline's traffic for that workload only.
-ROUND_TRAFFIC_BYTES = {(4096, 14336): 36.35e9}
+# DRAM bytes (read + written) of one round_kernel launch per workload, from one ncu capture of
+# the current kernel version (dram__bytes_read.sum + dram__bytes_write.sum, 1 pass); reported
+# as the roofline's traffic. Empty while the kernel has changed since its last capture (the
+# capture before the per-group grid steps and codebook Q measured 26.98 + 9.37 GB on
+# down_4096x14336).
+ROUND_TRAFFIC_BYTES: dict = {}
 
 
 def _roofline(per, m, n, rounding="nearest", gram_dims=None):
