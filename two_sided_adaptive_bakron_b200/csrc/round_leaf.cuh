@@ -198,7 +198,7 @@ __device__ __forceinline__ void solve_leaf_pushes(int lane, LeafBuf& B, LeafXchg
     X.part[1][0][j] = wT[1];
     X.part[1][1][j] = wR[1];
     pair_sync(bar);                          // slots 0 and 1 are in place
-    pair_sync(bar);                          // round 0: step 0 is being computed
+    pair_sync(bar);                          // first exchange: step 0 is being computed
 #pragma unroll 1
     for (int s0 = 0; s0 < NSLOT; s0 += UW) {
 #pragma unroll
