@@ -21,7 +21,11 @@ Sources (web pages on the method):
   - section 3: the Kronecker factors themselves: the one-sided input second moment
     H_1 = E[x^T x] (also Sketch A's starting point) and Sketch B, one power-iteration round from
     the identity, (H_I)_1 = E_s[G_s^T G_s] / m and (H_O)_1 = E_s[G_s G_s^T] / n over the
-    per-sequence weight gradients G_s (m x n).
+    per-sequence weight gradients G_s (m x n); Sketch A, the alternating reweighted second
+    moments over tokens (x_t the input row, g_t the output gradient row),
+        (H_I)_i = E_t[x_t^T x_t <(H_O)_{i-1}, g_t^T g_t>] / |(H_O)_{i-1}|_F^2,
+        (H_O)_i = E_t[g_t^T g_t <(H_I)_{i-1}, x_t^T x_t>] / |(H_I)_{i-1}|_F^2,
+    started from (H_I)_0 = E[x^T x], (H_O)_0 = I.
 
 Readings taken where the pages are garbled or silent (each one is listed in the design notes):
 * index ranges ``:i`` / ``:j`` are exclusive (rows k < i, columns l < j);
@@ -76,7 +80,7 @@ __all__ = [
     "proxy_loss", "proxy_loss_kron", "brute_force_fixed_points", "gptq_obs",
     "code_range", "fixed_point_pre_rows", "band_check", "grid_quotient",
     "philox4x64_10", "dither", "quantize_stochastic", "damped_gram", "sketch_b",
-    "damped_gram_rows", "codebook_midpoints", "quantize_codebook", "scale_of",
+    "damped_gram_rows", "codebook_midpoints", "quantize_codebook", "scale_of", "sketch_a",
     "gf27_chi", "hadamard28", "hadamard", "rht_signs", "rht_matrix", "rht", "hadamard_rows",
 ]
 
@@ -488,6 +492,23 @@ def damped_gram_rows(X, damp: float, rows) -> np.ndarray:
     mean_diag = float(np.mean(np.einsum("ti,ti->i", X, X))) / N
     out[np.arange(rows.size), rows] += damp * mean_diag
     return out
+
+
+def sketch_a(X, G, iterations: int, damp: float) -> tuple[np.ndarray, np.ndarray]:
+    """Sketch A: ``iterations`` rounds of the alternating update from (H_I)_0 = E[x^T x],
+    (H_O)_0 = I over the token rows of X (T x n, inputs) and G (T x m, output gradients), both
+    factors of a round computed from the previous round's pair; the returned pair is damped
+    (the iterations use the undamped factors). Returns (H_O, H_I) in fp64."""
+    X = np.asarray(X, dtype=np.float64)
+    G = np.asarray(G, dtype=np.float64)
+    T = X.shape[0]
+    HI = X.T @ X / T
+    HO = np.eye(G.shape[1])
+    for _ in range(iterations):
+        w_in = np.einsum("ta,ab,tb->t", G, HO, G) / np.sum(HO * HO)    # <H_O, g^T g> / |H_O|^2
+        w_out = np.einsum("ta,ab,tb->t", X, HI, X) / np.sum(HI * HI)   # <H_I, x^T x> / |H_I|^2
+        HI, HO = (X * w_in[:, None]).T @ X / T, (G * w_out[:, None]).T @ G / T
+    return _damp(HO, damp), _damp(HI, damp)
 
 
 def sketch_b(G, damp: float) -> tuple[np.ndarray, np.ndarray]:

@@ -10,12 +10,15 @@ other than itself:
   identity, identical rows giving a rank-one v v^T, scaling by c giving c^2;
 * Sketch B against the explicit Fisher E_s[vec(G_s) vec(G_s)^T] (mn x mn, row-major vec) and
   its two partial traces, which is what one power-iteration step from the identity computes;
-* the damping adds damp * mean(diag) to the diagonal only.
+* the damping adds damp * mean(diag) to the diagonal only;
+* Sketch A: no round is the one-sided start, one round written out token by token, tokens
+  that all share one x and one g keep x^T x and g^T g as the factors' shapes, and the
+  c^2 scaling of both factors when the gradients scale by c.
 """
 import numpy as np
 import pytest
 
-from oracle import damped_gram, damped_gram_rows, sketch_b
+from oracle import damped_gram, damped_gram_rows, sketch_a, sketch_b
 
 
 def _rng(seed):
@@ -107,3 +110,52 @@ def test_gram_rows_is_the_gram_restricted():
     rows = np.array([0, 5, 22, 5])
     np.testing.assert_allclose(damped_gram_rows(X, 0.03, rows), damped_gram(X, 0.03)[rows],
                                rtol=1e-12, atol=1e-14)
+
+
+# ----------------------------------------------------------------------------- Sketch A
+def test_sketch_a_zero_iterations_is_the_one_sided_start():
+    rng = _rng(8)
+    X, G = rng.standard_normal((50, 6)), rng.standard_normal((50, 4))
+    HO, HI = sketch_a(X, G, 0, 0.01)
+    np.testing.assert_allclose(HI, damped_gram(X, 0.01), rtol=1e-12)
+    np.testing.assert_allclose(HO, (1 + 0.01) * np.eye(4), rtol=1e-12)
+
+
+def test_sketch_a_one_iteration_by_explicit_sums():
+    # the first round written out token by token: w_t = g_t g_t^T / m (H_O = I), and
+    # H_O weights x_t H_1 x_t^T / |H_1|_F^2
+    rng = _rng(9)
+    T, n, m = 7, 3, 2
+    X, G = rng.standard_normal((T, n)), rng.standard_normal((T, m))
+    H1 = sum(np.outer(X[t], X[t]) for t in range(T)) / T
+    HI_ref = sum(np.outer(X[t], X[t]) * (G[t] @ G[t]) / m for t in range(T)) / T
+    HO_ref = sum(np.outer(G[t], G[t]) * (X[t] @ H1 @ X[t]) / np.sum(H1 * H1)
+                 for t in range(T)) / T
+    HO, HI = sketch_a(X, G, 1, 0.0)
+    np.testing.assert_allclose(HI, HI_ref, rtol=1e-12)
+    np.testing.assert_allclose(HO, HO_ref, rtol=1e-12)
+
+
+def test_sketch_a_separable_tokens_keep_the_shapes():
+    # every token has the same x and g: each round returns x^T x and g^T g with a scalar
+    # factor, so the normalised factors are fixed points from the first round on
+    rng = _rng(10)
+    x, g = rng.standard_normal(5), rng.standard_normal(3)
+    X, G = np.tile(x, (9, 1)), np.tile(g, (9, 1))
+    for it in (1, 2, 3):
+        HO, HI = sketch_a(X, G, it, 0.0)
+        np.testing.assert_allclose(HI / np.linalg.norm(HI), np.outer(x, x) / np.linalg.norm(
+            np.outer(x, x)), rtol=1e-12, atol=1e-14)
+        np.testing.assert_allclose(HO / np.linalg.norm(HO), np.outer(g, g) / np.linalg.norm(
+            np.outer(g, g)), rtol=1e-12, atol=1e-14)
+
+
+def test_sketch_a_scale_invariance():
+    # scaling the gradients by c scales both factors of the first round by c^2: H_I through
+    # its weights g H_O g^T (H_O = I), H_O through g^T g (its weights depend on X alone)
+    rng = _rng(11)
+    X, G = rng.standard_normal((40, 6)), rng.standard_normal((40, 4))
+    HO1, HI1 = sketch_a(X, G, 1, 0.0)
+    HO2, HI2 = sketch_a(X, 3.0 * G, 1, 0.0)
+    np.testing.assert_allclose(HI2, 9.0 * HI1, rtol=1e-12)
+    np.testing.assert_allclose(HO2, 9.0 * HO1, rtol=1e-12)
