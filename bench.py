@@ -207,6 +207,13 @@ def whole_job_value(world: int, m: int, n: int, ms_per_step: float) -> float:
     return world * m * n / (ms_per_step * 1e-3)
 
 
+def _gram_device(wl):
+    """Where the input generator forms the large Gram products: the GPU when there is one
+    (the inputs only; the oracle itself runs on the host)."""
+    import torch
+    return "cuda" if wl.m * wl.n > (1 << 22) and torch.cuda.is_available() else None
+
+
 def oracle_sample(wl, arrays=None, seconds_target: float = 12.0):
     """Times the oracle's whole path on leading r x 2r sub-layers of the workload, growing r by
     1.25x until one run takes a quarter of ``seconds_target``; returns the last (r, c, s)."""
@@ -215,7 +222,7 @@ def oracle_sample(wl, arrays=None, seconds_target: float = 12.0):
     import oracle
     from two_sided_adaptive_bakron_b200.workloads import make_workload
     if arrays is None:
-        arrays = make_workload(wl, device="cuda" if wl.m * wl.n > (1 << 22) else None)
+        arrays = make_workload(wl, device=_gram_device(wl))
     Ws, HO, HI, s, bits = arrays
     r = 16.0
     with threadpool_limits(limits=1):
@@ -246,7 +253,7 @@ def run_reference(args):
     import oracle
     from two_sided_adaptive_bakron_b200.workloads import WORKLOADS, make_workload
     wl = WORKLOADS[args.workload]
-    arrays = make_workload(wl, device="cuda" if wl.m * wl.n > (1 << 22) else None)
+    arrays = make_workload(wl, device=_gram_device(wl))
     Ws, HO, HI, s, bits = arrays
     # sizing run (also the first warm-up), then the remaining warm-ups, then K timed steps
     rr, c, _ = oracle_sample(wl, arrays, seconds_target=args.ref_seconds)
