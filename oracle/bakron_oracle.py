@@ -64,8 +64,12 @@ Readings taken where the pages are garbled or silent (each one is listed in the 
   16 (j % 4) and up), u = (field + 1/2) / 2^16. x is the fp32 quotient as for nearest rounding,
   and x + u is one fp32 addition.
 
-Parity status: every function below is pinned by ``tests/test_oracle.py`` against closed
-forms, textbook routines (numpy Cholesky, the GPTQ/OBS update on the vectorised problem),
+Parity status: every function below is pinned against things other than itself by
+``tests/test_oracle.py`` (factorisation, rule, loss), ``test_oracle_stochastic.py`` (Philox and
+stochastic Q), ``test_oracle_hessian.py`` (the Kronecker factors), ``test_oracle_quantizer.py``
+(per-group steps, codebooks) and ``test_oracle_incoherence.py`` (the Hadamard transform):
+closed forms, library routines (numpy Cholesky and Philox, scipy's Hadamard matrix), a
+different algorithm (GPTQ in its optimal-brain-surgeon form on the vectorised problem),
 special cases and brute force. No worked numerical example is printed on the pages, so there
 is no golden value from the pages themselves.
 """
