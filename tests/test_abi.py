@@ -127,3 +127,14 @@ def test_rht_rejects_bad_arguments_on_host(libpath):
     lib.bakron_row_scales.restype = ci
     lib.bakron_row_scales.argtypes = [vp, ci, ci, ci, ctypes.c_float, vp, vp]
     assert lib.bakron_row_scales(fake, 4, 4, 4, 0.0, fake, None) == -1
+
+
+def test_missing_library_fails_loudly(monkeypatch):
+    """There is no CPU fallback: without the built library every call raises."""
+    from two_sided_adaptive_bakron_b200 import bakron
+    monkeypatch.setattr(bakron, "_lib", None)
+    monkeypatch.setattr(bakron, "LIB_PATH", "/nonexistent/libbakron.so")
+    with pytest.raises(RuntimeError, match="missing"):
+        bakron.bakron_version()
+    with pytest.raises(RuntimeError, match="missing"):
+        bakron.bakron_round_workspace_bytes(8, 8)
