@@ -20,6 +20,10 @@
  *     a chain of calls sticks, and bakron_read_status() reads it.
  *   - Nothing traps: device-side waits are bounded and give up with BAKRON_ERR_TIMEOUT.
  *   - Identical inputs give bitwise identical outputs.
+ *   - Host threads: any entry point may be called from several host threads at once (the
+ *     library's own host state, e.g. the SM count per device, is set up once under a lock);
+ *     calls whose buffers, workspaces or status words overlap race on the device unless the
+ *     caller orders their streams.
  */
 #ifndef BAKRON_H_
 #define BAKRON_H_
@@ -276,7 +280,8 @@ const char* bakron_status_string(int code);
  * (diagnostics: lets a benchmark count its launches). */
 unsigned long long bakron_kernel_launches(void);
 
-/* Library version as 10000*major + 100*minor + patch. */
+/* Library version as 10000*major + 100*minor + patch (0.2.0: stochastic Q, the pluggable
+ * base quantizer, the Kronecker-factor and incoherence-processing entry points). */
 int bakron_version(void);
 
 #ifdef __cplusplus

@@ -50,4 +50,4 @@ extern "C" const char* bakron_status_string(int code) {
     }
 }
 
-extern "C" int bakron_version(void) { return 100; }
+extern "C" int bakron_version(void) { return 200; }
