@@ -33,16 +33,19 @@ Readings taken where the pages are garbled or silent (each one is listed in the 
   (the section-4 text also calls it "unit lower"; only the upper reading makes the rule causal
   and the bound hold);
 * Q is round-half-to-even of pre/s_i followed by a clamp to [-2^(b-1), 2^(b-1)-1], per-row
-  scale s_i; s_i = 0 gives code 0. The pages fix no precision for this integer decision, so
-  it is taken in the precision of the CUDA kernels: pre is rounded to fp32 and divided by s_i
-  with one correctly rounded fp32 division before round-half-even (pre itself stays fp64);
+  scale s_i; s_i = 0 gives code 0. The pages fix no precision for this integer decision, so it
+  is the plain one: the real quotient pre/s_i, formed here as one fp64 division of the fp64
+  pre by the (fp32) scale. For inputs that are fp32 values (identity factors, where pre = W*)
+  this decides exactly: a nonzero distance between pre/s and a half-integer is then far above
+  the fp64 rounding of the quotient;
 * E = W* - W always includes the clamp error;
 * the proxy loss is tr(H_O dW H_I dW^T) with no factor 1/2;
 * the base quantizer is pluggable ([BaKron] summary: the solver is modular in the base
   quantizer): the grid step may be per row and column group, s_ij = scales[i, j // group_size],
   and Q may round to a sorted scalar codebook c_0 < ... < c_{K-1} instead of the integers:
-  the code is the index of the nearest entry to x = pre / s_ij (the fp32 quotient), decided
-  against the fp32 midpoints fl32((c_k + c_{k+1}) / 2), a tie going to the lower entry, and
+  the quantizer is given by its decision thresholds, the fp32 midpoints
+  mu_k = fl32((c_k + c_{k+1}) / 2): the code is the number of thresholds strictly below the
+  quotient x = pre / s_ij (real, as for the integer grid), a tie going to the lower entry, and
   W_ij = s_ij c_code;
 * incoherence processing ([YAQA] section 4: like LDLQ, lower the incoherence of the Hessian
   factors before quantising) is the randomised Hadamard transform T_d = H_d S_d / sqrt(d) on
@@ -61,8 +64,9 @@ Readings taken where the pages are garbled or silent (each one is listed in the 
   generator, so u is drawn by Philox4x64-10 (Salmon, Moraes, Dror, Shaw, "Parallel random
   numbers: as easy as 1, 2, 3", SC 2011), keyed by (seed, 0) with counter (j // 16, i, 0, 0);
   entry (i, j) takes the 16-bit field j % 16 of the 256-bit block (word (j % 16) // 4, bits
-  16 (j % 4) and up), u = (field + 1/2) / 2^16. x is the fp32 quotient as for nearest rounding,
-  and x + u is one fp32 addition.
+  16 (j % 4) and up), u = (field + 1/2) / 2^16. x is the real quotient as for nearest
+  rounding, and x + u is formed in fp64 (u has 17 significant bits, so the sum is the real
+  one to fp64 precision).
 
 Parity status: every function below is pinned against things other than itself by
 ``tests/test_oracle.py`` (factorisation, rule, loss), ``test_oracle_stochastic.py`` (Philox and
@@ -124,12 +128,11 @@ def udu(H: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
 # Base quantizer Q ([YAQA] section 4: nearest rounding; reading: half-even, then clamp).
 # ---------------------------------------------------------------------------------------------
 def grid_quotient(pre, s):
-    """pre / s as the rounding decision sees it: fp32(pre) / fp32(s), one correctly rounded
-    fp32 division (elementwise on arrays), returned as fp64."""
+    """The quotient pre / s on which Q decides: the real quotient, formed as one fp64 division
+    (elementwise on arrays)."""
     with np.errstate(divide="ignore", invalid="ignore"):
-        q = np.float32(pre) / np.float32(s) if np.isscalar(pre) and np.isscalar(s) else \
-            np.asarray(pre, dtype=np.float32) / np.asarray(s, dtype=np.float32)
-    return np.asarray(q, dtype=np.float64)
+        q = np.asarray(pre, dtype=np.float64) / np.asarray(s, dtype=np.float64)
+    return q
 
 
 def quantize(pre: float, s: float, bits: int) -> int:
@@ -181,12 +184,12 @@ def dither(rows, n: int, seed: int) -> np.ndarray:
 
 
 def quantize_stochastic(pre: float, s: float, bits: int, u: float) -> int:
-    """Stochastic code for one entry: clamp(floor(x + u)), x the fp32 quotient pre / s and
-    x + u one fp32 addition; s == 0 gives 0."""
+    """Stochastic code for one entry: clamp(floor(x + u)), x the quotient pre / s and x + u
+    both in fp64; s == 0 gives 0."""
     lo, hi = code_range(bits)
     if s == 0.0:
         return 0
-    y = np.float32(grid_quotient(pre, s)) + np.float32(u)
+    y = float(grid_quotient(pre, s)) + float(u)
     return int(min(max(float(np.floor(y)), lo), hi))
 
 
@@ -201,7 +204,7 @@ def codebook_midpoints(codebook) -> np.ndarray:
 
 
 def quantize_codebook(pre: float, s: float, codebook) -> int:
-    """Index of the nearest codebook entry to the fp32 quotient pre / s: the number of
+    """Index of the nearest codebook entry to the quotient pre / s: the number of fp32
     midpoints strictly below it (a tie goes to the lower entry); s == 0 gives index 0."""
     if s == 0.0:
         return 0
@@ -359,7 +362,7 @@ def band_check(pre, codes, scales, bits, band=1e-3, dither=None, codebook=None, 
         frac = np.abs(x - np.floor(x) - 0.5)
     else:
         u = np.asarray(dither, dtype=np.float64)
-        q = np.clip(np.floor(xq.astype(np.float32) + u.astype(np.float32)), lo, hi)
+        q = np.clip(np.floor(xq + u), lo, hi)
         frac = np.abs(x + u - np.rint(x + u))
     q = np.where(s > 0, q, 0.0)
     in_band = frac < band
@@ -597,8 +600,8 @@ def brute_force_fixed_points(Wstar, L_O, L_I, scales, bits, chunk=4096, dither=N
         elif dither is None:
             Q = np.clip(np.rint(xq), lo, hi)
         else:
-            u = np.asarray(dither, dtype=np.float32)[None]
-            Q = np.clip(np.floor(xq.astype(np.float32) + u), lo, hi)
+            u = np.asarray(dither, dtype=np.float64)[None]
+            Q = np.clip(np.floor(xq + u), lo, hi)
         ok = np.all(Q == C, axis=(1, 2))
         found.extend(C[ok])
     return found

@@ -14,11 +14,14 @@ transposed factor, a wrong triangle, a wrong sign, the wrong rounding mode) fail
   (YAQA article, section 4);
 * invariance of the codes under H -> c H.
 """
+from fractions import Fraction
+
 import numpy as np
 import pytest
 
-from oracle import (brute_force_fixed_points, code_range, fixed_point_pre, gptq_obs, grid_quotient,
-                    proxy_loss, proxy_loss_kron, quantize, round_naive, round_row_sweep, udu)
+from oracle import (band_check, brute_force_fixed_points, code_range, fixed_point_pre,
+                    fixed_point_pre_rows, gptq_obs, grid_quotient, proxy_loss, proxy_loss_kron,
+                    quantize, round_naive, round_row_sweep, udu)
 from two_sided_adaptive_bakron_b200.workloads import make_workload, random_problem
 
 
@@ -63,9 +66,37 @@ def test_quantize_half_even_and_clamp():
     assert quantize(-9.7, 1.0, 4) == -8
     assert quantize(3.0, 0.0, 4) == 0     # zero scale row
     assert code_range(3) == (-4, 3)
-    # the decision is taken on the fp32 quotient: 0.7499999999 rounds to fp32 0.75 -> 1
-    assert quantize(0.7499999999, 1.0, 4) == 1
+    # the decision is on the real quotient: just below / above a half-integer (an fp32 quotient
+    # would land on the tie and round to even instead)
+    assert quantize(1.4999999999, 1.0, 4) == 1
+    assert quantize(2.5000000001, 1.0, 4) == 3
+    assert quantize(2.5, 1.0, 4) == 2 and quantize(3.5, 1.0, 4) == 4
     assert quantize(-7.5, 1.0, 4) == -8
+
+
+def _exact_round(pre, s, bits):
+    """Round half to even of the exact rational pre / s, then the clamp (Python fractions)."""
+    lo, hi = code_range(bits)
+    return min(max(round(Fraction(float(pre)) / Fraction(float(s))), lo), hi)
+
+
+def test_quantize_equals_exact_rational_rounding_near_boundaries():
+    # fp32 inputs placed on and within a few ulps of half-integer multiples of the grid step,
+    # where a correctly rounded fp32 quotient would often fall on the tie itself
+    rng = np.random.default_rng(17)
+    hits = 0
+    for _ in range(4000):
+        s = np.float32(rng.uniform(1e-3, 1.0))
+        k = int(rng.integers(-8, 8))
+        pre = np.float32((k + 0.5) * float(s))
+        pre = np.nextafter(pre, np.float32(np.inf) if rng.random() < 0.5 else np.float32(-np.inf)) \
+            if rng.random() < 0.7 else pre
+        exact = _exact_round(pre, s, 4)
+        assert quantize(float(pre), float(s), 4) == exact, (pre, s)
+        fp32q = np.float32(pre) / np.float32(s)
+        hits += int(fp32q - np.floor(fp32q) == 0.5 and Fraction(float(pre)) / Fraction(float(s))
+                    != Fraction(float(fp32q)))
+    assert hits > 100   # the inputs do reach the cases where the fp32 quotient would mislead
 
 
 # ----------------------------------------------------------------------------- special cases
@@ -74,9 +105,8 @@ def test_identity_factors_give_round_to_nearest(m, n, bits, seed):
     Ws, HO, HI, s, _ = random_problem(m, n, bits, seed, kind="identity")
     LO, _, LI, _ = _factors(HO, HI)
     C, _ = round_naive(Ws, LO, LI, s, bits)
-    lo, hi = code_range(bits)
-    # round to nearest, the quotient taken as one fp32 division (the decision precision)
-    rtn = np.clip(np.rint(Ws.astype(np.float32) / s[:, None].astype(np.float32)), lo, hi)
+    # round to nearest of the exact quotient (every row's largest entry sits near a tie)
+    rtn = np.array([[_exact_round(Ws[i, j], s[i], bits) for j in range(n)] for i in range(m)])
     np.testing.assert_array_equal(C, rtn)
 
 
@@ -201,3 +231,50 @@ def test_loss_identity_and_trace_bound(name):
     lo, hi = code_range(bits)
     inner = (C > lo) & (C < hi)
     assert np.all(np.abs(delta[inner]) <= 0.5 * s[:, None].repeat(C.shape[1], 1)[inner] + 1e-12)
+
+
+# ----------------------------------------------------------------------------- the checkers
+@pytest.mark.parametrize("m,n,seed", [(1, 1, 0), (13, 29, 1), (40, 7, 2), (64, 128, 3)])
+def test_fixed_point_pre_rows_equals_full_closed_form(m, n, seed):
+    # the row-restricted closed form (the checker of every large-shape test) against the full
+    # one and against the raster definition's own pre values, for solved and arbitrary W
+    Ws, HO, HI, s, bits = random_problem(m, n, 2, seed)
+    LO, _, LI, _ = _factors(HO, HI)
+    C, W, P = round_naive(Ws, LO, LI, s, bits, return_pre=True)
+    rng = np.random.default_rng(seed)
+    rows = np.unique(np.concatenate([[0, m - 1], rng.integers(0, m, 5)]))
+    full = fixed_point_pre(Ws, W, LO, LI)
+    got = fixed_point_pre_rows(Ws, W, LO, LI, rows)
+    np.testing.assert_allclose(got, full[rows], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(got, P[rows], rtol=0, atol=1e-12)
+    shuffled = rows[::-1].copy()                      # any row order
+    np.testing.assert_allclose(fixed_point_pre_rows(Ws, W, LO, LI, shuffled), full[shuffled],
+                               rtol=0, atol=1e-12)
+    Wr = rng.standard_normal((m, n))                  # the identity holds for any W
+    np.testing.assert_allclose(fixed_point_pre_rows(Ws, Wr, LO, LI, rows),
+                               fixed_point_pre(Ws, Wr, LO, LI)[rows], rtol=0, atol=1e-12)
+
+
+def test_band_check_nearest_flags_wrong_codes():
+    Ws, HO, HI, s, bits = make_workload("small_64x128")
+    LO, _, LI, _ = _factors(HO, HI)
+    C, W = round_naive(Ws, LO, LI, s, bits)
+    pre = fixed_point_pre(Ws, W, LO, LI)
+    assert band_check(pre, C, s, bits, 1e-3)[:2] == (0, 0)
+    lo, hi = code_range(bits)
+    # a code moved by one step, far from a boundary, is a mismatch outside the band
+    x = pre / s[:, None]
+    far = np.argwhere((np.abs(x - np.floor(x) - 0.5) > 0.1) & (C > lo) & (C < hi))
+    i, j = far[len(far) // 2]
+    Cb = C.copy()
+    Cb[i, j] += 1
+    assert band_check(pre, Cb, s, bits, 1e-3)[:2] == (1, 1)
+    # the same move where pre/s sits 1e-4 steps from a half-integer is exempt (in the band)
+    pre2 = pre.copy()
+    pre2[i, j] = (np.floor(x[i, j]) + 0.5 + 1e-4) * s[i]
+    Cc = C.copy()
+    Cc[i, j] = np.floor(x[i, j])                     # nearest would be floor + 1
+    mism, outside, in_band = band_check(pre2, Cc, s, bits, 1e-3)
+    assert (mism, outside) == (1, 0) and in_band >= 1
+    # and the band is what exempts it: with a narrower band the same entry is flagged
+    assert band_check(pre2, Cc, s, bits, 1e-5)[:2] == (1, 1)

@@ -76,7 +76,8 @@ def test_identity_factors_round_to_nearest_per_group_and_codebook():
     C, _ = round_naive(Ws, Z_O, Z_I, sg, bits, group_size=gs)
     lo, hi = code_range(bits)
     sfull = np.repeat(sg, gs, axis=1)[:, :n]
-    np.testing.assert_array_equal(C, np.clip(np.rint(Ws / sfull), lo, hi))
+    np.testing.assert_array_equal(
+        C, np.clip(np.rint(Ws.astype(np.float64) / sfull.astype(np.float64)), lo, hi))
     sc = _group_scales(Ws, gs, 1.0)
     C, W = round_naive(Ws, Z_O, Z_I, sc, 3, codebook=CB3, group_size=gs)
     sfull = np.repeat(sc, gs, axis=1)[:, :n].astype(np.float64)

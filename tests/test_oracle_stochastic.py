@@ -89,9 +89,11 @@ def test_quantize_stochastic_cases():
     assert quantize_stochastic(3.0, 0.0, 4, 0.5) == 0
     # integers stay put for any u < 1
     assert quantize_stochastic(2.0, 0.5, 4, 0.99998) == 4
-    # the sum is one fp32 addition: 0.49999997 (fp32) + 0.5 rounds to 1.0
+    # the sum is the real one: 0.49999997 (fp32) + 0.5 stays below 1 (an fp32 addition would
+    # round it up to 1.0)
     x = float(np.float32(0.5) - np.float32(2.0 ** -25))
-    assert quantize_stochastic(x, 1.0, 4, 0.5) == 1
+    assert quantize_stochastic(x, 1.0, 4, 0.5) == 0
+    assert quantize_stochastic(0.5, 1.0, 4, 0.5) == 1
 
 
 def test_stochastic_q_is_unbiased():
@@ -119,9 +121,17 @@ def test_stochastic_q_is_unbiased():
 @pytest.mark.parametrize("kind", ["identity", "kron"])
 def test_half_dither_is_nearest(kind):
     # floor(x + 1/2) is nearest rounding except at exact ties, where it rounds up instead of to
-    # even; with identity factors every row's largest entry sits on a tie (s = max|W*| / 3.5)
+    # even. With identity factors pre = W*; power-of-two grid steps and entries placed on
+    # half-integer multiples of them make exact ties.
     m, n, bits = 12, 20, 3
     Ws, HO, HI, s, _ = random_problem(m, n, bits, 2, kind=kind)
+    if kind == "identity":
+        rng = np.random.default_rng(3)
+        s = (2.0 ** -(3 + np.arange(m) % 3)).astype(np.float32)
+        Ws = Ws.copy()
+        for i in range(m):
+            cols = rng.choice(n, 4, replace=False)
+            Ws[i, cols] = (rng.integers(-4, 3, 4) + 0.5) * s[i]
     LO, _ = udu(HO)
     LI, _ = udu(HI)
     C0, W0, P0 = round_naive(Ws, LO, LI, s, bits, return_pre=True)
@@ -129,8 +139,9 @@ def test_half_dither_is_nearest(kind):
     xq = grid_quotient(P0, np.broadcast_to(s[:, None], P0.shape))
     tie = xq - np.floor(xq) == 0.5
     if kind == "identity":
-        assert tie.sum() >= m // 2      # most rows: fp32 scales do not always land exactly
+        assert tie.sum() == 4 * m
         np.testing.assert_array_equal(C1[tie], np.minimum(np.floor(xq[tie]) + 1, code_range(bits)[1]))
+        assert np.all(C0[tie] % 2 == 0)
     else:
         assert tie.sum() == 0
     np.testing.assert_array_equal(C0[~tie], C1[~tie])
@@ -198,7 +209,6 @@ def test_stochastic_row_sweep_and_closed_form(m, n, bits, seed):
     # stochastic codes differ from nearest on a good share of the entries
     C0, _ = round_naive(Ws, LO, LI, s, bits)
     assert np.mean(C0 != C) > 0.1
-    # the grid decision uses the fp32 quotient
+    # the grid decision is floor(pre / s + u) on the real values
     i, j = 1, 2
-    xq = grid_quotient(P[i, j], s[i])
-    assert C[i, j] == np.clip(np.floor(np.float32(xq) + np.float32(U[i, j])), *code_range(bits))
+    assert C[i, j] == np.clip(np.floor(P[i, j] / s[i] + U[i, j]), *code_range(bits))
