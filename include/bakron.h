@@ -42,7 +42,8 @@ typedef enum {
     BAKRON_ERR_CUDA = -3,         /* a CUDA launch or runtime call failed                */
     BAKRON_ERR_TIMEOUT = -4,      /* a device-side dependency wait gave up               */
     BAKRON_ERR_WORKSPACE = -5,    /* workspace NULL, too small or misaligned (256 B)     */
-    BAKRON_ERR_NONFINITE = -6     /* a non-finite value met on the device                */
+    BAKRON_ERR_NONFINITE = -6,    /* a non-finite value met on the device                */
+    BAKRON_ERR_CAPTURE = -7       /* a set-up step that cannot run under stream capture  */
 } bakron_status;
 
 /* ------------------------------------------------------------------------------------------
@@ -79,9 +80,13 @@ int bakron_ldl(const float* H, int n, float* L, float* D,
  *   n        [in]  1 <= n <= bakron_ldl_noalloc_max_n() (2048); larger n returns
  *                  BAKRON_ERR_INVALID_ARG without touching the device.
  * The first call on a device looks up the array's device address (cudaGetSymbolAddress) with
- * that device current; make that first call before any stream capture. Calls share the
- * array: two calls that overlap on the GPU (different streams or host threads) race. Nothing
- * in the array needs to start at zero. Allocates nothing.
+ * that device current, and caches it with the id of the device's current CUDA context; a call
+ * that finds a different context current (the context was destroyed and created again, e.g.
+ * by cudaDeviceReset) looks the address up again. Make the first call on a device, and the
+ * first after such a reset, before any stream capture: a lookup while `stream` is capturing is
+ * refused with BAKRON_ERR_CAPTURE, the capture untouched. Calls share the array: two calls that
+ * overlap on the GPU (different streams or host threads) race. Nothing in the array needs to
+ * start at zero. Allocates nothing.
  * ---------------------------------------------------------------------------------------- */
 int bakron_ldl_noalloc(const float* H, int n, float* L, float* D, int* dev_status,
                        void* stream);
@@ -99,7 +104,9 @@ int bakron_ldl_noalloc_max_n(void);
  *
  * where a_i is column i of L_O (entries k < i), b_j is column j of L_I (entries l < j), and
  * ":i" means indices 0..i-1. Equivalently W = Q(W* + (I+L_O)^T E (I+L_I) - E) holds at every
- * entry (the closed form used to check results).
+ * entry (the closed form used to check results). pre_ij is accumulated in fp32 (products as
+ * 3xTF32 on the tensor cores); the rounding decision is exact for that fp32 value, i.e. it
+ * rounds the real quotient pre_ij / s_i, not an fp32 approximation of it.
  *
  *   Wstar    [in]  m x n.
  *   m, n     [in]  1 <= m, n; m*n < 2^31.
@@ -127,8 +134,8 @@ int bakron_round(const float* Wstar, int m, int n, const float* L_O, const float
  *   code_ij = clamp(floor(x_ij + u_ij), -2^(bits-1), 2^(bits-1) - 1),   x_ij = pre_ij / s_i,
  *
  * so that, away from the clamp, s_i code_ij is an unbiased rounding of pre_ij: it takes the
- * grid point above with probability frac(x_ij). x_ij is the correctly rounded fp32 quotient
- * and x_ij + u_ij one fp32 addition. The variate u_ij = (k_ij + 1/2) / 2^16, where k_ij is the
+ * grid point above with probability frac(x_ij). The decision is exact for the kernel's fp32
+ * pre_ij: floor of the real x_ij + u_ij. The variate u_ij = (k_ij + 1/2) / 2^16, where k_ij is the
  * 16-bit field (j mod 16) (least significant first: word (j mod 16) / 4, bits 16 (j mod 4)
  * and up) of the Philox4x64-10 block (Salmon, Moraes, Dror, Shaw, "Parallel random numbers:
  * as easy as 1, 2, 3", SC 2011) with key (seed, 0) and counter (j / 16, i, 0, 0).
@@ -152,7 +159,7 @@ int bakron_round_stochastic(const float* Wstar, int m, int n, const float* L_O,
  *   with a codebook c_0 < ... < c_{K-1}, K = 2^bits:
  *            code_ij = the index k of the entry nearest to x = pre_ij / s_ij, decided against
  *                      the fp32 midpoints fl32((c_k + c_{k+1}) / 2) (a tie goes to the lower
- *                      entry; x is the correctly rounded fp32 quotient),
+ *                      entry; x is the real quotient of the kernel's fp32 pre_ij),
  *            W_ij    = s_ij c_k.
  *
  *   scales   [in]  m x G grid steps (device), s_ij >= 0 (0: code 0 and W 0 on that row part;

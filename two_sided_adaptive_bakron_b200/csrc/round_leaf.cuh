@@ -59,14 +59,17 @@ static_assert(offsetof(LeafBuf, LOr) % 16 == 0 && offsetof(LeafBuf, LIc) % 16 ==
 // zero for d > j and LOr for r + d >= 32, so no push needs a guard (a lane j < d gets its own
 // u back from the shuffle and multiplies it by zero). The step loop stays rolled (4 steps per
 // iteration) over a sliding window of 36 slot registers, so every register index is static.
-// Q divides by s_r as one correctly rounded fp32 division: the quotient is formed as
-// pre * (1/s_r), whose distance to the division's result is below 2e-7 |x|, and the exact
-// division is taken instead whenever that quotient lies within 1e-6 max(1,|x|) of a rounding
-// boundary, so the decision always equals the division's. Stochastic Q (kStochastic) decides on
-// y = x + u (one fp32 addition) with floor: its boundaries are the integers, and the exact
-// division is taken whenever y lies within 1e-6 max(1,|y|) of one; the two y differ by at most
-// 2e-7 |x| + 2^-24 (|y| + |y'|) <= 5.2e-7 max(1,|y|) since |x| <= |y| + 1, so outside that
-// zone both lie between the same integers.
+// Q decides on the real quotient pre / s_r of the fp32 pre. It is estimated as
+// x = pre * (1/s_r), within 1.2e-7 |x| of the real quotient (two correctly rounded steps);
+// where x lies more than 1e-6 max(1,|x|) from every rounding boundary b, the estimate decides.
+// Inside that zone the side is taken from the sign of r = fmaf(-b, s_r, pre): b * s_r is exact
+// inside the fma (b has at most 24 significant bits) and the single rounding of the fma keeps
+// the sign of the exact residual pre - b s_r, so the decision is the real one (r == 0 is an
+// exact tie). The boundaries: k + 1/2 for nearest rounding (a tie goes to the even code); for
+// stochastic Q (kStochastic, floor(pre/s + u)) the points pre/s = k - u, k an integer, with
+// k - u exact in fp32 for |k| <= 128 (u has 17 significant bits), which covers every k that the
+// clamp does not absorb, and y = x + u estimated within 1.2e-7 |x| + 2^-24 |y| <= 5e-7 max(1,|y|);
+// for a codebook its fp32 midpoints.
 //
 // The wavefront runs on two warps: the solver warp runs the element chain (the slot's sum, Q,
 // e, u and the distance-1 terms), the helper warp the distance >= 2 pushes one step behind.
@@ -90,7 +93,7 @@ __device__ __forceinline__ void pair_sync(int id) {
 // Codebook Q: cb (shared memory) holds the entries, mid (any memory, read once per leaf) the
 // decision thresholds fl32((c_k + c_{k+1}) / 2), +inf past the last one; the code is the number
 // of thresholds below x (a tie goes to the lower entry), found by independent compares that
-// also give the distance to the nearest threshold for the exact-division guard.
+// also give the distance to the nearest threshold for the exact decision near one.
 template <QKind kQ>
 __device__ __forceinline__ void solve_leaf_chain(int lane, int rows, int cols, float qlo,
                                                  float qhi, LeafBuf& B, LeafXchg& X, int bar,
@@ -124,7 +127,7 @@ __device__ __forceinline__ void solve_leaf_chain(int lane, int rows, int cols, f
             float q = 0.f, qv = 0.f;         // the code and its grid value
             if (sr > 0.f) {
                 if constexpr (kQ == QKind::kCodebook) {
-                    float x = pre * inv;
+                    const float x = pre * inv;
                     int k = 0;
                     float dmin = __int_as_float(0x7f800000);
 #pragma unroll
@@ -133,25 +136,35 @@ __device__ __forceinline__ void solve_leaf_chain(int lane, int rows, int cols, f
                         dmin = fminf(dmin, fabsf(x - md[t]));
                     }
                     if (dmin < 1e-6f * fmaxf(1.f, fabsf(x))) {
-                        x = __fdiv_rn(pre, sr);
+                        // exact: pre/s > mu_t iff pre - mu_t s > 0 (+inf thresholds give -inf)
                         k = 0;
 #pragma unroll
-                        for (int t = 0; t < kMaxCodebook - 1; ++t) k += (x > md[t]) ? 1 : 0;
+                        for (int t = 0; t < kMaxCodebook - 1; ++t)
+                            k += (__fmaf_rn(-md[t], sr, pre) > 0.f) ? 1 : 0;
                     }
                     q = (float)k;
                     qv = cb[k];
                 } else if constexpr (kQ == QKind::kStochastic) {
                     const float uv = ((float)(uint16_t)B.oC[rr * LB + j] + 0.5f) * (1.f / 65536.f);
-                    float y = __fadd_rn(__fmul_rn(pre, inv), uv);
-                    const float t = fabsf(y - rintf(y));
-                    if (t < 1e-6f * fmaxf(1.f, fabsf(y))) y = __fadd_rn(__fdiv_rn(pre, sr), uv);
-                    q = fminf(fmaxf(floorf(y), qlo), qhi);
+                    const float y = __fadd_rn(__fmul_rn(pre, inv), uv);
+                    const float k = rintf(y);
+                    float f = floorf(y);
+                    if (fabsf(y - k) < 1e-6f * fmaxf(1.f, fabsf(y)))
+                        // exact: pre/s + u >= k iff pre - (k - u) s >= 0
+                        f = (__fmaf_rn(-__fsub_rn(k, uv), sr, pre) >= 0.f) ? k : k - 1.f;
+                    q = fminf(fmaxf(f, qlo), qhi);
                     qv = q;
                 } else {
-                    float x = pre * inv;
-                    const float t = fabsf(x - rintf(x));
-                    if (0.5f - t < 1e-6f * fmaxf(1.f, fabsf(x))) x = __fdiv_rn(pre, sr);
-                    q = fminf(fmaxf(rintf(x), qlo), qhi);
+                    const float x = pre * inv;
+                    float c = rintf(x);
+                    const float t = fabsf(x - c);
+                    if (0.5f - t < 1e-6f * fmaxf(1.f, fabsf(x))) {
+                        // exact: the side of b = floor(x) + 1/2 from the sign of pre - b s; a
+                        // zero residual is a tie, which goes to the even neighbour
+                        const float lo = floorf(x), r = __fmaf_rn(-(lo + 0.5f), sr, pre);
+                        c = r > 0.f ? lo + 1.f : (r < 0.f ? lo : rintf(lo + 0.5f));
+                    }
+                    q = fminf(fmaxf(c, qlo), qhi);
                     qv = q;
                 }
             }
