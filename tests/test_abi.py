@@ -29,6 +29,14 @@ def test_host_side_queries_without_gpu(libpath):
     assert bakron.bakron_version() >= 100
     assert bakron.status_string(0) == "ok"
     assert "timed out" in bakron.status_string(-4)
+    assert "capture" in bakron.status_string(bakron.BAKRON_ERR_CAPTURE)
+    # every status the header declares has its own message
+    import re
+    with open(bakron.HEADER_PATH) as f:
+        codes = [int(v) for v in re.findall(r"BAKRON_ERR_\w+ = (-\d+)", f.read())]
+    assert len(codes) >= 7
+    assert len({bakron.status_string(c) for c in codes}) == len(codes)
+    assert all(bakron.status_string(c) != "unknown status" for c in codes)
     assert bakron.bakron_round_workspace_bytes(0, 5) == 0
     m, n = 100, 37
     assert bakron.bakron_round_workspace_bytes(m, n) >= 2 * 4 * m * n

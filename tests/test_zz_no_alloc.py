@@ -56,3 +56,38 @@ def test_noalloc_ldl_rejects_too_large(bk):
     D = torch.empty((n,), device="cuda")
     st = bk.new_status("cuda")
     assert bk.bakron_ldl_noalloc(H, L, D, st) == bk.BAKRON_ERR_INVALID_ARG
+
+
+def test_noalloc_first_call_under_capture_is_refused(bk):
+    """The first call in a fresh process, made while its stream captures a CUDA graph, must
+    not look up the scratch address (that may load the module): it returns BAKRON_ERR_CAPTURE
+    and leaves the capture intact; the same call after the capture works."""
+    import os
+    import subprocess
+    import sys
+    code = r"""
+import numpy as np, torch
+from two_sided_adaptive_bakron_b200 import bakron as bk
+from two_sided_adaptive_bakron_b200.workloads import random_problem
+_, H_np, _, _, _ = random_problem(64, 3, 2, 5)
+H = torch.from_numpy(H_np).cuda()
+L = torch.empty((64, 64), device='cuda'); D = torch.empty((64,), device='cuda')
+st = bk.new_status('cuda')
+bk.lib()
+s = torch.cuda.Stream()
+torch.cuda.synchronize()
+g = torch.cuda.CUDAGraph()
+with torch.cuda.graph(g, stream=s):
+    rc = bk.bakron_ldl_noalloc(H, L, D, st, stream=s)
+print('CAPTURED', rc)
+rc2 = bk.bakron_ldl_noalloc(H, L, D, st)
+print('AFTER', rc2, bk.bakron_read_status(st))
+Lr, Dr = bk.ldl(H)
+print('SAME', bool(torch.equal(L, Lr) and torch.equal(D, Dr)))
+"""
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, "-c", code], cwd=root, capture_output=True, text=True,
+                       timeout=300)
+    assert r.returncode == 0, r.stderr
+    assert f"CAPTURED {bk.BAKRON_ERR_CAPTURE}" in r.stdout, r.stdout
+    assert "AFTER 0 0" in r.stdout and "SAME True" in r.stdout, r.stdout

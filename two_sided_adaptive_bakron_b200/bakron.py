@@ -32,6 +32,7 @@ BAKRON_ERR_CUDA = -3
 BAKRON_ERR_TIMEOUT = -4
 BAKRON_ERR_WORKSPACE = -5
 BAKRON_ERR_NONFINITE = -6
+BAKRON_ERR_CAPTURE = -7
 
 _c_size_t, _c_int, _vp = ctypes.c_size_t, ctypes.c_int, ctypes.c_void_p
 _SIGNATURES = {

@@ -46,6 +46,7 @@ extern "C" const char* bakron_status_string(int code) {
         case BAKRON_ERR_TIMEOUT: return "device-side dependency wait timed out";
         case BAKRON_ERR_WORKSPACE: return "workspace missing, too small or misaligned";
         case BAKRON_ERR_NONFINITE: return "non-finite value on the device";
+        case BAKRON_ERR_CAPTURE: return "set-up step refused under stream capture";
         default: return "unknown status";
     }
 }
