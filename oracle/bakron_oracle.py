@@ -327,9 +327,8 @@ def fixed_point_pre_rows(Wstar, W, L_O, L_I, rows):
     Ws = np.asarray(Wstar, dtype=np.float64)
     E = Ws - np.asarray(W, dtype=np.float64)
     m, n = E.shape
-    LO = np.asarray(L_O, dtype=np.float64)
     LI = np.asarray(L_I, dtype=np.float64)
-    AoT_R = LO[:, rows].T.copy()
+    AoT_R = np.asarray(np.asarray(L_O)[:, rows], dtype=np.float64).T.copy()   # (L_O^T)[R, :]
     AoT_R[np.arange(rows.size), rows] += 1.0
     T = AoT_R @ E
     return Ws[rows] + T + T @ LI - E[rows]
@@ -371,9 +370,11 @@ def band_check(pre, codes, scales, bits, band=1e-3, dither=None, codebook=None, 
 
 
 def proxy_loss(dW, H_O, H_I) -> float:
-    """tr(H_O dW H_I dW^T) in fp64 ([YAQA] section 4 proxy; no factor 1/2)."""
+    """tr(H_O dW H_I dW^T) in fp64 ([YAQA] section 4 proxy; no factor 1/2), the trace of the
+    product written out: tr(A dW^T) = sum_ij A_ij dW_ij with A = H_O dW H_I."""
     d = np.asarray(dW, dtype=np.float64)
-    return float(np.trace(np.asarray(H_O, np.float64) @ d @ np.asarray(H_I, np.float64) @ d.T))
+    A = np.asarray(H_O, np.float64) @ d @ np.asarray(H_I, np.float64)
+    return float(np.sum(A * d))
 
 
 def proxy_loss_kron(dW, H_O, H_I) -> float:

@@ -18,7 +18,8 @@ import pytest
 
 torch = pytest.importorskip("torch")
 
-from oracle import damped_gram, damped_gram_rows, sketch_b
+from oracle import (band_check, damped_gram, damped_gram_rows, fixed_point_pre, proxy_loss,
+                    sketch_b)
 from two_sided_adaptive_bakron_b200.workloads import make_layer_samples
 
 pytestmark = pytest.mark.gpu
@@ -109,11 +110,18 @@ def test_sketch_b_factors_feed_the_solver(bk):
     H_O, H_I = bk.sketch_b(_dev(G), 0.01)
     Ws = (np.random.default_rng(10).standard_normal((m, n)) / np.sqrt(n)).astype(np.float32)
     s = (np.abs(Ws).max(axis=1) / np.float32((1 << (bits - 1)) - 0.5)).astype(np.float32)
-    codes, W, loss, _, _ = bk.solve(_dev(Ws), H_O, H_I, _dev(s), bits)
-    assert np.isfinite(float(loss.item())) and float(loss.item()) > 0
+    codes, W, loss, (L_O, _), (L_I, _) = bk.solve(_dev(Ws), H_O, H_I, _dev(s), bits)
     lo, hi = -(1 << (bits - 1)), (1 << (bits - 1)) - 1
-    c = codes.cpu().numpy()
+    c = codes.cpu().numpy().astype(np.int64)
     assert c.min() >= lo and c.max() <= hi
+    # the codes are the rule's fixed point with the factors the library made of these factors
+    Wn = W.cpu().numpy()
+    pre = fixed_point_pre(Ws, Wn, L_O.cpu().numpy(), L_I.cpu().numpy())
+    mism, outside, _ = band_check(pre, c, s, bits, 1e-3)
+    assert outside == 0 and mism <= 1e-3 * c.size
+    # and the loss is that of the residual under the Sketch-B factors themselves
+    ref = proxy_loss(Ws - Wn, H_O.cpu().numpy(), H_I.cpu().numpy())
+    assert abs(float(loss.item()) - ref) <= 1e-3 * ref
 
 
 def test_invalid_arguments(bk):

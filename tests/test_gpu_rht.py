@@ -8,7 +8,8 @@ rotated solve, against the fp64 oracle (run on a B200), through the C ABI.
   worst case of the arithmetic: each butterfly level adds at most sqrt(2) u of the norm
   (u = 2^-24), an order-28 sum at most 27 sqrt(28) u of its inputs' norm, over both sides;
   typical errors are near 1e-7.
-* Full size (4096 x 14336): sampled entries against the oracle's rows of T, the round trip and
+* Full size (the 4096 x 14336 and 28672 x 8192 layers, and shapes that reach the row lengths
+  2048, 16384 and 32768): sampled entries against the oracle's rows of T, the round trip and
   the norm.
 * Grid steps: bitwise equal to fp32 max / divisor.
 * The rotated solve: the proxy loss in the rotated basis equals the oracle's loss of the
@@ -76,8 +77,10 @@ def test_in_place(bk):
     np.testing.assert_array_equal(d.cpu().numpy(), bk.rht(_dev(X), 9, 10).cpu().numpy())
 
 
-def test_full_size_sampled_and_round_trip(bk):
-    r, c = 4096, 14336
+# the layer shapes of the benchmark workloads (4096 x 14336, 28672 x 8192) and the row
+# lengths that no smaller test reaches: 2048, 8192, 16384, 28672 and 32768
+@pytest.mark.parametrize("r,c", [(4096, 14336), (28672, 8192), (2048, 16384), (512, 32768)])
+def test_full_size_sampled_and_round_trip(bk, r, c):
     X = np.random.default_rng(11).standard_normal((r, c)).astype(np.float32)
     Xd = _dev(X)
     Y = bk.rht(Xd, 12, 13)
@@ -85,8 +88,8 @@ def test_full_size_sampled_and_round_trip(bk):
     nx = float(torch.linalg.norm(Xd.double()))
     assert float(torch.linalg.norm(back.double() - Xd.double())) <= 4e-5 * nx
     assert abs(float(torch.linalg.norm(Y.double())) - nx) <= 2e-5 * nx
-    rows = np.array([0, 1, 2047, 4095])
-    cols = np.array([0, 511, 512, 7000, 14335])
+    rows = np.unique(np.array([0, 1, r // 2 - 1, r // 2, r - 1]))
+    cols = np.unique(np.array([0, c // 28 - 1, c // 28, c // 2, c - 1]))
     Tr = _t_rows(r, 12, rows)
     Tc = _t_rows(c, 13, cols)
     ref = Tr @ X.astype(np.float64) @ Tc.T
