@@ -27,14 +27,18 @@
 //    The solver and helper warps run the in-leaf wavefront (round_leaf.cuh); the solver then
 //    publishes E and U^T and releases the leaf's flag, the helper publishes the U and E^T
 //    planes and counts the leaf into its super-block, and the loaders copy out codes and W.
-//  * GEMM CTAs run the far-field pushes as 3xTF32 tcgen05 tile tasks (128 x 128, K = one
-//    super-block): E of super-block (A', C) into T_far of a target (A, C) with A >= A' + 2, and
-//    U of (A, C') into R_far of (A, C) with C >= C' + 2, i.e. the divide-and-conquer
-//    off-diagonal products as dense block products. Tasks are ordered by their source
-//    super-block in the order the sources finish (anti-diagonal, then row), nearest targets
-//    first; each output tile takes its sources in increasing order (a per-tile counter), so
-//    sums are deterministic, and a tile's successive sources are one super-block apart in
-//    time, so that order rarely has to wait.
+//  * GEMM CTAs run the far-field pushes as 3xTF32 tcgen05 tile tasks (128 x 128): E of the
+//    super-blocks (A', C) into T_far of a target (A, C) with A >= A' + 2, and U of (A, C')
+//    into R_far of (A, C) with C >= C' + 2, i.e. the divide-and-conquer off-diagonal products
+//    as dense block products. A target takes its sources in batches by distance, {2}, {3},
+//    {4, 5}, {6 .. 9}, {10 .. 17}, ... (consecutive super-blocks, so one batch is one product
+//    over their joint K range): the nearest source, which is needed soonest, alone, the older
+//    ones in ever longer products, so a target with c sources takes about log2(c) additions of
+//    its tile instead of c. Tasks are ordered by their newest source super-block in the order
+//    the sources finish (anti-diagonal, then row), nearest targets first, and handed out one at
+//    a time from a global counter, so a free CTA always takes the oldest task nobody has taken;
+//    each output tile takes its batches oldest first (a per-tile counter), so sums are
+//    deterministic.
 // Every task depends only on tasks that come earlier in one global order (leaves by
 // anti-diagonal, the pushes of a super-block right after its last leaf and before the first
 // leaf two super-blocks on), so the persistent CTAs always make progress; every wait is
@@ -59,6 +63,7 @@ using leaf::QKind;
 using leaf::kMaxCodebook;
 using leaf::solve_leaf_chain;
 using leaf::solve_leaf_pushes;
+using leaf::swz;
 
 constexpr int SB = 256;              // super-block edge
 constexpr int LPB = SB / LB;         // leaves per super-block edge
@@ -95,6 +100,7 @@ struct FusedArgs {
     int* cntT;           // [TM * TN] far sources added into the T_far tile
     int* cntR;           // [TM * TN] far sources added into the R_far tile
     int* abort_word;
+    int* task_next;      // next push task to hand out (GEMM CTAs take tasks from it)
     int* status;
     const int* task_pre; // [nsb + 1] first push task of each source super-block (in order)
     const int2* task_sb; // [nsb] (A, C) of the source super-blocks, anti-diagonal order
@@ -126,10 +132,11 @@ struct LeafMaps {
 constexpr int NRING = 4;             // sources in flight per leaf group (box-load path)
 constexpr int kBox = LB * LB;        // floats of one 32 x 32 box
 
-struct alignas(128) LeafGroupSmem {
+struct alignas(1024) LeafGroupSmem {
+    // box-load path: NRING stages of two boxes (swizzled copies: 1024-byte aligned); plain
+    // path: sA, sB in stage 0
+    float ring[NRING][2][kBox];
     LeafBuf buf[2];
-    // box-load path: NRING stages of two boxes; plain path: sA, sB in stage 0
-    alignas(128) float ring[NRING][2][kBox];
     uint64_t rfull[NRING];       // box loads of a ring stage landed
     uint64_t sbar;               // W* and the diagonal blocks landed
     uint64_t tbar;               // T_far and R_far landed
@@ -143,17 +150,36 @@ struct LeafCtaSmem {
     LeafGroupSmem g[2];
     float qcb[kMaxCodebook];     // the codebook (read with a per-lane index)
 };
-static_assert(sizeof(LeafGroupSmem) % 128 == 0 && offsetof(LeafGroupSmem, buf) % 128 == 0 &&
-                  offsetof(LeafGroupSmem, ring) % 128 == 0,
-              "leaf group layout: 16-byte staging rows, 128-byte box destinations");
+static_assert(sizeof(LeafGroupSmem) % 1024 == 0 && offsetof(LeafGroupSmem, buf) % 128 == 0 &&
+                  offsetof(LeafGroupSmem, ring) % 1024 == 0 && (kBox * 4) % 1024 == 0,
+              "leaf group layout: 16-byte staging rows, 128-byte box destinations, 1024-byte "
+              "swizzled box destinations");
 
 constexpr size_t kGemmSmem = tc::gemm_smem_bytes<BN, STAGES>();
-constexpr size_t kLeafSmem = sizeof(LeafCtaSmem) + 128;   // + alignment slack
+constexpr size_t kLeafSmem = sizeof(LeafCtaSmem) + 1024;  // + alignment slack
 constexpr size_t kSmem = kLeafSmem > kGemmSmem ? kLeafSmem : kGemmSmem;
 static_assert(kSmem <= 227 * 1024, "shared memory above the per-CTA limit");
+static_assert(kGemmSmem + 256 <= kSmem, "room for the push CTAs' task ring after the barriers");
 
 __device__ __forceinline__ int leaves_in(int extent_leaves, int blk) {
     return min(LPB, extent_leaves - blk * LPB);
+}
+
+// Batch j of a target's far sources: the super-blocks at distances bd_min(j) .. bd_max(j)
+// (2, 3, 4-5, 6-9, 10-17, ...). A target at index X along the push direction has its sources at
+// distances 2 .. X, in n_batches(X) batches; a source at index Xs is the newest source of
+// batch j of the target Xs + bd_min(j), for the n_ready(Xs, NX) such targets inside the matrix.
+__host__ __device__ constexpr int bd_min(int j) { return j < 2 ? 2 + j : (1 << (j - 1)) + 2; }
+__host__ __device__ constexpr int bd_max(int j) { return j < 2 ? 2 + j : (1 << j) + 1; }
+__host__ __device__ inline int n_batches(int X) {
+    int j = 0;
+    while (bd_min(j) <= X) ++j;
+    return j;
+}
+__host__ __device__ inline int n_ready(int Xs, int NX) {
+    int j = 0;
+    while (Xs + bd_min(j) < NX) ++j;
+    return j;
 }
 
 // Walks the leaves in anti-diagonal order (d = I + J, then I); g must not decrease.
@@ -207,18 +233,22 @@ __device__ __forceinline__ void mma_16x8x8_tf32(float (&d)[4], const uint32_t (&
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
 
-// One source's contribution D[m][n] += sum_k X[k][m] Y[k][n] (X, Y: 32 x 32, row stride 32) on
-// the tensor cores, 3xTF32 as in the GEMM engine (hi = tf32 truncation, lo = x - hi,
-// hi*hi + hi*lo + lo*hi). Warp w of the group holds rows 16w .. 16w + 15, all 32 columns:
-// acc[nt] is the m16n8 accumulator of columns 8nt .. 8nt + 7 (element q at row
-// 16w + g + 8 (q >> 1), column 8nt + 2t + (q & 1), g = lane / 4, t = lane % 4).
+// One source's contribution D[m][n] += sum_k X[k][m] Y[k][n] (X, Y: 32 x 32 tiles in the
+// swizzled layout swz) on the tensor cores, 3xTF32 as in the GEMM engine (hi = tf32
+// truncation, lo = x - hi, hi*hi + hi*lo + lo*hi). Warp w of the group holds rows
+// 16w .. 16w + 15, all 32 columns: acc[nt] is the m16n8 accumulator of columns 8nt .. 8nt + 7
+// (element q at row 16w + g + 8 (q >> 1), column 8nt + 2t + (q & 1), g = lane / 4,
+// t = lane % 4). Within each group of 8 k the fragment's k = t is taken from tile row 2t and
+// k = t + 4 from row 2t + 1 (the same permutation for X and Y leaves the sum unchanged), so
+// that every fragment load of the swizzled tiles hits 32 distinct banks.
 __device__ __forceinline__ void product_mma(const float* X, const float* Y, int w, int lane,
                                             float (&acc)[4][4]) {
     const int g = lane >> 2, t = lane & 3;
 #pragma unroll
     for (int k0 = 0; k0 < LB; k0 += 8) {
-        const float a[4] = {X[(k0 + t) * LB + 16 * w + g], X[(k0 + t) * LB + 16 * w + g + 8],
-                            X[(k0 + t + 4) * LB + 16 * w + g], X[(k0 + t + 4) * LB + 16 * w + g + 8]};
+        const int ka = k0 + 2 * t, kb = ka + 1;
+        const float a[4] = {X[swz(ka, 16 * w + g)], X[swz(ka, 16 * w + g + 8)],
+                            X[swz(kb, 16 * w + g)], X[swz(kb, 16 * w + g + 8)]};
         uint32_t ah[4], al[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -228,7 +258,7 @@ __device__ __forceinline__ void product_mma(const float* X, const float* Y, int 
         }
 #pragma unroll
         for (int nt = 0; nt < 4; ++nt) {
-            const float b[2] = {Y[(k0 + t) * LB + 8 * nt + g], Y[(k0 + t + 4) * LB + 8 * nt + g]};
+            const float b[2] = {Y[swz(ka, 8 * nt + g)], Y[swz(kb, 8 * nt + g)]};
             uint32_t bh[2], bl[2];
 #pragma unroll
             for (int i = 0; i < 2; ++i) {
@@ -305,9 +335,8 @@ __device__ void leaf_loaders(const FusedArgs& a, const LeafMaps* maps, LeafGroup
         const int i0 = I * LB, j0 = J * LB;
         const int rows = min(LB, m - i0), cols = min(LB, n - j0);
         // what does not depend on other leaves: W*, the diagonal blocks, the scales
-        const float* dLO;                        // diagonal blocks, row stride dld
+        const float* dLO;                        // diagonal blocks, swizzled 32 x 32 tiles
         const float* dLI;
-        int dld;
         if (box) {
             if (lead) {
                 sm100::mbar_arrive_expect_tx(&sm.sbar, 3 * kBox * 4);
@@ -317,18 +346,16 @@ __device__ void leaf_loaders(const FusedArgs& a, const LeafMaps* maps, LeafGroup
             }
             dLO = sm.ring[0][0];
             dLI = sm.ring[0][1];
-            dld = LB;
         } else {
 #pragma unroll 4
             for (int q = 0; q < (LB * LB) / NLOAD; ++q) {
                 const int e = lt + q * NLOAD, r = e >> 5, c = e & 31;
                 B.W[e] = (r < rows && c < cols) ? __ldg(&a.Ws[(size_t)(i0 + r) * n + j0 + c]) : 0.f;
-                sA[r * LB + c] = (r < rows && c < rows) ? __ldg(&a.LO[(size_t)(i0 + r) * m + i0 + c]) : 0.f;
-                sB[r * LB + c] = (r < cols && c < cols) ? __ldg(&a.LI[(size_t)(j0 + r) * n + j0 + c]) : 0.f;
+                sA[swz(r, c)] = (r < rows && c < rows) ? __ldg(&a.LO[(size_t)(i0 + r) * m + i0 + c]) : 0.f;
+                sB[swz(r, c)] = (r < cols && c < cols) ? __ldg(&a.LI[(size_t)(j0 + r) * n + j0 + c]) : 0.f;
             }
             dLO = sA;
             dLI = sB;
-            dld = LB;
         }
         if (lt < LB) {
             // the leaf's grid step: per row, or per row and column group (one group per leaf)
@@ -353,8 +380,10 @@ __device__ void leaf_loaders(const FusedArgs& a, const LeafMaps* maps, LeafGroup
         if (lead) {
             const int tile = (I * LB / TB) * a.TN + (J * LB / TB);
             bool ok = true;
-            if (A >= 2) ok = wait_geq(&a.cntT[tile], A - 1, a.abort_word, a.status, a.limit_ns);
-            if (ok && C >= 2) ok = wait_geq(&a.cntR[tile], C - 1, a.abort_word, a.status, a.limit_ns);
+            if (A >= 2)
+                ok = wait_geq(&a.cntT[tile], n_batches(A), a.abort_word, a.status, a.limit_ns);
+            if (ok && C >= 2)
+                ok = wait_geq(&a.cntR[tile], n_batches(C), a.abort_word, a.status, a.limit_ns);
             if (ok && box) {
                 // T_far / R_far were written through the generic proxy on other SMs
                 asm volatile("fence.proxy.async.global;" ::: "memory");
@@ -369,8 +398,8 @@ __device__ void leaf_loaders(const FusedArgs& a, const LeafMaps* maps, LeafGroup
         if (*(volatile int*)&sm.stop) break;
         for (int e = lt; e < LB * LS; e += NLOAD) {
             const int x = e / LS, dd = e % LS;
-            B.LOr[e] = (dd >= 1 && dd < LB && x + dd < LB) ? dLO[x * dld + x + dd] : 0.f;
-            B.LIc[e] = (dd >= 1 && dd < LB && x - dd >= 0) ? dLI[(x - dd) * dld + x] : 0.f;
+            B.LOr[e] = (dd >= 1 && dd < LB && x + dd < LB) ? dLO[swz(x, x + dd)] : 0.f;
+            B.LIc[e] = (dd >= 1 && dd < LB && x - dd >= 0) ? dLI[swz(x - dd, x)] : 0.f;
         }
         // this thread's accumulator elements (m16n8 layout, see product_mma)
         const int eg = lane >> 2, et = lane & 3;
@@ -530,8 +559,8 @@ __device__ void leaf_loaders(const FusedArgs& a, const LeafMaps* maps, LeafGroup
 #pragma unroll
                 for (int q = 0; q < 16; ++q) {
                     const int e = lt + q * NLOAD, r = e >> 5, c = e & 31;
-                    sA[r * LB + c] = pf[q];        // sA[k = source row / column][leaf row]
-                    sB[r * LB + c] = pf[16 + q];   // sB[k][leaf col]
+                    sA[swz(r, c)] = pf[q];         // sA[k = source row / column][leaf row]
+                    sB[swz(r, c)] = pf[16 + q];    // sB[k][leaf col]
                 }
                 if (idx + 1 < nf.nsrc) {
                     if (!wait_recent(idx + 1)) { stop = true; break; }
@@ -638,7 +667,7 @@ __device__ void leaf_solver(const FusedArgs& a, LeafGroupSmem& sm, int lane, int
         }
         if (lane < rows) {
             for (int c = 0; c < cols; ++c)
-                __stcg(&a.Ut[(size_t)(j0 + c) * a.ldm + i0 + lane], B.oUt[c * LB + lane]);
+                __stcg(&a.Ut[(size_t)(j0 + c) * a.ldm + i0 + lane], B.oUt[swz(c, lane)]);
         }
         __threadfence();
         __syncwarp();
@@ -722,16 +751,19 @@ __device__ void leaf_role(const FusedArgs& a, const LeafMaps* maps, uint8_t* sme
 struct PushTask {
     bool valid;
     bool vert;      // E into T_far (else U into R_far)
-    int src;        // source super-block index along the column (vert) / row
+    int src_lo;     // the batch's source super-blocks along the column (vert) / row ...
+    int src_hi;     // ... src_lo .. src_hi, src_hi the newest
+    int pos;        // the batch's place in the tile's order of additions
     int A, C;       // target super-block
     int tr, tc;     // target 128 x 128 tile
+    int k0;         // first K index (row / column of the sources)
     int nkb;        // k-blocks of 32
 };
 
-// Task t: source super-block (A', C') by binary search over the prefix, then (target, tile)
-// inside it. Its targets are (A'+2+d, C') for the vertical push (d < nvt) and (A', C'+2+d) for
-// the horizontal one (d < nht), nearest first (vertical, horizontal, then the next distance),
-// 4 tiles each.
+// Task t: its newest source super-block (A', C') by binary search over the prefix, then
+// (target, tile) inside it: the targets (A' + bd_min(j), C') of the vertical push
+// (j < n_ready(A', MS)) and (A', C' + bd_min(j)) of the horizontal one, nearest first
+// (vertical, horizontal, then the next batch), 4 tiles each.
 __device__ __forceinline__ PushTask decode_task(const FusedArgs& a, int t) {
     int lo = 0, hi = a.nsb - 1;
     while (lo < hi) {
@@ -741,23 +773,27 @@ __device__ __forceinline__ PushTask decode_task(const FusedArgs& a, int t) {
     }
     const int2 sc = __ldg(&a.task_sb[lo]);
     const int local = t - __ldg(&a.task_pre[lo]);
-    const int nvt = max(a.MS - sc.x - 2, 0), nht = max(a.NS - sc.y - 2, 0);
-    const int mn = min(nvt, nht);
+    const int nvj = n_ready(sc.x, a.MS), nhj = n_ready(sc.y, a.NS);
+    const int mn = min(nvj, nhj);
     const int u = local >> 2, q = local & 3;
-    int d;
+    int j;
     bool vert;
-    if (u < 2 * mn) { d = u >> 1; vert = (u & 1) == 0; }
-    else { d = mn + (u - 2 * mn); vert = nvt > nht; }
+    if (u < 2 * mn) { j = u >> 1; vert = (u & 1) == 0; }
+    else { j = mn + (u - 2 * mn); vert = nvj > nhj; }
     PushTask p;
     p.vert = vert;
-    p.A = vert ? sc.x + 2 + d : sc.x;
-    p.C = vert ? sc.y : sc.y + 2 + d;
-    p.src = vert ? sc.x : sc.y;
+    const int X = (vert ? sc.x : sc.y) + bd_min(j);       // the target along the direction
+    p.A = vert ? X : sc.x;
+    p.C = vert ? sc.y : X;
+    p.src_hi = vert ? sc.x : sc.y;
+    p.src_lo = max(0, X - bd_max(j));
+    p.pos = n_batches(X) - 1 - j;                         // oldest batch first
     p.tr = 2 * p.A + (q >> 1);
     p.tc = 2 * p.C + (q & 1);
     p.valid = p.tr * TB < a.m && p.tc * TB < a.n;
-    const int kext = vert ? min(SB, a.m - p.src * SB) : min(SB, a.n - p.src * SB);
-    p.nkb = (kext + tc::BK - 1) / tc::BK;
+    const int dim = vert ? a.m : a.n;
+    p.k0 = p.src_lo * SB;
+    p.nkb = (min((p.src_hi + 1) * SB, dim) - p.k0 + tc::BK - 1) / tc::BK;
     return p;
 }
 
@@ -767,6 +803,26 @@ __device__ __forceinline__ void gemm_sync() {   // the six warps of the push pip
 
 __device__ __forceinline__ void epi_sync() {
     asm volatile("bar.sync 1, 128;" ::: "memory");
+}
+
+// Task ids travel from the producer (which takes them from the global counter) to the MMA
+// issuer and the epilogue through a ring of kTaskFifo slots; -1 ends the stream.
+constexpr int kTaskFifo = 8;
+struct TaskFifo {
+    int id[kTaskFifo];
+    uint64_t full[kTaskFifo];    // the producer wrote the slot (1 arrival)
+    uint64_t empty[kTaskFifo];   // the MMA issuer and the epilogue read it (2 arrivals)
+};
+
+// The consumer side: the n-th task id (or -1 at the end, -2 if a wait gave up).
+__device__ __forceinline__ int fifo_pop(TaskFifo& q, int nth, int* status, uint64_t limit_ns,
+                                        volatile int* s_abort) {
+    const int f = nth % kTaskFifo;
+    if (!tc::wait_or_abort(&q.full[f], (nth / kTaskFifo) & 1, status, limit_ns, s_abort))
+        return -2;
+    const int t = q.id[f];
+    sm100::mbar_arrive(&q.empty[f]);
+    return t;
 }
 
 // Tensor-core far-field pushes (same warp roles as the GEMM engine: warp 0 TMA, warp 1 MMA,
@@ -789,10 +845,12 @@ __device__ void gemm_role(const CUtensorMap* loth, const CUtensorMap* lotl, cons
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
     volatile int* s_abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
     volatile int* s_go = s_abort + 1;
+    volatile int* s_task = s_go + 1;
+    TaskFifo& fifo = *reinterpret_cast<TaskFifo*>(
+        (reinterpret_cast<uintptr_t>(s_task + 1) + 7) & ~uintptr_t(7));
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (warp >= 6) return;   // the push pipeline uses warps 0 .. 5
-    const int gid = blockIdx.x - a.leaf_ctas, ng = gridDim.x - a.leaf_ctas;
     const int total = __ldg(&a.task_pre[a.nsb]);
 
     if (threadIdx.x == 0) {
@@ -805,6 +863,10 @@ __device__ void gemm_role(const CUtensorMap* loth, const CUtensorMap* lotl, cons
             sm100::mbar_init(&acc_empty[b], 4);
         }
         sm100::mbar_init(drain, 1);
+        for (int f = 0; f < kTaskFifo; ++f) {
+            sm100::mbar_init(&fifo.full[f], 1);
+            sm100::mbar_init(&fifo.empty[f], 2);
+        }
         *s_abort = 0;
         *s_go = 0;
         sm100::fence_mbar_init();
@@ -831,12 +893,31 @@ __device__ void gemm_role(const CUtensorMap* loth, const CUtensorMap* lotl, cons
             sm100::prefetch_tmap(uh);   sm100::prefetch_tmap(ul);
             sm100::prefetch_tmap(lith); sm100::prefetch_tmap(litl);
             uint32_t g = 0;
-            for (int t = gid; t < total && !*s_abort; t += ng) {
-                const PushTask p = decode_task(a, t);
-                if (!p.valid) continue;
-                const int sA = p.vert ? p.src : p.A, sC = p.vert ? p.C : p.src;
-                const int need = leaves_in(a.Mt, sA) * leaves_in(a.Nt, sC);
-                if (!wait_geq(&a.sb_done[sA * a.NS + sC], need, a.abort_word, a.status, a.limit_ns)) {
+            for (int nt = 0; !*s_abort; ++nt) {
+                // the next valid task from the global counter, or the end of the stream
+                int t;
+                PushTask p;
+                do {
+                    t = atomicAdd(a.task_next, 1);
+                    if (t >= total) break;
+                    p = decode_task(a, t);
+                } while (!p.valid);
+                const int f = nt % kTaskFifo;
+                if (nt >= kTaskFifo &&
+                    !tc::wait_or_abort(&fifo.empty[f], ((nt / kTaskFifo) & 1) ^ 1, a.status,
+                                       a.limit_ns, s_abort))
+                    break;
+                fifo.id[f] = t < total ? t : -1;
+                sm100::mbar_arrive(&fifo.full[f]);
+                if (t >= total) break;
+                bool ready = true;      // every source super-block of the batch is complete
+                for (int sx = p.src_lo; sx <= p.src_hi && ready; ++sx) {
+                    const int sA = p.vert ? sx : p.A, sC = p.vert ? p.C : sx;
+                    const int need = leaves_in(a.Mt, sA) * leaves_in(a.Nt, sC);
+                    ready = wait_geq(&a.sb_done[sA * a.NS + sC], need, a.abort_word, a.status,
+                                     a.limit_ns);
+                }
+                if (!ready) {
                     *s_abort = 1;
                     break;
                 }
@@ -855,7 +936,7 @@ __device__ void gemm_role(const CUtensorMap* loth, const CUtensorMap* lotl, cons
                         break;
                     }
                     sm100::mbar_arrive_expect_tx(&full[s], Cf::kStageBytes);
-                    const int kx = p.src * SB + kb * tc::BK;
+                    const int kx = p.k0 + kb * tc::BK;
                     sm100::tma_load_2d(stage_ptr(s, 0), ma_h, kx, p.tr * TB, &full[s]);
                     sm100::tma_load_2d(stage_ptr(s, 1), ma_l, kx, p.tr * TB, &full[s]);
                     sm100::tma_load_2d(stage_ptr(s, 2), mb_h, kx, p.tc * TB, &full[s]);
@@ -875,9 +956,10 @@ __device__ void gemm_role(const CUtensorMap* loth, const CUtensorMap* lotl, cons
             constexpr uint32_t idesc = sm100::idesc_tf32(tc::BM, BN);
             uint32_t g = 0;
             int i = 0;
-            for (int t = gid; t < total && !*s_abort; t += ng) {
+            for (int nt = 0; !*s_abort; ++nt) {
+                const int t = fifo_pop(fifo, nt, a.status, a.limit_ns, s_abort);
+                if (t < 0) break;
                 const PushTask p = decode_task(a, t);
-                if (!p.valid) continue;
                 const int b = i & 1;
                 if (i >= 2 &&
                     !tc::wait_or_abort(&acc_empty[b], ((i >> 1) & 1) ^ 1, a.status, a.limit_ns, s_abort))
@@ -924,20 +1006,29 @@ __device__ void gemm_role(const CUtensorMap* loth, const CUtensorMap* lotl, cons
         const int quarter = warp & 3;
         float* stage = epi_stage + (warp - tc::kEpiWarp0) * (32 * 33);
         int i = 0;
-        for (int t = gid; t < total; t += ng) {
-            const PushTask p = decode_task(a, t);
-            if (!p.valid) continue;
+        for (int nt = 0;; ++nt) {
             const int b = i & 1;
-            int* cnt = (p.vert ? a.cntT : a.cntR) + (size_t)p.tr * a.TN + p.tc;
             if (threadIdx.x == tc::kEpiWarp0 * 32) {
-                bool ok = tc::wait_or_abort(&acc_full[b], (i >> 1) & 1, a.status, a.limit_ns, s_abort);
-                // the tile takes its sources in order
-                if (ok) ok = wait_geq(cnt, p.src, a.abort_word, a.status, a.limit_ns);
-                if (!ok) { *s_abort = 1; atomicExch(a.abort_word, 1); }
+                const int t = fifo_pop(fifo, nt, a.status, a.limit_ns, s_abort);
+                bool ok = t >= 0;
+                if (ok) {
+                    const PushTask q = decode_task(a, t);
+                    int* c = (q.vert ? a.cntT : a.cntR) + (size_t)q.tr * a.TN + q.tc;
+                    ok = tc::wait_or_abort(&acc_full[b], (i >> 1) & 1, a.status, a.limit_ns,
+                                           s_abort);
+                    // the tile takes its batches in order
+                    if (ok) ok = wait_geq(c, q.pos, a.abort_word, a.status, a.limit_ns);
+                    if (!ok) { *s_abort = 1; atomicExch(a.abort_word, 1); }
+                } else if (t == -2) {
+                    atomicExch(a.abort_word, 1);
+                }
+                *s_task = t;
                 *s_go = ok ? 1 : 0;
             }
             epi_sync();
             if (!*s_go) break;
+            const PushTask p = decode_task(a, *s_task);
+            int* cnt = (p.vert ? a.cntT : a.cntR) + (size_t)p.tr * a.TN + p.tc;
             sm100::tc_fence_after();
             float* Cm = p.vert ? a.Tf : a.Rf;
             const int row0 = p.tr * TB + quarter * 32;
@@ -962,7 +1053,7 @@ __device__ void gemm_role(const CUtensorMap* loth, const CUtensorMap* lotl, cons
             __threadfence();
             sm100::tc_fence_before();
             epi_sync();
-            if (threadIdx.x == tc::kEpiWarp0 * 32) st_release_gpu(cnt, p.src + 1);
+            if (threadIdx.x == tc::kEpiWarp0 * 32) st_release_gpu(cnt, p.pos + 1);
             if (lane == 0) sm100::mbar_arrive(&acc_empty[b]);
             ++i;
         }
@@ -981,9 +1072,9 @@ round_kernel(const __grid_constant__ CUtensorMap loth, const __grid_constant__ C
              const __grid_constant__ LeafMaps lmaps, const __grid_constant__ FusedArgs a) {
     extern __shared__ __align__(1024) uint8_t round_smem[];
     if ((int)blockIdx.x < a.leaf_ctas) {
-        // box-copy destinations need 128-byte alignment of the leaf layout's base
+        // swizzled box-copy destinations need 1024-byte alignment of the leaf layout's base
         uint8_t* base = reinterpret_cast<uint8_t*>(
-            (reinterpret_cast<uintptr_t>(round_smem) + 127) & ~uintptr_t(127));
+            (reinterpret_cast<uintptr_t>(round_smem) + 1023) & ~uintptr_t(1023));
         leaf_role(a, &lmaps, base);
         return;
     }
@@ -999,7 +1090,7 @@ __global__ void task_prefix_kernel(int MS, int NS, int* pre, int2* sb) {
             const int C = d - A;
             pre[idx] = acc;
             sb[idx] = make_int2(A, C);
-            acc += 4 * (max(MS - A - 2, 0) + max(NS - C - 2, 0));
+            acc += 4 * (n_ready(A, MS) + n_ready(C, NS));
             ++idx;
         }
     }
@@ -1147,6 +1238,7 @@ int round_impl(const float* Wstar, int m, int n, const float* L_O, const float* 
     a.cntT = a.sb_done + L.nsb;
     a.cntR = a.cntT + (size_t)L.TM * L.TN;
     a.abort_word = a.cntR + (size_t)L.TM * L.TN;
+    a.task_next = a.abort_word + 32;   // in the zeroed slack at the end of the int region
     a.status = dev_status;
     a.task_pre = task_pre;
     a.task_sb = task_sb;
@@ -1169,10 +1261,10 @@ int round_impl(const float* Wstar, int m, int n, const float* L_O, const float* 
     auto al16 = [](const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15) == 0; };
     a.box_loads = (m % 4 == 0 && n % 4 == 0 && al16(Wstar) && al16(L_O) && al16(L_I)) ? 1 : 0;
     if (a.box_loads) {
-        if ((e = tc::make_box_map(&lm.lo, L_O, m, m, m, LB))) return e;
-        if ((e = tc::make_box_map(&lm.li, L_I, n, n, n, LB))) return e;
-        if ((e = tc::make_box_map(&lm.e, E, m, n, n, LB))) return e;
-        if ((e = tc::make_box_map(&lm.ut, Ut, n, m, L.ldm, LB))) return e;
+        if ((e = tc::make_box_map(&lm.lo, L_O, m, m, m, LB, true))) return e;
+        if ((e = tc::make_box_map(&lm.li, L_I, n, n, n, LB, true))) return e;
+        if ((e = tc::make_box_map(&lm.e, E, m, n, n, LB, true))) return e;
+        if ((e = tc::make_box_map(&lm.ut, Ut, n, m, L.ldm, LB, true))) return e;
         if ((e = tc::make_box_map(&lm.ws, Wstar, m, n, n, LB))) return e;
         if ((e = tc::make_box_map(&lm.tf, Tf, m, n, n, LB))) return e;
         if ((e = tc::make_box_map(&lm.rf, Rf, m, n, n, LB))) return e;

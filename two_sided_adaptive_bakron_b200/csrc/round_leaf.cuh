@@ -24,6 +24,14 @@ constexpr int UW = 4;            // wavefront steps per unrolled group
 constexpr int WIN = LB + UW;     // register window of slots
 constexpr int LS = LB + 4;       // row stride of the skewed diagonal blocks (16-byte rows)
 
+// Element (r, c) of a 32 x 32 fp32 tile in the layout a tensor copy with 128-byte swizzle
+// gives (a 1024-byte aligned tile of 128-byte rows): the 16-byte chunk c / 4 of row r sits at
+// chunk (c / 4) ^ (r % 8). The near-field fragment loads (a K index 2t or 2t + 1 against a row
+// or column index g, see product_mma) then touch 32 distinct banks.
+__device__ __forceinline__ int swz(int r, int c) {
+    return r * LB + ((((c >> 2) ^ r) & 7) << 2) + (c & 3);
+}
+
 // One staging buffer: a leaf's inputs and outputs (shared memory, floats). LOr and LIc rows
 // are read as float4 (16-byte rows); W, T and R may be filled by tensor (box) copies, whose
 // shared-memory destination must sit on a 128-byte boundary.
@@ -36,7 +44,7 @@ struct alignas(128) LeafBuf {
     float S[2 * LB];             // s_r and its reciprocal
     float oE[LB * LB], oU[LB * LB];
     float oEt[LB * LB];          // E transposed (for the transposed planes)
-    float oUt[LB * LB];          // U transposed
+    float oUt[LB * LB];          // U transposed, element (c, r) at swz(c, r)
     // the codes; before the wavefront, with stochastic Q, the 16-bit fields k of the leaf's
     // variates u = (k + 1/2) / 2^16 (each is read by the lane that then writes the code there)
     alignas(16) int16_t oC[LB * LB];
@@ -176,7 +184,7 @@ __device__ __forceinline__ void solve_leaf_chain(int lane, int rows, int cols, f
             B.oE[rr * LB + j] = e;
             B.oEt[j * LB + rr] = e;
             B.oU[rr * LB + j] = u;
-            B.oUt[j * LB + rr] = u;
+            B.oUt[swz(j, rr)] = u;
         }
         X.eu[s & 1][0][j] = e;
         X.eu[s & 1][1][j] = u;

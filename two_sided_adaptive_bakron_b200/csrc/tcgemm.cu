@@ -75,15 +75,18 @@ int sm_count() {
     return cached[dev];
 }
 
-int make_box_map(CUtensorMap* map, const float* base, int rows, int cols, int ld, int box) {
+int make_box_map(CUtensorMap* map, const float* base, int rows, int cols, int ld, int box,
+                 bool swizzle128) {
     auto fn = encode_fn();
     if (!fn) return BAKRON_ERR_CUDA;
+    if (swizzle128 && box * sizeof(float) != 128) return BAKRON_ERR_INVALID_ARG;
     cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
     cuuint64_t strides[1] = {(cuuint64_t)ld * sizeof(float)};
     cuuint32_t boxd[2] = {(cuuint32_t)box, (cuuint32_t)box};
     cuuint32_t estr[2] = {1, 1};
     CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(base), dims,
-                    strides, boxd, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                    strides, boxd, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? BAKRON_OK : BAKRON_ERR_CUDA;
 }

@@ -20,9 +20,12 @@ int make_kmajor_map(CUtensorMap* map, const float* base, int rows, int kcols, in
                     int box_rows);
 
 // 2-D fp32 tensor map of a row-major matrix (rows x cols, row stride ld elements, ld % 4 == 0,
-// base 16-byte aligned) with a box x box box, no swizzle (the box lands as a dense row-major
-// tile), out-of-range elements read as zero.
-int make_box_map(CUtensorMap* map, const float* base, int rows, int cols, int ld, int box);
+// base 16-byte aligned) with a box x box box, out-of-range elements read as zero. Without
+// swizzle the box lands as a dense row-major tile; with swizzle128 (box = 32: 128-byte rows)
+// the 16-byte chunk c of row r lands at chunk c ^ (r % 8), and the destination must be
+// 1024-byte aligned.
+int make_box_map(CUtensorMap* map, const float* base, int rows, int cols, int ld, int box,
+                 bool swizzle128 = false);
 
 // Splits an fp32 matrix (rows x cols, row stride ld_src) into hi/lo planes (row stride
 // ld_dst). transpose = 1 writes the planes of the transposed matrix (cols x rows).
