@@ -17,7 +17,17 @@
 //                                             outer block right away (K = 128), the rest once
 //                                             per outer block (K = 512, upper block triangle),
 //                                             so the trailing matrix is streamed n/512 times.
+// Look-ahead (n > kLookaheadMin): the diagonal blocks form a chain of single-CTA kernels that
+// would leave the GPU mostly idle, so each outer block's trailing update is split and moved to
+// a side stream. There, (a) the next outer block's 512 columns are updated first, on the whole
+// GPU, and the caller's stream waits only for that before it goes on with the next block's
+// diagonal chain; (b) the rest of the trailing matrix follows on all but kReserveSms SMs, which
+// stay free for that chain. The side stream runs (a) of outer block o - 1 after (b) of o, the
+// only other update of those columns. The panel planes alternate between two sets, so (b) can
+// still read outer block o's planes while o - 1's panels are written.
 #include <algorithm>
+#include <atomic>
+#include <mutex>
 
 #include "ldl_diag.cuh"
 #include "tcgemm_host.cuh"
@@ -83,8 +93,20 @@ struct EpiPanel {
     __device__ void tile_done(const tc::Problem&, int, int) {}
 };
 
+// Above this size the factorisation runs with look-ahead (two plane sets, a side stream);
+// at or below it, sequentially on the caller's stream with one plane set.
+constexpr int kLookaheadMin = 2048;
+constexpr int kReserveSms = 24;   // SMs the bulk update leaves to the diagonal chain
+
+inline int plane_sets(int n) { return n > kLookaheadMin ? 2 : 1; }
+
+struct Planes {
+    float *x_hi, *x_lo, *u_hi, *u_lo;   // X and U_AB of an outer block (n x NBO each)
+};
+
 struct LdlWs {
-    float *inv_hi, *inv_lo, *p_hi, *p_lo, *x_hi, *x_lo, *u_hi, *u_lo;
+    float *inv_hi, *inv_lo, *p_hi, *p_lo;
+    Planes set[2];
 };
 
 template <class F>
@@ -93,11 +115,54 @@ void ldl_ws_layout(int n, F&& take) {
     take((size_t)NBI * NBI);        // inv_lo
     take((size_t)n * NBI);          // p_hi  (panel of H')
     take((size_t)n * NBI);          // p_lo
-    take((size_t)n * NBO);          // x_hi  (X of the outer block)
-    take((size_t)n * NBO);          // x_lo
-    take((size_t)n * NBO);          // u_hi  (U_AB of the outer block)
-    take((size_t)n * NBO);          // u_lo
+    for (int k = 0; k < plane_sets(n); ++k) {
+        take((size_t)n * NBO);      // x_hi  (X of the outer block)
+        take((size_t)n * NBO);      // x_lo
+        take((size_t)n * NBO);      // u_hi  (U_AB of the outer block)
+        take((size_t)n * NBO);      // u_lo
+    }
 }
+
+// Side streams for the look-ahead, created once per device and never destroyed (a small pool,
+// taken round robin, so that factorisations enqueued at the same time on different streams do
+// not all share one side stream).
+constexpr int kSidePool = 4;
+constexpr int kMaxDevices = 64;
+std::mutex g_side_mu;
+cudaStream_t g_side[kMaxDevices][kSidePool] = {};
+std::atomic<unsigned> g_side_next{0};
+
+int side_stream(cudaStream_t* out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+        return BAKRON_ERR_CUDA;
+    const unsigned k = g_side_next.fetch_add(1, std::memory_order_relaxed) % kSidePool;
+    std::lock_guard<std::mutex> lock(g_side_mu);
+    if (!g_side[dev][k] &&
+        cudaStreamCreateWithFlags(&g_side[dev][k], cudaStreamNonBlocking) != cudaSuccess) {
+        g_side[dev][k] = nullptr;
+        return BAKRON_ERR_CUDA;
+    }
+    *out = g_side[dev][k];
+    return BAKRON_OK;
+}
+
+// Events of one call, released when the call has enqueued everything (their pending waits
+// still complete).
+struct CallEvents {
+    static constexpr int kCount = 3;
+    cudaEvent_t ev[kCount] = {};
+    int n = 0;
+    ~CallEvents() {
+        for (int i = 0; i < n; ++i) cudaEventDestroy(ev[i]);
+    }
+    int make() {
+        for (n = 0; n < kCount; ++n)
+            if (cudaEventCreateWithFlags(&ev[n], cudaEventDisableTiming) != cudaSuccess)
+                return BAKRON_ERR_CUDA;
+        return BAKRON_OK;
+    }
+};
 
 }  // namespace
 }  // namespace bakron
@@ -117,10 +182,13 @@ extern "C" int bakron_ldl(const float* H, int n, float* L, float* D, void* ws, s
     if (!ws_ok(ws, ws_bytes, bakron_ldl_workspace_bytes(n))) return BAKRON_ERR_WORKSPACE;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     WsCarver c(ws);
-    float* bufs[8];
+    float* bufs[12];
     int bi = 0;
     ldl_ws_layout(n, [&](size_t k) { bufs[bi++] = c.take<float>(k); });
-    LdlWs w{bufs[0], bufs[1], bufs[2], bufs[3], bufs[4], bufs[5], bufs[6], bufs[7]};
+    const int nsets = plane_sets(n);
+    LdlWs w{bufs[0], bufs[1], bufs[2], bufs[3], {}};
+    for (int k = 0; k < nsets; ++k)
+        w.set[k] = Planes{bufs[4 + 4 * k], bufs[5 + 4 * k], bufs[6 + 4 * k], bufs[7 + 4 * k]};
 
     if (cudaFuncSetAttribute(ldl_diag::diag_block_kernel,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -128,17 +196,31 @@ extern "C" int bakron_ldl(const float* H, int n, float* L, float* D, void* ws, s
         return BAKRON_ERR_CUDA;
     int e;
     // Tensor maps over the outer-block planes (fixed for the whole call).
-    CUtensorMap m_xh, m_xl, m_uh, m_ul;
-    if ((e = tc::make_kmajor_map(&m_xh, w.x_hi, n, NBO, NBO, tc::BM))) return e;
-    if ((e = tc::make_kmajor_map(&m_xl, w.x_lo, n, NBO, NBO, tc::BM))) return e;
-    if ((e = tc::make_kmajor_map(&m_uh, w.u_hi, n, NBO, NBO, BN))) return e;
-    if ((e = tc::make_kmajor_map(&m_ul, w.u_lo, n, NBO, NBO, BN))) return e;
+    CUtensorMap m_xh[2], m_xl[2], m_uh[2], m_ul[2];
+    for (int k = 0; k < nsets; ++k) {
+        if ((e = tc::make_kmajor_map(&m_xh[k], w.set[k].x_hi, n, NBO, NBO, tc::BM))) return e;
+        if ((e = tc::make_kmajor_map(&m_xl[k], w.set[k].x_lo, n, NBO, NBO, tc::BM))) return e;
+        if ((e = tc::make_kmajor_map(&m_uh[k], w.set[k].u_hi, n, NBO, NBO, BN))) return e;
+        if ((e = tc::make_kmajor_map(&m_ul[k], w.set[k].u_lo, n, NBO, NBO, BN))) return e;
+    }
+    // look-ahead: a side stream and the call's events (ready: an outer block's panels are
+    // written; next: the next outer block's columns are updated; join: the side stream's end)
+    const bool ahead = nsets == 2;
+    cudaStream_t side = nullptr;
+    CallEvents evs;
+    if (ahead) {
+        if ((e = side_stream(&side))) return e;
+        if ((e = evs.make())) return e;
+    }
+    cudaEvent_t ev_ready = evs.ev[0], ev_next = evs.ev[1], ev_join = evs.ev[2];
 
     const int eb = 1184;
     copy_upper_kernel<<<eb, 256, 0, st>>>(H, L, n);
     count_launches(1);
-    for (int ko1 = n; ko1 > 0; ko1 -= NBO) {
+    for (int ko1 = n, o = 0; ko1 > 0; ko1 -= NBO, ++o) {
         const int ko0 = std::max(0, ko1 - NBO);
+        const int ps = ahead ? (o & 1) : 0;      // this outer block's plane set
+        const Planes& pw = w.set[ps];
         for (int t = 0, kb1 = ko1; kb1 > ko0; ++t, kb1 -= NBI) {
             // plane columns of this inner block, counted from the end of the outer block so
             // that they stay 128-aligned even when the outer block is a partial one
@@ -156,7 +238,7 @@ extern "C" int bakron_ldl(const float* H, int n, float* L, float* D, void* ws, s
             if ((e = tc::make_kmajor_map(&m_il, w.inv_lo, NBI, b, NBI, BN))) return e;
             tc::ProblemList pl(BN);
             pl.add(0, 0, 0, 0, kb0, b, b, 0, 0);
-            EpiPanel ep{L, n, D, kb0, w.x_hi, w.x_lo, w.u_hi, w.u_lo, NBO, c_off};
+            EpiPanel ep{L, n, D, kb0, pw.x_hi, pw.x_lo, pw.u_hi, pw.u_lo, NBO, c_off};
             if ((e = tc::launch_gemm3x<BN, STAGES>(m_ph, m_pl, m_ih, m_il, pl, ep, dev_status, st)))
                 return e;
             // columns of the outer block still pending: H'[0:kb0, ko0:kb0] -= X U_AB^T
@@ -164,19 +246,51 @@ extern "C" int bakron_ldl(const float* H, int n, float* L, float* D, void* ws, s
                 tc::ProblemList wl(BN);
                 wl.add(0, c_off, ko0, c_off, kb0, kb0 - ko0, b, 0, ko0, -1.f);
                 tc::EpiStore es{L, n, 1, 1};
-                if ((e = tc::launch_gemm3x<BN, STAGES>(m_xh, m_xl, m_uh, m_ul, wl, es, dev_status,
-                                                       st)))
+                if ((e = tc::launch_gemm3x<BN, STAGES>(m_xh[ps], m_xl[ps], m_uh[ps], m_ul[ps], wl,
+                                                       es, dev_status, st)))
                     return e;
             }
         }
-        // the rest of the trailing matrix, once per outer block: upper block triangle
-        if (ko0 > 0) {
+        if (ko0 == 0) continue;
+        // the rest of the trailing matrix, once per outer block: upper block triangle of
+        // [0, ko0)^2, K = this outer block's columns
+        const int K = ko1 - ko0;
+        tc::EpiStore es{L, n, 1, 1};
+        if (!ahead) {
             tc::ProblemList tl(BN);
-            tl.add(0, 0, 0, 0, ko0, ko0, ko1 - ko0, 0, 0, -1.f, /*upper_only=*/1);
-            tc::EpiStore es{L, n, 1, 1};
-            if ((e = tc::launch_gemm3x<BN, STAGES>(m_xh, m_xl, m_uh, m_ul, tl, es, dev_status, st)))
+            tl.add(0, 0, 0, 0, ko0, ko0, K, 0, 0, -1.f, /*upper_only=*/1);
+            if ((e = tc::launch_gemm3x<BN, STAGES>(m_xh[0], m_xl[0], m_uh[0], m_ul[0], tl, es,
+                                                   dev_status, st)))
+                return e;
+            continue;
+        }
+        // look-ahead, on the side stream once this outer block's panels are written: (a) the
+        // columns [ca, ko0) of the next outer block (after (b) of the previous outer block,
+        // which updated them too and read the plane set the next panels overwrite), then (b)
+        // the bulk [0, ca)^2
+        const int ca = std::max(0, ko0 - NBO);
+        if ((e = cuda_err(cudaEventRecord(ev_ready, st)))) return e;
+        if ((e = cuda_err(cudaStreamWaitEvent(side, ev_ready, 0)))) return e;
+        tc::ProblemList al(BN);
+        al.add(0, 0, ca, 0, ca, ko0 - ca, K, 0, ca, -1.f);                      // rows above
+        al.add(ca, 0, ca, 0, ko0 - ca, ko0 - ca, K, ca, ca, -1.f, /*upper_only=*/1);
+        if ((e = tc::launch_gemm3x<BN, STAGES>(m_xh[ps], m_xl[ps], m_uh[ps], m_ul[ps], al, es,
+                                               dev_status, side)))
+            return e;
+        if ((e = cuda_err(cudaEventRecord(ev_next, side)))) return e;
+        if (ca > 0) {
+            tc::ProblemList bl(BN);
+            bl.add(0, 0, 0, 0, ca, ca, K, 0, 0, -1.f, /*upper_only=*/1);
+            if ((e = tc::launch_gemm3x<BN, STAGES>(m_xh[ps], m_xl[ps], m_uh[ps], m_ul[ps], bl, es,
+                                                   dev_status, side,
+                                                   std::max(1, tc::sm_count() - kReserveSms))))
                 return e;
         }
+        if ((e = cuda_err(cudaStreamWaitEvent(st, ev_next, 0)))) return e;
+    }
+    if (ahead) {   // the side stream's last work joins the caller's stream
+        if ((e = cuda_err(cudaEventRecord(ev_join, side)))) return e;
+        if ((e = cuda_err(cudaStreamWaitEvent(st, ev_join, 0)))) return e;
     }
     clear_lower_kernel<<<eb, 256, 0, st>>>(L, n);
     count_launches(1);
