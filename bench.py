@@ -489,10 +489,9 @@ def _e2e(args, torch, bk, solver, stream, dev, ws, m, n, bits, Ws, HO, HI, sc,
 
 
 # DRAM bytes (read + written) of one round_kernel launch per workload, from one ncu capture of
-# the current kernel version (dram__bytes_read.sum + dram__bytes_write.sum, 1 pass); reported
-# as the roofline's traffic. Empty while the kernel has changed since its last capture (the
-# capture before the per-group grid steps and codebook Q measured 26.98 + 9.37 GB on
-# down_4096x14336).
+# the current kernel version (dram__bytes_read.sum + dram__bytes_write.sum; 1 pass on the
+# 4096 x 14336 bench command, part of --set full on 4096^2); reported as the roofline's
+# traffic. Emptied whenever the kernel changes, until it is captured again.
 ROUND_TRAFFIC_BYTES: dict = {}
 
 

@@ -39,6 +39,7 @@ constexpr int NBI = 128;   // inner block: diagonal factorisation in one CTA
 static_assert(NBI == ldl_diag::NB, "diagonal kernel block width");
 constexpr int NBO = 512;   // outer block: K of the trailing update
 constexpr int BN = 128;
+constexpr int BNP = 64;    // panel tiles 128 x 64: twice the CTAs on the chain's critical path
 constexpr int STAGES = 3;
 
 __global__ void copy_upper_kernel(const float* __restrict__ H, float* __restrict__ L, int n) {
@@ -59,7 +60,7 @@ __global__ void clear_lower_kernel(float* __restrict__ L, int n) {
     }
 }
 
-// Panel epilogue: x = (H'_AB U_BB^{-T})[i][c]; U_AB = x / D_c goes to L; x and U_AB also go
+// Panel epilogue: x = (H'_AB U_BB^{-T})[i][c]; U_AB = x (1 / D_c) goes to L; x and U_AB also go
 // to the hi/lo planes used by the trailing updates (column offset c_off in the outer block).
 struct EpiPanel {
     float* L;
@@ -74,13 +75,13 @@ struct EpiPanel {
     int c_off;
     __device__ void chunk(const tc::Problem& P, int row0, int c, int, int, const float* v) {
         if (c >= P.N) return;
-        const float dc = D[kb0 + c];
+        const float rdc = 1.0f / D[kb0 + c];
 #pragma unroll 8
         for (int rr = 0; rr < 32; ++rr) {
             const int row = row0 + rr;
             if (row >= P.M) break;
             const float x = v[rr * 33];
-            const float u = __fdiv_rn(x, dc);
+            const float u = x * rdc;
             L[(size_t)row * n + kb0 + c] = u;
             const size_t o = (size_t)row * ldx + c_off + c;
             const float xh_ = sm100::tf32_hi(x), uh_ = sm100::tf32_hi(u);
@@ -234,12 +235,12 @@ extern "C" int bakron_ldl(const float* H, int n, float* L, float* D, void* ws, s
             CUtensorMap m_ph, m_pl, m_ih, m_il;
             if ((e = tc::make_kmajor_map(&m_ph, w.p_hi, kb0, b, NBI, tc::BM))) return e;
             if ((e = tc::make_kmajor_map(&m_pl, w.p_lo, kb0, b, NBI, tc::BM))) return e;
-            if ((e = tc::make_kmajor_map(&m_ih, w.inv_hi, NBI, b, NBI, BN))) return e;
-            if ((e = tc::make_kmajor_map(&m_il, w.inv_lo, NBI, b, NBI, BN))) return e;
-            tc::ProblemList pl(BN);
+            if ((e = tc::make_kmajor_map(&m_ih, w.inv_hi, NBI, b, NBI, BNP))) return e;
+            if ((e = tc::make_kmajor_map(&m_il, w.inv_lo, NBI, b, NBI, BNP))) return e;
+            tc::ProblemList pl(BNP);
             pl.add(0, 0, 0, 0, kb0, b, b, 0, 0);
             EpiPanel ep{L, n, D, kb0, pw.x_hi, pw.x_lo, pw.u_hi, pw.u_lo, NBO, c_off};
-            if ((e = tc::launch_gemm3x<BN, STAGES>(m_ph, m_pl, m_ih, m_il, pl, ep, dev_status, st)))
+            if ((e = tc::launch_gemm3x<BNP, STAGES>(m_ph, m_pl, m_ih, m_il, pl, ep, dev_status, st)))
                 return e;
             // columns of the outer block still pending: H'[0:kb0, ko0:kb0] -= X U_AB^T
             if (kb0 > ko0) {

@@ -120,8 +120,10 @@ struct FusedArgs {
 // 32 x 32 fp32 box maps (no swizzle) of the matrices a leaf reads; only valid when m and n are
 // multiples of 4 (16-byte row strides), otherwise the loaders use plain loads.
 struct LeafMaps {
-    CUtensorMap lo;   // L_O (m x m)
-    CUtensorMap li;   // L_I (n x n)
+    CUtensorMap lo;   // L_O (m x m), 128-byte swizzle (near-field operands)
+    CUtensorMap li;   // L_I (n x n), 128-byte swizzle
+    CUtensorMap lod;  // L_O, no swizzle (the leaf's diagonal block)
+    CUtensorMap lid;  // L_I, no swizzle
     CUtensorMap e;    // E (m x n)
     CUtensorMap ut;   // U^T (n x m, row stride ldm)
     CUtensorMap ws;   // W* (m x n)
@@ -334,18 +336,19 @@ __device__ void leaf_loaders(const FusedArgs& a, const LeafMaps* maps, LeafGroup
         const int A = I / LPB, C = J / LPB;
         const int i0 = I * LB, j0 = J * LB;
         const int rows = min(LB, m - i0), cols = min(LB, n - j0);
-        // what does not depend on other leaves: W*, the diagonal blocks, the scales
-        const float* dLO;                        // diagonal blocks, swizzled 32 x 32 tiles
-        const float* dLI;
+        // what does not depend on other leaves: W*, the diagonal blocks, the scales. With box
+        // loads the diagonal blocks land in B.T / B.R (row-major), which the far-field sums
+        // overwrite once the blocks are skewed into LOr / LIc, after the older near-field
+        // products (so that those start right away).
+        const float* dLO = sA;                   // plain path: diagonal blocks, swizzled tiles
+        const float* dLI = sB;
         if (box) {
             if (lead) {
                 sm100::mbar_arrive_expect_tx(&sm.sbar, 3 * kBox * 4);
                 sm100::tma_load_2d(B.W, &maps->ws, j0, i0, &sm.sbar);
-                sm100::tma_load_2d(sm.ring[0][0], &maps->lo, i0, i0, &sm.sbar);
-                sm100::tma_load_2d(sm.ring[0][1], &maps->li, j0, j0, &sm.sbar);
+                sm100::tma_load_2d(B.T, &maps->lod, i0, i0, &sm.sbar);
+                sm100::tma_load_2d(B.R, &maps->lid, j0, j0, &sm.sbar);
             }
-            dLO = sm.ring[0][0];
-            dLI = sm.ring[0][1];
         } else {
 #pragma unroll 4
             for (int q = 0; q < (LB * LB) / NLOAD; ++q) {
@@ -354,8 +357,6 @@ __device__ void leaf_loaders(const FusedArgs& a, const LeafMaps* maps, LeafGroup
                 sA[swz(r, c)] = (r < rows && c < rows) ? __ldg(&a.LO[(size_t)(i0 + r) * m + i0 + c]) : 0.f;
                 sB[swz(r, c)] = (r < cols && c < cols) ? __ldg(&a.LI[(size_t)(j0 + r) * n + j0 + c]) : 0.f;
             }
-            dLO = sA;
-            dLI = sB;
         }
         if (lt < LB) {
             // the leaf's grid step: per row, or per row and column group (one group per leaf)
@@ -377,29 +378,25 @@ __device__ void leaf_loaders(const FusedArgs& a, const LeafMaps* maps, LeafGroup
             dst[1] = make_ulonglong2(w[2], w[3]);
         }
         // far field: every super-block at least two steps above / to the left has been added
-        if (lead) {
-            const int tile = (I * LB / TB) * a.TN + (J * LB / TB);
+        // (the box path waits for it after its older near-field products, see below)
+        const int ftile = (I * LB / TB) * a.TN + (J * LB / TB);
+        auto far_ready = [&]() -> bool {
             bool ok = true;
             if (A >= 2)
-                ok = wait_geq(&a.cntT[tile], n_batches(A), a.abort_word, a.status, a.limit_ns);
+                ok = wait_geq(&a.cntT[ftile], n_batches(A), a.abort_word, a.status, a.limit_ns);
             if (ok && C >= 2)
-                ok = wait_geq(&a.cntR[tile], n_batches(C), a.abort_word, a.status, a.limit_ns);
-            if (ok && box) {
-                // T_far / R_far were written through the generic proxy on other SMs
-                asm volatile("fence.proxy.async.global;" ::: "memory");
-                sm100::mbar_arrive_expect_tx(&sm.tbar, 2 * kBox * 4);
-                sm100::tma_load_2d(B.T, &maps->tf, j0, i0, &sm.tbar);
-                sm100::tma_load_2d(B.R, &maps->rf, j0, i0, &sm.tbar);
+                ok = wait_geq(&a.cntR[ftile], n_batches(C), a.abort_word, a.status, a.limit_ns);
+            return ok;
+        };
+        if (!box) {
+            if (lead) sm.stop = far_ready() ? 0 : 1;
+            group_sync(g);
+            if (*(volatile int*)&sm.stop) break;
+            for (int e = lt; e < LB * LS; e += NLOAD) {
+                const int x = e / LS, dd = e % LS;
+                B.LOr[e] = (dd >= 1 && dd < LB && x + dd < LB) ? dLO[swz(x, x + dd)] : 0.f;
+                B.LIc[e] = (dd >= 1 && dd < LB && x - dd >= 0) ? dLI[swz(x - dd, x)] : 0.f;
             }
-            if (ok && box && !sm100::mbar_wait(&sm.sbar, k & 1, a.status, a.limit_ns)) ok = false;
-            sm.stop = ok ? 0 : 1;
-        }
-        group_sync(g);
-        if (*(volatile int*)&sm.stop) break;
-        for (int e = lt; e < LB * LS; e += NLOAD) {
-            const int x = e / LS, dd = e % LS;
-            B.LOr[e] = (dd >= 1 && dd < LB && x + dd < LB) ? dLO[swz(x, x + dd)] : 0.f;
-            B.LIc[e] = (dd >= 1 && dd < LB && x - dd >= 0) ? dLI[swz(x - dd, x)] : 0.f;
         }
         // this thread's accumulator elements (m16n8 layout, see product_mma)
         const int eg = lane >> 2, et = lane & 3;
@@ -436,7 +433,7 @@ __device__ void leaf_loaders(const FusedArgs& a, const LeafMaps* maps, LeafGroup
             ok = __all_sync(0xffffffffu, ok);
             if (lane == 0) sm.stop = ok ? 0 : 1;
         }
-        group_sync(g);   // also: the skew is done with the diagonal blocks in ring stage 0
+        group_sync(g);   // plain path: also, the skew is done with the diagonal blocks in sA / sB
         if (*(volatile int*)&sm.stop) break;
         bool stop = false;
         float acc[2][4][4];                      // box path: this warp's direction, all 32 rows
@@ -474,12 +471,8 @@ __device__ void leaf_loaders(const FusedArgs& a, const LeafMaps* maps, LeafGroup
                     sm100::tma_load_2d(sm.ring[st][1], &maps->li, j0, sl * LB, &sm.rfull[st]);
                 }
             };
-            if (lane == 0) {
-                // the older sources' flags were acquired before the group barrier above
-                asm volatile("fence.proxy.async.global;" ::: "memory");
-                for (int i = 0; i < min(2, nold_d); ++i) issue(i);
-            }
-            for (int i = 0; i < ns; ++i) {
+            // one source's product; false when a wait gave up
+            auto product = [&](int i) -> bool {
                 const bool recent = i == nold_d;
                 if (recent) {   // its flag first (the local one needs none)
                     int okr = 1;
@@ -497,20 +490,61 @@ __device__ void leaf_loaders(const FusedArgs& a, const LeafMaps* maps, LeafGroup
                             }
                         }
                     }
-                    if (!__shfl_sync(0xffffffffu, okr, 0)) { stop = true; break; }
+                    if (!__shfl_sync(0xffffffffu, okr, 0)) return false;
                 }
                 const uint32_t q = rq + i, st = 2 * lw + (q & 1);
                 bool okw = sm100::mbar_wait(&sm.rfull[st], (q >> 1) & 1, a.status, a.limit_ns);
                 if (okw && loc && recent)   // the previous leaf's wavefront is done
                     okw = sm100::mbar_wait(&sm.solved[b ^ 1], ((k - 1) >> 1) & 1, a.status,
                                            a.limit_ns);
-                if (!__all_sync(0xffffffffu, okw)) { stop = true; break; }
+                if (!__all_sync(0xffffffffu, okw)) return false;
                 const float* X = (loc && recent) ? P.oUt : sm.ring[st][0];
                 product_mma(X, sm.ring[st][1], 0, lane, acc[0]);
                 product_mma(X, sm.ring[st][1], 1, lane, acc[1]);
                 __syncwarp();   // the stage is free again
                 if (lane == 0 && i + 2 < nold_d) issue(i + 2);
+                return true;
+            };
+            if (lane == 0) {
+                // the older sources' flags were acquired before the group barrier above
+                asm volatile("fence.proxy.async.global;" ::: "memory");
+                for (int i = 0; i < min(2, nold_d); ++i) issue(i);
             }
+            for (int i = 0; i < nold_d && !stop; ++i) stop = !product(i);
+            if (!vdir && !stop) {
+                // the horizontal warp (whose older sources finish first), between its older and
+                // its recent source: the diagonal blocks (in B.T / B.R) into LOr / LIc, then the
+                // far field into B.T / B.R
+                int ok = 1;
+                if (lane == 0) ok = sm100::mbar_wait(&sm.sbar, k & 1, a.status, a.limit_ns);
+                if (__shfl_sync(0xffffffffu, ok, 0)) {
+                    for (int e = lane; e < LB * LS; e += 32) {
+                        const int x = e / LS, dd = e % LS;
+                        B.LOr[e] = (dd >= 1 && dd < LB && x + dd < LB) ? B.T[x * LB + x + dd] : 0.f;
+                        B.LIc[e] = (dd >= 1 && dd < LB && x - dd >= 0) ? B.R[(x - dd) * LB + x] : 0.f;
+                    }
+                    __syncwarp();
+                    if (lane == 0) {
+                        ok = far_ready();
+                        if (ok) {
+                            // the skew's reads of B.T / B.R (generic proxy) come before the
+                            // copies that overwrite them; T_far / R_far were written through
+                            // the generic proxy on other SMs
+                            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                            asm volatile("fence.proxy.async.global;" ::: "memory");
+                            sm100::mbar_arrive_expect_tx(&sm.tbar, 2 * kBox * 4);
+                            sm100::tma_load_2d(B.T, &maps->tf, j0, i0, &sm.tbar);
+                            sm100::tma_load_2d(B.R, &maps->rf, j0, i0, &sm.tbar);
+                        }
+                    }
+                }
+                if (!__shfl_sync(0xffffffffu, ok, 0)) stop = true;
+            }
+            if (!stop && ns > nold_d) stop = !product(nold_d);
+            if (!vdir && !stop && lane == 0 &&
+                !sm100::mbar_wait(&sm.tbar, k & 1, a.status, a.limit_ns))
+                stop = true;   // the far-field sums have landed in B.T / B.R
+            stop = __shfl_sync(0xffffffffu, stop ? 1 : 0, 0) != 0;
             rq += ns;
             if (stop && lane == 0) {
                 atomicExch(a.abort_word, 1);
@@ -574,10 +608,6 @@ __device__ void leaf_loaders(const FusedArgs& a, const LeafMaps* maps, LeafGroup
         // box path: the two warps may stop independently; they agree through sm.stop after the
         // barrier below (a warp leaving alone would strand the other at a named barrier)
         if (stop && !box) break;
-        if (box && lead && !sm100::mbar_wait(&sm.tbar, k & 1, a.status, a.limit_ns)) {
-            atomicExch(a.abort_word, 1);
-            sm.stop = 1;
-        }
         group_sync(g);
         if (*(volatile int*)&sm.stop) break;
         if (box) {
@@ -1081,20 +1111,56 @@ round_kernel(const __grid_constant__ CUtensorMap loth, const __grid_constant__ C
     gemm_role(&loth, &lotl, &eth, &etl, &uh, &ul, &lith, &litl, a, round_smem);
 }
 
-// Push tasks per source super-block, in the order the sources finish (anti-diagonal, then row).
-__global__ void task_prefix_kernel(int MS, int NS, int* pre, int2* sb) {
-    if (threadIdx.x != 0 || blockIdx.x != 0) return;
-    int idx = 0, acc = 0;
-    for (int d = 0; d < MS + NS - 1; ++d) {
-        for (int A = max(0, d - NS + 1); A <= min(d, MS - 1); ++A) {
-            const int C = d - A;
-            pre[idx] = acc;
-            sb[idx] = make_int2(A, C);
-            acc += 4 * (n_ready(A, MS) + n_ready(C, NS));
-            ++idx;
-        }
+// Push tasks per source super-block, in the order the sources finish (anti-diagonal, then row):
+// pre[idx] = the first task of the idx-th source, sb[idx] its (A, C). One block: each thread
+// takes a contiguous range of source indices, counts their tasks, and a block scan of the
+// per-thread counts gives every range its first task.
+constexpr int kPrefixThreads = 1024;
+__global__ void __launch_bounds__(kPrefixThreads)
+task_prefix_kernel(int MS, int NS, int* pre, int2* sb) {
+    __shared__ int part[kPrefixThreads];
+    const int nsb = MS * NS, tid = threadIdx.x;
+    const int per = (nsb + kPrefixThreads - 1) / kPrefixThreads;
+    const int i0 = min(nsb, tid * per), i1 = min(nsb, i0 + per);
+    // the diagonal d of source index i0 and the index of that diagonal's first source
+    int d = 0, base = 0;
+    while (true) {
+        const int cnt = min(d, MS - 1) - max(0, d - NS + 1) + 1;
+        if (i0 < base + cnt || d >= MS + NS - 2) break;
+        base += cnt;
+        ++d;
     }
-    pre[idx] = acc;
+    auto walk = [&](auto&& f) {   // visits (idx, A, C) for idx in [i0, i1), in order
+        int dd = d, bb = base;
+        for (int i = i0; i < i1; ++i) {
+            int lo = max(0, dd - NS + 1), hi = min(dd, MS - 1);
+            while (i >= bb + hi - lo + 1) {
+                bb += hi - lo + 1;
+                ++dd;
+                lo = max(0, dd - NS + 1);
+                hi = min(dd, MS - 1);
+            }
+            const int A = lo + (i - bb);
+            f(i, A, dd - A);
+        }
+    };
+    int mine = 0;
+    walk([&](int, int A, int C) { mine += 4 * (n_ready(A, MS) + n_ready(C, NS)); });
+    part[tid] = mine;
+    __syncthreads();
+    for (int off = 1; off < kPrefixThreads; off <<= 1) {   // inclusive scan
+        const int v = tid >= off ? part[tid - off] : 0;
+        __syncthreads();
+        part[tid] += v;
+        __syncthreads();
+    }
+    int acc = part[tid] - mine;
+    walk([&](int i, int A, int C) {
+        pre[i] = acc;
+        sb[i] = make_int2(A, C);
+        acc += 4 * (n_ready(A, MS) + n_ready(C, NS));
+    });
+    if (tid == kPrefixThreads - 1) pre[nsb] = part[tid];
 }
 
 struct Layout {
@@ -1211,7 +1277,7 @@ int round_impl(const float* Wstar, int m, int n, const float* L_O, const float* 
     // static operands of the pushes: L_O^T and L_I^T as hi/lo planes
     tc::split_planes(L_O, m, m, m, lot_hi, lot_lo, L.ldm, 1, st);
     tc::split_planes(L_I, n, n, n, lit_hi, lit_lo, L.ldn, 1, st);
-    task_prefix_kernel<<<1, 32, 0, st>>>(L.MS, L.NS, task_pre, task_sb);
+    task_prefix_kernel<<<1, kPrefixThreads, 0, st>>>(L.MS, L.NS, task_pre, task_sb);
     count_launches(1);
 
     CUtensorMap m_loth, m_lotl, m_eth, m_etl, m_uh, m_ul, m_lith, m_litl;
@@ -1263,6 +1329,8 @@ int round_impl(const float* Wstar, int m, int n, const float* L_O, const float* 
     if (a.box_loads) {
         if ((e = tc::make_box_map(&lm.lo, L_O, m, m, m, LB, true))) return e;
         if ((e = tc::make_box_map(&lm.li, L_I, n, n, n, LB, true))) return e;
+        if ((e = tc::make_box_map(&lm.lod, L_O, m, m, m, LB))) return e;
+        if ((e = tc::make_box_map(&lm.lid, L_I, n, n, n, LB))) return e;
         if ((e = tc::make_box_map(&lm.e, E, m, n, n, LB, true))) return e;
         if ((e = tc::make_box_map(&lm.ut, Ut, n, m, L.ldm, LB, true))) return e;
         if ((e = tc::make_box_map(&lm.ws, Wstar, m, n, n, LB))) return e;
