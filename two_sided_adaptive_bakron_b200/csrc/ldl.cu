@@ -25,6 +25,10 @@
 // stay free for that chain. The side stream runs (a) of outer block o - 1 after (b) of o, the
 // only other update of those columns. The panel planes alternate between two sets, so (b) can
 // still read outer block o's planes while o - 1's panels are written.
+// Inside an outer block, likewise, the caller's stream applies a panel only to the next
+// diagonal block before factoring it; a second side stream applies the same panel to the next
+// panel's input columns (which the caller's stream waits for before that panel) and then to the
+// later columns of the outer block (waited for before the diagonal block after next).
 #include <algorithm>
 #include <atomic>
 #include <mutex>
@@ -133,25 +137,29 @@ std::mutex g_side_mu;
 cudaStream_t g_side[kMaxDevices][kSidePool] = {};
 std::atomic<unsigned> g_side_next{0};
 
-int side_stream(cudaStream_t* out) {
+// Two distinct side streams of the current device's pool.
+int side_streams(cudaStream_t* a, cudaStream_t* b) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
         return BAKRON_ERR_CUDA;
-    const unsigned k = g_side_next.fetch_add(1, std::memory_order_relaxed) % kSidePool;
+    const unsigned k = g_side_next.fetch_add(2, std::memory_order_relaxed) % kSidePool;
     std::lock_guard<std::mutex> lock(g_side_mu);
-    if (!g_side[dev][k] &&
-        cudaStreamCreateWithFlags(&g_side[dev][k], cudaStreamNonBlocking) != cudaSuccess) {
-        g_side[dev][k] = nullptr;
-        return BAKRON_ERR_CUDA;
+    cudaStream_t* out[2] = {a, b};
+    for (unsigned i = 0; i < 2; ++i) {
+        cudaStream_t& s = g_side[dev][(k + i) % kSidePool];
+        if (!s && cudaStreamCreateWithFlags(&s, cudaStreamNonBlocking) != cudaSuccess) {
+            s = nullptr;
+            return BAKRON_ERR_CUDA;
+        }
+        *out[i] = s;
     }
-    *out = g_side[dev][k];
     return BAKRON_OK;
 }
 
 // Events of one call, released when the call has enqueued everything (their pending waits
 // still complete).
 struct CallEvents {
-    static constexpr int kCount = 3;
+    static constexpr int kCount = 6;
     cudaEvent_t ev[kCount] = {};
     int n = 0;
     ~CallEvents() {
@@ -204,16 +212,20 @@ extern "C" int bakron_ldl(const float* H, int n, float* L, float* D, void* ws, s
         if ((e = tc::make_kmajor_map(&m_uh[k], w.set[k].u_hi, n, NBO, NBO, BN))) return e;
         if ((e = tc::make_kmajor_map(&m_ul[k], w.set[k].u_lo, n, NBO, NBO, BN))) return e;
     }
-    // look-ahead: a side stream and the call's events (ready: an outer block's panels are
-    // written; next: the next outer block's columns are updated; join: the side stream's end)
+    // look-ahead: two side streams and the call's events (ready: an outer block's panels are
+    // written; next: the next outer block's columns are updated; join: the side stream's end;
+    // panel: a panel is written; npanel: the next panel's input columns are updated; rest:
+    // the later columns of the outer block are updated)
     const bool ahead = nsets == 2;
-    cudaStream_t side = nullptr;
+    cudaStream_t side = nullptr, s3 = nullptr;
     CallEvents evs;
     if (ahead) {
-        if ((e = side_stream(&side))) return e;
+        if ((e = side_streams(&side, &s3))) return e;
         if ((e = evs.make())) return e;
     }
     cudaEvent_t ev_ready = evs.ev[0], ev_next = evs.ev[1], ev_join = evs.ev[2];
+    cudaEvent_t ev_panel = evs.ev[3], ev_npanel = evs.ev[4], ev_rest = evs.ev[5];
+    bool npanel_pending = false, rest_pending = false;
 
     const int eb = 1184;
     copy_upper_kernel<<<eb, 256, 0, st>>>(H, L, n);
@@ -230,6 +242,10 @@ extern "C" int bakron_ldl(const float* H, int n, float* L, float* D, void* ws, s
                                                                   w.inv_lo, dev_status);
             count_launches(1);
             if (kb0 == 0) continue;
+            if (npanel_pending) {   // this panel's input columns, updated by the previous panel
+                if ((e = cuda_err(cudaStreamWaitEvent(st, ev_npanel, 0)))) return e;
+                npanel_pending = false;
+            }
             // panel: X = H'[0:kb0, B] U_BB^{-T}
             tc::split_planes(L + kb0, kb0, b, n, w.p_hi, w.p_lo, NBI, 0, st);
             CUtensorMap m_ph, m_pl, m_ih, m_il;
@@ -244,13 +260,49 @@ extern "C" int bakron_ldl(const float* H, int n, float* L, float* D, void* ws, s
                 return e;
             // columns of the outer block still pending: H'[0:kb0, ko0:kb0] -= X U_AB^T
             if (kb0 > ko0) {
-                tc::ProblemList wl(BN);
-                wl.add(0, c_off, ko0, c_off, kb0, kb0 - ko0, b, 0, ko0, -1.f);
                 tc::EpiStore es{L, n, 1, 1};
-                if ((e = tc::launch_gemm3x<BN, STAGES>(m_xh[ps], m_xl[ps], m_uh[ps], m_ul[ps], wl,
+                if (!ahead) {
+                    tc::ProblemList wl(BN);
+                    wl.add(0, c_off, ko0, c_off, kb0, kb0 - ko0, b, 0, ko0, -1.f);
+                    if ((e = tc::launch_gemm3x<BN, STAGES>(m_xh[ps], m_xl[ps], m_uh[ps],
+                                                           m_ul[ps], wl, es, dev_status, st)))
+                        return e;
+                    continue;
+                }
+                // the next inner block [nb0, kb0): its input columns above it and the later
+                // columns [ko0, nb0) on the second side stream, its diagonal block here
+                const int nb0 = std::max(ko0, kb0 - NBI);
+                if ((e = cuda_err(cudaEventRecord(ev_panel, st)))) return e;
+                if ((e = cuda_err(cudaStreamWaitEvent(s3, ev_panel, 0)))) return e;
+                tc::ProblemList nl(BN);
+                nl.add(0, c_off, nb0, c_off, nb0, kb0 - nb0, b, 0, nb0, -1.f);
+                if ((e = tc::launch_gemm3x<BN, STAGES>(m_xh[ps], m_xl[ps], m_uh[ps], m_ul[ps], nl,
+                                                       es, dev_status, s3)))
+                    return e;
+                if ((e = cuda_err(cudaEventRecord(ev_npanel, s3)))) return e;
+                npanel_pending = true;
+                if (nb0 > ko0) {
+                    tc::ProblemList rl(BN);
+                    rl.add(0, c_off, ko0, c_off, nb0, nb0 - ko0, b, 0, ko0, -1.f);
+                    if ((e = tc::launch_gemm3x<BN, STAGES>(m_xh[ps], m_xl[ps], m_uh[ps],
+                                                           m_ul[ps], rl, es, dev_status, s3)))
+                        return e;
+                }
+                // the previous panel's later columns hold the next diagonal block: they go first
+                if (rest_pending && (e = cuda_err(cudaStreamWaitEvent(st, ev_rest, 0)))) return e;
+                if ((e = cuda_err(cudaEventRecord(ev_rest, s3)))) return e;
+                rest_pending = true;
+                tc::ProblemList tl(BN);
+                tl.add(nb0, c_off, nb0, c_off, kb0 - nb0, kb0 - nb0, b, nb0, nb0, -1.f,
+                       /*upper_only=*/1);
+                if ((e = tc::launch_gemm3x<BN, STAGES>(m_xh[ps], m_xl[ps], m_uh[ps], m_ul[ps], tl,
                                                        es, dev_status, st)))
                     return e;
             }
+        }
+        if (rest_pending) {   // everything the second side stream did for this outer block
+            if ((e = cuda_err(cudaStreamWaitEvent(st, ev_rest, 0)))) return e;
+            rest_pending = npanel_pending = false;
         }
         if (ko0 == 0) continue;
         // the rest of the trailing matrix, once per outer block: upper block triangle of
