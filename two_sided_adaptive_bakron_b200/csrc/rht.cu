@@ -10,7 +10,8 @@
 // rounding; the proxy loss is the same in both bases.
 //
 // One CTA transforms one row with the row in registers: the signs (one Philox4x64-10 block per
-// 256 indices, keyed (seed, 0) at counter (i / 256, 0, 1, 0), bit i % 256, set = -1), the
+// 256 indices, keyed (seed, 0) at counter (i / 256, 0, 1, 0), bit i % 256, set = -1; drawn once
+// per call by rht_signs_kernel, copied by every row's CTA), the
 // Sylvester butterflies over each 2^k segment (the fast Walsh-Hadamard transform: a pair
 // (i, i ^ h) with 2h <= 2^k never leaves its segment), by warp shuffles, shared memory or
 // inside a thread depending on the stride, then the order-28 stage across segments, and the
@@ -98,10 +99,22 @@ struct H28f {
 // textbook order (strides 1, 2, 4, ..., then the order-28 sums in index order).
 constexpr int kRowThreads = 512;
 
+// The sign words of T_d: words[4 b + q] = word q of the Philox4x64-10 block keyed (seed, 0) at
+// counter (b, 0, 1, 0), for the (d + 255) / 256 blocks b; bit i % 64 of word i / 64 is index i.
+__global__ void rht_signs_kernel(int d, unsigned long long seed, uint64_t* __restrict__ words) {
+    const int nblk = (d + 255) / 256;
+    for (int b = blockIdx.x * blockDim.x + threadIdx.x; b < nblk; b += gridDim.x * blockDim.x) {
+        uint64_t w[4];
+        philox4x64_10((uint64_t)b, 0, 1, 0, seed, 0, w);
+        for (int q = 0; q < 4; ++q) words[4 * b + q] = w[q];
+    }
+}
+
 template <int U, int OUTER, bool kInverse>
 __global__ void __launch_bounds__(kRowThreads)
 rht_rows_kernel(const float* __restrict__ X, float* __restrict__ Y, int d, int T,
-                unsigned long long seed, float scale, const __grid_constant__ H28f H) {
+                const uint64_t* __restrict__ signs, float scale,
+                const __grid_constant__ H28f H) {
     constexpr int E = OUTER * U;
     extern __shared__ __align__(16) uint8_t rht_smem[];
     float* buf = reinterpret_cast<float*>(rht_smem);                    // d floats (exchange)
@@ -109,12 +122,8 @@ rht_rows_kernel(const float* __restrict__ X, float* __restrict__ Y, int d, int T
     const size_t row = blockIdx.x;
     const int t = threadIdx.x;
     const bool own = t < T;                   // blockDim.x = max(T, 32)
-    const int nblk = (d + 255) / 256;
-    for (int b = t; b < nblk; b += blockDim.x) {
-        uint64_t w[4];
-        philox4x64_10((uint64_t)b, 0, 1, 0, seed, 0, w);
-        for (int q = 0; q < 4; ++q) sw[4 * b + q] = w[q];
-    }
+    const int nwords = 4 * ((d + 255) / 256);
+    for (int q = t; q < nwords; q += blockDim.x) sw[q] = __ldg(&signs[q]);
     const float* x = X + row * (size_t)d;
     float v[E];
 #pragma unroll
@@ -214,7 +223,7 @@ __global__ void row_scales_kernel(const float* __restrict__ W, int n, int group,
 }
 
 template <int U, int OUTER, bool kInverse>
-int launch_rows(const float* X, float* Y, int rows, int d, unsigned long long seed,
+int launch_rows(const float* X, float* Y, int rows, int d, const uint64_t* signs,
                 const H28f& H, cudaStream_t st) {
     const int T = d / (OUTER * U);
     const size_t smem = (size_t)((d + 3) & ~3) * sizeof(float) +
@@ -224,41 +233,41 @@ int launch_rows(const float* X, float* Y, int rows, int d, unsigned long long se
         cudaSuccess)
         return BAKRON_ERR_CUDA;
     const float scale = 1.0f / sqrtf((float)d);
-    kern<<<rows, T < 32 ? 32 : T, smem, st>>>(X, Y, d, T, seed, scale, H);
+    kern<<<rows, T < 32 ? 32 : T, smem, st>>>(X, Y, d, T, signs, scale, H);
     count_launches(1);
     return cuda_err(cudaGetLastError());
 }
 
 // T = min(seg, 512) threads, U = seg / T columns of each segment per thread.
 template <bool kInverse>
-int rows_pass_dir(const float* X, float* Y, int rows, int d, unsigned long long seed,
+int rows_pass_dir(const float* X, float* Y, int rows, int d, const uint64_t* signs,
                   const H28f& H, cudaStream_t st) {
     int seg = 0;
     const int outer = factor(d, seg);
     const int U = seg <= kRowThreads ? 1 : seg / kRowThreads;
     if (outer == 28) {
         switch (U) {
-            case 1: return launch_rows<1, 28, kInverse>(X, Y, rows, d, seed, H, st);
-            case 2: return launch_rows<2, 28, kInverse>(X, Y, rows, d, seed, H, st);
+            case 1: return launch_rows<1, 28, kInverse>(X, Y, rows, d, signs, H, st);
+            case 2: return launch_rows<2, 28, kInverse>(X, Y, rows, d, signs, H, st);
             default: return BAKRON_ERR_INVALID_ARG;
         }
     }
     switch (U) {
-        case 1: return launch_rows<1, 1, kInverse>(X, Y, rows, d, seed, H, st);
-        case 2: return launch_rows<2, 1, kInverse>(X, Y, rows, d, seed, H, st);
-        case 4: return launch_rows<4, 1, kInverse>(X, Y, rows, d, seed, H, st);
-        case 8: return launch_rows<8, 1, kInverse>(X, Y, rows, d, seed, H, st);
-        case 16: return launch_rows<16, 1, kInverse>(X, Y, rows, d, seed, H, st);
-        case 32: return launch_rows<32, 1, kInverse>(X, Y, rows, d, seed, H, st);
-        case 64: return launch_rows<64, 1, kInverse>(X, Y, rows, d, seed, H, st);
+        case 1: return launch_rows<1, 1, kInverse>(X, Y, rows, d, signs, H, st);
+        case 2: return launch_rows<2, 1, kInverse>(X, Y, rows, d, signs, H, st);
+        case 4: return launch_rows<4, 1, kInverse>(X, Y, rows, d, signs, H, st);
+        case 8: return launch_rows<8, 1, kInverse>(X, Y, rows, d, signs, H, st);
+        case 16: return launch_rows<16, 1, kInverse>(X, Y, rows, d, signs, H, st);
+        case 32: return launch_rows<32, 1, kInverse>(X, Y, rows, d, signs, H, st);
+        case 64: return launch_rows<64, 1, kInverse>(X, Y, rows, d, signs, H, st);
         default: return BAKRON_ERR_INVALID_ARG;
     }
 }
 
-int rows_pass(const float* X, float* Y, int rows, int d, unsigned long long seed, int inverse,
+int rows_pass(const float* X, float* Y, int rows, int d, const uint64_t* signs, int inverse,
               const H28f& H, cudaStream_t st) {
-    return inverse ? rows_pass_dir<true>(X, Y, rows, d, seed, H, st)
-                   : rows_pass_dir<false>(X, Y, rows, d, seed, H, st);
+    return inverse ? rows_pass_dir<true>(X, Y, rows, d, signs, H, st)
+                   : rows_pass_dir<false>(X, Y, rows, d, signs, H, st);
 }
 
 void transpose(const float* X, float* Y, int r, int c, cudaStream_t st) {
@@ -281,10 +290,14 @@ extern "C" int bakron_rht_supported(int d) {
     return factor(d, seg) != 0 ? 1 : 0;
 }
 
+inline size_t sign_words(int d) { return 4 * (size_t)((d + 255) / 256); }
+
 extern "C" size_t bakron_rht_workspace_bytes(int rows, int cols) {
     if (rows < 1 || cols < 1) return 0;
     WsSizer z;
     z.take<float>((size_t)rows * cols);
+    z.take<uint64_t>(sign_words(cols));
+    z.take<uint64_t>(sign_words(rows));
     return z.bytes();
 }
 
@@ -306,12 +319,18 @@ extern "C" int bakron_rht(const float* X, int rows, int cols, uint64_t seed_rows
     }();
     WsCarver c(ws);
     float* t = c.take<float>((size_t)rows * cols);
+    uint64_t* sc_words = c.take<uint64_t>(sign_words(cols));
+    uint64_t* sr_words = c.take<uint64_t>(sign_words(rows));
+    // the signs of T_c and T_r, drawn once for every row
+    rht_signs_kernel<<<(cols / 256 + 64) / 64, 64, 0, st>>>(cols, seed_cols, sc_words);
+    rht_signs_kernel<<<(rows / 256 + 64) / 64, 64, 0, st>>>(rows, seed_rows, sr_words);
+    count_launches(2);
     int e;
     // Y = X T_c^T (inverse: X T_c): each row x -> T_c x (inverse: T_c^T x)
-    if ((e = rows_pass(X, Y, rows, cols, seed_cols, inverse, H, st))) return e;
+    if ((e = rows_pass(X, Y, rows, cols, sc_words, inverse, H, st))) return e;
     // then T_r Y (inverse: T_r^T Y) as a row pass over Y^T
     transpose(Y, t, rows, cols, st);
-    if ((e = rows_pass(t, t, cols, rows, seed_rows, inverse, H, st))) return e;
+    if ((e = rows_pass(t, t, cols, rows, sr_words, inverse, H, st))) return e;
     transpose(t, Y, cols, rows, st);
     return cuda_err(cudaGetLastError());
 }
