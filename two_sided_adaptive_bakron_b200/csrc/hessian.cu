@@ -13,7 +13,9 @@
 //   Sketch B, H_I:      P = [G_1; ...; G_S]^T          (d = n, K = S m)
 //   Sketch B, H_O:      P = [G_1, G_2, ..., G_S]       (d = m, K = S n)
 // The product runs on the 3xTF32 tcgen05 GEMM engine over the upper block triangle only
-// (d (d + 1) K / 2 multiply-adds). Then the diagonal is summed in fp64 in a fixed order and one
+// (d (d + 1) K / 2 multiply-adds) in chunks of kChunkK samples: the tensor core's fp32
+// accumulator is restarted every chunk and the chunk sums are added in round-to-nearest fp32,
+// so the accumulation error stays at one chunk's level instead of growing with K. Then the diagonal is summed in fp64 in a fixed order and one
 // kernel transposes the upper triangle into the lower one through shared memory while adding
 // damp * mean(diag) to the diagonal, so H is exactly symmetric.
 #include <algorithm>
@@ -25,6 +27,8 @@ namespace {
 
 constexpr int BN = 128;   // square tiles (BM == BN) for the upper block triangle
 constexpr int STAGES = 3;
+constexpr int kChunkKb = 8;                 // k-blocks per accumulator chunk
+constexpr int kChunkK = kChunkKb * tc::BK;  // = 256 samples
 constexpr int kMaxSplitRows = 65535 * 32;   // the transposed plane split's grid limit
 
 // out[0] = sum_i H[i][i], one block, fixed order.
@@ -76,7 +80,8 @@ int gram_from_planes(float* p_hi, float* p_lo, int d, int K, int ldk, float damp
     tc::ProblemList pl(BN);
     pl.add(0, 0, 0, 0, d, d, K, 0, 0, 1.f / (float)K, /*upper_only=*/1);
     tc::EpiStore epi{H, d, /*accumulate=*/0, /*upper=*/1};
-    if ((e = tc::launch_gemm3x<BN, STAGES>(mh, ml, mh, ml, pl, epi, dev_status, st))) return e;
+    if ((e = tc::launch_gemm3x<BN, STAGES, kChunkKb>(mh, ml, mh, ml, pl, epi, dev_status, st)))
+        return e;
     diag_sum_kernel<<<1, 1024, 0, st>>>(H, d, dsum);
     const int nt = (d + 31) / 32;
     mirror_damp_kernel<<<dim3(nt, nt), dim3(32, 8), 0, st>>>(H, d, dsum, damp);

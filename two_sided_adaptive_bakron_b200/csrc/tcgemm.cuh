@@ -18,6 +18,14 @@
 //                     32 (w % 4) .. + 31 = tile rows), then the Epi functor, then the
 //                     accumulator goes back to the MMA issuer, so a tile's epilogue overlaps
 //                     the next tile's MMAs.
+// Chunked accumulation (CHUNK > 0): the tensor core's fp32 accumulator does not round to
+// nearest, so its error grows with the number of MMAs summed into it. With CHUNK > 0 the issuer
+// restarts the accumulator every CHUNK k-blocks and hands each partial sum over like a tile;
+// the epilogue adds the partials in registers (fp32, round to nearest, in k order) and runs the
+// Epi functor once per tile on their sum. The accumulator then never holds more than
+// 3 CHUNK BK / 8 instructions' worth of products, whatever K is. This mode takes four TMEM
+// accumulators (4 x BN columns), so the issuer can run two chunks ahead of an epilogue that
+// is still writing out the previous tile.
 // A launch may hold several problems (a grouped GEMM): the operand tensor maps cover whole
 // planes and every problem only moves the tile origins.
 // Every mbarrier wait is bounded and also gives up when another role has raised the CTA's
@@ -114,22 +122,35 @@ __device__ __forceinline__ bool decode_tile(const Problems& P, int BNv, int t, i
     return false;
 }
 
-template <int BN, int STAGES, class Epi>
+// k-blocks per accumulator hand-off and hand-offs per tile (K = 0: one, of zeros)
+template <int CHUNK>
+__device__ __forceinline__ int chunk_len(int nkb) { return CHUNK > 0 ? CHUNK : (nkb > 0 ? nkb : 1); }
+template <int CHUNK>
+__device__ __forceinline__ int chunk_count(int nkb) {
+    return nkb > 0 ? (nkb + chunk_len<CHUNK>(nkb) - 1) / chunk_len<CHUNK>(nkb) : 1;
+}
+
+template <int BN, int STAGES, class Epi, int CHUNK = 0>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm3x_kernel(const __grid_constant__ CUtensorMap a_hi, const __grid_constant__ CUtensorMap a_lo,
               const __grid_constant__ CUtensorMap b_hi, const __grid_constant__ CUtensorMap b_lo,
               const __grid_constant__ Problems probs, const Epi epi, int* status,
               uint64_t limit_ns) {
     using C = Cfg<BN>;
+    // accumulators in TMEM: two, or four for chunked accumulation, so that the epilogue may
+    // still be writing a finished tile while the issuer fills the next tile's first chunks
+    constexpr int NACC = (CHUNK > 0 && 4 * BN <= 512) ? 4 : 2;
+    constexpr uint32_t kTmemCols = NACC * BN;
+    static_assert((2 * STAGES + 2 * NACC + 1) * 8 + 8 <= 256, "barrier area");
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     float* epi_stage = reinterpret_cast<float*>(smem + STAGES * C::kStageBytes);
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * C::kStageBytes + C::kEpiBytes);
     uint64_t* empty = full + STAGES;
-    uint64_t* acc_full = empty + STAGES;   // [2] accumulator ready for the epilogue
-    uint64_t* acc_empty = acc_full + 2;    // [2] accumulator read out (4 epilogue warps)
-    uint64_t* drain = acc_empty + 2;       // error path: all MMAs retired
+    uint64_t* acc_full = empty + STAGES;   // [NACC] accumulator ready for the epilogue
+    uint64_t* acc_empty = acc_full + NACC; // [NACC] accumulator read out (4 epilogue warps)
+    uint64_t* drain = acc_empty + NACC;    // error path: all MMAs retired
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
     volatile int* s_abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -141,7 +162,7 @@ gemm3x_kernel(const __grid_constant__ CUtensorMap a_hi, const __grid_constant__ 
             sm100::mbar_init(&full[s], 1);
             sm100::mbar_init(&empty[s], 1);
         }
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < NACC; ++b) {
             sm100::mbar_init(&acc_full[b], 1);
             sm100::mbar_init(&acc_empty[b], 4);
         }
@@ -150,7 +171,7 @@ gemm3x_kernel(const __grid_constant__ CUtensorMap a_hi, const __grid_constant__ 
         sm100::fence_mbar_init();
     }
     if (warp == 1) {
-        sm100::tmem_alloc(tmem_slot, C::kTmemCols);
+        sm100::tmem_alloc(tmem_slot, kTmemCols);
         sm100::tmem_relinquish();
     }
     sm100::tc_fence_before();
@@ -201,46 +222,53 @@ gemm3x_kernel(const __grid_constant__ CUtensorMap a_hi, const __grid_constant__ 
         if (lane == 0) {
             constexpr uint32_t idesc = sm100::idesc_tf32(BM, BN);
             uint32_t g = 0;   // k-blocks consumed
-            int i = 0;        // tiles of this CTA
-            for (int t = blockIdx.x; t < total && !*s_abort; t += gridDim.x, ++i) {
+            uint32_t u = 0;   // accumulator hand-offs (one per tile, or per chunk)
+            bool ok = true;
+            for (int t = blockIdx.x; t < total && ok && !*s_abort; t += gridDim.x) {
                 int pi, m0, n0;
                 if (!decode_tile(probs, BN, t, pi, m0, n0)) break;
                 const int nkb = (probs.p[pi].K + BK - 1) / BK;
-                const int b = i & 1;
-                if (i >= 2 &&
-                    !wait_or_abort(&acc_empty[b], ((i >> 1) & 1) ^ 1, status, limit_ns, s_abort))
-                    break;
-                sm100::tc_fence_after();
-                const uint32_t acc = tmem + (uint32_t)(b * BN);
-                bool ok = true;
-                for (int kb = 0; kb < nkb; ++kb, ++g) {
-                    const int s = g % STAGES;
-                    if (!wait_or_abort(&full[s], (g / STAGES) & 1, status, limit_ns, s_abort)) {
+                const int per = chunk_len<CHUNK>(nkb), nch = chunk_count<CHUNK>(nkb);
+                for (int j = 0; j < nch; ++j, ++u) {
+                    const int b = u % NACC;
+                    if (u >= NACC &&
+                        !wait_or_abort(&acc_empty[b], ((u / NACC) & 1) ^ 1, status, limit_ns,
+                                       s_abort)) {
                         ok = false;
                         break;
                     }
                     sm100::tc_fence_after();
-                    const uint32_t ah = sm100::smem_u32(stage_ptr(s, 0));
-                    const uint32_t al = sm100::smem_u32(stage_ptr(s, 1));
-                    const uint32_t bh = sm100::smem_u32(stage_ptr(s, 2));
-                    const uint32_t bl = sm100::smem_u32(stage_ptr(s, 3));
+                    const uint32_t acc = tmem + (uint32_t)(b * BN);
+                    const int kb0 = j * per, kb1 = min(nkb, kb0 + per);
+                    for (int kb = kb0; kb < kb1; ++kb, ++g) {
+                        const int s = g % STAGES;
+                        if (!wait_or_abort(&full[s], (g / STAGES) & 1, status, limit_ns, s_abort)) {
+                            ok = false;
+                            break;
+                        }
+                        sm100::tc_fence_after();
+                        const uint32_t ah = sm100::smem_u32(stage_ptr(s, 0));
+                        const uint32_t al = sm100::smem_u32(stage_ptr(s, 1));
+                        const uint32_t bh = sm100::smem_u32(stage_ptr(s, 2));
+                        const uint32_t bl = sm100::smem_u32(stage_ptr(s, 3));
 #pragma unroll
-                    for (int kk = 0; kk < BK / 8; ++kk) {
-                        const uint32_t off = kk * 32;  // 8 tf32 = 32 bytes along the swizzled row
-                        const uint64_t dah = sm100::desc_kmajor_sw128(ah + off);
-                        const uint64_t dal = sm100::desc_kmajor_sw128(al + off);
-                        const uint64_t dbh = sm100::desc_kmajor_sw128(bh + off);
-                        const uint64_t dbl = sm100::desc_kmajor_sw128(bl + off);
-                        const uint32_t acc0 = (kb > 0 || kk > 0) ? 1u : 0u;
-                        sm100::mma_tf32(acc, dah, dbh, idesc, acc0);
-                        sm100::mma_tf32(acc, dah, dbl, idesc, 1u);
-                        sm100::mma_tf32(acc, dal, dbh, idesc, 1u);
+                        for (int kk = 0; kk < BK / 8; ++kk) {
+                            const uint32_t off = kk * 32;  // 8 tf32 = 32 bytes along the swizzled row
+                            const uint64_t dah = sm100::desc_kmajor_sw128(ah + off);
+                            const uint64_t dal = sm100::desc_kmajor_sw128(al + off);
+                            const uint64_t dbh = sm100::desc_kmajor_sw128(bh + off);
+                            const uint64_t dbl = sm100::desc_kmajor_sw128(bl + off);
+                            const uint32_t acc0 = (kb > kb0 || kk > 0) ? 1u : 0u;
+                            sm100::mma_tf32(acc, dah, dbh, idesc, acc0);
+                            sm100::mma_tf32(acc, dah, dbl, idesc, 1u);
+                            sm100::mma_tf32(acc, dal, dbh, idesc, 1u);
+                        }
+                        sm100::mma_commit(&empty[s]);
                     }
-                    sm100::mma_commit(&empty[s]);
+                    if (!ok) break;
+                    if (nkb > 0) sm100::mma_commit(&acc_full[b]);
+                    else sm100::mbar_arrive(&acc_full[b]);   // K = 0: the epilogue writes zeros
                 }
-                if (!ok) break;
-                if (nkb > 0) sm100::mma_commit(&acc_full[b]);
-                else sm100::mbar_arrive(&acc_full[b]);   // K = 0: the epilogue writes zeros
             }
             if (*s_abort) {
                 sm100::mma_commit(drain);
@@ -252,44 +280,86 @@ gemm3x_kernel(const __grid_constant__ CUtensorMap a_hi, const __grid_constant__ 
         Epi e = epi;
         const int quarter = warp & 3;   // TMEM lanes this warp may read
         float* stage = epi_stage + (warp - kEpiWarp0) * (32 * 33);
-        int i = 0;
-        for (int t = blockIdx.x; t < total; t += gridDim.x, ++i) {
+        uint32_t u = 0;   // accumulator hand-offs, in the issuer's order
+        bool ok = true;
+        // lane 0 waits for hand-off u; the warp learns the outcome
+        auto take = [&](uint32_t uu) {
+            bool r = true;
+            if (lane == 0)
+                r = wait_or_abort(&acc_full[uu % NACC], (uu / NACC) & 1, status, limit_ns, s_abort);
+            r = __shfl_sync(0xffffffffu, r ? 1 : 0, 0) != 0;
+            if (r) sm100::tc_fence_after();
+            return r;
+        };
+        auto give_back = [&](uint32_t uu) {
+            sm100::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) sm100::mbar_arrive(&acc_empty[uu % NACC]);
+        };
+        auto taddr = [&](uint32_t uu, int c0) {
+            return tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)((uu % NACC) * BN + c0);
+        };
+        for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
             int pi, m0, n0;
             if (!decode_tile(probs, BN, t, pi, m0, n0)) break;
             const Problem& P = probs.p[pi];
-            const int b = i & 1;
-            bool ok = true;
-            if (lane == 0) ok = wait_or_abort(&acc_full[b], (i >> 1) & 1, status, limit_ns, s_abort);
-            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-            if (!ok) break;
-            sm100::tc_fence_after();
             const bool have = P.K > 0;
+            if constexpr (CHUNK == 0) {
+                if (!(ok = take(u))) break;
 #pragma unroll 1
-            for (int c0 = 0; c0 < BN; c0 += 32) {
-                float v[32];
-                if (have) {
-                    sm100::tmem_ld32(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(b * BN + c0), v);
-                } else {
+                for (int c0 = 0; c0 < BN; c0 += 32) {
+                    float v[32];
+                    if (have) {
+                        sm100::tmem_ld32(taddr(u, c0), v);
+                    } else {
 #pragma unroll
-                    for (int q = 0; q < 32; ++q) v[q] = 0.f;
+                        for (int q = 0; q < 32; ++q) v[q] = 0.f;
+                    }
+#pragma unroll
+                    for (int q = 0; q < 32; ++q) stage[lane * 33 + q] = v[q];
+                    __syncwarp();
+                    // lane = column n0 + c0 + lane, element rr of the chunk at stage[rr * 33 + lane]
+                    e.chunk(P, m0 + quarter * 32, n0 + c0 + lane, m0, n0, stage + lane);
+                    __syncwarp();
                 }
+                give_back(u++);
+            } else {
+                const int nch = chunk_count<CHUNK>((P.K + BK - 1) / BK);
+                float sum[BN / 32][32];
 #pragma unroll
-                for (int q = 0; q < 32; ++q) stage[lane * 33 + q] = v[q];
-                __syncwarp();
-                // lane = column n0 + c0 + lane, element rr of the chunk at stage[rr * 33 + lane]
-                e.chunk(P, m0 + quarter * 32, n0 + c0 + lane, m0, n0, stage + lane);
-                __syncwarp();
+                for (int c = 0; c < BN / 32; ++c)
+#pragma unroll
+                    for (int q = 0; q < 32; ++q) sum[c][q] = 0.f;
+                for (int j = 0; j < nch; ++j) {
+                    if (!(ok = take(u))) break;
+                    if (have) {
+#pragma unroll
+                        for (int c = 0; c < BN / 32; ++c) {
+                            float v[32];
+                            sm100::tmem_ld32(taddr(u, c * 32), v);
+#pragma unroll
+                            for (int q = 0; q < 32; ++q) sum[c][q] += v[q];
+                        }
+                    }
+                    give_back(u++);
+                }
+                if (!ok) break;
+#pragma unroll
+                for (int c = 0; c < BN / 32; ++c) {
+#pragma unroll
+                    for (int q = 0; q < 32; ++q) stage[lane * 33 + q] = sum[c][q];
+                    __syncwarp();
+                    e.chunk(P, m0 + quarter * 32, n0 + c * 32 + lane, m0, n0, stage + lane);
+                    __syncwarp();
+                }
             }
             e.tile_done(P, t, quarter);
-            sm100::tc_fence_before();
-            __syncwarp();
-            if (lane == 0) sm100::mbar_arrive(&acc_empty[b]);
         }
     }
     __syncwarp();   // the producer and MMA warps reconverge with their idle lanes
     sm100::tc_fence_before();
     __syncthreads();
-    if (warp == 1) sm100::tmem_dealloc(tmem, C::kTmemCols);
+    if (warp == 1) sm100::tmem_dealloc(tmem, kTmemCols);
 }
 
 }  // namespace tc

@@ -146,8 +146,9 @@ struct ProblemList {
 int sm_count();
 
 // Launches the grouped GEMM with min(tiles, max_ctas) persistent CTAs (max_ctas <= 0: one per
-// SM). A smaller max_ctas leaves SMs free for work on other streams.
-template <int BN, int STAGES, class Epi>
+// SM). A smaller max_ctas leaves SMs free for work on other streams. CHUNK > 0 restarts the
+// accumulator every CHUNK k-blocks and sums the partials in round-to-nearest fp32.
+template <int BN, int STAGES, int CHUNK = 0, class Epi>
 int launch_gemm3x(const CUtensorMap& ah, const CUtensorMap& al, const CUtensorMap& bh,
                   const CUtensorMap& bl, const ProblemList& L, const Epi& epi, int* status,
                   cudaStream_t st, int max_ctas = 0) {
@@ -157,7 +158,7 @@ int launch_gemm3x(const CUtensorMap& ah, const CUtensorMap& al, const CUtensorMa
         if ((L.P.p[i].a_k0 & 3) || (L.P.p[i].b_k0 & 3)) return BAKRON_ERR_INVALID_ARG;
     constexpr size_t smem = gemm_smem_bytes<BN, STAGES>();
     static_assert(smem <= 227 * 1024, "GEMM shared memory above the per-CTA limit");
-    auto kern = gemm3x_kernel<BN, STAGES, Epi>;
+    auto kern = gemm3x_kernel<BN, STAGES, Epi, CHUNK>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
         cudaSuccess)
         return BAKRON_ERR_CUDA;
