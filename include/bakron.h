@@ -257,9 +257,10 @@ int bakron_sketch_b(const float* G, int S, int m, int n, float damp, float* H_O,
  *   rows, cols [in] each 2^k or 28 * 2^k, at most 32768 (bakron_rht_supported tells).
  *   Y        [out] rows x cols.
  *   ws       [in]  at least bakron_rht_workspace_bytes(rows, cols) bytes, 256-B aligned.
- * Returns BAKRON_ERR_INVALID_ARG for an unsupported size. Four passes over the matrix: the
- * signs, butterflies and order-28 stage along rows in shared memory, then the same along
- * columns through two tiled transposes.
+ * Returns BAKRON_ERR_INVALID_ARG for an unsupported size. Three passes over the matrix: the
+ * signs, butterflies and order-28 stage along each row (one CTA per row), then the same along
+ * the columns in place on Y, on 32-column tiles: strides below 512 in one pass, the larger
+ * strides and the order-28 stage in the next. The workspace holds the sign words only.
  * ---------------------------------------------------------------------------------------- */
 int bakron_rht_supported(int d);
 size_t bakron_rht_workspace_bytes(int rows, int cols);

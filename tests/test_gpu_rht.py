@@ -97,6 +97,25 @@ def test_full_size_sampled_and_round_trip(bk, r, c):
     assert np.abs(got - ref).max() <= 1e-4
 
 
+# column lengths that select the column passes' remaining variants: 28 2^k with 2^k between 32
+# and 512 (896), 2^k above 4096 (8192, 16384, 32768: up to 64 rows per thread in the strided
+# pass) and 28 * 512 (14336: order-28 stage alone in the strided pass)
+@pytest.mark.parametrize("r,c", [(896, 64), (8192, 32), (14336, 28), (16384, 28), (32768, 32)])
+def test_column_lengths_sampled_and_round_trip(bk, r, c):
+    X = np.random.default_rng(r + c).standard_normal((r, c)).astype(np.float32)
+    Xd = _dev(X)
+    Y = bk.rht(Xd, 21, 22)
+    back = bk.rht(Y, 21, 22, inverse=True)
+    nx = float(torch.linalg.norm(Xd.double()))
+    assert float(torch.linalg.norm(back.double() - Xd.double())) <= 4e-5 * nx
+    assert abs(float(torch.linalg.norm(Y.double())) - nx) <= 2e-5 * nx
+    rows = np.unique(np.array([0, 1, 511, 512, r // 28, r // 2, r - 1]))
+    cols = np.arange(c)
+    ref = _t_rows(r, 21, rows) @ X.astype(np.float64) @ _t_rows(c, 22, cols).T
+    got = Y.cpu().numpy()[np.ix_(rows, cols)]
+    assert np.abs(got - ref).max() <= 1e-4
+
+
 @pytest.mark.parametrize("m,n,group,div", [(5, 37, 37, 1.5), (64, 128, 32, 3.5), (3, 100, 7, 1.0)])
 def test_row_scales_exact(bk, m, n, group, div):
     W = np.random.default_rng(m + n).standard_normal((m, n)).astype(np.float32)

@@ -15,8 +15,13 @@
 // Sylvester butterflies over each 2^k segment (the fast Walsh-Hadamard transform: a pair
 // (i, i ^ h) with 2h <= 2^k never leaves its segment), by warp shuffles, shared memory or
 // inside a thread depending on the stride, then the order-28 stage across segments, and the
-// 1/sqrt(d) scale. The column transform is a row transform of the transpose (tiled 32 x 32
-// transposes through shared memory). Every pass reads and writes the matrix once: HBM-bound.
+// 1/sqrt(d) scale. The column transform runs in place on the result in two more passes, on
+// tiles of 32 columns (one 128-byte segment per row): the butterflies of strides below
+// B = min(2^k, 512) inside 512-row tiles (registers, one shared-memory exchange), then, one
+// thread per column and row residue mod B, the larger strides, the order-28 stage and the
+// scale. Every pass reads and writes the matrix once: HBM-bound. Each sum is formed in the
+// same order on both sides (the textbook order: strides 1, 2, 4, ..., then the order-28 sums in
+// index order), so a column's result is bitwise that of the row pass applied to it.
 #include <cmath>
 #include <cstring>
 
@@ -99,6 +104,11 @@ struct H28f {
 // textbook order (strides 1, 2, 4, ..., then the order-28 sums in index order).
 constexpr int kRowThreads = 512;
 
+// x * (bit ? -1 : +1), as a flip of the sign bit: the same bits as the multiplication
+__device__ __forceinline__ float flip_if(float x, uint64_t bit) {
+    return __uint_as_float(__float_as_uint(x) ^ ((uint32_t)bit << 31));
+}
+
 // The sign words of T_d: words[4 b + q] = word q of the Philox4x64-10 block keyed (seed, 0) at
 // counter (b, 0, 1, 0), for the (d + 255) / 256 blocks b; bit i % 64 of word i / 64 is index i.
 __global__ void rht_signs_kernel(int d, unsigned long long seed, uint64_t* __restrict__ words) {
@@ -129,10 +139,10 @@ rht_rows_kernel(const float* __restrict__ X, float* __restrict__ Y, int d, int T
 #pragma unroll
     for (int e = 0; e < E; ++e) v[e] = own ? x[t + T * e] : 0.f;
     __syncthreads();                          // the sign words are in place
-    auto sgn = [&](int j) { return ((sw[j >> 6] >> (j & 63)) & 1ull) ? -1.f : 1.f; };
+    auto sbit = [&](int j) { return (sw[j >> 6] >> (j & 63)) & 1ull; };
     if (!kInverse && own) {
 #pragma unroll
-        for (int e = 0; e < E; ++e) v[e] *= sgn(t + T * e);
+        for (int e = 0; e < E; ++e) v[e] = flip_if(v[e], sbit(t + T * e));
     }
     for (int h = 1; h < T && h < 32; h <<= 1) {
         const bool hi = (t & h) != 0;
@@ -186,23 +196,141 @@ rht_rows_kernel(const float* __restrict__ X, float* __restrict__ Y, int d, int T
 #pragma unroll
     for (int e = 0; e < E; ++e) {
         const int j = t + T * e;
-        y[j] = (kInverse ? v[e] * sgn(j) : v[e]) * scale;
+        y[j] = (kInverse ? flip_if(v[e], sbit(j)) : v[e]) * scale;
     }
 }
 
-// Y (c x r) = X^T for X (r x c), 32 x 32 tiles.
-__global__ void transpose_kernel(const float* __restrict__ X, float* __restrict__ Y, int r,
-                                 int c) {
-    __shared__ float t[32][33];
-    const int r0 = blockIdx.y * 32, c0 = blockIdx.x * 32;
-    for (int k = threadIdx.y; k < 32; k += 8) {
-        const int rr = r0 + k, cc = c0 + threadIdx.x;
-        if (rr < r && cc < c) t[k][threadIdx.x] = X[(size_t)rr * c + cc];
+// Column transform, first pass: Y (r x c, in place) along its rows i, the signs (forward)
+// and the butterflies of strides 1 .. B / 2 of every B-row slab (B = min(2^k, 512), so a slab
+// never leaves a 512-row tile). CTA = 512 consecutive rows x 32 columns, thread (w, lane) =
+// column lane. Phase 1: rows 32 w + e (e < 32) in registers, strides 1 .. 16 inside the thread;
+// phase 2 (B > 32), after one exchange through shared memory: rows w + 16 e, strides
+// 32 .. 256 inside the thread. kFinal (d = 2^k <= 512, nothing left for the second pass): the
+// scale and, inverse, the signs.
+constexpr int kSlabRows = 512;
+constexpr int kSlabThreads = 512;
+constexpr size_t kSlabSmem = (size_t)kSlabRows * 32 * sizeof(float);
+
+__device__ __forceinline__ uint64_t sign_bit(const uint64_t* __restrict__ words, int i) {
+    return (__ldg(&words[i >> 6]) >> (i & 63)) & 1ull;
+}
+
+template <bool kInverse, bool kFinal>
+__global__ void __launch_bounds__(kSlabThreads)
+rht_cols_slab_kernel(float* __restrict__ Y, int r, int c, int B,
+                     const uint64_t* __restrict__ signs, float scale) {
+    extern __shared__ __align__(16) float slab[];   // [512][32]
+    const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int r0 = blockIdx.y * kSlabRows, col = blockIdx.x * 32 + lane;
+    const bool cok = col < c;
+    float v[32];
+    // the thread's 32 rows share one sign word (rows 32 w .. 32 w + 31 of a 64-aligned tile)
+    const uint64_t sw = (r0 + 32 * w < r) ? __ldg(&signs[(r0 + 32 * w) >> 6]) : 0ull;
+    const int sb = (r0 + 32 * w) & 63;
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+        const int row = r0 + 32 * w + e;
+        v[e] = (cok && row < r) ? Y[(size_t)row * c + col] : 0.f;
+        if (!kInverse) v[e] = flip_if(v[e], (sw >> (sb + e)) & 1ull);
     }
-    __syncthreads();
-    for (int k = threadIdx.y; k < 32; k += 8) {
-        const int cc = c0 + k, rr = r0 + threadIdx.x;
-        if (rr < r && cc < c) Y[(size_t)cc * r + rr] = t[threadIdx.x][k];
+#pragma unroll
+    for (int q = 1; q < 32; q <<= 1) {        // strides 1 .. 16 (row bits 0 .. 4)
+        if (q >= B) break;
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+            if ((e & q) == 0) {
+                const float a = v[e], b = v[e | q];
+                v[e] = a + b;
+                v[e | q] = a - b;
+            }
+        }
+    }
+    const bool two = B > 32;
+    if (two) {                                // rows w + 16 e: row bits 4 .. 8 in the thread
+#pragma unroll
+        for (int e = 0; e < 32; ++e) slab[(32 * w + e) * 32 + lane] = v[e];
+        __syncthreads();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) v[e] = slab[(w + 16 * e) * 32 + lane];
+#pragma unroll
+        for (int q = 2; q < 32; q <<= 1) {    // strides 32 .. 256 (e bits 1 .. 4)
+            if (16 * q >= B) break;
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+                if ((e & q) == 0) {
+                    const float a = v[e], b = v[e | q];
+                    v[e] = a + b;
+                    v[e | q] = a - b;
+                }
+            }
+        }
+    }
+    if (!cok) return;
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+        const int row = r0 + (two ? w + 16 * e : 32 * w + e);
+        if (row >= r) continue;
+        float y = v[e];
+        if (kFinal) y = (kInverse ? flip_if(y, sign_bit(signs, row)) : y) * scale;
+        Y[(size_t)row * c + col] = y;
+    }
+}
+
+// Column transform, second pass, for d = OUTER * 2^k rows with 2^k = HI * B: thread = one
+// column and one row residue i0 < B, holding the A = OUTER * HI rows i0 + B (q HI + h) (q <
+// OUTER: the order-28 index, h < HI). The butterflies of strides B .. 2^k / 2 (the h bits), the
+// order-28 stage across q, then the scale and, inverse, the signs. No shared memory, no barrier.
+// G is H_28^T forward and H_28 inverse, read as G[c][a] (a column of G per output: the same
+// access pattern in both directions, which keeps the table in the constant bank).
+constexpr int kStridedThreads = 64;   // small CTAs: several per SM, their phases interleave
+
+template <int OUTER, int HI, bool kInverse>
+__global__ void __launch_bounds__(kStridedThreads)
+rht_cols_strided_kernel(float* __restrict__ Y, int c, int B, const uint64_t* __restrict__ signs,
+                        float scale, const __grid_constant__ H28f G) {
+    constexpr int A = OUTER * HI;
+    const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int i0 = blockIdx.y * (kStridedThreads / 32) + w;
+    const int col = blockIdx.x * 32 + lane;
+    if (i0 >= B || col >= c) return;
+    // 32-bit element offsets (r c < 2^31): one register per row instead of a 64-bit address
+    const unsigned off0 = (unsigned)i0 * (unsigned)c + (unsigned)col;
+    const unsigned step = (unsigned)B * (unsigned)c;
+    float v[A];
+#pragma unroll
+    for (int a = 0; a < A; ++a) v[a] = Y[off0 + a * step];
+#pragma unroll
+    for (int q = 1; q < HI; q <<= 1) {
+#pragma unroll
+        for (int a = 0; a < A; ++a) {
+            if ((a & q) == 0) {
+                const float x = v[a], y = v[a | q];
+                v[a] = x + y;
+                v[a | q] = x - y;
+            }
+        }
+    }
+    // each output row is written as soon as it is formed: sum_c G[c][a] v[c HI + h] for the
+    // order-28 stage, v itself otherwise
+    auto put = [&](int a, float y) {
+        const int row = i0 + B * a;
+        Y[off0 + a * step] = (kInverse ? flip_if(y, sign_bit(signs, row)) : y) * scale;
+    };
+    if (OUTER == 28) {
+#pragma unroll
+        for (int h = 0; h < HI; ++h) {
+#pragma unroll
+            for (int a = 0; a < 28; ++a) {
+                float acc = 0.f;
+#pragma unroll
+                for (int cc = 0; cc < 28; ++cc)
+                    acc = fmaf(G.h[cc][a], v[cc * HI + h], acc);
+                put(a * HI + h, acc);
+            }
+        }
+    } else {
+#pragma unroll
+        for (int a = 0; a < A; ++a) put(a, v[a]);
     }
 }
 
@@ -270,9 +398,68 @@ int rows_pass(const float* X, float* Y, int rows, int d, const uint64_t* signs, 
                    : rows_pass_dir<false>(X, Y, rows, d, signs, H, st);
 }
 
-void transpose(const float* X, float* Y, int r, int c, cudaStream_t st) {
-    transpose_kernel<<<dim3((c + 31) / 32, (r + 31) / 32), dim3(32, 8), 0, st>>>(X, Y, r, c);
+template <bool kInverse, bool kFinal>
+int launch_slab(float* Y, int r, int c, int B, const uint64_t* signs, float scale,
+                cudaStream_t st) {
+    auto kern = rht_cols_slab_kernel<kInverse, kFinal>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kSlabSmem) != cudaSuccess)
+        return BAKRON_ERR_CUDA;
+    kern<<<dim3((c + 31) / 32, (r + kSlabRows - 1) / kSlabRows), kSlabThreads, kSlabSmem, st>>>(
+        Y, r, c, B, signs, scale);
     count_launches(1);
+    return cuda_err(cudaGetLastError());
+}
+
+template <int OUTER, int HI, bool kInverse>
+int launch_strided(float* Y, int c, int B, const uint64_t* signs, float scale, const H28f& H,
+                   cudaStream_t st) {
+    H28f G;   // H^T forward, H inverse
+    for (int a = 0; a < 28; ++a)
+        for (int cc = 0; cc < 28; ++cc) G.h[cc][a] = kInverse ? H.h[cc][a] : H.h[a][cc];
+    rht_cols_strided_kernel<OUTER, HI, kInverse>
+        <<<dim3((c + 31) / 32, (B + kStridedThreads / 32 - 1) / (kStridedThreads / 32)),
+           kStridedThreads, 0, st>>>(Y, c, B, signs, scale, G);
+    count_launches(1);
+    return cuda_err(cudaGetLastError());
+}
+
+// Y <- T_r Y (inverse: T_r^T Y) for Y (r x c), in place: the slab pass, then (unless d = 2^k
+// <= 512) the strided pass.
+template <bool kInverse>
+int cols_pass_dir(float* Y, int r, int c, const uint64_t* signs, const H28f& H,
+                  cudaStream_t st) {
+    int seg = 0;
+    const int outer = factor(r, seg);
+    const int B = seg < kSlabRows ? seg : kSlabRows;
+    const int hi = seg / B;
+    const float scale = 1.0f / sqrtf((float)r);
+    const bool final_slab = outer == 1 && hi == 1;
+    int e = final_slab ? launch_slab<kInverse, true>(Y, r, c, B, signs, scale, st)
+                       : launch_slab<kInverse, false>(Y, r, c, B, signs, scale, st);
+    if (e || final_slab) return e;
+    if (outer == 28) {
+        switch (hi) {
+            case 1: return launch_strided<28, 1, kInverse>(Y, c, B, signs, scale, H, st);
+            case 2: return launch_strided<28, 2, kInverse>(Y, c, B, signs, scale, H, st);
+            default: return BAKRON_ERR_INVALID_ARG;
+        }
+    }
+    switch (hi) {
+        case 2: return launch_strided<1, 2, kInverse>(Y, c, B, signs, scale, H, st);
+        case 4: return launch_strided<1, 4, kInverse>(Y, c, B, signs, scale, H, st);
+        case 8: return launch_strided<1, 8, kInverse>(Y, c, B, signs, scale, H, st);
+        case 16: return launch_strided<1, 16, kInverse>(Y, c, B, signs, scale, H, st);
+        case 32: return launch_strided<1, 32, kInverse>(Y, c, B, signs, scale, H, st);
+        case 64: return launch_strided<1, 64, kInverse>(Y, c, B, signs, scale, H, st);
+        default: return BAKRON_ERR_INVALID_ARG;
+    }
+}
+
+int cols_pass(float* Y, int r, int c, const uint64_t* signs, int inverse, const H28f& H,
+              cudaStream_t st) {
+    return inverse ? cols_pass_dir<true>(Y, r, c, signs, H, st)
+                   : cols_pass_dir<false>(Y, r, c, signs, H, st);
 }
 
 }  // namespace
@@ -295,7 +482,6 @@ inline size_t sign_words(int d) { return 4 * (size_t)((d + 255) / 256); }
 extern "C" size_t bakron_rht_workspace_bytes(int rows, int cols) {
     if (rows < 1 || cols < 1) return 0;
     WsSizer z;
-    z.take<float>((size_t)rows * cols);
     z.take<uint64_t>(sign_words(cols));
     z.take<uint64_t>(sign_words(rows));
     return z.bytes();
@@ -318,7 +504,6 @@ extern "C" int bakron_rht(const float* X, int rows, int cols, uint64_t seed_rows
         return f;
     }();
     WsCarver c(ws);
-    float* t = c.take<float>((size_t)rows * cols);
     uint64_t* sc_words = c.take<uint64_t>(sign_words(cols));
     uint64_t* sr_words = c.take<uint64_t>(sign_words(rows));
     // the signs of T_c and T_r, drawn once for every row
@@ -328,10 +513,8 @@ extern "C" int bakron_rht(const float* X, int rows, int cols, uint64_t seed_rows
     int e;
     // Y = X T_c^T (inverse: X T_c): each row x -> T_c x (inverse: T_c^T x)
     if ((e = rows_pass(X, Y, rows, cols, sc_words, inverse, H, st))) return e;
-    // then T_r Y (inverse: T_r^T Y) as a row pass over Y^T
-    transpose(Y, t, rows, cols, st);
-    if ((e = rows_pass(t, t, cols, rows, sr_words, inverse, H, st))) return e;
-    transpose(t, Y, cols, rows, st);
+    // then T_r Y (inverse: T_r^T Y) along the columns, in place
+    if ((e = cols_pass(Y, rows, cols, sr_words, inverse, H, st))) return e;
     return cuda_err(cudaGetLastError());
 }
 
