@@ -260,7 +260,8 @@ int bakron_sketch_b(const float* G, int S, int m, int n, float damp, float* H_O,
  * Returns BAKRON_ERR_INVALID_ARG for an unsupported size. Three passes over the matrix: the
  * signs, butterflies and order-28 stage along each row (one CTA per row), then the same along
  * the columns in place on Y, on 32-column tiles: strides below 512 in one pass, the larger
- * strides and the order-28 stage in the next. The workspace holds the sign words only.
+ * strides and the order-28 stage in the next. The workspace holds the sign words and the
+ * 28 x 28 matrix of the order-28 stage.
  * ---------------------------------------------------------------------------------------- */
 int bakron_rht_supported(int d);
 size_t bakron_rht_workspace_bytes(int rows, int cols);

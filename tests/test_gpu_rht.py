@@ -47,7 +47,8 @@ def _t_rows(d, seed, idx):
 
 @pytest.mark.parametrize("r,c,i,j,inverse", [(1, 1, 0, 0, 0), (2, 28, 1, 27, 0),
                                              (28, 4, 13, 2, 1), (56, 64, 55, 0, 0),
-                                             (112, 448, 77, 300, 1), (64, 896, 5, 895, 0)])
+                                             (112, 448, 77, 300, 1), (64, 896, 5, 895, 0),
+                                             (4, 1792, 3, 1000, 0), (2, 3584, 1, 3583, 1)])
 def test_spike_is_exact(bk, r, c, i, j, inverse):
     X = np.zeros((r, c), dtype=np.float32)
     X[i, j] = 1.0
@@ -61,7 +62,8 @@ def test_spike_is_exact(bk, r, c, i, j, inverse):
 
 
 @pytest.mark.parametrize("r,c,inverse", [(1, 28, 0), (28, 28, 1), (64, 112, 0), (448, 32, 1),
-                                         (1024, 224, 0), (128, 128, 1)])
+                                         (1024, 224, 0), (128, 128, 1), (28, 1792, 1),
+                                         (8, 3584, 0)])
 def test_random_matches_oracle(bk, r, c, inverse):
     X = np.random.default_rng(r * 7 + c).standard_normal((r, c)).astype(np.float32)
     Y = bk.rht(_dev(X), 5, 6, inverse=bool(inverse)).cpu().numpy().astype(np.float64)
@@ -113,6 +115,24 @@ def test_column_lengths_sampled_and_round_trip(bk, r, c):
     cols = np.arange(c)
     ref = _t_rows(r, 21, rows) @ X.astype(np.float64) @ _t_rows(c, 22, cols).T
     got = Y.cpu().numpy()[np.ix_(rows, cols)]
+    assert np.abs(got - ref).max() <= 1e-4
+
+
+# row lengths 28 S (S = 256, 512, 1024) of the tensor-core row pass, both directions (the
+# inverse through the round trip), on a few rows; sampled columns across segment boundaries
+@pytest.mark.parametrize("r,c", [(8, 7168), (16, 14336), (4, 28672)])
+def test_row_lengths_sampled_and_round_trip(bk, r, c):
+    X = np.random.default_rng(r + c).standard_normal((r, c)).astype(np.float32)
+    Xd = _dev(X)
+    Y = bk.rht(Xd, 31, 32)
+    back = bk.rht(Y, 31, 32, inverse=True)
+    nx = float(torch.linalg.norm(Xd.double()))
+    assert float(torch.linalg.norm(back.double() - Xd.double())) <= 4e-5 * nx
+    assert abs(float(torch.linalg.norm(Y.double())) - nx) <= 2e-5 * nx
+    S = c // 28
+    cols = np.unique(np.array([0, 1, 7, 8, 31, 32, S - 1, S, 5 * S + 17, c // 2, c - 2, c - 1]))
+    ref = _t_rows(r, 31, np.arange(r)) @ X.astype(np.float64) @ _t_rows(c, 32, cols).T
+    got = Y.cpu().numpy()[:, cols]
     assert np.abs(got - ref).max() <= 1e-4
 
 

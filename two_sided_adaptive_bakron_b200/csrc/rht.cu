@@ -15,19 +15,21 @@
 // Sylvester butterflies over each 2^k segment (the fast Walsh-Hadamard transform: a pair
 // (i, i ^ h) with 2h <= 2^k never leaves its segment), by warp shuffles, shared memory or
 // inside a thread depending on the stride, then the order-28 stage across segments, and the
-// 1/sqrt(d) scale. The column transform runs in place on the result in two more passes, on
-// tiles of 32 columns (one 128-byte segment per row): the butterflies of strides below
-// B = min(2^k, 512) inside 512-row tiles (registers, one shared-memory exchange), then, one
-// thread per column and row residue mod B, the larger strides, the order-28 stage and the
-// scale. Every pass reads and writes the matrix once: HBM-bound. Each sum is formed in the
-// same order on both sides (the textbook order: strides 1, 2, 4, ..., then the order-28 sums in
-// index order), so a column's result is bitwise that of the row pass applied to it.
+// 1/sqrt(d) scale. Rows of 28 * 2^k >= 1792 take a variant that stages the row in shared
+// memory and forms the order-28 stage on the tensor cores (rht_rows28_kernel). The column
+// transform runs in place on the result in two more passes, on tiles of 32 columns (one
+// 128-byte segment per row): the butterflies of strides below B = min(2^k, 512) inside 512-row
+// tiles (registers, one shared-memory exchange), then, one thread per column and row residue
+// mod B, the larger strides, the order-28 stage and the scale. Every pass reads and writes the
+// matrix once: HBM-bound. The butterflies and the column passes' order-28 sums are formed in
+// the textbook order (strides 1, 2, 4, ..., then the order-28 sums in index order).
 #include <cmath>
 #include <cstring>
 
 #include "bakron_internal.h"
 #include "common.cuh"
 #include "philox.cuh"
+#include "sm100.cuh"
 
 namespace bakron {
 namespace {
@@ -200,6 +202,162 @@ rht_rows_kernel(const float* __restrict__ X, float* __restrict__ Y, int d, int T
     }
 }
 
+// Row pass for d = 28 S, S = 32 NQ = 2^k between 64 and 1024 (the order-28 stage on the tensor
+// cores). One CTA per row; the row is staged in shared memory as 28 segments of NQ chunks of
+// 32 positions, a chunk padded to 33 floats and a segment to SP = 33 NQ + pad floats with
+// SP = 8 (mod 32), so that the accesses of all three phases spread over the banks.
+//   phase 0: the row into shared memory with coalesced float4 loads;
+//   phase 1: one thread per chunk: the chunk's 32 positions in registers, the signs (forward),
+//            the butterflies of strides 1 .. 16;
+//   phase 2: one thread per segment and position residue mod 32: its NQ positions, strides
+//            32 .. S / 2;
+//   phase 3: out[a][p] = sum_c G[a][c] v[c][p] (G = gtab: H_28 forward, H_28^T inverse,
+//            zero-padded to 32 x 32) as m16n8k8 tf32 MMAs, 8 positions per tile: G is exact in tf32 and
+//            v = hi + lo (hi the tf32 truncation), two MMAs per tile, so a product is within
+//            2^-21 of exact; then the scale, the inverse's signs and the store.
+// The butterflies are those of the textbook order; the order-28 sums are accumulated by the
+// tensor core (not the fmaf chain of rht_rows_kernel), which moves the last bits only.
+constexpr int kRows28Threads = 256;
+
+template <int NQ>
+__host__ __device__ constexpr int rows28_sp() { return 33 * NQ + ((8 - NQ % 32) + 32) % 32; }
+template <int NQ>
+constexpr size_t rows28_smem() { return (size_t)28 * rows28_sp<NQ>() * sizeof(float); }
+
+template <int NQ, bool kInverse>
+__global__ void __launch_bounds__(kRows28Threads, 2)
+rht_rows28_kernel(const float* __restrict__ X, float* __restrict__ Y,
+                  const uint64_t* __restrict__ signs, float scale,
+                  const float* __restrict__ gtab) {
+    constexpr int S = 32 * NQ, D = 28 * S, NCH = 28 * NQ, SP = rows28_sp<NQ>();
+    static_assert(SP % 32 == 8, "segment stride");
+    extern __shared__ __align__(16) float seg[];   // [28][SP]
+    const size_t row = blockIdx.x;
+    const float* x = X + row * D;
+    float* y = Y + row * D;
+    const int t = threadIdx.x, lane = t & 31, w = t >> 5;
+    // phase 0: the row into shared memory, coalesced (lane q takes positions 4 q .. 4 q + 3)
+    const float4* src = reinterpret_cast<const float4*>(x);
+#pragma unroll 4
+    for (int q = t; q < D / 4; q += kRows28Threads) {
+        const float4 f = src[q];
+        const int j = 4 * q;
+        float* d = seg + (j / S) * SP + 33 * ((j % S) >> 5) + (j & 31);
+        d[0] = f.x;
+        d[1] = f.y;
+        d[2] = f.z;
+        d[3] = f.w;
+    }
+    __syncthreads();
+    // phase 1
+    for (int ch = t; ch < NCH; ch += kRows28Threads) {
+        float* cp = seg + (ch / NQ) * SP + 33 * (ch % NQ);
+        float v[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = cp[i];
+        if (!kInverse) {
+            const uint64_t sw = __ldg(&signs[(32 * ch) >> 6]);
+            const int sb = (32 * ch) & 63;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = flip_if(v[i], (sw >> (sb + i)) & 1ull);
+        }
+#pragma unroll
+        for (int q = 1; q < 32; q <<= 1) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                if ((i & q) == 0) {
+                    const float a = v[i], b = v[i | q];
+                    v[i] = a + b;
+                    v[i | q] = a - b;
+                }
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < 32; ++i) cp[i] = v[i];
+    }
+    __syncthreads();
+    // phase 2
+    if (NQ > 1) {
+        for (int gi = t; gi < 28 * 32; gi += kRows28Threads) {
+            float* base = seg + (gi >> 5) * SP + (gi & 31);
+            float v[NQ];
+#pragma unroll
+            for (int i = 0; i < NQ; ++i) v[i] = base[33 * i];
+#pragma unroll
+            for (int q = 1; q < NQ; q <<= 1) {
+#pragma unroll
+                for (int i = 0; i < NQ; ++i) {
+                    if ((i & q) == 0) {
+                        const float a = v[i], b = v[i | q];
+                        v[i] = a + b;
+                        v[i | q] = a - b;
+                    }
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < NQ; ++i) base[33 * i] = v[i];
+        }
+        __syncthreads();
+    }
+    // phase 3: fragments as laid out by mma.m16n8k8 (g = lane / 4, tq = lane % 4): A rows g,
+    // g + 8 and columns tq, tq + 4 of a 16 x 8 tile; B rows (k) tq, tq + 4 of column (n) g;
+    // C rows g, g + 8 and columns 2 tq, 2 tq + 1
+    const int g = lane >> 2, tq = lane & 3;
+    auto gval = [&](int m, int k) {
+        return (m < 28 && k < 28) ? __ldg(&gtab[28 * m + k]) : 0.f;
+    };
+    uint32_t af[2][4][4];
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+        for (int s4 = 0; s4 < 4; ++s4) {
+            const int m0 = 16 * mt + g, k0 = 8 * s4 + tq;
+            af[mt][s4][0] = __float_as_uint(gval(m0, k0));
+            af[mt][s4][1] = __float_as_uint(gval(m0 + 8, k0));
+            af[mt][s4][2] = __float_as_uint(gval(m0, k0 + 4));
+            af[mt][s4][3] = __float_as_uint(gval(m0 + 8, k0 + 4));
+        }
+    for (int ng = w; ng < S / 8; ng += kRows28Threads / 32) {
+        const int p = 8 * ng + g;                 // this lane's B column: position p
+        const float* colp = seg + 33 * (p >> 5) + (p & 31);
+        uint32_t bh[4][2], bl[4][2];
+#pragma unroll
+        for (int s4 = 0; s4 < 4; ++s4)
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                const int k = 8 * s4 + tq + 4 * hf;
+                const float xv = k < 28 ? colp[k * SP] : 0.f;
+                const float hv = sm100::tf32_hi(xv);
+                bh[s4][hf] = __float_as_uint(hv);
+                bl[s4][hf] = __float_as_uint(xv - hv);
+            }
+        float acc[2][4] = {};
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+            for (int s4 = 0; s4 < 4; ++s4) {
+                sm100::mma_16x8x8_tf32(acc[mt], af[mt][s4], bh[s4]);
+                sm100::mma_16x8x8_tf32(acc[mt], af[mt][s4], bl[s4]);
+            }
+        const int p0 = 8 * ng + 2 * tq;
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const int a = 16 * mt + g + 8 * hh;
+                if (a >= 28) continue;
+                const int j = a * S + p0;         // even: j and j + 1 share a sign word
+                float v0 = acc[mt][2 * hh], v1 = acc[mt][2 * hh + 1];
+                if (kInverse) {
+                    const uint64_t sw = __ldg(&signs[j >> 6]);
+                    v0 = flip_if(v0, (sw >> (j & 63)) & 1ull);
+                    v1 = flip_if(v1, (sw >> ((j & 63) + 1)) & 1ull);
+                }
+                *reinterpret_cast<float2*>(y + j) = make_float2(v0 * scale, v1 * scale);
+            }
+    }
+}
+
 // Column transform, first pass: Y (r x c, in place) along its rows i, the signs (forward)
 // and the butterflies of strides 1 .. B / 2 of every B-row slab (B = min(2^k, 512), so a slab
 // never leaves a 512-row tile). CTA = 512 consecutive rows x 32 columns, thread (w, lane) =
@@ -334,6 +492,43 @@ rht_cols_strided_kernel(float* __restrict__ Y, int c, int B, const uint64_t* __r
     }
 }
 
+// The second column pass for d = 28 * 2^k rows with 2^k = 2 B (28672 rows): the same work as
+// rht_cols_strided_kernel<28, 2> split over a lane pair, so that each thread carries one
+// order-28 stage (half the unrolled code, which otherwise overflows the instruction cache).
+// Lanes l and l + 16 share column 16 * blockIdx.x + (l & 15) and row residue i0; lane half h
+// holds the 28 rows i0 + B (2 q + h). The stride-B butterfly takes the partner's value by a
+// shuffle (lower half a + b, upper half a - b, as in the textbook order).
+template <bool kInverse>
+__global__ void __launch_bounds__(kStridedThreads)
+rht_cols_strided28x2_kernel(float* __restrict__ Y, int c, int B,
+                            const uint64_t* __restrict__ signs, float scale,
+                            const __grid_constant__ H28f G) {
+    const int w = threadIdx.x >> 5, lane = threadIdx.x & 31, h = lane >> 4;
+    const int i0 = blockIdx.y * (kStridedThreads / 32) + w;
+    const int col = blockIdx.x * 16 + (lane & 15);
+    if (i0 >= B) return;                      // the whole warp
+    const bool ok = col < c;                  // inactive lanes still take part in the shuffles
+    const unsigned off0 = (unsigned)(i0 + B * h) * (unsigned)c + (unsigned)col;
+    const unsigned step = 2u * (unsigned)B * (unsigned)c;
+    float v[28];
+#pragma unroll
+    for (int q = 0; q < 28; ++q) v[q] = ok ? Y[off0 + q * step] : 0.f;
+#pragma unroll
+    for (int q = 0; q < 28; ++q) {
+        const float p = __shfl_xor_sync(0xffffffffu, v[q], 16);
+        v[q] = h ? p - v[q] : v[q] + p;
+    }
+    if (!ok) return;
+#pragma unroll
+    for (int a = 0; a < 28; ++a) {
+        float acc = 0.f;
+#pragma unroll
+        for (int cc = 0; cc < 28; ++cc) acc = fmaf(G.h[cc][a], v[cc], acc);
+        const int row = i0 + B * (2 * a + h);
+        Y[off0 + a * step] = (kInverse ? flip_if(acc, sign_bit(signs, row)) : acc) * scale;
+    }
+}
+
 // scales[i * G + g] = max_{j in group g} |W[i][j]| / divisor; one CTA per row, one warp per
 // group at a time.
 __global__ void row_scales_kernel(const float* __restrict__ W, int n, int group, int G,
@@ -366,13 +561,39 @@ int launch_rows(const float* X, float* Y, int rows, int d, const uint64_t* signs
     return cuda_err(cudaGetLastError());
 }
 
-// T = min(seg, 512) threads, U = seg / T columns of each segment per thread.
+template <int NQ, bool kInverse>
+int launch_rows28(const float* X, float* Y, int rows, const uint64_t* signs, const float* gtab,
+                  cudaStream_t st) {
+    constexpr size_t smem = rows28_smem<NQ>();
+    auto kern = rht_rows28_kernel<NQ, kInverse>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess)
+        return BAKRON_ERR_CUDA;
+    const float scale = 1.0f / sqrtf((float)(28 * 32 * NQ));
+    kern<<<rows, kRows28Threads, smem, st>>>(X, Y, signs, scale, gtab);
+    count_launches(1);
+    return cuda_err(cudaGetLastError());
+}
+
+// Rows of 28 S with S >= 64 (and 16-byte aligned matrices): the tensor-core row pass;
+// otherwise T = min(seg, 512) threads, U = seg / T columns of each segment per thread.
 template <bool kInverse>
 int rows_pass_dir(const float* X, float* Y, int rows, int d, const uint64_t* signs,
-                  const H28f& H, cudaStream_t st) {
+                  const H28f& H, const float* gtab, cudaStream_t st) {
     int seg = 0;
     const int outer = factor(d, seg);
     const int U = seg <= kRowThreads ? 1 : seg / kRowThreads;
+    const bool aligned = ((reinterpret_cast<uintptr_t>(X) | reinterpret_cast<uintptr_t>(Y)) & 15) == 0;
+    if (outer == 28 && aligned) {
+        switch (seg) {
+            case 64: return launch_rows28<2, kInverse>(X, Y, rows, signs, gtab, st);
+            case 128: return launch_rows28<4, kInverse>(X, Y, rows, signs, gtab, st);
+            case 256: return launch_rows28<8, kInverse>(X, Y, rows, signs, gtab, st);
+            case 512: return launch_rows28<16, kInverse>(X, Y, rows, signs, gtab, st);
+            case 1024: return launch_rows28<32, kInverse>(X, Y, rows, signs, gtab, st);
+            default: break;
+        }
+    }
     if (outer == 28) {
         switch (U) {
             case 1: return launch_rows<1, 28, kInverse>(X, Y, rows, d, signs, H, st);
@@ -393,9 +614,9 @@ int rows_pass_dir(const float* X, float* Y, int rows, int d, const uint64_t* sig
 }
 
 int rows_pass(const float* X, float* Y, int rows, int d, const uint64_t* signs, int inverse,
-              const H28f& H, cudaStream_t st) {
-    return inverse ? rows_pass_dir<true>(X, Y, rows, d, signs, H, st)
-                   : rows_pass_dir<false>(X, Y, rows, d, signs, H, st);
+              const H28f& H, const float* gtab, cudaStream_t st) {
+    return inverse ? rows_pass_dir<true>(X, Y, rows, d, signs, H, gtab, st)
+                   : rows_pass_dir<false>(X, Y, rows, d, signs, H, gtab, st);
 }
 
 template <bool kInverse, bool kFinal>
@@ -424,6 +645,19 @@ int launch_strided(float* Y, int c, int B, const uint64_t* signs, float scale, c
     return cuda_err(cudaGetLastError());
 }
 
+template <bool kInverse>
+int launch_strided28x2(float* Y, int c, int B, const uint64_t* signs, float scale,
+                       const H28f& H, cudaStream_t st) {
+    H28f G;   // H^T forward, H inverse
+    for (int a = 0; a < 28; ++a)
+        for (int cc = 0; cc < 28; ++cc) G.h[cc][a] = kInverse ? H.h[cc][a] : H.h[a][cc];
+    rht_cols_strided28x2_kernel<kInverse>
+        <<<dim3((c + 15) / 16, (B + kStridedThreads / 32 - 1) / (kStridedThreads / 32)),
+           kStridedThreads, 0, st>>>(Y, c, B, signs, scale, G);
+    count_launches(1);
+    return cuda_err(cudaGetLastError());
+}
+
 // Y <- T_r Y (inverse: T_r^T Y) for Y (r x c), in place: the slab pass, then (unless d = 2^k
 // <= 512) the strided pass.
 template <bool kInverse>
@@ -441,7 +675,7 @@ int cols_pass_dir(float* Y, int r, int c, const uint64_t* signs, const H28f& H,
     if (outer == 28) {
         switch (hi) {
             case 1: return launch_strided<28, 1, kInverse>(Y, c, B, signs, scale, H, st);
-            case 2: return launch_strided<28, 2, kInverse>(Y, c, B, signs, scale, H, st);
+            case 2: return launch_strided28x2<kInverse>(Y, c, B, signs, scale, H, st);
             default: return BAKRON_ERR_INVALID_ARG;
         }
     }
@@ -479,11 +713,20 @@ extern "C" int bakron_rht_supported(int d) {
 
 inline size_t sign_words(int d) { return 4 * (size_t)((d + 255) / 256); }
 
+// gtab[28 m + k] = the order-28 matrix applied in this call: H_28 forward, H_28^T inverse. The
+// tensor-core row pass builds its fragments from it with per-lane loads from global memory
+// (per-lane reads of a kernel parameter would serialise on the constant cache).
+__global__ void rht_h28_table_kernel(const __grid_constant__ H28f H, int inverse, float* gtab) {
+    const int t = threadIdx.x;
+    if (t < 28 * 28) gtab[t] = inverse ? H.h[t % 28][t / 28] : H.h[t / 28][t % 28];
+}
+
 extern "C" size_t bakron_rht_workspace_bytes(int rows, int cols) {
     if (rows < 1 || cols < 1) return 0;
     WsSizer z;
     z.take<uint64_t>(sign_words(cols));
     z.take<uint64_t>(sign_words(rows));
+    z.take<float>(28 * 28);
     return z.bytes();
 }
 
@@ -506,13 +749,16 @@ extern "C" int bakron_rht(const float* X, int rows, int cols, uint64_t seed_rows
     WsCarver c(ws);
     uint64_t* sc_words = c.take<uint64_t>(sign_words(cols));
     uint64_t* sr_words = c.take<uint64_t>(sign_words(rows));
+    float* gtab = c.take<float>(28 * 28);
+    rht_h28_table_kernel<<<1, 28 * 28, 0, st>>>(H, inverse, gtab);
+    count_launches(1);
     // the signs of T_c and T_r, drawn once for every row
     rht_signs_kernel<<<(cols / 256 + 64) / 64, 64, 0, st>>>(cols, seed_cols, sc_words);
     rht_signs_kernel<<<(rows / 256 + 64) / 64, 64, 0, st>>>(rows, seed_rows, sr_words);
     count_launches(2);
     int e;
     // Y = X T_c^T (inverse: X T_c): each row x -> T_c x (inverse: T_c^T x)
-    if ((e = rows_pass(X, Y, rows, cols, sc_words, inverse, H, st))) return e;
+    if ((e = rows_pass(X, Y, rows, cols, sc_words, inverse, H, gtab, st))) return e;
     // then T_r Y (inverse: T_r^T Y) along the columns, in place
     if ((e = cols_pass(Y, rows, cols, sr_words, inverse, H, st))) return e;
     return cuda_err(cudaGetLastError());

@@ -226,15 +226,6 @@ __device__ __forceinline__ void publish_rest(const FusedArgs& a, const LeafBuf& 
     }
 }
 
-__device__ __forceinline__ void mma_16x8x8_tf32(float (&d)[4], const uint32_t (&a)[4],
-                                                const uint32_t (&b)[2]) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-        "{%8,%9}, {%0,%1,%2,%3};"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
-}
-
 // One source's contribution D[m][n] += sum_k X[k][m] Y[k][n] (X, Y: 32 x 32 tiles in the
 // swizzled layout swz) on the tensor cores, 3xTF32 as in the GEMM engine (hi = tf32
 // truncation, lo = x - hi, hi*hi + hi*lo + lo*hi). Warp w of the group holds rows
@@ -268,9 +259,9 @@ __device__ __forceinline__ void product_mma(const float* X, const float* Y, int 
                 bh[i] = __float_as_uint(h);
                 bl[i] = __float_as_uint(b[i] - h);
             }
-            mma_16x8x8_tf32(acc[nt], ah, bh);
-            mma_16x8x8_tf32(acc[nt], ah, bl);
-            mma_16x8x8_tf32(acc[nt], al, bh);
+            sm100::mma_16x8x8_tf32(acc[nt], ah, bh);
+            sm100::mma_16x8x8_tf32(acc[nt], ah, bl);
+            sm100::mma_16x8x8_tf32(acc[nt], al, bh);
         }
     }
 }

@@ -158,6 +158,18 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// ------------------------------------------------------------------------------ mma.sync
+// d += a b for one m16n8k8 tile with tf32 operands (the bit patterns of fp32 values; the low 13
+// mantissa bits are ignored) and fp32 accumulators, in the fragment layout of mma.m16n8k8.
+__device__ __forceinline__ void mma_16x8x8_tf32(float (&d)[4], const uint32_t (&a)[4],
+                                                const uint32_t (&b)[2]) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
 // ------------------------------------------------------------------------------ 3xTF32 split
 // hi keeps the 10 explicit mantissa bits a tf32 operand carries; lo = x - hi is exact in fp32.
 __device__ __forceinline__ float tf32_hi(float x) {
