@@ -27,8 +27,9 @@
 // still read outer block o's planes while o - 1's panels are written.
 // Inside an outer block, likewise, the caller's stream applies a panel only to the next
 // diagonal block before factoring it; a second side stream applies the same panel to the next
-// panel's input columns (which the caller's stream waits for before that panel) and then to the
-// later columns of the outer block (waited for before the diagonal block after next).
+// panel's input columns (which the caller's stream waits for before that panel; this update
+// also writes that panel's hi/lo operand planes, so the panel needs no split pass) and then to
+// the later columns of the outer block (waited for before the diagonal block after next).
 #include <algorithm>
 #include <atomic>
 #include <mutex>
@@ -93,6 +94,42 @@ struct EpiPanel {
             xl[o] = x - xh_;
             uh[o] = uh_;
             ul[o] = u - uh_;
+        }
+    }
+    __device__ void tile_done(const tc::Problem&, int, int) {}
+};
+
+// C += weight * acc (as tc::EpiStore with accumulation, for blocks strictly above the
+// diagonal), the result also written as hi/lo planes at (c_row0 + r, c_col0 + c - pcol0), row
+// stride ldp: the update of the next panel's input columns leaves that panel's operand planes
+// behind, so the panel needs no separate split pass on the chain.
+struct EpiStorePlanes {
+    float* C;
+    int ldc;
+    float* hi;
+    float* lo;
+    int ldp;
+    int pcol0;
+    __device__ void chunk(const tc::Problem& P, int row0, int col, int, int, const float* v) {
+        if (col >= P.N) return;
+        const int gc = P.c_col0 + col;
+        float old[32];
+#pragma unroll
+        for (int rr = 0; rr < 32; ++rr) {
+            const int gr = P.c_row0 + row0 + rr;
+            old[rr] = (row0 + rr < P.M) ? C[(size_t)gr * ldc + gc] : 0.f;
+        }
+#pragma unroll
+        for (int rr = 0; rr < 32; ++rr) {
+            const int gr = P.c_row0 + row0 + rr;
+            if (row0 + rr < P.M) {
+                const float x = old[rr] + P.weight * v[rr * 33];
+                C[(size_t)gr * ldc + gc] = x;
+                const size_t o = (size_t)gr * ldp + (gc - pcol0);
+                const float h = sm100::tf32_hi(x);
+                hi[o] = h;
+                lo[o] = x - h;
+            }
         }
     }
     __device__ void tile_done(const tc::Problem&, int, int) {}
@@ -242,12 +279,14 @@ extern "C" int bakron_ldl(const float* H, int n, float* L, float* D, void* ws, s
                                                                   w.inv_lo, dev_status);
             count_launches(1);
             if (kb0 == 0) continue;
-            if (npanel_pending) {   // this panel's input columns, updated by the previous panel
+            // panel: X = H'[0:kb0, B] U_BB^{-T}; its operand planes come from the update of
+            // these columns by the previous panel (look-ahead), else from a split pass here
+            if (npanel_pending) {
                 if ((e = cuda_err(cudaStreamWaitEvent(st, ev_npanel, 0)))) return e;
                 npanel_pending = false;
+            } else {
+                tc::split_planes(L + kb0, kb0, b, n, w.p_hi, w.p_lo, NBI, 0, st);
             }
-            // panel: X = H'[0:kb0, B] U_BB^{-T}
-            tc::split_planes(L + kb0, kb0, b, n, w.p_hi, w.p_lo, NBI, 0, st);
             CUtensorMap m_ph, m_pl, m_ih, m_il;
             if ((e = tc::make_kmajor_map(&m_ph, w.p_hi, kb0, b, NBI, tc::BM))) return e;
             if ((e = tc::make_kmajor_map(&m_pl, w.p_lo, kb0, b, NBI, tc::BM))) return e;
@@ -276,8 +315,9 @@ extern "C" int bakron_ldl(const float* H, int n, float* L, float* D, void* ws, s
                 if ((e = cuda_err(cudaStreamWaitEvent(s3, ev_panel, 0)))) return e;
                 tc::ProblemList nl(BN);
                 nl.add(0, c_off, nb0, c_off, nb0, kb0 - nb0, b, 0, nb0, -1.f);
+                EpiStorePlanes ep_next{L, n, w.p_hi, w.p_lo, NBI, nb0};
                 if ((e = tc::launch_gemm3x<BN, STAGES>(m_xh[ps], m_xl[ps], m_uh[ps], m_ul[ps], nl,
-                                                       es, dev_status, s3)))
+                                                       ep_next, dev_status, s3)))
                     return e;
                 if ((e = cuda_err(cudaEventRecord(ev_npanel, s3)))) return e;
                 npanel_pending = true;
