@@ -99,13 +99,15 @@ struct EpiPanel {
     __device__ void tile_done(const tc::Problem&, int, int) {}
 };
 
-// C += weight * acc (as tc::EpiStore with accumulation, for blocks strictly above the
-// diagonal), the result also written as hi/lo planes at (c_row0 + r, c_col0 + c - pcol0), row
-// stride ldp: the update of the next panel's input columns leaves that panel's operand planes
-// behind, so the panel needs no separate split pass on the chain.
+// C += weight * acc (as tc::EpiStore with accumulation; `upper`: only entries with global
+// column >= global row), and every result at global (row, col) with row < pcol0 <= col also as
+// hi/lo planes at (row, col - pcol0), row stride ldp: the update of the next panel's input
+// columns leaves that panel's operand planes behind, so the panel needs no separate split pass
+// on the chain.
 struct EpiStorePlanes {
     float* C;
     int ldc;
+    int upper;
     float* hi;
     float* lo;
     int ldp;
@@ -117,18 +119,21 @@ struct EpiStorePlanes {
 #pragma unroll
         for (int rr = 0; rr < 32; ++rr) {
             const int gr = P.c_row0 + row0 + rr;
-            old[rr] = (row0 + rr < P.M) ? C[(size_t)gr * ldc + gc] : 0.f;
+            const bool ok = (row0 + rr < P.M) && (!upper || gc >= gr);
+            old[rr] = ok ? C[(size_t)gr * ldc + gc] : 0.f;
         }
 #pragma unroll
         for (int rr = 0; rr < 32; ++rr) {
             const int gr = P.c_row0 + row0 + rr;
-            if (row0 + rr < P.M) {
+            if ((row0 + rr < P.M) && (!upper || gc >= gr)) {
                 const float x = old[rr] + P.weight * v[rr * 33];
                 C[(size_t)gr * ldc + gc] = x;
-                const size_t o = (size_t)gr * ldp + (gc - pcol0);
-                const float h = sm100::tf32_hi(x);
-                hi[o] = h;
-                lo[o] = x - h;
+                if (gr < pcol0 && gc >= pcol0) {
+                    const size_t o = (size_t)gr * ldp + (gc - pcol0);
+                    const float h = sm100::tf32_hi(x);
+                    hi[o] = h;
+                    lo[o] = x - h;
+                }
             }
         }
     }
@@ -263,6 +268,7 @@ extern "C" int bakron_ldl(const float* H, int n, float* L, float* D, void* ws, s
     cudaEvent_t ev_ready = evs.ev[0], ev_next = evs.ev[1], ev_join = evs.ev[2];
     cudaEvent_t ev_panel = evs.ev[3], ev_npanel = evs.ev[4], ev_rest = evs.ev[5];
     bool npanel_pending = false, rest_pending = false;
+    bool first_planes = false;   // the look-ahead update left the next first panel's planes
 
     const int eb = 1184;
     copy_upper_kernel<<<eb, 256, 0, st>>>(H, L, n);
@@ -279,14 +285,16 @@ extern "C" int bakron_ldl(const float* H, int n, float* L, float* D, void* ws, s
                                                                   w.inv_lo, dev_status);
             count_launches(1);
             if (kb0 == 0) continue;
-            // panel: X = H'[0:kb0, B] U_BB^{-T}; its operand planes come from the update of
-            // these columns by the previous panel (look-ahead), else from a split pass here
+            // panel: X = H'[0:kb0, B] U_BB^{-T}; with look-ahead its operand planes come from
+            // the last update of these columns (the previous panel's, or for an outer block's
+            // first panel the previous outer block's look-ahead update), else from a split here
             if (npanel_pending) {
                 if ((e = cuda_err(cudaStreamWaitEvent(st, ev_npanel, 0)))) return e;
                 npanel_pending = false;
-            } else {
+            } else if (!(first_planes && t == 0)) {
                 tc::split_planes(L + kb0, kb0, b, n, w.p_hi, w.p_lo, NBI, 0, st);
             }
+            first_planes = false;
             CUtensorMap m_ph, m_pl, m_ih, m_il;
             if ((e = tc::make_kmajor_map(&m_ph, w.p_hi, kb0, b, NBI, tc::BM))) return e;
             if ((e = tc::make_kmajor_map(&m_pl, w.p_lo, kb0, b, NBI, tc::BM))) return e;
@@ -315,7 +323,7 @@ extern "C" int bakron_ldl(const float* H, int n, float* L, float* D, void* ws, s
                 if ((e = cuda_err(cudaStreamWaitEvent(s3, ev_panel, 0)))) return e;
                 tc::ProblemList nl(BN);
                 nl.add(0, c_off, nb0, c_off, nb0, kb0 - nb0, b, 0, nb0, -1.f);
-                EpiStorePlanes ep_next{L, n, w.p_hi, w.p_lo, NBI, nb0};
+                EpiStorePlanes ep_next{L, n, 1, w.p_hi, w.p_lo, NBI, nb0};
                 if ((e = tc::launch_gemm3x<BN, STAGES>(m_xh[ps], m_xl[ps], m_uh[ps], m_ul[ps], nl,
                                                        ep_next, dev_status, s3)))
                     return e;
@@ -367,9 +375,14 @@ extern "C" int bakron_ldl(const float* H, int n, float* L, float* D, void* ws, s
         tc::ProblemList al(BN);
         al.add(0, 0, ca, 0, ca, ko0 - ca, K, 0, ca, -1.f);                      // rows above
         al.add(ca, 0, ca, 0, ko0 - ca, ko0 - ca, K, ca, ca, -1.f, /*upper_only=*/1);
-        if ((e = tc::launch_gemm3x<BN, STAGES>(m_xh[ps], m_xl[ps], m_uh[ps], m_ul[ps], al, es,
-                                               dev_status, side)))
+        // it also leaves the operand planes of the next outer block's first panel (columns
+        // [fb0, ko0), rows above them)
+        const int fb0 = std::max(ca, ko0 - NBI);
+        EpiStorePlanes ep_first{L, n, 1, w.p_hi, w.p_lo, NBI, fb0};
+        if ((e = tc::launch_gemm3x<BN, STAGES>(m_xh[ps], m_xl[ps], m_uh[ps], m_ul[ps], al,
+                                               ep_first, dev_status, side)))
             return e;
+        first_planes = true;
         if ((e = cuda_err(cudaEventRecord(ev_next, side)))) return e;
         if (ca > 0) {
             tc::ProblemList bl(BN);
