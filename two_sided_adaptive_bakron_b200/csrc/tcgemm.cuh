@@ -11,8 +11,8 @@
 // Persistent pipeline (at most one 192-thread CTA per SM, tiles t = blockIdx.x + i * gridDim.x):
 //   warp 0 / lane 0 : TMA producer, STAGES-deep ring of {A_hi, A_lo, B_hi, B_lo} k-blocks of
 //                     32 fp32 (one 128-byte swizzle row) that runs on across tiles;
-//   warp 1 / lane 0 : MMA issuer, 4 k-steps of 8 x 3 tcgen05.mma per k-block into one of two
-//                     TMEM accumulators (2 x BN columns); tcgen05.commit frees the stage and,
+//   warp 1 / lane 0 : MMA issuer, 4 k-steps of 8 x 3 tcgen05.mma per k-block into one of the
+//                     TMEM accumulators (two of BN columns); tcgen05.commit frees the stage and,
 //                     after a tile's last k-block, hands the accumulator to the epilogue;
 //   warps 2 .. 5    : epilogue, tcgen05.ld of the accumulator (warp w reads TMEM lanes
 //                     32 (w % 4) .. + 31 = tile rows), then the Epi functor, then the
@@ -24,7 +24,7 @@
 // the epilogue adds the partials in registers (fp32, round to nearest, in k order) and runs the
 // Epi functor once per tile on their sum. The accumulator then never holds more than
 // 3 CHUNK BK / 8 instructions' worth of products, whatever K is. This mode takes four TMEM
-// accumulators (4 x BN columns), so the issuer can run two chunks ahead of an epilogue that
+// accumulators (4 x BN columns), so the issuer can fill up to three chunks while the epilogue
 // is still writing out the previous tile.
 // A launch may hold several problems (a grouped GEMM): the operand tensor maps cover whole
 // planes and every problem only moves the tile origins.
