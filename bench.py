@@ -444,8 +444,9 @@ def _e2e(args, torch, bk, solver, stream, dev, ws, m, n, bits, Ws, HO, HI, sc,
     from pinned host memory to the device (W*, the scales and either H_O, H_I or, with
     --hessian, the samples X and G), runs the whole path, and copies the codes and the loss
     back. A step's input copies run on a copy stream into one of two device input sets while
-    the previous step computes (the copy engines and the SMs work at the same time); every
-    copy of every step lies inside the timed region."""
+    the previous step computes, and its results are copied device to device into a staging
+    buffer and read back on a third stream while the next step computes (the copy engines and
+    the SMs work at the same time); every copy of every step lies inside the timed region."""
     hW = torch.from_numpy(Ws_np).pin_memory()
     hs = torch.from_numpy(s_np).pin_memory()
     if hess is None:
@@ -460,9 +461,13 @@ def _e2e(args, torch, bk, solver, stream, dev, ws, m, n, bits, Ws, HO, HI, sc,
              torch.empty_like(shapes[1])) for _ in range(2)]
     hcodes = torch.empty((m, n), dtype=torch.int8).pin_memory()
     hloss = torch.empty((1,), dtype=torch.float64).pin_memory()
+    dcodes = torch.empty((m, n), dtype=torch.int8, device=dev)     # staging for the read-back
+    dloss = torch.empty((1,), dtype=torch.float64, device=dev)
     h2d = sum(x.numel() * x.element_size() for x in (hW, hs) + h_in)
     d2h = m * n + 8
     copy_stream = torch.cuda.Stream(device=dev)
+    back_stream = torch.cuda.Stream(device=dev)
+    staged, read_back = torch.cuda.Event(), torch.cuda.Event()
     copied = [torch.cuda.Event(), torch.cuda.Event()]
     consumed = [torch.cuda.Event(), torch.cuda.Event()]
     used = [False, False]
@@ -491,8 +496,17 @@ def _e2e(args, torch, bk, solver, stream, dev, ws, m, n, bits, Ws, HO, HI, sc,
                 solver.run(dW2, HO, HI, ds2, bits, stream, seed=seed, **(quant or {}))
             consumed[b].record(stream)
             used[b] = True
-            hcodes.copy_(solver.codes, non_blocking=True)
-            hloss.copy_(solver.loss, non_blocking=True)
+            # the staging buffer is free once the previous step's read-back has finished
+            if k > 0:
+                stream.wait_event(read_back)
+            dcodes.copy_(solver.codes, non_blocking=True)
+            dloss.copy_(solver.loss, non_blocking=True)
+            staged.record(stream)
+            back_stream.wait_event(staged)
+            with torch.cuda.stream(back_stream):
+                hcodes.copy_(dcodes, non_blocking=True)
+                hloss.copy_(dloss, non_blocking=True)
+            read_back.record(back_stream)
 
     run_steps(1)
     torch.cuda.synchronize()
@@ -503,6 +517,7 @@ def _e2e(args, torch, bk, solver, stream, dev, ws, m, n, bits, Ws, HO, HI, sc,
     e0.record(stream)
     copy_stream.wait_event(e0)        # the first prefetch starts inside the timed region
     run_steps(args.steps)
+    stream.wait_event(read_back)      # the last read-back ends inside the timed region
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, dev)
