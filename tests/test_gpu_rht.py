@@ -6,7 +6,10 @@ rotated solve, against the fp64 oracle (run on a B200), through the C ABI.
   pattern and the magnitude are compared exactly (all index and sign logic of both passes).
 * Random inputs: relative Frobenius error at most 2e-5 against the oracle. The bound is the
   worst case of the arithmetic: each butterfly level adds at most sqrt(2) u of the norm
-  (u = 2^-24), an order-28 sum at most 27 sqrt(28) u of its inputs' norm, over both sides;
+  (u = 2^-24), an order-28 sum at most 27 sqrt(28) u of its inputs' norm, over both sides.
+  Rows of 28 * 2^k >= 1792 form the order-28 sums on the tensor cores: the data split hi + lo
+  (lo truncated to tf32: at most 2^-21 of the value), 56 terms accumulated in fp32 without
+  round-to-nearest (at most 2^-23 of the running sum each), about 7e-6 of the inputs' norm;
   typical errors are near 1e-7.
 * Full size (the 4096 x 14336 and 28672 x 8192 layers, and shapes that reach the row lengths
   2048, 16384 and 32768): sampled entries against the oracle's rows of T, the round trip and
